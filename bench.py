@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the routed quantized-expert MoE FFN layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one full MoE layer forward (router -> top-10 -> grouping -> fused
+dequant gate/up + SwiGLU -> down -> gate-weighted combine with the shared
+expert) over one batch of decode tokens, through the C ABI.  Headline
+workload: 512 experts, hidden 2048, expert intermediate 768, top-10 + 1 shared,
+4-bit blocks of 32 with fp16 scales, 16 decode tokens.  Steps rotate over
+distinct seeded layer instances (and 16 distinct token batches), so the
+expert bytes a step touches are never still in the 126 MB L2 from an earlier
+step.  Prints one JSON line (rank 0).  Under torchrun every rank runs its own
+replica (no data-path collective: the path shards by independent batches).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+EXPERT_BYTES = {4: 2654208, 2: 1769472}     # packed gate/up + down of one expert (H=2048, I=768)
+GU_BYTES = {4: 1769472, 2: 1179648}
+ROUTER_BYTES = 512 * 2048 * 2
+METRIC = "MoE-layer decode tokens/s (512 experts, top-10 + shared, H=2048, I=768, 4-bit/32, 16 tokens)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tokens", type=int, default=16)
+    ap.add_argument("--instances", type=int, default=48, help="distinct layer instances rotated over")
+    ap.add_argument("--no-detail", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=2)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ utils ---
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+# --------------------------------------------------------------- oracle ---
+
+def oracle_sample(tokens: int):
+    """Times the CPU oracle (as it stands) on the first `tokens` tokens of the
+    headline workload.  Input generation happens before the clock starts."""
+    import moe_inputs as mi
+    import oracle as orc
+    shape = mi.FULL4
+    x = mi.hidden_states_bf16(16, shape.hidden, 0, 0)[:tokens]
+    rw = mi.router_weight_bf16(shape, 0, 0)
+    logits = orc.router_logits(orc.bf16_to_f64(x), rw, None)
+    need = sorted(set(orc.select_topk(logits, shape.top_k).reshape(-1).tolist()))
+    packed = {e: mi.expert_packed(shape, 0, 0, e) for e in need}
+    sh = mi.shared_packed(shape, 0, 0)
+    lay = orc.OracleLayer(experts=shape.experts, hidden=shape.hidden, inter=shape.inter, top_k=shape.top_k,
+                          bits=shape.bits, block=shape.block, router_w_bits=rw, router_bias=None,
+                          expert=lambda e: packed[e], shared=lambda: sh, cache_size=4)
+    t0 = time.perf_counter()
+    orc.layer_forward(lay, x)
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{tokens} decode tokens of the 16-token headline batch (layer 0, seed 0), float64 numpy; "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = max(1, args.steps if args.steps < 5 else 1)
+    tot_tok, tot_t = 0, 0.0
+    cb = None
+    for _ in range(steps):
+        cb = oracle_sample(args.cpu_sample_tokens)
+        tot_tok += args.cpu_sample_tokens
+        tot_t += args.cpu_sample_tokens / cb["value"]
+    v = tot_tok / tot_t
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": 0, "ms_per_step": 1000.0 * tot_t / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "full-shape MoE layer decode, 16 tokens, 4-bit/32 (CPU oracle on a token sample)",
+                       "experts": 512, "hidden": 2048, "inter": 768, "top_k": 10, "shared": 1, "bits": 4,
+                       "block": 32, "tokens": 16},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- GPU ---
+
+class Runner:
+    def __init__(self, torch, q, mi, md):
+        self.torch, self.q, self.mi, self.md = torch, q, mi, md
+
+    def layers(self, shape, n, zipf=False, seed=0):
+        return [self.q.LayerWeights(**self.md.device_layer_tensors(shape, seed, l, zipf=zipf)) for l in range(n)]
+
+    def xbatches(self, shape, T, n, seed=0, base=100):
+        return [self.torch.from_numpy(self.mi.hidden_states_bf16(T, shape.hidden, seed, base + b).view(np.int16))
+                .to("cuda") for b in range(n)]
+
+    def touched(self, shape, cfg, layers, xs, steps):
+        """Distinct routed experts each step selects (from the routing itself)."""
+        torch, q = self.torch, self.q
+        T = xs[0].shape[0]
+        ws = torch.empty(q.moe_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+        idx = torch.empty((T, shape.top_k), dtype=torch.int32, device="cuda")
+        wt = torch.empty((T, shape.top_k), dtype=torch.float32, device="cuda")
+        cnt = torch.empty(shape.experts, dtype=torch.int32, device="cuda")
+        us = []
+        for i in range(steps):
+            w = layers[i % len(layers)]
+            q.moe_route(cfg, w.router_w, w.router_bias, xs[i % len(xs)], idx, wt, ws, counts=cnt)
+            us.append(int((cnt > 0).sum().item()))
+        return us
+
+    def timed_graph(self, fn, K, W, chunk=32):
+        """Warm-up W steps, then exactly K steps replayed from CUDA graphs of
+        `chunk` steps (remainder in a second graph); returns elapsed ms."""
+        torch = self.torch
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for i in range(max(W, 1)):
+                fn(i)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        graphs = []
+        full, rem = divmod(K, chunk)
+        for n, offset in ((chunk if full else 0, 0), (rem, full * chunk)):
+            if n == 0:
+                graphs.append(None)
+                continue
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for i in range(n):
+                    fn(offset + i)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        return graphs, full
+
+    def replay(self, graphs, full):
+        torch = self.torch
+        st = torch.cuda.current_stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(st)
+        for _ in range(full):
+            graphs[0].replay()
+        if graphs[1] is not None:
+            graphs[1].replay()
+        b.record(st)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+
+def barrier(dist, world):
+    if world > 1:
+        dist.barrier()
+
+
+def max_over_ranks(dist, world, v: float) -> float:
+    if world <= 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(dist, world, v: float) -> float:
+    if world <= 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    import moe_inputs as mi
+    import moe_inputs.device as md
+    import quantized_expert_ffn_moe_b200 as q
+    q.load_library()          # fails loudly if the CUDA library is missing
+    md.load()
+    R = Runner(torch, q, mi, md)
+    hbm_peak, tf_peak, tf_sust, peak_src = measured_peaks()
+    shape = mi.FULL4
+    cfg = q.config_of(shape.experts, shape.hidden, shape.inter, shape.top_k, True, shape.bits, shape.block)
+    T, K, W = args.tokens, args.steps, max(3, args.warmup)
+    NI = args.instances
+    pool = R.layers(shape, NI)
+    NX = 16
+    xs = R.xbatches(shape, T, NX)
+    ys = [torch.empty_like(xs[0]) for _ in range(4)]
+    ws = torch.empty(q.moe_workspace_bytes(cfg, max(T, 4096)), dtype=torch.uint8, device="cuda")
+
+    def step(i):
+        q.moe_layer_forward(cfg, pool[i % NI], xs[i % NX], ys[i % 4], ws)
+
+    # ---- headline: exactly K steps, device-timed, max over ranks
+    graphs, full = R.timed_graph(step, K, W)
+    barrier(dist, world)
+    clk = Clocks(local)
+    clk.start()
+    ms = R.replay(graphs, full)
+    clocks = clk.stop()
+    del graphs
+    ms = max_over_ranks(dist, world, ms)
+    tokens_all = sum_over_ranks(dist, world, float(T * K))
+    value = tokens_all / (ms / 1000.0)
+    ms_step = ms / K
+    assert q.moe_device_status(ws) == 0, "device-side check failed"
+
+    # ---- bytes the steps touch, and per-phase times (events on the launch stream)
+    us = R.touched(shape, cfg, pool, xs, NI * 2)
+    mean_u = float(np.mean(us))
+    touched_bytes = (mean_u + 1) * EXPERT_BYTES[4] + ROUTER_BYTES + 2 * T * 2048 * 2
+    n_prof = min(256, K)
+    torch.cuda.synchronize()
+    q.moe_profile_begin(n_prof)
+    for i in range(n_prof):
+        step(i)
+    phase_ms, calls = q.moe_profile_end()
+    gu_ms = phase_ms[1] / calls
+    gu_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * GU_BYTES[4]
+    roofline = {"bound": "hbm", "kernel": "ffn_tma_kernel<gate/up>", "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9,
+                "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": None,
+                "peak_source": f"{peak_src} (copy bandwidth)",
+                "phase_us": {"route": 1000 * phase_ms[0] / calls, "gate_up": 1000 * phase_ms[1] / calls,
+                             "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls}}
+    roofline["frac"] = roofline["achieved"] / hbm_peak
+
+    # ---- end to end: pinned host x -> device -> layer -> host y, every step
+    x_host = [xs[i].cpu().pin_memory() for i in range(NX)]
+    y_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(4)]
+    xd = torch.empty_like(xs[0])
+
+    def e2e_step(i):
+        xd.copy_(x_host[i % NX], non_blocking=True)
+        q.moe_layer_forward(cfg, pool[i % NI], xd, ys[i % 4], ws)
+        y_host[i % 4].copy_(ys[i % 4], non_blocking=True)
+
+    Ke = min(K, 4000)
+    graphs, full = R.timed_graph(e2e_step, Ke, W)
+    barrier(dist, world)
+    ems = max_over_ranks(dist, world, R.replay(graphs, full))
+    del graphs
+    e2e = {"value": sum_over_ranks(dist, world, float(T * Ke)) / (ems / 1000.0), "unit": "tokens/s",
+           "h2d_bytes_per_step": T * 2048 * 2, "d2h_bytes_per_step": T * 2048 * 2,
+           "path": "pinned host x -> device, moe_layer_forward, device y -> pinned host, per step"}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp16x2 dequant-dot + fp32 accumulate (bf16 activations, 4-bit codes)", "data": "synthetic",
+            "config": {"workload": "full-shape MoE layer decode (512 experts, H 2048, I 768, top-10 + shared, "
+                                   "4-bit/32 fp16 scales), 16 tokens per step",
+                       "tokens": T, "experts": 512, "hidden": 2048, "inter": 768, "top_k": 10, "shared": 1,
+                       "bits": 4, "block": 32, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: steps rotate over {NI} distinct layer instances "
+                             f"({NI * (512 * EXPERT_BYTES[4] + EXPERT_BYTES[4] + ROUTER_BYTES) / 1e9:.1f} GB) "
+                             f"and {NX} token batches"},
+            "hbm": {"touched_bytes_per_step": touched_bytes, "distinct_experts_per_step": mean_u,
+                    "achieved_gbs": touched_bytes / (ms_step * 1e-3) / 1e9,
+                    "frac_of_measured": touched_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak,
+                    "frac_of_8tbs": touched_bytes / (ms_step * 1e-3) / 8e12},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": 5 * K, "clocks": clocks}
+
+    # ---- secondary workloads of the same layer family
+    if not args.no_detail:
+        line["detail"] = detail(R, args, pool, ws, W, hbm_peak, tf_peak, dist, world)
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    if world == 1:
+        line["cpu_baseline"] = oracle_sample(args.cpu_sample_tokens)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
+    torch, q, mi = R.torch, R.q, R.mi
+    out = {}
+    shape = mi.FULL4
+    cfg = q.config_of(512, 2048, 768, 10, True, 4, 32)
+    NI = len(pool4)
+
+    def layer_rate(cfg, shape, pool, T, K, bits, name, zipf=False):
+        xs = R.xbatches(shape, T, 8, base=300 + T)
+        ys = [torch.empty_like(xs[0]) for _ in range(2)]
+
+        def step(i):
+            q.moe_layer_forward(cfg, pool[i % len(pool)], xs[i % len(xs)], ys[i % 2], ws)
+        graphs, full = R.timed_graph(step, K, 3, chunk=min(32, K))
+        barrier(dist, world)
+        ms = max_over_ranks(dist, world, R.replay(graphs, full))
+        us = R.touched(shape, cfg, pool, xs, min(K, 2 * len(pool)))
+        mb = (np.mean(us) + 1) * EXPERT_BYTES[bits] + ROUTER_BYTES
+        r = {"tokens": T, "steps": K, "us_per_step": 1000 * ms / K, "tokens_per_s": T * K / (ms / 1000),
+             "distinct_experts": float(np.mean(us)), "touched_mb": mb / 1e6,
+             "achieved_gbs": mb / (ms / K * 1e-3) / 1e9}
+        r["frac_of_measured_hbm"] = r["achieved_gbs"] / hbm_peak
+        if T > 64:
+            flops = 9437184.0 * (T * 10 + T)
+            r["tflops"] = flops / (ms / K * 1e-3) / 1e12
+            r["frac_of_measured_bf16"] = r["tflops"] / tf_peak
+        out[name] = r
+
+    for T in (1, 4):
+        layer_rate(cfg, shape, pool4, T, 4000, 4, f"decode4_t{T}")
+    layer_rate(cfg, shape, pool4, 4096, 8, 4, "prefill4_t4096")
+    # 2-bit skewed routing
+    s2 = mi.FULL2
+    cfg2 = q.config_of(512, 2048, 768, 10, True, 2, 16)
+    pool2 = R.layers(s2, 16, zipf=True)
+    for T in (1, 8, 64):
+        layer_rate(cfg2, s2, pool2, T, 2000, 2, f"zipf2_t{T}", zipf=True)
+    del pool2
+    torch.cuda.empty_cache()
+    # 48-layer stack: residual stream through all layers resident in HBM
+    if NI >= 48:
+        for T in (1, 32):
+            xs = R.xbatches(shape, T, 4, base=500 + T)
+            xw = torch.empty_like(xs[0])
+
+            def sstep(i):
+                xw.copy_(xs[i % 4])
+                q.moe_stack_forward(cfg, pool4[:48], xw, ws)
+            K = 20 if T == 1 else 10
+            graphs, full = R.timed_graph(sstep, K, 2, chunk=K)
+            barrier(dist, world)
+            ms = max_over_ranks(dist, world, R.replay(graphs, full))
+            out[f"stack48_t{T}"] = {"tokens": T, "steps": K, "ms_per_step": ms / K,
+                                    "tokens_per_s": T * K / (ms / 1000)}
+    return out
+
+
+if __name__ == "__main__":
+    main()

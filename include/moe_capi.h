@@ -1,0 +1,149 @@
+/*
+ * moe_capi.h -- C ABI of the routed, quantized-expert MoE FFN layer for B200
+ * (sm_100a).  Library: libmoe.so (built in-tree into quantized_expert_ffn_moe_b200/).
+ *
+ * The operation.  The transformer block's FFN is replaced by many parallel
+ * expert sub-networks plus a light gating network (router) that picks the
+ * Top-K experts per token ("Running a 125B Model on a Single RTX 5090: Strata
+ * Benchmarks Qwen3.8 Flash Next", section "Layer 1: On-Demand MoE Expert
+ * Scheduling"); 512 experts per layer with 10 selected per token ("Strata Open
+ * Source Project: Run a 125B Model Locally on a Home PC", section "How Strata
+ * Makes Your Entire PC Work Together"); one shared expert is active for every
+ * token besides the routed ones ("How a 125B Model Reaches 100 Tok/s on an RTX
+ * 4090", section "The model is large on paper, sparse in practice"); expert
+ * weights are symmetric, group-wise quantised 4-bit or 2-bit integers
+ * ("Running Massive Language Models on Consumer Hardware Without Breaking the
+ * Bank", section "Quantization Techniques That Actually Work").
+ *
+ * Per token x (bf16, hidden H):
+ *   l_e   = sum_h x_h Wr[e,h] (+ b_e)                  fp32 accumulation
+ *   S     = the k largest l_e, slots by descending logit, ties -> smaller e
+ *   w_j   = softmax over the selected logits (= full softmax renormalised)
+ *   FFN_e = W_down,e (silu(W_gate,e x) * (W_up,e x)),   W = (code - 2^(b-1)) * scale
+ *   out   = FFN_shared(x) + sum_j w_j FFN_{S_j}(x)      slot order, fp32, -> bf16
+ *
+ * Packed weight format (all arrays row-major, dense, caller-owned, device
+ * memory, 16-byte aligned):
+ *   codes : one byte holds 8/bits elements of a row; element j of a row is at
+ *           byte j*bits/8, bit offset (j*bits)%8 (lower element in lower bits);
+ *           stored code c = q + 2^(bits-1), q in [-(2^(bits-1)-1), 2^(bits-1)-1]
+ *   scales: one IEEE fp16 per block of `block` consecutive elements of a row
+ *   gate/up: one [2I, H] matrix per expert, row 2i = gate row i, row 2i+1 =
+ *           up row i; down: [H, I] per expert.  Experts are stacked densely.
+ * Supported: bits/block in {4/32, 2/16}; H % 256 == 0; I % 128 == 0;
+ * 1 <= k <= 16, k <= E <= 1024; shared_inter in {0, inter}.
+ *
+ * Conventions.  All calls are asynchronous on `stream` (a cudaStream_t passed
+ * as void*; NULL = legacy default stream) and never allocate or free device
+ * memory: scratch comes from the caller's `workspace` (device, 256-byte
+ * aligned, at least moe_workspace_bytes()).  Arguments are validated on the
+ * host before any launch; on error nothing is launched and a negative
+ * moe_status is returned.  T == 0 returns MOE_OK and launches nothing.  The
+ * same inputs give bitwise identical outputs on every call (no float atomics).
+ * Calls that share a workspace must not overlap in time on the device.
+ */
+#ifndef MOE_CAPI_H
+#define MOE_CAPI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,   /* null/misaligned pointer, negative size         */
+  MOE_ERR_UNSUPPORTED = -2,   /* shape or format outside the supported set       */
+  MOE_ERR_WORKSPACE = -3,     /* workspace smaller than moe_workspace_bytes()    */
+  MOE_ERR_CUDA = -4,          /* a CUDA runtime call failed (see moe_status_str) */
+  MOE_ERR_DEVICE_CHECK = -5,  /* a kernel's own check failed (moe_device_status) */
+  MOE_ERR_TIMEOUT = -6        /* a bounded device wait gave up                   */
+} moe_status;
+
+typedef struct moe_config {
+  int32_t num_experts;   /* E                                    */
+  int32_t hidden;        /* H                                    */
+  int32_t inter;         /* I, intermediate size of each expert  */
+  int32_t top_k;         /* k                                    */
+  int32_t shared_inter;  /* 0 = no shared expert, else == inter  */
+  int32_t bits;          /* 4 or 2                               */
+  int32_t block;         /* 32 (4-bit) or 16 (2-bit)             */
+} moe_config;
+
+/* One layer's weights; every pointer is device memory owned by the caller. */
+typedef struct moe_layer_weights {
+  const uint8_t*  gate_up_codes;          /* [E][2I][H*bits/8]                  */
+  const uint16_t* gate_up_scales;         /* [E][2I][H/block] fp16 bits         */
+  const uint8_t*  down_codes;             /* [E][H][I*bits/8]                   */
+  const uint16_t* down_scales;            /* [E][H][I/block]                    */
+  const uint8_t*  shared_gate_up_codes;   /* [2I][H*bits/8]; NULL if no shared  */
+  const uint16_t* shared_gate_up_scales;  /* [2I][H/block]                      */
+  const uint8_t*  shared_down_codes;      /* [H][I*bits/8]                      */
+  const uint16_t* shared_down_scales;     /* [H][I/block]                       */
+  const uint16_t* router_w;               /* [E][H] bf16 bits                   */
+  const float*    router_bias;            /* [E] fp32, or NULL (no bias)        */
+} moe_layer_weights;
+
+/* Bytes of device workspace needed by moe_route / moe_layer_forward /
+ * moe_stack_forward for up to max_tokens tokens.  Returns 0 for an invalid or
+ * unsupported config or max_tokens < 0. */
+size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens);
+
+/* Router and grouping only (the selection and gate weights of the operation
+ * above, plus the per-expert token lists).  Inputs: router_w [E][H] bf16,
+ * router_bias [E] or NULL, x [T][H] bf16.  Outputs (device, caller-owned):
+ *   topk_idx [T][k] int32 (slots by descending logit), topk_w [T][k] fp32,
+ *   expert_counts [E], expert_offsets [E+1] (exclusive prefix sum),
+ *   pairs [T*k]: pair ids t*k+j sorted by expert, then by token.
+ * Any output pointer may be NULL except topk_idx and topk_w. */
+int moe_route(const moe_config* cfg, const uint16_t* router_w, const float* router_bias,
+              const uint16_t* x, int32_t T, int32_t* topk_idx, float* topk_w,
+              int32_t* expert_counts, int32_t* expert_offsets, int32_t* pairs,
+              void* workspace, size_t ws_bytes, void* stream);
+
+/* One MoE layer: y[T][H] (bf16) = out as defined above for x[T][H] (bf16).
+ * x and y may not overlap.  T <= 64 takes the decode path (grouped GEMV on
+ * CUDA cores); larger T takes the prefill path. */
+int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w,
+                      const uint16_t* x, int32_t T, uint16_t* y,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* L layers in sequence on the residual stream, in place:
+ *   for l in 0..L-1:  x <- bf16(x + moe_l(bf16(rmsnorm(x))))
+ * rmsnorm(x) = x / sqrt(mean(x^2) + 1e-6) per token (weight 1).
+ * layers: HOST array of L weight structs (device pointers inside).
+ * topk_trace: NULL, or device int32 [L][T][k] that receives each layer's
+ * selection (for validation). */
+int moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, int32_t L,
+                      uint16_t* x_inout, int32_t T, int32_t* topk_trace,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Reads back the device check word kept in the workspace (synchronises the
+ * device).  *code_out = 0 when no kernel reported a failed check. */
+int moe_device_status(const void* workspace, int32_t* code_out);
+
+/* Test hook: rows [row0, row0+rows) of a packed matrix with `cols` columns,
+ * decoded by the same device routine the GEMV kernels use, written as fp32
+ * out[rows][cols].  Not on the timed path. */
+int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t* scales,
+                     int32_t row0, int32_t rows, int32_t cols, float* out, void* stream);
+
+/* Measurement hook.  moe_profile_begin(n) makes the next n layer calls
+ * record CUDA events around their four phases on the call's stream (route,
+ * gate/up + SwiGLU, down, combine); moe_profile_end() waits for those events
+ * and returns the summed milliseconds per phase in ms_out[4] and the number of
+ * recorded calls in *calls.  Events are host-side driver objects; no device
+ * memory is allocated.  Not thread-safe; meant for benchmarks. */
+int moe_profile_begin(int32_t max_calls);
+int moe_profile_end(float* ms_out, int32_t* calls);
+
+/* Static description of a status code. */
+const char* moe_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_CAPI_H */

@@ -1,0 +1,161 @@
+// Device side of the seeded input generator (libmoe_inputs.so).  Same recipe
+// as moe_inputs/gen.py, using only integer arithmetic and single correctly
+// rounded fp32 operations so that both sides produce identical bytes:
+//   SplitMix64 output function as a counter-based hash, Irwin-Hall sum of the
+//   four 16-bit fields as an approximate normal deviate, fp32 masters, and the
+//   symmetric absmax block encoder of the packed weight format.
+// This library prepares inputs only; it is not part of the MoE layer.
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace {
+
+constexpr uint64_t kGolden = 0x9E3779B97F4A7C15ull;
+enum { ROLE_ROUTER = 0, ROLE_GATE = 1, ROLE_UP = 2, ROLE_DOWN = 3, ROLE_SH_GATE = 4, ROLE_SH_UP = 5,
+       ROLE_SH_DOWN = 6 };
+
+__host__ __device__ inline uint64_t mix64(uint64_t z) {
+  z ^= z >> 30;
+  z *= 0xBF58476D1CE4E5B9ull;
+  z ^= z >> 27;
+  z *= 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return z;
+}
+
+__host__ __device__ inline uint64_t stream_key(uint64_t seed, uint64_t layer, uint64_t role, uint64_t expert) {
+  uint64_t k = mix64(seed);
+  k = mix64(k + layer);
+  k = mix64(k + role);
+  k = mix64(k + expert);
+  return k;
+}
+
+__device__ inline float normal_at(uint64_t key, uint64_t i, float c) {
+  const uint64_t z = mix64(key + (i + 1) * kGolden);
+  const int s = int(z & 0xFFFF) + int((z >> 16) & 0xFFFF) + int((z >> 32) & 0xFFFF) + int(z >> 48);
+  const int d = 2 * s - 262140;
+  return __fmul_rn(float(d), c);
+}
+
+struct PoolArgs {
+  uint64_t seed;
+  int layer, E, H, I, bits, block;
+  int e0, ne, shared;
+  float c;
+  uint8_t* gu_codes;
+  uint16_t* gu_scales;
+  uint8_t* d_codes;
+  uint16_t* d_scales;
+};
+
+// One thread per quantisation block.
+__global__ void gen_pool_kernel(PoolArgs a) {
+  const long long gu_blocks = (long long)2 * a.I * (a.H / a.block);
+  const long long d_blocks = (long long)a.H * (a.I / a.block);
+  const long long per_expert = gu_blocks + d_blocks;
+  const long long total = per_expert * a.ne;
+  const int qmax = (1 << (a.bits - 1)) - 1;
+  for (long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x; tid < total;
+       tid += (long long)gridDim.x * blockDim.x) {
+    const int slot = int(tid / per_expert);
+    long long b = tid % per_expert;
+    const int expert = a.shared ? 0 : a.e0 + slot;
+    int role, row, col0, K;
+    bool is_gu = b < gu_blocks;
+    int packed_row;
+    if (is_gu) {
+      const int bpr = a.H / a.block;
+      packed_row = int(b / bpr);
+      col0 = int(b % bpr) * a.block;
+      row = packed_row >> 1;
+      role = (packed_row & 1) ? (a.shared ? ROLE_SH_UP : ROLE_UP) : (a.shared ? ROLE_SH_GATE : ROLE_GATE);
+      K = a.H;
+    } else {
+      b -= gu_blocks;
+      const int bpr = a.I / a.block;
+      packed_row = int(b / bpr);
+      col0 = int(b % bpr) * a.block;
+      row = packed_row;
+      role = a.shared ? ROLE_SH_DOWN : ROLE_DOWN;
+      K = a.I;
+    }
+    const uint64_t key = stream_key(a.seed, (uint64_t)a.layer, (uint64_t)role, (uint64_t)expert);
+    float w[32];
+    float amax = 0.f;
+    for (int j = 0; j < a.block; ++j) {
+      w[j] = normal_at(key, (uint64_t)row * K + col0 + j, a.c);
+      amax = fmaxf(amax, fabsf(w[j]));
+    }
+    const __half s16 = __float2half_rn(__fdiv_rn(amax, float(qmax)));
+    const float sf = __half2float(s16);
+    uint32_t packed[4] = {0, 0, 0, 0};   // up to 16 bytes of codes per block
+    for (int j = 0; j < a.block; ++j) {
+      int q = 0;
+      if (sf != 0.f) {
+        q = int(rintf(__fdiv_rn(w[j], sf)));
+        q = q < -qmax ? -qmax : (q > qmax ? qmax : q);
+      }
+      const uint32_t code = uint32_t(q + (1 << (a.bits - 1)));
+      const int bit = j * a.bits;
+      packed[bit >> 5] |= code << (bit & 31);
+    }
+    const int code_bytes = a.block * a.bits / 8;
+    const size_t row_bytes = size_t(K) * a.bits / 8;
+    uint8_t* cdst;
+    uint16_t* sdst;
+    if (is_gu) {
+      cdst = a.gu_codes + size_t(slot) * 2 * a.I * (size_t(a.H) * a.bits / 8) + size_t(packed_row) * row_bytes;
+      sdst = a.gu_scales + size_t(slot) * 2 * a.I * (a.H / a.block) + size_t(packed_row) * (K / a.block);
+    } else {
+      cdst = a.d_codes + size_t(slot) * a.H * (size_t(a.I) * a.bits / 8) + size_t(packed_row) * row_bytes;
+      sdst = a.d_scales + size_t(slot) * a.H * (a.I / a.block) + size_t(packed_row) * (K / a.block);
+    }
+    cdst += size_t(col0) * a.bits / 8;
+    for (int q = 0; q < code_bytes / 4; ++q) reinterpret_cast<uint32_t*>(cdst)[q] = packed[q];
+    sdst[col0 / a.block] = __half_as_ushort(s16);
+  }
+}
+
+__global__ void gen_bf16_kernel(uint64_t key, uint64_t start, uint64_t n, float c, uint16_t* out) {
+  for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n; i += (uint64_t)gridDim.x * blockDim.x) {
+    const __nv_bfloat16 b = __float2bfloat16_rn(normal_at(key, start + i, c));
+    out[i] = __bfloat16_as_ushort(b);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+// Packed pool of experts [e0, e0+ne) of one layer (shared == 0), or of the
+// shared expert (shared == 1, ne == 1).  Outputs are device buffers laid out
+// as in include/moe_capi.h, starting at the first generated expert.
+// c = fp32 sigma / 75674.45 (bits 0x348de3bd for sigma 0.02).
+int moe_gen_pool(uint64_t seed, int layer, int E, int H, int I, int bits, int block, int e0, int ne, int shared,
+                 float c, uint8_t* gu_codes, uint16_t* gu_scales, uint8_t* d_codes, uint16_t* d_scales,
+                 void* stream) {
+  if (!((bits == 4 && block == 32) || (bits == 2 && block == 16))) return -2;
+  if (ne <= 0 || (shared && ne != 1) || (!shared && (e0 < 0 || e0 + ne > E))) return -1;
+  if (!gu_codes || !gu_scales || !d_codes || !d_scales) return -1;
+  if (H % block || I % block) return -2;
+  PoolArgs a{(uint64_t)seed, layer, E, H, I, bits, block, e0, ne, shared, c, gu_codes, gu_scales, d_codes, d_scales};
+  gen_pool_kernel<<<148 * 16, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+// n bf16 values N(0, sigma) of stream `key`, elements start .. start+n-1.
+int moe_gen_normal_bf16(uint64_t key, uint64_t start, uint64_t n, float c, uint16_t* out, void* stream) {
+  if (!out) return -1;
+  if (n == 0) return 0;
+  gen_bf16_kernel<<<148 * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(key, start, n, c, out);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+uint64_t moe_gen_stream_key(uint64_t seed, int layer, int role, int expert) {
+  return stream_key(seed, (uint64_t)layer, (uint64_t)role, (uint64_t)expert);
+}
+
+}  // extern "C"

@@ -1,0 +1,99 @@
+// Gate-weighted combine: out[t] = Y[shared, t] + sum_j Y[(t, j)] in fixed slot
+// order (the gate weight is already inside Y), fp32, rounded once to bf16.
+// The shared expert is added with weight 1 ("How a 125B Model Reaches 100
+// Tok/s on an RTX 4090", section "The model is large on paper, sparse in
+// practice": 10 routed experts plus one shared expert are active per token).
+// In the stack the residual add and the next layer's RMSNorm are fused here:
+// x <- bf16(x + out), xhat <- bf16(x / sqrt(mean(x^2) + 1e-6)).
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCombThreads = 256;
+
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(
+    const float* __restrict__ Y, const int* __restrict__ inv, int T, int k, int H, int shared,
+    uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next) {
+  pdl_wait();
+  const int t = blockIdx.x;
+  const int P_routed = T * k;
+  int pos[16];
+  for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+  float ss = 0.f;
+  constexpr int VPT = 8;                      // elements per thread per step
+  for (int h0 = threadIdx.x * VPT; h0 < H; h0 += kCombThreads * VPT) {
+    float acc[VPT];
+    if (shared) {
+      const float4 a = *reinterpret_cast<const float4*>(Y + size_t(P_routed + t) * H + h0);
+      const float4 b = *reinterpret_cast<const float4*>(Y + size_t(P_routed + t) * H + h0 + 4);
+      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) acc[i] = 0.f;
+    }
+    for (int j = 0; j < k; ++j) {
+      const float* row = Y + size_t(pos[j]) * H + h0;
+      const float4 a = *reinterpret_cast<const float4*>(row);
+      const float4 b = *reinterpret_cast<const float4*>(row + 4);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    uint16_t* dst = out + size_t(t) * H + h0;
+    uint16_t ob[VPT];
+    if (residual) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(dst);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += __uint_as_float(xw[i] << 16);
+        acc[2 * i + 1] += __uint_as_float(xw[i] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const __nv_bfloat16 b = __float2bfloat16_rn(acc[i]);
+      ob[i] = *reinterpret_cast<const uint16_t*>(&b);
+      const float r = __bfloat162float(b);
+      ss = fmaf(r, r, ss);
+    }
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob);
+  }
+  if (xhat_next) {
+    __shared__ float red[kCombThreads / 32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    for (int i = 0; i < kCombThreads / 32; ++i) tot += red[i];
+    const float r = 1.0f / sqrtf(tot / float(H) + 1e-6f);
+    for (int h0 = threadIdx.x * VPT; h0 < H; h0 += kCombThreads * VPT) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(out + size_t(t) * H + h0);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+      uint16_t hb[VPT];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat16 lo = __float2bfloat16_rn(__uint_as_float(xw[i] << 16) * r);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(__uint_as_float(xw[i] & 0xFFFF0000u) * r);
+        hb[2 * i] = *reinterpret_cast<const uint16_t*>(&lo);
+        hb[2 * i + 1] = *reinterpret_cast<const uint16_t*>(&hi);
+      }
+      *reinterpret_cast<uint4*>(xhat_next + size_t(t) * H + h0) = *reinterpret_cast<const uint4*>(hb);
+    }
+  }
+  pdl_launch_dependents();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const LayerArgs& a) {
+  const moe_config& c = a.cfg;
+  return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, a.stream,
+                    reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
+                    a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next);
+}
+
+}  // namespace moe

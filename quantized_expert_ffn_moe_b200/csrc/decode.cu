@@ -1,0 +1,556 @@
+// Decode path: grouped GEMV over the packed rows of the selected experts.
+//
+// Per selected expert e with token list L_e (and the shared expert with all T
+// tokens): gate/up pass h = silu(W_gate x) * (W_up x), down pass
+// Y = w_(t,e) * W_down h.  The expert FFN replaces the dense FFN
+// ("Running a 125B Model on a Single RTX 5090: Strata Benchmarks Qwen3.8 Flash
+// Next", section "Layer 1: On-Demand MoE Expert Scheduling"); decode is bound
+// by moving expert weights, not by arithmetic ("125 billion parameters on one
+// gaming GPU -- first impressions of Strata + Qwen 3.8 Flash Next", section "In
+// brief": compute isn't the blocker).
+//
+// Design: every CTA takes an equal contiguous share of all (expert, row-group)
+// work units, so HBM bytes are balanced across SMs.  A warp holds the packed
+// bytes of RW x 2 rows in registers (128-bit read-only loads, each 16-byte
+// piece being one 4-bit block of 32 or four 2-bit blocks of 16), decodes them
+// to exact small integers in fp16, multiplies with the activation vector
+// staged in shared memory as fp16 (pre-scaled per token by a power of two so
+// that block partial sums cannot overflow), accumulates each block in fp16x2
+// and the blocks in fp32 with the block's fp16 scale, then reduces across the
+// lanes of the row with shuffles.  No atomics: every output element is written
+// once.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kNCW = 8;                     // consumer warps
+constexpr int kThreads = (kNCW + 1) * 32;   // + one producer warp
+constexpr int kStages = 4;                  // shared-memory ring depth
+constexpr int kSmemBudget = 220 * 1024;
+constexpr int kMaxNTC = 64;
+
+enum Mode { GATEUP = 0, DOWN = 1 };
+
+template <int BITS, int LPR, int CPL>
+struct Geom {
+  static constexpr int RW = 32 / LPR;                 // lane groups (row pairs) per warp
+  static constexpr int W16 = BITS == 4 ? 32 : 64;     // weights per 16-byte piece
+  static constexpr int K = LPR * CPL * W16;           // reduction length
+  static constexpr int NPART = BITS == 4 ? 1 : 2;     // 16-byte activation slots per code word
+  static constexpr int G = BITS == 4 ? 8 : 16;        // elements per code word
+  static constexpr int BLOCK = BITS == 4 ? 32 : 16;
+  static constexpr int SPR = K / BLOCK;               // scales per row
+  static constexpr int RB = K * BITS / 8;             // code bytes per row
+  static constexpr int RPS = kNCW * RW * 2;           // rows per pipeline stage
+  static constexpr int CODE_BYTES = RPS * RB;
+  static constexpr int SCALE_BYTES = RPS * SPR * 2;
+  static constexpr int STAGE_BYTES = (CODE_BYTES + SCALE_BYTES + 127) / 128 * 128;
+};
+
+// Offset (in halves) of element h of a staged activation row: the order in
+// which a lane of a row group meets the decoded half2 pairs (see decode_q4x8 /
+// decode_q2x16), laid out so that the lanes of a group read consecutive
+// 16-byte slots.
+template <int BITS, int LPR, int CPL>
+__device__ __forceinline__ int staged_offset(int h) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  const int c = h / Gm::W16, o = h % Gm::W16;
+  const int s = c / LPR, lr = c % LPR;
+  const int m = o / Gm::G, j = o % Gm::G;
+  const int slot = decode_slot(BITS, j);
+  const int part = slot >> 3, within = slot & 7;
+  return ((((s * 4 + m) * Gm::NPART + part) * LPR + lr) << 3) + within;
+}
+
+struct FfnArgs {
+  const uint8_t* codes;          // routed pool
+  const uint16_t* scales;
+  const uint8_t* sh_codes;       // shared expert (or null)
+  const uint16_t* sh_scales;
+  size_t expert_code_bytes;      // per routed expert
+  size_t expert_scale_count;
+  int rows;                      // rows per expert (2I gate/up, H down)
+  int out_cols;                  // columns of the output buffer (I gate/up, H down)
+  int ntc;                       // tokens staged per chunk
+  const uint16_t* xin;           // GATEUP: [T][K] bf16 activations
+  const float* hin;              // DOWN:   [P][K] fp32 intermediate
+  float* out;                    // GATEUP: h [P][I]; DOWN: Y [P][H]
+  int* status;
+  RouteView rv;
+};
+
+// Token range of a slot: routed expert e -> its sorted positions; the shared
+// expert (id E) -> positions T*k .. T*k+T-1.
+__device__ __forceinline__ void slot_tokens(const RouteView& rv, int slot, int* e_out, int* p0, int* n) {
+  const int e = __ldcg(rv.ulist + slot);
+  *e_out = e;
+  if (e >= rv.E) {
+    *p0 = rv.T * rv.k;
+    *n = rv.T;
+  } else {
+    *p0 = __ldcg(rv.offsets + e);
+    *n = __ldcg(rv.offsets + e + 1) - *p0;
+  }
+}
+
+// Cursor over the work units (slot, token chunk, row stage) of one CTA.
+struct Cursor {
+  int slot, chunk, stage, nchunks;
+};
+
+__device__ __forceinline__ int chunks_of(int n, int ntc) { return (n + ntc - 1) / ntc; }
+
+template <int MODE, int BITS, int LPR, int CPL>
+__global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  constexpr int K = Gm::K;
+  const int ntc = a.ntc;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  unsigned char* ring = smem + 256;
+  __half* xs = reinterpret_cast<__half*>(ring + kStages * Gm::STAGE_BYTES);     // [ntc][K]
+  float* tok_inv = reinterpret_cast<float*>(xs + size_t(ntc) * K);
+  float* tok_w = tok_inv + kMaxNTC;
+  int* tok_pos = reinterpret_cast<int*>(tok_w + kMaxNTC);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool producer = warp == kNCW;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kNCW);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  // The weights never depend on the previous kernel; routing was final before
+  // that kernel started.  Only the activations (h in the down pass) do.
+  if (MODE == GATEUP || !producer) pdl_wait();
+  pdl_launch_dependents();
+
+  const RouteView& rv = a.rv;
+  const int nslots = __ldcg(rv.status + ST_UCOUNT) + rv.shared;
+  const int total = __ldcg(rv.woff + nslots);
+  const int w0 = int((long long)total * blockIdx.x / gridDim.x);
+  const int w1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
+  if (w0 >= w1) return;
+  const int spe = a.rows / Gm::RPS;
+
+  // slot holding work unit w0: largest u with woff[u] <= w0
+  int lo = 0, hi = nslots - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldcg(rv.woff + mid) <= w0) lo = mid; else hi = mid - 1;
+  }
+  Cursor cur;
+  {
+    int e, p0, n;
+    slot_tokens(rv, lo, &e, &p0, &n);
+    const int within = w0 - __ldcg(rv.woff + lo);
+    cur.slot = lo;
+    cur.chunk = within / spe;
+    cur.stage = within % spe;
+    cur.nchunks = chunks_of(n, ntc);
+  }
+  auto advance = [&](Cursor& c) {
+    if (++c.stage == spe) {
+      c.stage = 0;
+      if (++c.chunk == c.nchunks) {
+        c.chunk = 0;
+        ++c.slot;
+        if (c.slot < nslots) {
+          int e, p0, n;
+          slot_tokens(rv, c.slot, &e, &p0, &n);
+          c.nchunks = chunks_of(n, ntc);
+        }
+      }
+    }
+  };
+
+  if (producer) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int w = w0; w < w1; ++w, advance(cur)) {
+        const int slot = issued % kStages;
+        if (*abort_flag) break;
+        if (issued >= kStages && !mbar_wait(&empty[slot], ((issued / kStages) - 1) & 1, abort_flag)) {
+          *abort_flag = 1;
+          report_error(a.status, MOE_ERR_TIMEOUT, 1);
+          break;
+        }
+        const int e = __ldcg(rv.ulist + cur.slot);
+        const bool sh = e >= rv.E;
+        const uint8_t* cb = sh ? a.sh_codes : a.codes + size_t(e) * a.expert_code_bytes;
+        const uint16_t* sb = sh ? a.sh_scales : a.scales + size_t(e) * a.expert_scale_count;
+        const size_t row0 = size_t(cur.stage) * Gm::RPS;
+        unsigned char* dst = ring + slot * Gm::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + Gm::SCALE_BYTES);
+        bulk_g2s(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot]);
+        bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * Gm::SPR, Gm::SCALE_BYTES, &full[slot]);
+        ++issued;
+      }
+      // never leave with copies in flight
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        if (!mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 2);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int grp = lane / LPR, lr = lane % LPR;
+  const int rl0 = (warp * Gm::RW + grp) * 2;     // local rows rl0, rl0+1 of each stage
+  int e = 0, p0 = 0, n = 0, nc = 0;
+  for (int w = w0, i = 0; w < w1; ++w, ++i, advance(cur)) {
+    if (w == w0 || cur.stage == 0) {
+      // (re)stage the activations of this slot's token chunk
+      slot_tokens(rv, cur.slot, &e, &p0, &n);
+      const bool is_shared = e >= rv.E;
+      const int tbase = cur.chunk * ntc;
+      nc = min(ntc, n - tbase);
+      named_bar_sync(1, kNCW * 32);
+      for (int tl = warp; tl < nc; tl += kNCW) {
+        const int p = p0 + tbase + tl;
+        const int row = (MODE == GATEUP) ? (is_shared ? p - rv.T * rv.k : __ldcg(rv.pairs + p) / rv.k) : p;
+        float vmax = 0.f;
+        if (MODE == GATEUP) {
+          const uint16_t* src = a.xin + size_t(row) * K;
+          for (int h = lane * 8; h < K; h += 256) {
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src + h));
+            const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+              vmax = fmaxf(vmax, fabsf(__uint_as_float(q[z] << 16)));
+              vmax = fmaxf(vmax, fabsf(__uint_as_float(q[z] & 0xFFFF0000u)));
+            }
+          }
+        } else {
+          const float* src = a.hin + size_t(row) * K;
+          for (int h = lane * 4; h < K; h += 128) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(src + h));
+            vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        int sh = 0;
+        if (vmax > 0.f) {
+          int ex;
+          frexpf(vmax, &ex);
+          sh = min(max(8 - ex, -100), 100);      // max |x * 2^sh| in [128, 256)
+        }
+        const float mul = ldexpf(1.f, sh);
+        __half* dst = xs + size_t(tl) * K;
+        for (int g0 = lane * Gm::G; g0 < K; g0 += 32 * Gm::G) {
+          float v[Gm::G];
+          if (MODE == GATEUP) {
+            const uint16_t* src = a.xin + size_t(row) * K + g0;
+#pragma unroll
+            for (int q = 0; q < Gm::G / 8; ++q) {
+              const uint4 u = __ldcg(reinterpret_cast<const uint4*>(src + 8 * q));
+              const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int z = 0; z < 4; ++z) {
+                v[8 * q + 2 * z] = __uint_as_float(wd[z] << 16);
+                v[8 * q + 2 * z + 1] = __uint_as_float(wd[z] & 0xFFFF0000u);
+              }
+            }
+          } else {
+            const float* src = a.hin + size_t(row) * K + g0;
+#pragma unroll
+            for (int q = 0; q < Gm::G / 4; ++q) {
+              const float4 u = __ldcg(reinterpret_cast<const float4*>(src + 4 * q));
+              v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+            }
+          }
+          __align__(16) __half hv[Gm::G];
+#pragma unroll
+          for (int j = 0; j < Gm::G; ++j) hv[decode_slot(BITS, j)] = __float2half_rn(v[j] * mul);
+          const int base = staged_offset<BITS, LPR, CPL>(g0);
+#pragma unroll
+          for (int part = 0; part < Gm::NPART; ++part)
+            *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+        }
+        if (lane == 0) {
+          tok_inv[tl] = ldexpf(1.f, -sh);
+          tok_pos[tl] = p;
+          tok_w[tl] = (MODE == DOWN && !is_shared) ? __ldcg(rv.topk_w + __ldcg(rv.pairs + p)) : 1.f;
+        }
+      }
+      named_bar_sync(1, kNCW * 32);
+    }
+
+    const int slot = i % kStages;
+    bool ok = !*abort_flag;
+    if (ok && !mbar_wait(&full[slot], (i / kStages) & 1, abort_flag)) {
+      ok = false;
+      *abort_flag = 1;
+      report_error(a.status, MOE_ERR_TIMEOUT, 3);
+    }
+    if (ok) {
+      const unsigned char* st = ring + slot * Gm::STAGE_BYTES;
+      const unsigned char* crow0 = st + rl0 * Gm::RB;
+      const unsigned char* srow0 = st + Gm::CODE_BYTES + rl0 * Gm::SPR * 2;
+      const int r0 = cur.stage * Gm::RPS + rl0;    // row of the expert matrix
+#pragma unroll 1
+      for (int tp = 0; tp < nc; tp += 2) {
+        const bool two = tp + 1 < nc;
+        float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int s = 0; s < CPL; ++s) {
+          const int c = s * LPR + lr;
+          uint4 cw[2];
+          cw[0] = *reinterpret_cast<const uint4*>(crow0 + c * 16);
+          cw[1] = *reinterpret_cast<const uint4*>(crow0 + Gm::RB + c * 16);
+          const uint32_t wd[2][4] = {{cw[0].x, cw[0].y, cw[0].z, cw[0].w}, {cw[1].x, cw[1].y, cw[1].z, cw[1].w}};
+          if (BITS == 4) {
+            float sc[2];
+#pragma unroll
+            for (int rho = 0; rho < 2; ++rho)
+              sc[rho] = __half2float(*reinterpret_cast<const __half*>(srow0 + rho * Gm::SPR * 2 + c * 2));
+            __half2 hacc[2][2];
+#pragma unroll
+            for (int rho = 0; rho < 2; ++rho) hacc[rho][0] = hacc[rho][1] = __float2half2_rn(0.f);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              __half2 q[2][4];
+              decode_q4x8(wd[0][m], q[0]);
+              decode_q4x8(wd[1][m], q[1]);
+              const int off = ((s * 4 + m) * LPR + lr) * 8;
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                if (t == 0 || two) {
+                  const uint4 xv = *reinterpret_cast<const uint4*>(xs + size_t(tp + t) * K + off);
+                  const __half2 x2[4] = {u32_as_h2(xv.x), u32_as_h2(xv.y), u32_as_h2(xv.z), u32_as_h2(xv.w)};
+#pragma unroll
+                  for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+                    for (int z = 0; z < 4; ++z) hacc[rho][t] = __hfma2(q[rho][z], x2[z], hacc[rho][t]);
+                }
+              }
+            }
+#pragma unroll
+            for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                const float2 f = __half22float2(hacc[rho][t]);
+                acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
+              }
+          } else {
+            uint2 scp[2];
+#pragma unroll
+            for (int rho = 0; rho < 2; ++rho)
+              scp[rho] = *reinterpret_cast<const uint2*>(srow0 + rho * Gm::SPR * 2 + c * 8);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              __half2 q[2][8];
+              decode_q2x16(wd[0][m], q[0]);
+              decode_q2x16(wd[1][m], q[1]);
+              const int off = ((s * 4 + m) * 2 * LPR + lr) * 8;
+              float sc[2];
+#pragma unroll
+              for (int rho = 0; rho < 2; ++rho) {
+                const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
+                sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
+              }
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                if (t == 0 || two) {
+                  const __half* xr = xs + size_t(tp + t) * K + off;
+                  const uint4 xa = *reinterpret_cast<const uint4*>(xr);
+                  const uint4 xb = *reinterpret_cast<const uint4*>(xr + LPR * 8);
+                  const __half2 x2[8] = {u32_as_h2(xa.x), u32_as_h2(xa.y), u32_as_h2(xa.z), u32_as_h2(xa.w),
+                                         u32_as_h2(xb.x), u32_as_h2(xb.y), u32_as_h2(xb.z), u32_as_h2(xb.w)};
+#pragma unroll
+                  for (int rho = 0; rho < 2; ++rho) {
+                    __half2 h2 = __float2half2_rn(0.f);
+#pragma unroll
+                    for (int z = 0; z < 8; ++z) h2 = __hfma2(q[rho][z], x2[z], h2);
+                    const float2 f = __half22float2(h2);
+                    acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
+                  }
+                }
+              }
+            }
+          }
+        }
+        // reduce across the LPR lanes of each row
+#pragma unroll
+        for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) acc[rho][t] += __shfl_xor_sync(0xffffffffu, acc[rho][t], o);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int tl = tp + t;
+          if (tl < nc && lr == (t % LPR)) {
+            const float inv = tok_inv[tl];
+            const int p = tok_pos[tl];
+            if (MODE == GATEUP) {
+              const float g = acc[0][t] * inv, u = acc[1][t] * inv;
+              a.out[size_t(p) * a.out_cols + (r0 >> 1)] = g / (1.f + expf(-g)) * u;
+            } else {
+              const float wgt = tok_w[tl] * inv;
+              *reinterpret_cast<float2*>(a.out + size_t(p) * a.out_cols + r0) = make_float2(acc[0][t] * wgt, acc[1][t] * wgt);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+  }
+}
+
+// --------------------------------------------------------- dequant hook
+// Writes out[r][j] = q * scale for rows row0.. of a packed matrix, with the
+// same word decoders the GEMV uses (test hook, not on the timed path).
+template <int BITS>
+__global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
+                                    int row0, int rows, int cols, float* __restrict__ out) {
+  constexpr int G = BITS == 4 ? 8 : 16;
+  constexpr int BLOCK = BITS == 4 ? 32 : 16;
+  const int words_per_row = cols / G;
+  const long long total = (long long)rows * words_per_row;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int r = int(i / words_per_row), wi = int(i % words_per_row);
+    const size_t row = size_t(row0 + r);
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(codes + row * (cols * BITS / 8) + size_t(wi) * 4);
+    __half2 q[G / 2];
+    if (BITS == 4) decode_q4x8(v, q); else decode_q2x16(v, q);
+    for (int j = 0; j < G; ++j) {
+      const int col = wi * G + j;
+      const int sl = decode_slot(BITS, j);
+      const __half qh = (sl & 1) ? __high2half(q[sl >> 1]) : __low2half(q[sl >> 1]);
+      const float sc = __half2float(__ushort_as_half(scales[row * (cols / BLOCK) + col / BLOCK]));
+      out[size_t(r) * cols + col] = __half2float(qh) * sc;
+    }
+  }
+}
+
+template <int BITS, int LPR, int CPL>
+PassPlan plan_of(int rows, int K) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  PassPlan p;
+  p.spe = rows / Gm::RPS;
+  const int avail = kSmemBudget - 256 - kStages * Gm::STAGE_BYTES - kMaxNTC * 12;
+  p.ntc = min(kMaxNTC, (avail / (K * 2)) & ~1);
+  return p;
+}
+
+template <int MODE, int BITS, int LPR, int CPL>
+cudaError_t launch_one(FfnArgs fa, int num_sms, cudaStream_t s) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  auto kern = ffn_tma_kernel<MODE, BITS, LPR, CPL>;
+  const size_t smem = 256 + size_t(kStages) * Gm::STAGE_BYTES + size_t(fa.ntc) * Gm::K * 2 + kMaxNTC * 12;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, dim3(num_sms), dim3(kThreads), smem, s, fa);
+}
+
+// 16-byte pieces per row C -> lanes per row (largest power of two <= 32
+// dividing C) and pieces per lane.
+#define MOE_C_CASES(X) X(2, 2, 1) X(4, 4, 1) X(8, 8, 1) X(12, 4, 3) X(16, 16, 1) X(24, 8, 3) \
+                       X(32, 32, 1) X(48, 16, 3) X(64, 32, 2) X(96, 32, 3) X(128, 32, 4)
+
+template <int MODE, int BITS>
+cudaError_t dispatch(int K, FfnArgs fa, int num_sms, cudaStream_t s) {
+  const int C = K * BITS / 8 / 16;
+  switch (C) {
+#define X(c, lpr, cpl) case c: return launch_one<MODE, BITS, lpr, cpl>(fa, num_sms, s);
+    MOE_C_CASES(X)
+#undef X
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int BITS>
+bool plan_for(int rows, int K, PassPlan* p) {
+  const int C = K * BITS / 8 / 16;
+  switch (C) {
+#define X(c, lpr, cpl) \
+  case c: { using Gm = Geom<BITS, lpr, cpl>; if (rows % Gm::RPS) return false; *p = plan_of<BITS, lpr, cpl>(rows, K); return p->ntc >= 2; }
+    MOE_C_CASES(X)
+#undef X
+    default: return false;
+  }
+}
+
+bool plans(int bits, int H, int I, PassPlan* gu, PassPlan* dn) {
+  if (bits == 4) return plan_for<4>(2 * I, H, gu) && plan_for<4>(H, I, dn);
+  return plan_for<2>(2 * I, H, gu) && plan_for<2>(H, I, dn);
+}
+
+}  // namespace
+
+bool decode_shape_supported(int bits, int H, int I) {
+  PassPlan g, d;
+  return plans(bits, H, I, &g, &d);
+}
+
+void decode_plans(const moe_config& c, PassPlan* gu, PassPlan* dn) { plans(c.bits, c.hidden, c.inter, gu, dn); }
+
+cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
+  const moe_config& c = a.cfg;
+  const int H = c.hidden, I = c.inter, bits = c.bits;
+  PassPlan pg, pd;
+  if (!plans(bits, H, I, &pg, &pd)) return cudaErrorInvalidValue;
+  RouteView rv;
+  rv.T = a.T; rv.k = c.top_k; rv.E = c.num_experts; rv.shared = c.shared_inter > 0 ? 1 : 0;
+  rv.status = reinterpret_cast<const int*>(a.ws + a.L.status);
+  rv.ulist = reinterpret_cast<const int*>(a.ws + a.L.ulist);
+  rv.offsets = reinterpret_cast<const int*>(a.ws + a.L.offsets);
+  rv.pairs = reinterpret_cast<const int*>(a.ws + a.L.pairs);
+  rv.inv = reinterpret_cast<const int*>(a.ws + a.L.inv);
+  rv.topk_w = reinterpret_cast<const float*>(a.ws + a.L.topk_w);
+
+  FfnArgs g{};
+  g.codes = a.w.gate_up_codes; g.scales = a.w.gate_up_scales;
+  g.sh_codes = a.w.shared_gate_up_codes; g.sh_scales = a.w.shared_gate_up_scales;
+  g.expert_code_bytes = size_t(2 * I) * H * bits / 8;
+  g.expert_scale_count = size_t(2 * I) * (H / c.block);
+  g.rows = 2 * I; g.out_cols = I; g.ntc = pg.ntc;
+  g.xin = a.x; g.hin = nullptr;
+  g.out = reinterpret_cast<float*>(a.ws + a.L.h);
+  g.status = reinterpret_cast<int*>(a.ws + a.L.status);
+  g.rv = rv;
+  g.rv.woff = reinterpret_cast<const int*>(a.ws + a.L.woff_gu);
+  cudaError_t err = bits == 4 ? dispatch<GATEUP, 4>(H, g, a.num_sms, a.stream)
+                              : dispatch<GATEUP, 2>(H, g, a.num_sms, a.stream);
+  if (err != cudaSuccess) return err;
+  if (between) cudaEventRecord(between, a.stream);
+
+  FfnArgs d{};
+  d.codes = a.w.down_codes; d.scales = a.w.down_scales;
+  d.sh_codes = a.w.shared_down_codes; d.sh_scales = a.w.shared_down_scales;
+  d.expert_code_bytes = size_t(H) * I * bits / 8;
+  d.expert_scale_count = size_t(H) * (I / c.block);
+  d.rows = H; d.out_cols = H; d.ntc = pd.ntc;
+  d.xin = nullptr; d.hin = reinterpret_cast<const float*>(a.ws + a.L.h);
+  d.out = reinterpret_cast<float*>(a.ws + a.L.y);
+  d.status = reinterpret_cast<int*>(a.ws + a.L.status);
+  d.rv = rv;
+  d.rv.woff = reinterpret_cast<const int*>(a.ws + a.L.woff_dn);
+  return bits == 4 ? dispatch<DOWN, 4>(I, d, a.num_sms, a.stream) : dispatch<DOWN, 2>(I, d, a.num_sms, a.stream);
+}
+
+cudaError_t launch_dequant_rows(int bits, int, const uint8_t* codes, const uint16_t* scales, int row0, int rows,
+                                int cols, float* out, cudaStream_t s) {
+  const int G = bits == 4 ? 8 : 16;
+  const long long total = (long long)rows * (cols / G);
+  const long long want = (total + 255) / 256;
+  const int blocks = int(want < 4096 ? want : 4096);
+  if (bits == 4) dequant_rows_kernel<4><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, out);
+  else dequant_rows_kernel<2><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,255 @@
+// C ABI of libmoe.so: argument validation and launch sequencing.  The
+// operation and the conventions are documented in include/moe_capi.h.
+#include "moe_internal.cuh"
+
+
+namespace moe {
+cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
+                              const uint16_t* x, int T, char* ws, const Layout& L, int* api_counts,
+                              int* api_offsets, int* api_pairs, cudaStream_t s);
+}
+
+using namespace moe;
+
+namespace {
+
+
+int num_sms_current() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int validate_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->num_experts <= 0 || c->hidden <= 0 || c->inter <= 0 || c->top_k <= 0 || c->shared_inter < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->num_experts > 1024 || c->num_experts % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->top_k > 16 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
+  if (!((c->bits == 4 && c->block == 32) || (c->bits == 2 && c->block == 16))) return MOE_ERR_UNSUPPORTED;
+  const int H = c->hidden;
+  if (!(H == 256 || H == 512 || H == 1024 || H == 2048 || H == 4096)) return MOE_ERR_UNSUPPORTED;
+  if (c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->shared_inter != 0 && c->shared_inter != c->inter) return MOE_ERR_UNSUPPORTED;
+  if (!decode_shape_supported(c->bits, H, c->inter)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int validate_weights(const moe_config* c, const moe_layer_weights* w) {
+  if (!w) return MOE_ERR_INVALID_ARG;
+  const void* req[] = {w->gate_up_codes, w->gate_up_scales, w->down_codes, w->down_scales, w->router_w};
+  for (const void* p : req)
+    if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  if (c->shared_inter > 0) {
+    const void* sh[] = {w->shared_gate_up_codes, w->shared_gate_up_scales, w->shared_down_codes,
+                        w->shared_down_scales};
+    for (const void* p : sh)
+      if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  }
+  if (w->router_bias && !aligned(w->router_bias, 4)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int check_ws(const moe_config* c, int T, void* ws, size_t ws_bytes) {
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_workspace_bytes(c, T)) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Optional per-phase event recording (moe_profile_begin / moe_profile_end).
+struct Profile {
+  bool on = false;
+  int cap = 0, used = 0;
+  cudaEvent_t* ev = nullptr;    // [cap][5]
+};
+Profile g_prof;
+
+void prof_mark(int call, int phase, cudaStream_t s) {
+  if (call >= 0) cudaEventRecord(g_prof.ev[call * 5 + phase], s);
+}
+
+// One layer on the stream: route, gate/up + SwiGLU, down, combine.
+int run_layer(const LayerArgs& a) {
+  const int call = (g_prof.on && g_prof.used < g_prof.cap) ? g_prof.used++ : -1;
+  prof_mark(call, 0, a.stream);
+  cudaError_t e = launch_route_full(a.cfg, a.w.router_w, a.w.router_bias, a.x, a.T, a.ws, a.L, nullptr,
+                                    nullptr, nullptr, a.stream);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  prof_mark(call, 1, a.stream);
+  e = launch_decode_ffn(a, call >= 0 ? g_prof.ev[call * 5 + 2] : nullptr);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  prof_mark(call, 3, a.stream);
+  e = launch_combine(a);
+  prof_mark(call, 4, a.stream);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens) {
+  if (validate_config(cfg) != MOE_OK || max_tokens < 0) return 0;
+  return make_layout(*cfg, max_tokens).total;
+}
+
+int moe_route(const moe_config* cfg, const uint16_t* router_w, const float* router_bias, const uint16_t* x,
+              int32_t T, int32_t* topk_idx, float* topk_w, int32_t* expert_counts, int32_t* expert_offsets,
+              int32_t* pairs, void* workspace, size_t ws_bytes, void* stream) {
+  int st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!router_w || !aligned(router_w, 16) || !x || !aligned(x, 16) || !topk_idx || !topk_w)
+    return MOE_ERR_INVALID_ARG;
+  if (router_bias && !aligned(router_bias, 4)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(cfg, T, workspace, ws_bytes)) != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const Layout L = make_layout(*cfg, T);
+  if (cudaMemsetAsync(ws + L.status, 0, ST_COUNT * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = launch_route_full(*cfg, router_w, router_bias, x, T, ws, L, expert_counts, expert_offsets,
+                                    pairs, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t n = size_t(T) * cfg->top_k;
+  if (cudaMemcpyAsync(topk_idx, ws + L.topk_idx, n * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaMemcpyAsync(topk_w, ws + L.topk_w, n * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
+                      uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
+  int st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if ((st = validate_weights(cfg, w)) != MOE_OK) return st;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = size_t(T) * cfg->hidden * 2;
+  const char* xb = reinterpret_cast<const char*>(x);
+  const char* yb = reinterpret_cast<const char*>(y);
+  if (xb < yb + bytes && yb < xb + bytes) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(cfg, T, workspace, ws_bytes)) != MOE_OK) return st;
+  LayerArgs a{};
+  a.cfg = *cfg; a.w = *w; a.T = T; a.x = x; a.y = y; a.residual = false; a.xhat_next = nullptr;
+  a.ws = static_cast<char*>(workspace);
+  a.L = make_layout(*cfg, T);
+  a.num_sms = num_sms_current();
+  a.stream = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  return run_layer(a);
+}
+
+int moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, int32_t L, uint16_t* x_inout,
+                      int32_t T, int32_t* topk_trace, void* workspace, size_t ws_bytes, void* stream) {
+  int st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || L < 0 || !layers) return MOE_ERR_INVALID_ARG;
+  if (T == 0 || L == 0) return MOE_OK;
+  for (int l = 0; l < L; ++l)
+    if ((st = validate_weights(cfg, &layers[l])) != MOE_OK) return st;
+  if (!x_inout || !aligned(x_inout, 16)) return MOE_ERR_INVALID_ARG;
+  if (topk_trace && !aligned(topk_trace, 4)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(cfg, T, workspace, ws_bytes)) != MOE_OK) return st;
+  LayerArgs a{};
+  a.cfg = *cfg; a.T = T;
+  a.ws = static_cast<char*>(workspace);
+  a.L = make_layout(*cfg, T);
+  a.num_sms = num_sms_current();
+  a.stream = static_cast<cudaStream_t>(stream);
+  uint16_t* xhat = reinterpret_cast<uint16_t*>(a.ws + a.L.xhat);
+  if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_rmsnorm(x_inout, xhat, T, cfg->hidden, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  for (int l = 0; l < L; ++l) {
+    a.w = layers[l];
+    a.x = xhat;
+    a.y = x_inout;
+    a.residual = true;
+    a.xhat_next = (l + 1 < L) ? xhat : nullptr;
+    if ((st = run_layer(a)) != MOE_OK) return st;
+    if (topk_trace) {
+      const size_t n = size_t(T) * cfg->top_k;
+      if (cudaMemcpyAsync(topk_trace + size_t(l) * n, a.ws + a.L.topk_idx, n * 4, cudaMemcpyDeviceToDevice,
+                          a.stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+  }
+  return MOE_OK;
+}
+
+int moe_device_status(const void* workspace, int32_t* code_out) {
+  if (!workspace || !code_out) return MOE_ERR_INVALID_ARG;
+  int32_t v[2] = {0, 0};
+  if (cudaMemcpy(v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  *code_out = v[0];
+  return v[0] == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
+}
+
+int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t* scales, int32_t row0,
+                     int32_t rows, int32_t cols, float* out, void* stream) {
+  if (!cfg || !codes || !scales || !out || row0 < 0 || rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  if (!((cfg->bits == 4 && cfg->block == 32) || (cfg->bits == 2 && cfg->block == 16))) return MOE_ERR_UNSUPPORTED;
+  if (cols % cfg->block != 0 || (cols * cfg->bits / 8) % 4 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(codes, 4) || !aligned(scales, 2) || !aligned(out, 4)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  return cuda_status(launch_dequant_rows(cfg->bits, cfg->block, codes, scales, row0, rows, cols, out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int moe_profile_begin(int32_t max_calls) {
+  if (max_calls <= 0 || g_prof.on) return MOE_ERR_INVALID_ARG;
+  g_prof.ev = new cudaEvent_t[size_t(max_calls) * 5];
+  for (int i = 0; i < max_calls * 5; ++i)
+    if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+  g_prof.cap = max_calls;
+  g_prof.used = 0;
+  g_prof.on = true;
+  return MOE_OK;
+}
+
+int moe_profile_end(float* ms_out, int32_t* calls) {
+  if (!g_prof.on || !ms_out || !calls) return MOE_ERR_INVALID_ARG;
+  int st = MOE_OK;
+  for (int p = 0; p < 4; ++p) ms_out[p] = 0.f;
+  for (int c = 0; c < g_prof.used; ++c) {
+    for (int p = 0; p < 4; ++p) {
+      float ms = 0.f;
+      if (cudaEventSynchronize(g_prof.ev[c * 5 + p + 1]) != cudaSuccess ||
+          cudaEventElapsedTime(&ms, g_prof.ev[c * 5 + p], g_prof.ev[c * 5 + p + 1]) != cudaSuccess)
+        st = MOE_ERR_CUDA;
+      ms_out[p] += ms;
+    }
+  }
+  *calls = g_prof.used;
+  for (int i = 0; i < g_prof.cap * 5; ++i) cudaEventDestroy(g_prof.ev[i]);
+  delete[] g_prof.ev;
+  g_prof = Profile{};
+  return st;
+}
+
+const char* moe_status_str(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument (null, misaligned or negative)";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case MOE_ERR_WORKSPACE: return "workspace smaller than moe_workspace_bytes()";
+    case MOE_ERR_CUDA: return "a CUDA runtime call failed";
+    case MOE_ERR_DEVICE_CHECK: return "a device-side check failed";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,283 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libmoe.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/moe_capi.h"
+
+namespace moe {
+
+// ------------------------------------------------------------ workspace ---
+// One call's scratch, carved from the caller's workspace.  Every region starts
+// on a 256-byte boundary.  P = T*k (+ T when the shared expert is present)
+// counts token-expert pairs; pair positions are expert-major (sorted), the
+// shared expert's pairs come last at positions T*k + t.
+enum StatusSlot {
+  ST_ERROR = 0,      // first failed device check (0 = none)
+  ST_ERROR_AUX = 1,  // detail of that check
+  ST_UCOUNT = 2,     // number of distinct routed experts selected
+  ST_COUNT = 16
+};
+
+struct Layout {
+  size_t status, logits, topk_idx, topk_w, counts, offsets, pairs, inv, ulist, woff_gu, woff_dn, xhat, h, y, xs,
+      total;
+  int P;
+};
+
+__host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+inline Layout make_layout(const moe_config& c, int T) {
+  Layout L{};
+  const int S = c.shared_inter > 0 ? 1 : 0;
+  const int P = T * c.top_k + S * T;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  L.status = take(ST_COUNT * 4);
+  L.logits = take(size_t(T) * c.num_experts * 4);
+  L.topk_idx = take(size_t(T) * c.top_k * 4);
+  L.topk_w = take(size_t(T) * c.top_k * 4);
+  L.counts = take(size_t(c.num_experts) * 4);
+  L.offsets = take(size_t(c.num_experts + 1) * 4);
+  L.pairs = take(size_t(T) * c.top_k * 4);
+  L.inv = take(size_t(T) * c.top_k * 4);
+  L.ulist = take(size_t(c.num_experts + 1) * 4);
+  L.woff_gu = take(size_t(c.num_experts + 2) * 4);
+  L.woff_dn = take(size_t(c.num_experts + 2) * 4);
+  L.xhat = take(size_t(T) * c.hidden * 2);
+  L.h = take(size_t(P) * c.inter * 4);
+  L.y = take(size_t(P) * c.hidden * 4);
+  L.xs = take(size_t(P) * c.hidden * 2);
+  L.total = o;
+  L.P = P;
+  return L;
+}
+
+// Everything a kernel of the layer needs to find the routing results.
+struct RouteView {
+  int T, k, E, shared;              // shared: 1 when the shared expert exists
+  const int* status;                // [ST_COUNT]
+  const int* ulist;                 // [E+1] touched experts ascending, E = shared
+  const int* offsets;               // [E+1]
+  const int* pairs;                 // [T*k] pair id t*k+j at each routed position
+  const int* inv;                   // [T*k] position of pair t*k+j
+  const float* topk_w;              // [T*k]
+  const int* woff;                  // [nslots+1] work-unit prefix of one GEMV pass
+};
+
+// Work decomposition of one decode GEMV pass, shared by the grouping kernel
+// (which writes the per-slot work prefix) and the GEMV kernel.
+struct PassPlan {
+  int ntc;    // tokens staged per chunk
+  int spe;    // stages (row groups) per expert
+};
+
+// -------------------------------------------------------------- device ---
+__device__ __forceinline__ void pdl_wait() {
+#if defined(__CUDA_ARCH__) && __CUDA_ARCH__ >= 900
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+#if defined(__CUDA_ARCH__) && __CUDA_ARCH__ >= 900
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+
+// Streaming 16-byte load of read-once weight bytes: read-only path, no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_stream4(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint2 ld_stream8(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint16_t ld_stream2(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
+// ------------------------------------------------ mbarrier / bulk copy ---
+// Every wait is bounded: after kWaitLimitNs of wall time (or when the CTA's
+// abort flag is raised) it gives up and returns false; the caller records
+// MOE_ERR_TIMEOUT in the status word and skips the remaining work.
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase of `bar` with the given parity; false on timeout/abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+// 1-D TMA: `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// Records the first failure in the status word (0 = none).
+__device__ __forceinline__ void report_error(int* status, int code, int aux) {
+  if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, aux);
+}
+
+// (a & b) | c in one instruction.
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
+
+// In-register decode of packed codes to signed integers q = c - 2^(bits-1),
+// exact in fp16.  A 16-bit lane of the form 0x6400 | (c << n) is the fp16
+// number 1024 + c * 2^n; one fused multiply-add by 2^-n and -(1024/2^n +
+// offset) leaves q.  Each half2 carries two elements that sit 16 bits apart in
+// the source word, so the activation vector is stored in the matching order.
+//
+// 4-bit, one 32-bit word = 8 elements e0..e7 (e_j at bits 4j):
+//   out[0] = (q0, q4)  out[1] = (q1, q5)  out[2] = (q2, q6)  out[3] = (q3, q7)
+__device__ __forceinline__ void decode_q4x8(uint32_t v, __half2 out[4]) {
+  const uint32_t MAGIC = 0x64006400u;
+  const uint32_t lo0 = lop_and_or(v, 0x000F000Fu, MAGIC);
+  const uint32_t hi0 = lop_and_or(v, 0x00F000F0u, MAGIC);
+  const uint32_t v8 = v >> 8;
+  const uint32_t lo1 = lop_and_or(v8, 0x000F000Fu, MAGIC);
+  const uint32_t hi1 = lop_and_or(v8, 0x00F000F0u, MAGIC);
+  const __half2 sub_lo = u32_as_h2(0x64086408u);          // 1032 = 1024 + 8
+  const __half2 mul_hi = u32_as_h2(0x2C002C00u);          // 1/16
+  const __half2 add_hi = u32_as_h2(0xD480D480u);          // -72 = -(64 + 8)
+  out[0] = __hsub2(u32_as_h2(lo0), sub_lo);
+  out[1] = __hfma2(u32_as_h2(hi0), mul_hi, add_hi);
+  out[2] = __hsub2(u32_as_h2(lo1), sub_lo);
+  out[3] = __hfma2(u32_as_h2(hi1), mul_hi, add_hi);
+}
+
+// 2-bit, one 32-bit word = 16 elements e0..e15 (e_j at bits 2j):
+//   out[j] = (q_j, q_{j+8}) for j = 0..7
+__device__ __forceinline__ void decode_q2x16(uint32_t v, __half2 out[8]) {
+  const uint32_t MAGIC = 0x64006400u;
+  const __half2 sub1 = u32_as_h2(0x64026402u);            // 1026 = 1024 + 2
+  const __half2 m4 = u32_as_h2(0x34003400u), a4 = u32_as_h2(0xDC08DC08u);    // 1/4,  -258
+  const __half2 m16 = u32_as_h2(0x2C002C00u), a16 = u32_as_h2(0xD420D420u);  // 1/16, -66
+  const __half2 m64 = u32_as_h2(0x24002400u), a64 = u32_as_h2(0xCC80CC80u);  // 1/64, -18
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t w = half ? (v >> 8) : v;
+    out[4 * half + 0] = __hsub2(u32_as_h2(lop_and_or(w, 0x00030003u, MAGIC)), sub1);
+    out[4 * half + 1] = __hfma2(u32_as_h2(lop_and_or(w, 0x000C000Cu, MAGIC)), m4, a4);
+    out[4 * half + 2] = __hfma2(u32_as_h2(lop_and_or(w, 0x00300030u, MAGIC)), m16, a16);
+    out[4 * half + 3] = __hfma2(u32_as_h2(lop_and_or(w, 0x00C000C0u, MAGIC)), m64, a64);
+  }
+}
+
+// Position, inside a group of 8 (4-bit) or 16 (2-bit) consecutive elements,
+// of element j in the half2 order produced by the decoders above.
+__host__ __device__ inline int decode_slot(int bits, int j) {
+  return bits == 4 ? (j & 3) * 2 + (j >> 2) : (j & 7) * 2 + (j >> 3);
+}
+
+// ------------------------------------------------------------- launches ---
+struct LayerArgs {
+  moe_config cfg;
+  moe_layer_weights w;
+  int T;
+  const uint16_t* x;       // [T][H] bf16 layer input (post-norm when stacked)
+  uint16_t* y;             // [T][H] bf16 output (layer) or the residual stream (stack)
+  bool residual;           // y <- bf16(y + out) and refresh xhat for the next layer
+  uint16_t* xhat_next;     // stack: normalised input of the next layer (or nullptr)
+  char* ws;
+  Layout L;
+  int num_sms;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* xhat, int T, int H, cudaStream_t s);
+cudaError_t launch_route(const moe_config& c, const uint16_t* router_w, const float* bias,
+                         const uint16_t* x, int T, char* ws, const Layout& L, int num_sms,
+                         cudaStream_t s);
+cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between = nullptr);
+void decode_plans(const moe_config& c, PassPlan* gu, PassPlan* dn);
+cudaError_t launch_combine(const LayerArgs& a);
+cudaError_t launch_dequant_rows(int bits, int block, const uint8_t* codes, const uint16_t* scales,
+                                int row0, int rows, int cols, float* out, cudaStream_t s);
+bool decode_shape_supported(int bits, int H, int I);
+
+// Launch helper: programmatic dependent launch (the kernel may start while
+// the previous kernel on the stream drains; it calls pdl_wait() before
+// reading that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+}  // namespace moe

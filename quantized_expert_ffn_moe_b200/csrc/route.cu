@@ -1,0 +1,408 @@
+// Router logits, top-k selection with renormalised gates, and the counting
+// sort that turns the selection into per-expert token lists.
+//
+// The router is the light gating network that picks the Top-K experts per
+// token ("Running a 125B Model on a Single RTX 5090: Strata Benchmarks Qwen3.8
+// Flash Next", section "Layer 1: On-Demand MoE Expert Scheduling"); per layer
+// the GPU works out which 10 of 512 experts each token needs ("Strata Open
+// Source Project: Run a 125B Model Locally on a Home PC", section "The
+// 'Doorbell' Mechanism").  Gates: softmax over the selected logits (the full
+// softmax renormalised over the selection); ties go to the smaller expert.
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouterWarps = 4;        // experts per router CTA (one warp each)
+constexpr int kRouterTokTile = 16;     // tokens staged in shared memory at a time
+constexpr int kRouterTokBlock = 256;   // tokens per CTA along grid.y
+constexpr int kGroupThreads = 1024;    // the single grouping CTA
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(uint32_t(b) << 16);
+}
+
+// ------------------------------------------------------------------ rmsnorm
+// xhat[t] = bf16(x[t] / sqrt(mean(x[t]^2) + 1e-6)), one CTA of 256 threads per token.
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ x,
+                                                      uint16_t* __restrict__ xhat, int H) {
+  pdl_wait();
+  const int t = blockIdx.x;
+  const uint16_t* row = x + size_t(t) * H;
+  float ss = 0.f;
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const float v = bf16_bits_to_float(row[h]);
+    ss = fmaf(v, v, ss);
+  }
+  __shared__ float red[8];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+  const float r = 1.0f / sqrtf(tot / float(H) + 1e-6f);
+  pdl_launch_dependents();
+  for (int h = threadIdx.x; h < H; h += blockDim.x) {
+    const __nv_bfloat16 o = __float2bfloat16_rn(bf16_bits_to_float(row[h]) * r);
+    xhat[size_t(t) * H + h] = *reinterpret_cast<const uint16_t*>(&o);
+  }
+}
+
+// ---------------------------------------------------------- router logits
+// logits[t][e] = sum_h x[t][h] * Wr[e][h] (+ bias[e]) in fp32.  Each warp owns
+// one expert row; its lanes read 16-byte pieces of the row (a warp load is
+// 512 contiguous bytes) and the row stays in registers while the warp walks
+// the tokens, which are staged in shared memory kRouterTokTile at a time.
+template <int H>
+__global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(
+    const uint16_t* __restrict__ wr, const float* __restrict__ bias,
+    const uint16_t* __restrict__ x, int T, int E, float* __restrict__ logits) {
+  constexpr int PER_LANE = H / 256;   // 16-byte pieces per lane
+  extern __shared__ __align__(16) uint16_t xs[];   // [kRouterTokTile][H]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * kRouterWarps + warp;
+  uint4 wv[PER_LANE];
+  if (e < E) {
+    const uint16_t* row = wr + size_t(e) * H;
+#pragma unroll
+    for (int p = 0; p < PER_LANE; ++p) wv[p] = ld_stream16(row + (p * 32 + lane) * 8);
+  }
+  const float b = (e < E && bias) ? bias[e] : 0.f;
+  pdl_wait();   // x may be produced by the previous kernel
+  const int t_lo = blockIdx.y * kRouterTokBlock, t_hi = min(T, t_lo + kRouterTokBlock);
+  for (int t0 = t_lo; t0 < t_hi; t0 += kRouterTokTile) {
+    const int nt = min(kRouterTokTile, t_hi - t0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nt * H / 8; i += blockDim.x)
+      reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(x + size_t(t0) * H)[i];
+    __syncthreads();
+    if (e < E) {
+      for (int t = 0; t < nt; ++t) {
+        float acc = 0.f;
+#pragma unroll
+        for (int p = 0; p < PER_LANE; ++p) {
+          const uint4 xv = reinterpret_cast<const uint4*>(xs + t * H)[p * 32 + lane];
+          const uint32_t wa[4] = {wv[p].x, wv[p].y, wv[p].z, wv[p].w};
+          const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc = fmaf(__uint_as_float(wa[q] << 16), __uint_as_float(xa[q] << 16), acc);
+            acc = fmaf(__uint_as_float(wa[q] & 0xFFFF0000u), __uint_as_float(xa[q] & 0xFFFF0000u), acc);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) logits[size_t(t0 + t) * E + e] = acc + b;
+      }
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// ------------------------------------------------------------------ top-k
+// One warp selects the k largest of E logits: lane l holds experts l + 32m.
+// Each round takes the warp-wide maximum (ties to the smaller expert), the
+// owner marks it taken.  Gates are a softmax over the k selected logits.
+template <int NPL>
+__device__ void warp_topk(const float* __restrict__ lrow, int k, int E,
+                          int* __restrict__ idx_out, float* __restrict__ w_out) {
+  const int lane = threadIdx.x & 31;
+  float v[NPL];
+#pragma unroll
+  for (int m = 0; m < NPL; ++m) {
+    const int e = lane + 32 * m;
+    v[m] = e < E ? lrow[e] : -INFINITY;
+  }
+  uint32_t taken = 0;
+  float my_logit = -INFINITY;
+  int my_idx = 0;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int m = 0; m < NPL; ++m) {
+      const int e = lane + 32 * m;
+      const bool ok = !((taken >> m) & 1u) && e < E;
+      if (ok && (v[m] > bv || (v[m] == bv && e < be))) { bv = v[m]; be = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == j) { my_logit = bv; my_idx = be; }
+  }
+  const float top = __shfl_sync(0xffffffffu, my_logit, 0);
+  float ex = lane < k ? expf(my_logit - top) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < k) {
+    idx_out[lane] = my_idx;
+    w_out[lane] = ex / sum;
+  }
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                   int* __restrict__ idx, float* __restrict__ w) {
+  pdl_wait();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t < T) warp_topk<NPL>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
+  pdl_launch_dependents();
+}
+
+// -------------------------------------------------------------- grouping
+// Stable counting sort of the T*k (token, slot) pairs by expert, in one CTA of
+// 32 warps.  Warp w owns a contiguous token range; per-warp histograms give
+// each warp's starting rank inside every expert, then each warp walks its
+// tokens in order, so positions are sorted by expert, then by token.  Also
+// writes the ascending list of selected experts (the shared expert appended
+// as id E) and, when `fused_topk`, runs the top-k itself first (decode).
+template <int NPL>
+__global__ void __launch_bounds__(kGroupThreads) group_kernel(
+    const float* __restrict__ logits, int fused_topk, int* __restrict__ idx, float* __restrict__ w,
+    int T, int E, int k, int shared, int* __restrict__ status, int* __restrict__ counts_out,
+    int* __restrict__ offsets_out, int* __restrict__ pairs_out, int* __restrict__ inv_out,
+    int* __restrict__ ulist_out, int* __restrict__ api_counts, int* __restrict__ api_offsets,
+    int* __restrict__ api_pairs, PassPlan pg, PassPlan pd, int* __restrict__ woff_gu,
+    int* __restrict__ woff_dn) {
+  extern __shared__ int sm[];
+  constexpr int NW = kGroupThreads / 32;
+  int* hist = sm;                       // [NW][E]
+  int* offs = sm + NW * E;              // [E+1]
+  int* scan = offs + E + 1;             // [kGroupThreads] scan scratch
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  if (fused_topk) {
+    for (int t = warp; t < T; t += NW)
+      warp_topk<NPL>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
+    __syncthreads();
+    __threadfence_block();
+  }
+  for (int i = threadIdx.x; i < NW * E; i += kGroupThreads) hist[i] = 0;
+  __syncthreads();
+  const int tpw = (T + NW - 1) / NW;
+  const int t_begin = min(T, warp * tpw), t_end = min(T, t_begin + tpw);
+  for (int p = t_begin * k + lane; p < t_end * k; p += 32) {
+    const int e = idx[p];
+    if (e < 0 || e >= E) {              // never produced by the selection above
+      atomicCAS(status + ST_ERROR, 0, 1);
+      continue;
+    }
+    atomicAdd(&hist[warp * E + e], 1);
+  }
+  __syncthreads();
+  // per-expert exclusive prefix over warps; counts
+  for (int e = threadIdx.x; e < E; e += kGroupThreads) {
+    int run = 0;
+    for (int ww = 0; ww < NW; ++ww) {
+      const int c = hist[ww * E + e];
+      hist[ww * E + e] = run;
+      run += c;
+    }
+    offs[e] = run;                      // count for now
+  }
+  __syncthreads();
+  // exclusive scan of counts -> offsets (E <= kGroupThreads)
+  {
+    const int e = threadIdx.x;
+    const int c = e < E ? offs[e] : 0;
+    int v = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += n;
+    }
+    if (lane == 31) scan[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int s = scan[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += n;
+      }
+      scan[lane] = s;                   // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = v - c + (warp > 0 ? scan[warp - 1] : 0);
+    __syncthreads();
+    if (e < E) {
+      counts_out[e] = c;
+      offsets_out[e] = excl;
+      if (api_counts) api_counts[e] = c;
+      if (api_offsets) api_offsets[e] = excl;
+      offs[e] = excl;
+    }
+    if (e == E - 1) {
+      offsets_out[E] = excl + c;
+      if (api_offsets) api_offsets[E] = excl + c;
+      offs[E] = excl + c;
+    }
+    // touched-expert list: scan of flags
+    __syncthreads();
+    const int f = (e < E && c > 0) ? 1 : 0;
+    int fv = f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, fv, o);
+      if (lane >= o) fv += n;
+    }
+    if (lane == 31) scan[warp] = fv;
+    __syncthreads();
+    if (warp == 0) {
+      int s = scan[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += n;
+      }
+      scan[lane] = s;
+    }
+    __syncthreads();
+    const int fpos = fv - f + (warp > 0 ? scan[warp - 1] : 0);
+    if (f) ulist_out[fpos] = e;
+    if (threadIdx.x == 0) {
+      const int U = scan[NW - 1];
+      status[ST_UCOUNT] = U;
+      if (shared) ulist_out[U] = E;
+    }
+  }
+  __syncthreads();
+  // work prefix of the two GEMV passes over the slots (touched experts, then
+  // the shared expert): each slot contributes ceil(n / ntc) * stages units.
+  if (warp == 0) {
+    const int U = scan[NW - 1];
+    const int nslots = U + shared;
+    int run_g = 0, run_d = 0;
+    for (int base = 0; base < nslots; base += 32) {
+      const int u = base + lane;
+      int n = 0;
+      if (u < U) {
+        const int e = ulist_out[u];
+        n = offs[e + 1] - offs[e];
+      } else if (u < nslots) {
+        n = T;
+      }
+      int g = u < nslots ? (n + pg.ntc - 1) / pg.ntc * pg.spe : 0;
+      int d = u < nslots ? (n + pd.ntc - 1) / pd.ntc * pd.spe : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ng = __shfl_up_sync(0xffffffffu, g, o);
+        const int nd = __shfl_up_sync(0xffffffffu, d, o);
+        if (lane >= o) { g += ng; d += nd; }
+      }
+      if (u < nslots) {
+        woff_gu[u + 1] = run_g + g;
+        woff_dn[u + 1] = run_d + d;
+      }
+      run_g += __shfl_sync(0xffffffffu, g, 31);
+      run_d += __shfl_sync(0xffffffffu, d, 31);
+    }
+    if (lane == 0) {
+      woff_gu[0] = 0;
+      woff_dn[0] = 0;
+    }
+  }
+  // stable scatter: each warp walks its tokens in order
+  for (int t = t_begin; t < t_end; ++t) {
+    if (lane < k) {
+      const int q = t * k + lane;
+      const int e = idx[q];
+      if (e >= 0 && e < E) {
+        const int pos = offs[e] + hist[warp * E + e];
+        hist[warp * E + e] += 1;        // distinct experts within one token
+        pairs_out[pos] = q;
+        inv_out[q] = pos;
+        if (api_pairs) api_pairs[pos] = q;
+      }
+    }
+    __syncwarp();
+  }
+  pdl_launch_dependents();
+}
+
+template <int NPL>
+cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout& L, bool fused,
+                              int* api_counts, int* api_offsets, int* api_pairs, cudaStream_t s) {
+  const size_t smem = (size_t(32) * c.num_experts + c.num_experts + 1 + kGroupThreads) * sizeof(int);
+  auto kern = group_kernel<NPL>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  PassPlan pg{1, 1}, pd{1, 1};
+  decode_plans(c, &pg, &pd);
+  float* logits = reinterpret_cast<float*>(ws + L.logits);
+  int* idx = reinterpret_cast<int*>(ws + L.topk_idx);
+  float* w = reinterpret_cast<float*>(ws + L.topk_w);
+  if (!fused) {
+    err = launch_pdl(topk_kernel<NPL>, dim3((T + 7) / 8), dim3(256), 0, s, logits, T, c.num_experts,
+                     c.top_k, idx, w);
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(kern, dim3(1), dim3(kGroupThreads), smem, s, logits, fused ? 1 : 0, idx, w, T,
+                    c.num_experts, c.top_k, c.shared_inter > 0 ? 1 : 0,
+                    reinterpret_cast<int*>(ws + L.status), reinterpret_cast<int*>(ws + L.counts),
+                    reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
+                    reinterpret_cast<int*>(ws + L.inv), reinterpret_cast<int*>(ws + L.ulist), api_counts,
+                    api_offsets, api_pairs, pg, pd, reinterpret_cast<int*>(ws + L.woff_gu),
+                    reinterpret_cast<int*>(ws + L.woff_dn));
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* xhat, int T, int H, cudaStream_t s) {
+  return launch_pdl(rmsnorm_kernel, dim3(T), dim3(256), 0, s, x, xhat, H);
+}
+
+cudaError_t launch_router_logits(const moe_config& c, const uint16_t* router_w, const float* bias,
+                                 const uint16_t* x, int T, float* logits, cudaStream_t s) {
+  const dim3 grid((c.num_experts + kRouterWarps - 1) / kRouterWarps, (T + kRouterTokBlock - 1) / kRouterTokBlock);
+  const dim3 block(kRouterWarps * 32);
+  const size_t smem = size_t(kRouterTokTile) * c.hidden * 2;
+  void (*kern)(const uint16_t*, const float*, const uint16_t*, int, int, float*) = nullptr;
+  switch (c.hidden) {
+    case 256: kern = router_logits_kernel<256>; break;
+    case 512: kern = router_logits_kernel<512>; break;
+    case 1024: kern = router_logits_kernel<1024>; break;
+    case 2048: kern = router_logits_kernel<2048>; break;
+    case 4096: kern = router_logits_kernel<4096>; break;
+    default: return cudaErrorInvalidValue;
+  }
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, grid, block, smem, s, router_w, bias, x, T, c.num_experts, logits);
+}
+
+cudaError_t launch_topk_group_any(const moe_config& c, int T, char* ws, const Layout& L, bool fused,
+                                  int* api_counts, int* api_offsets, int* api_pairs, cudaStream_t s) {
+  switch (c.num_experts / 32) {
+    case 1: return launch_topk_group<1>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    case 2: return launch_topk_group<2>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    case 4: return launch_topk_group<4>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    case 8: return launch_topk_group<8>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    case 16: return launch_topk_group<16>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    case 32: return launch_topk_group<32>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
+                              const uint16_t* x, int T, char* ws, const Layout& L, int* api_counts,
+                              int* api_offsets, int* api_pairs, cudaStream_t s) {
+  cudaError_t err = launch_router_logits(c, router_w, bias, x, T, reinterpret_cast<float*>(ws + L.logits), s);
+  if (err != cudaSuccess) return err;
+  const bool fused = T <= 64;
+  return launch_topk_group_any(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+}
+
+cudaError_t launch_route(const moe_config& c, const uint16_t* router_w, const float* bias,
+                         const uint16_t* x, int T, char* ws, const Layout& L, int, cudaStream_t s) {
+  return launch_route_full(c, router_w, bias, x, T, ws, L, nullptr, nullptr, nullptr, s);
+}
+
+}  // namespace moe

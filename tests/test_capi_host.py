@@ -1,0 +1,144 @@
+"""Host-side tests of the C ABI: the library builds and loads, exports every
+symbol include/moe_capi.h declares, sizes its workspace, and rejects bad
+arguments before launching anything (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_expert_ffn_moe_b200 as q
+from quantized_expert_ffn_moe_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_capi.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return q.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(moe_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("moe_route", "moe_layer_forward", "moe_stack_forward", "moe_workspace_bytes"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(q.EXPORTS) <= set(declared_functions())
+
+
+FULL = dict(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=32)
+
+
+def cfg(**kw):
+    d = dict(FULL)
+    d.update(kw)
+    return q.config_of(d["experts"], d["hidden"], d["inter"], d["top_k"], d["shared"], d["bits"], d["block"])
+
+
+def test_workspace_bytes(lib):
+    a = q.moe_workspace_bytes(cfg(), 1)
+    b = q.moe_workspace_bytes(cfg(), 16)
+    c = q.moe_workspace_bytes(cfg(), 4096)
+    assert 0 < a < b < c
+    # scratch at T=4096: h (fp32) + Y (fp32) + gathered X (bf16) dominate
+    P = 4096 * 11
+    assert c >= P * (768 * 4 + 2048 * 4 + 2048 * 2)
+    assert q.moe_workspace_bytes(cfg(), 0) > 0
+    assert q.moe_workspace_bytes(cfg(), -1) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(bits=3), dict(bits=4, block=16), dict(bits=2, block=32), dict(hidden=300),
+                                dict(experts=500), dict(top_k=17), dict(inter=100), dict(experts=2048)])
+def test_unsupported_configs_report_zero_workspace(lib, kw):
+    assert q.moe_workspace_bytes(cfg(**kw), 16) == 0
+
+
+def test_tiny_and_2bit_configs_supported(lib):
+    assert q.moe_workspace_bytes(q.config_of(64, 256, 128, 4, True, 4, 32), 8) > 0
+    assert q.moe_workspace_bytes(cfg(bits=2, block=16), 64) > 0
+    assert q.moe_workspace_bytes(cfg(shared=False), 64) > 0
+
+
+def _fake_weights(shared=True, misalign=None):
+    # addresses are never dereferenced on these paths
+    base = 1 << 20
+    w = q._Weights()
+    for i, (name, _) in enumerate(q._Weights._fields_):
+        setattr(w, name, base * (i + 1))
+    if not shared:
+        for n in ("shared_gate_up_codes", "shared_gate_up_scales", "shared_down_codes", "shared_down_scales"):
+            setattr(w, n, None)
+    w.router_bias = None
+    if misalign:
+        setattr(w, misalign, getattr(w, misalign) + 8)
+    return w
+
+
+def _layer(lib, c, w, x=1 << 30, T=4, y=2 << 30, ws=3 << 30, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.moe_workspace_bytes(ctypes.byref(c), T)
+    return lib.moe_layer_forward(ctypes.byref(c), ctypes.byref(w), x, T, y, ws, ws_bytes, None)
+
+
+def test_layer_forward_argument_errors(lib):
+    c = cfg()
+    w = _fake_weights()
+    assert _layer(lib, c, w, T=0) == 0                       # empty batch: no-op
+    assert _layer(lib, c, w, T=-1) == q.MOE_OK - 1           # MOE_ERR_INVALID_ARG
+    assert _layer(lib, c, w, x=None) == -1
+    assert _layer(lib, c, w, x=(1 << 30) + 2) == -1          # misaligned x
+    assert _layer(lib, c, w, y=(1 << 30) + 1024) == -1       # y overlaps x
+    assert _layer(lib, c, w, ws=(3 << 30) + 16) == -1        # workspace not 256-aligned
+    assert _layer(lib, c, w, ws_bytes=100) == -3             # MOE_ERR_WORKSPACE
+    assert _layer(lib, c, _fake_weights(misalign="down_codes")) == -1
+    assert _layer(lib, c, _fake_weights(shared=False)) == -1  # shared expert configured but missing
+    assert _layer(lib, cfg(shared=False), _fake_weights(shared=False), ws_bytes=0) == -3
+    assert _layer(lib, cfg(bits=3), w) == -2                  # MOE_ERR_UNSUPPORTED
+    assert lib.moe_layer_forward(None, ctypes.byref(w), 1 << 30, 4, 2 << 30, 3 << 30, 1 << 40, None) == -1
+
+
+def test_route_and_stack_argument_errors(lib):
+    c = cfg()
+    n = lib.moe_workspace_bytes(ctypes.byref(c), 4)
+    assert lib.moe_route(ctypes.byref(c), 1 << 20, None, 1 << 30, 0, 1 << 31, 1 << 32, None, None, None,
+                         3 << 30, n, None) == 0
+    assert lib.moe_route(ctypes.byref(c), None, None, 1 << 30, 4, 1 << 31, 1 << 32, None, None, None,
+                         3 << 30, n, None) == -1
+    assert lib.moe_route(ctypes.byref(c), 1 << 20, None, 1 << 30, 4, None, 1 << 32, None, None, None,
+                         3 << 30, n, None) == -1
+    arr = (q._Weights * 2)(_fake_weights(), _fake_weights(misalign="router_w"))
+    assert lib.moe_stack_forward(ctypes.byref(c), arr, 2, 1 << 30, 4, None, 3 << 30, n, None) == -1
+    assert lib.moe_stack_forward(ctypes.byref(c), arr, 0, 1 << 30, 4, None, 3 << 30, n, None) == 0
+    assert lib.moe_stack_forward(ctypes.byref(c), arr, 1, 1 << 30, 0, None, 3 << 30, n, None) == 0
+    assert lib.moe_dequant_rows(ctypes.byref(cfg(bits=3)), 1 << 20, 1 << 21, 0, 1, 256, 1 << 22, None) == -2
+
+
+def test_status_strings(lib):
+    for s in (0, -1, -2, -3, -4, -5, -6):
+        assert q.moe_status_str(s) and q.moe_status_str(s) != "unknown status"
+    assert q.moe_status_str(42) == "unknown status"
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    import importlib
+    mod = importlib.import_module("quantized_expert_ffn_moe_b200")
+    with pytest.raises(RuntimeError):
+        mod._lib, saved = None, mod._lib
+        try:
+            mod.load_library(str(tmp_path / "missing.so"))
+        finally:
+            mod._lib = saved

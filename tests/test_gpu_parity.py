@@ -1,0 +1,273 @@
+"""GPU parity of the CUDA path against the float64 oracle, through the C ABI.
+
+Tolerances: integer work (grouping, decoded codes) is bit-exact; expert ids are
+bit-exact except inside the oracle's tie band (k-th and (k+1)-th logits within
+1e-5, where both choices are correct); gate weights within 1e-5 (fp32 logits
+and exp); layer outputs within max |err| <= 2e-2 * RMS(oracle output).
+"""
+
+import numpy as np
+import pytest
+
+import gpu_cases as gc
+import moe_inputs as mi
+import oracle as orc
+import quantized_expert_ffn_moe_b200 as q
+
+pytestmark = pytest.mark.gpu
+
+SHAPE_2BIT_TINY = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=2, block=16)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_expert_ffn_moe_b200 import build
+    from moe_inputs import build as ibuild
+    build.build()
+    ibuild.build()
+    q.load_library()
+
+
+# ------------------------------------------------------------ input bytes ---
+
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2], ids=["tiny4", "tiny2", "full4", "full2"])
+def test_device_generator_matches_host(shape):
+    """The device generator writes the same bytes as the numpy generator."""
+    w = gc.device_layer(shape, seed=3, layer=5)
+    for e in (0, 1, shape.experts - 1):
+        ref = mi.expert_packed(shape, 3, 5, e)
+        got = (w.gate_up_codes[e], w.gate_up_scales[e], w.down_codes[e], w.down_scales[e])
+        for r, g in zip(ref, got):
+            np.testing.assert_array_equal(g.cpu().numpy().view(r.dtype).reshape(r.shape), r)
+    ref = mi.shared_packed(shape, 3, 5)
+    got = (w.shared_gate_up_codes, w.shared_gate_up_scales, w.shared_down_codes, w.shared_down_scales)
+    for r, g in zip(ref, got):
+        np.testing.assert_array_equal(g.cpu().numpy().view(r.dtype).reshape(r.shape), r)
+    np.testing.assert_array_equal(gc.bits_to_np(w.router_w), mi.router_weight_bf16(shape, 3, 5))
+
+
+# ----------------------------------------------------------- dequant hook ---
+
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2], ids=["tiny4", "tiny2", "full4", "full2"])
+def test_device_decoder_bit_exact(shape):
+    torch = gc.torch()
+    w = gc.device_layer(shape, seed=1, layer=0)
+    cfg = gc.cfg_of(shape)
+    e = shape.experts // 2
+    gcodes, gsc, dcodes, dsc = mi.expert_packed(shape, 1, 0, e)
+    H, I = shape.hidden, shape.inter
+    out = torch.empty((2 * I, H), dtype=torch.float32, device="cuda")
+    q.moe_dequant_rows(cfg, w.gate_up_codes[e], w.gate_up_scales[e], 0, 2 * I, H, out)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64),
+                                  orc.dequantize(gcodes, gsc, 2 * I, H, shape.bits, shape.block))
+    out = torch.empty((H - 3, I), dtype=torch.float32, device="cuda")
+    q.moe_dequant_rows(cfg, w.down_codes[e], w.down_scales[e], 3, H - 3, I, out)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64),
+                                  orc.dequantize(dcodes, dsc, H, I, shape.bits, shape.block)[3:])
+
+
+# ----------------------------------------------------------------- router ---
+
+def _check_route(shape, seed, layer, x_bits, zipf=False):
+    w = gc.device_layer(shape, seed, layer, zipf=zipf)
+    idx, wt, counts, offsets, pairs = gc.run_route(shape, w, x_bits)
+    lay = gc.host_oracle_layer(shape, seed, layer, zipf=zipf)
+    logits = orc.router_logits(orc.bf16_to_f64(x_bits), lay.router_w_bits, lay.router_bias)
+    oidx = orc.select_topk(logits, shape.top_k)
+    gc.check_selection(logits, oidx, idx, shape.top_k)
+    # gate weights: the oracle's definition evaluated on the GPU's selection
+    np.testing.assert_allclose(wt, orc.gate_weights(logits, idx), atol=1e-5, rtol=0)
+    np.testing.assert_allclose(wt.sum(1), 1.0, atol=1e-5)
+    c, o, p = orc.group_by_expert(idx, shape.experts)
+    np.testing.assert_array_equal(counts, c)
+    np.testing.assert_array_equal(offsets, o)
+    np.testing.assert_array_equal(pairs, p)
+    return idx
+
+
+@pytest.mark.parametrize("T", [1, 3, 8, 64, 65, 300])
+def test_route_tiny(T):
+    _check_route(mi.TINY, 0, 0, mi.hidden_states_bf16(T, mi.TINY.hidden, 0, 7))
+
+
+@pytest.mark.parametrize("T", [1, 16, 64, 4096])
+def test_route_full(T):
+    _check_route(mi.FULL4, 0, 0, mi.hidden_states_bf16(T, mi.FULL4.hidden, 0, 9))
+
+
+def test_route_zipf_skew():
+    idx = _check_route(mi.FULL2, 0, 0, mi.hidden_states_bf16(64, 2048, 0, 4), zipf=True)
+    rank = np.rint(np.exp(mi.zipf_router_bias(mi.FULL2, 0, 0).astype(np.float64) / -mi.ZIPF_ALPHA))
+    assert np.mean(rank[idx] <= 102) > 0.85
+
+
+def test_route_exact_ties_go_to_smaller_index():
+    """All router rows equal: every logit ties, so the selection is experts
+    0..k-1 in order with equal gates."""
+    torch = gc.torch()
+    shape = mi.TINY
+    w = gc.device_layer(shape, 0, 0)
+    w.router_w = w.router_w[:1].repeat(shape.experts, 1).contiguous()
+    x = mi.hidden_states_bf16(5, shape.hidden, 0, 1)
+    idx, wt, counts, _, _ = gc.run_route(shape, w, x)
+    np.testing.assert_array_equal(idx, np.tile(np.arange(shape.top_k), (5, 1)))
+    np.testing.assert_allclose(wt, 1.0 / shape.top_k, atol=1e-7)
+    assert counts[: shape.top_k].tolist() == [5] * shape.top_k
+    del torch
+
+
+# ------------------------------------------------------------------ layer ---
+
+def _oracle_given(lay, x_bits, gpu_idx, differ):
+    over = {t: gpu_idx[t] for t in differ}
+    return orc.layer_forward(lay, x_bits, topk_override=over)
+
+
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY], ids=["tiny4", "tiny2"])
+@pytest.mark.parametrize("T", [1, 2, 7, 8, 17, 64, 100])
+def test_layer_tiny_live_oracle(shape, T):
+    x = mi.hidden_states_bf16(T, shape.hidden, 0, 0)
+    w = gc.device_layer(shape, 0, 0)
+    y = gc.run_layer(shape, w, x)
+    lay = gc.host_oracle_layer(shape, 0, 0, cache_size=shape.experts + 1)
+    idx = gc.run_route(shape, w, x)[0]
+    r = orc.layer_forward(lay, x)
+    differ = gc.check_selection(r["logits"], r["idx"], idx, shape.top_k)
+    if differ:
+        r = _oracle_given(lay, x, idx, differ)
+    gc.assert_close(y, r["out"])
+
+
+def test_layer_without_shared_expert():
+    shape = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=False, bits=4, block=32)
+    x = mi.hidden_states_bf16(9, shape.hidden, 0, 3)
+    w = gc.device_layer(shape, 2, 0)
+    y = gc.run_layer(shape, w, x)
+    r = orc.layer_forward(gc.host_oracle_layer(shape, 2, 0, cache_size=70), x)
+    gc.assert_close(y, r["out"])
+
+
+def _stored_layer_case(name, T_list):
+    case = gc.load_case(name)
+    E, H, I, k, sh, bits, bs = case["shape"].tolist()
+    shape = mi.MoeShape(E, H, I, k, bool(sh), bits, bs)
+    zipf = bool(case["zipf"])
+    w = gc.device_layer(shape, int(case["seed"]), 0, zipf=zipf)
+    xall = mi.hidden_states_bf16(int(case["T"]), H, int(case["seed"]), int(case["batch"]))
+    toks = case["tokens"]
+    for T in T_list:
+        x = xall[:T]
+        y = gc.run_layer(shape, w, x)
+        idx = gc.run_route(shape, w, x)[0]
+        sel = toks[toks < T]
+        rows = np.searchsorted(toks, sel)
+        ref = case["out_"][rows].astype(np.float64)
+        differ = gc.check_selection(case["logits"][rows], case["idx"][rows], idx[sel], k)
+        if differ:   # re-run the oracle on the GPU's (valid) selection for those tokens
+            lay = gc.host_oracle_layer(shape, int(case["seed"]), 0, zipf=zipf)
+            for i in differ:
+                r = orc.layer_forward(lay, x[sel[i]:sel[i] + 1], topk_override={0: idx[sel[i]]})
+                ref[i] = r["out"][0]
+        gc.assert_close(y[sel], ref)
+
+
+def test_layer_full4_decode_stored_oracle():
+    _stored_layer_case("full4_decode", [1, 4, 16])
+
+
+def test_layer_full2_zipf_decode_stored_oracle():
+    _stored_layer_case("full2_zipf_decode", [1, 2, 8, 33, 64])
+
+
+def test_layer_full4_prefill_stored_oracle():
+    _stored_layer_case("full4_prefill", [4096])
+
+
+def test_layer_is_deterministic():
+    torch = gc.torch()
+    shape = mi.FULL4
+    w = gc.device_layer(shape, 0, 0)
+    cfg = gc.cfg_of(shape)
+    x = gc.to_dev_bits(mi.hidden_states_bf16(16, shape.hidden, 0, 5))
+    ws = gc.workspace(cfg, 16)
+    y1, y2 = torch.empty_like(x), torch.empty_like(x)
+    q.moe_layer_forward(cfg, w, x, y1, ws)
+    q.moe_layer_forward(cfg, w, x, y2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_empty_batch_and_small_workspace():
+    torch = gc.torch()
+    shape = mi.TINY
+    w = gc.device_layer(shape, 0, 0)
+    cfg = gc.cfg_of(shape)
+    x = gc.to_dev_bits(mi.hidden_states_bf16(4, shape.hidden, 0, 0))
+    y = torch.full_like(x, 7)
+    ws = gc.workspace(cfg, 4)
+    assert q.moe_layer_forward(cfg, w, x, y, ws, tokens=0) == 0
+    torch.cuda.synchronize()
+    assert bool((y == 7).all())
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    assert q.moe_layer_forward(cfg, w, x, y, small, check=False) == -3
+
+
+# ------------------------------------------------------------------ stack ---
+
+def _gpu_stack(shape, layers_w, x_bits, trace=True):
+    torch = gc.torch()
+    cfg = gc.cfg_of(shape)
+    T = x_bits.shape[0]
+    x = gc.to_dev_bits(x_bits)
+    ws = gc.workspace(cfg, T)
+    tr = torch.empty((len(layers_w), T, shape.top_k), dtype=torch.int32, device="cuda") if trace else None
+    q.moe_stack_forward(cfg, layers_w, x, ws, topk_trace=tr)
+    torch.cuda.synchronize()
+    assert q.moe_device_status(ws) == 0
+    return mi.bf16_bits_to_f32(gc.bits_to_np(x)).astype(np.float64), (tr.cpu().numpy() if trace else None)
+
+
+STACK_BAND = 2e-3   # the residual streams of both sides differ by bf16 rounding flips after a few layers
+
+
+def test_stack_tiny_live_oracle():
+    shape = mi.TINY
+    L, T = 4, 6
+    ws = [gc.device_layer(shape, 0, l) for l in range(L)]
+    x = mi.hidden_states_bf16(T, shape.hidden, 0, 2)
+    got, trace = _gpu_stack(shape, ws, x)
+    lays = [gc.host_oracle_layer(shape, 0, l, cache_size=shape.experts + 1) for l in range(L)]
+
+    def choose(l, logits, idx):
+        over = {}
+        for t in range(T):
+            if not np.array_equal(trace[l, t], idx[t]):
+                assert orc.tie_band_ok(logits[t], trace[l, t], shape.top_k, STACK_BAND), (l, t)
+                over[t] = trace[l, t]
+        return over
+    r = orc.stack_forward(lays, x, choose_topk=choose)
+    gc.assert_close(got, r["x"])
+
+
+def test_stack_full48_decode_stored_oracle():
+    case = gc.load_case("full4_stack48_decode")
+    shape = mi.FULL4
+    L = int(case["layers"])
+    ws = [gc.device_layer(shape, 0, l) for l in range(L)]
+    x = mi.hidden_states_bf16(int(case["T"]), shape.hidden, 0, int(case["batch"]))
+    got, trace = _gpu_stack(shape, ws, x)
+    toks = case["tokens"]
+    compared = 0
+    for i, t in enumerate(toks):
+        same = all(np.array_equal(trace[l, t], case["trace_idx"][l, i]) for l in range(L))
+        for l in range(L):
+            assert orc.tie_band_ok(case["trace_logits"][l, i], trace[l, t], shape.top_k, STACK_BAND)
+        if same:
+            gc.assert_close(got[t], case["x_final"][i].astype(np.float64))
+            compared += 1
+    assert compared >= len(toks) // 2
