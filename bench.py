@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--instances", type=int, default=48, help="distinct layer instances rotated over")
     ap.add_argument("--no-detail", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--cpu-sample-tokens", type=int, default=2)
+    ap.add_argument("--quick", action="store_true",
+                    help="headline loop only (no e2e, detail or CPU baseline): the small case used for ncu")
     return ap.parse_args()
 
 
@@ -321,6 +323,10 @@ def main():
                              "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls}}
     roofline["frac"] = roofline["achieved"] / hbm_peak
 
+    if args.quick:
+        print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "steps": K, "ms_per_step": ms_step,
+                          "roofline": roofline, "quick": True}), flush=True)
+        return
     # ---- end to end: pinned host x -> device -> layer -> host y, every step
     x_host = [xs[i].cpu().pin_memory() for i in range(NX)]
     y_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(4)]

@@ -274,7 +274,7 @@ def stack_forward(layers, x_bits: np.ndarray, *, choose_topk=None) -> dict:
             override = choose_topk(l, probe["logits"], probe["idx"])
         r = layer_forward(layer, xb, rmsnorm=True, topk_override=override)
         x = round_bf16(x + r["out"])
-        trace.append({"idx": r["idx"], "logits": r["logits"]})
+        trace.append({"idx": r["idx"], "logits": r["logits"], "x": x.copy()})
     return {"x": x, "trace": trace}
 
 

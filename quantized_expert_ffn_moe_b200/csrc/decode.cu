@@ -81,31 +81,198 @@ struct FfnArgs {
   RouteView rv;
 };
 
-// Token range of a slot: routed expert e -> its sorted positions; the shared
-// expert (id E) -> positions T*k .. T*k+T-1.
-__device__ __forceinline__ void slot_tokens(const RouteView& rv, int slot, int* e_out, int* p0, int* n) {
-  const int e = __ldcg(rv.ulist + slot);
-  *e_out = e;
-  if (e >= rv.E) {
-    *p0 = rv.T * rv.k;
-    *n = rv.T;
-  } else {
-    *p0 = __ldcg(rv.offsets + e);
-    *n = __ldcg(rv.offsets + e + 1) - *p0;
-  }
-}
-
-// Cursor over the work units (slot, token chunk, row stage) of one CTA.
+// Walks the stages (slot, token chunk, row stage) whose start lies in this
+// CTA's share [w0, w1) of the pass's cost (see stage_cost); producer and
+// consumers walk the same sequence.
 struct Cursor {
-  int slot, chunk, stage, nchunks;
+  const RouteView* rv;
+  int nslots, spe, ntc;
+  int slot, n, p0, e, chunk, nc, stage;
+  long long pos;               // cost position of the current stage's start
+
+  __device__ void load_slot() {
+    slot_range(*rv, slot, &e, &p0, &n);
+    chunk = 0;
+    nc = min(ntc, n);
+    stage = 0;
+  }
+  __device__ void next_chunk() {
+    ++chunk;
+    stage = 0;
+    if (chunk * ntc >= n) {
+      if (++slot < nslots) load_slot();
+    } else {
+      nc = min(ntc, n - chunk * ntc);
+    }
+  }
+  __device__ void init(long long w0) {
+    int lo = 0, hi = nslots - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldcg(rv->woff + mid) <= w0) lo = mid; else hi = mid - 1;
+    }
+    slot = lo;
+    load_slot();
+    pos = __ldcg(rv->woff + lo);
+    while (slot < nslots) {
+      const long long c = stage_cost(nc), chunk_cost = c * spe;
+      if (pos + chunk_cost <= w0) {
+        pos += chunk_cost;
+        next_chunk();
+        continue;
+      }
+      const long long k = (w0 - pos + c - 1) / c;     // first stage starting at or after w0
+      if (k >= spe) {
+        pos += chunk_cost;
+        next_chunk();
+      } else {
+        stage = int(k);
+        pos += k * c;
+      }
+      break;
+    }
+  }
+  __device__ bool valid(long long w1) const { return slot < nslots && pos < w1; }
+  __device__ void advance() {
+    pos += stage_cost(nc);
+    if (++stage == spe) next_chunk();
+  }
 };
 
-__device__ __forceinline__ int chunks_of(int n, int ntc) { return (n + ntc - 1) / ntc; }
+// Two rows of one stage (codes + scales in shared memory) and their row index
+// in the expert matrix.
+struct Rows {
+  const unsigned char* codes;     // row rl0; row rl0+1 follows at +RB
+  const unsigned char* scales;    // row rl0; row rl0+1 follows at +SPR*2
+  int r0;
+};
+
+// Dot products of the lane group's two rows with NT staged tokens, reduced
+// over the LPR lanes of the row, then the epilogue.  Each block's products
+// accumulate in two independent fp16x2 chains (even / odd code words) and
+// are folded into fp32 with the block scale.  `nt` <= NT tokens are valid.
+template <int MODE, int BITS, int LPR, int CPL, int NT>
+__device__ __forceinline__ void rows_dot(const FfnArgs& a, const Rows& rw, const __half* xs, int tb, int lr,
+                                         const float* tok_inv, const float* tok_w, const int* tok_pos,
+                                         int nt = NT) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  constexpr int K = Gm::K;
+  float acc[2][NT];
+#pragma unroll
+  for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[rho][t] = 0.f;
+#pragma unroll
+  for (int s = 0; s < CPL; ++s) {
+    const int c = s * LPR + lr;
+    const uint4 cw0 = *reinterpret_cast<const uint4*>(rw.codes + c * 16);
+    const uint4 cw1 = *reinterpret_cast<const uint4*>(rw.codes + Gm::RB + c * 16);
+    const uint32_t wd[2][4] = {{cw0.x, cw0.y, cw0.z, cw0.w}, {cw1.x, cw1.y, cw1.z, cw1.w}};
+    if (BITS == 4) {
+      float sc[2];
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho)
+        sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * Gm::SPR * 2 + c * 2));
+      __half2 hacc[2][NT][2];
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) hacc[rho][t][0] = hacc[rho][t][1] = __float2half2_rn(0.f);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        __half2 q[2][4];
+        decode_q4x8(wd[0][m], q[0]);
+        decode_q4x8(wd[1][m], q[1]);
+        const __half* xcol = xs + ((s * 4 + m) * LPR + lr) * 8;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (NT == 4 && t >= nt) continue;
+          const uint4 xv = *reinterpret_cast<const uint4*>(xcol + size_t(t) * K);
+          const __half2 x2[4] = {u32_as_h2(xv.x), u32_as_h2(xv.y), u32_as_h2(xv.z), u32_as_h2(xv.w)};
+#pragma unroll
+          for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+            for (int z = 0; z < 4; ++z) hacc[rho][t][m & 1] = __hfma2(q[rho][z], x2[z], hacc[rho][t][m & 1]);
+        }
+      }
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (NT == 4 && t >= nt) continue;
+          const float2 f = __half22float2(__hadd2(hacc[rho][t][0], hacc[rho][t][1]));
+          acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
+        }
+    } else {
+      uint2 scp[2];
+#pragma unroll
+      for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        __half2 q[2][8];
+        decode_q2x16(wd[0][m], q[0]);
+        decode_q2x16(wd[1][m], q[1]);
+        const __half* xcol = xs + ((s * 4 + m) * 2 * LPR + lr) * 8;
+        float sc[2];
+#pragma unroll
+        for (int rho = 0; rho < 2; ++rho) {
+          const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
+          sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          if (NT == 4 && t >= nt) continue;
+          const __half* xr = xcol + size_t(t) * K;
+          const uint4 xa = *reinterpret_cast<const uint4*>(xr);
+          const uint4 xb = *reinterpret_cast<const uint4*>(xr + LPR * 8);
+          const __half2 x2[8] = {u32_as_h2(xa.x), u32_as_h2(xa.y), u32_as_h2(xa.z), u32_as_h2(xa.w),
+                                 u32_as_h2(xb.x), u32_as_h2(xb.y), u32_as_h2(xb.z), u32_as_h2(xb.w)};
+#pragma unroll
+          for (int rho = 0; rho < 2; ++rho) {
+            __half2 h0 = __hmul2(q[rho][0], x2[0]), h1 = __hmul2(q[rho][1], x2[1]);
+#pragma unroll
+            for (int z = 2; z < 8; z += 2) {
+              h0 = __hfma2(q[rho][z], x2[z], h0);
+              h1 = __hfma2(q[rho][z + 1], x2[z + 1], h1);
+            }
+            const float2 f = __half22float2(__hadd2(h0, h1));
+            acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
+          }
+        }
+      }
+    }
+  }
+  // reduce across the LPR lanes of each row
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    if (NT == 4 && t >= nt) continue;
+#pragma unroll
+    for (int rho = 0; rho < 2; ++rho)
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) acc[rho][t] += __shfl_xor_sync(0xffffffffu, acc[rho][t], o);
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int tl = tb + t;
+    if (t < nt && lr == (t % LPR)) {
+      const float inv = tok_inv[tl];
+      const int p = tok_pos[tl];
+      if (MODE == GATEUP) {
+        const float g = acc[0][t] * inv, u = acc[1][t] * inv;
+        a.out[size_t(p) * a.out_cols + (rw.r0 >> 1)] = g / (1.f + expf(-g)) * u;
+      } else {
+        const float wgt = tok_w[tl] * inv;
+        *reinterpret_cast<float2*>(a.out + size_t(p) * a.out_cols + rw.r0) = make_float2(acc[0][t] * wgt, acc[1][t] * wgt);
+      }
+    }
+  }
+}
 
 template <int MODE, int BITS, int LPR, int CPL>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
+  constexpr int NTB = 4;                        // tokens per register block
   const int ntc = a.ntc;
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -136,48 +303,22 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
 
   const RouteView& rv = a.rv;
   const int nslots = __ldcg(rv.status + ST_UCOUNT) + rv.shared;
-  const int total = __ldcg(rv.woff + nslots);
-  const int w0 = int((long long)total * blockIdx.x / gridDim.x);
-  const int w1 = int((long long)total * (blockIdx.x + 1) / gridDim.x);
+  const long long total = __ldcg(rv.woff + nslots);
+  const long long w0 = total * blockIdx.x / gridDim.x;
+  const long long w1 = total * (blockIdx.x + 1) / gridDim.x;
   if (w0 >= w1) return;
-  const int spe = a.rows / Gm::RPS;
-
-  // slot holding work unit w0: largest u with woff[u] <= w0
-  int lo = 0, hi = nslots - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldcg(rv.woff + mid) <= w0) lo = mid; else hi = mid - 1;
-  }
   Cursor cur;
-  {
-    int e, p0, n;
-    slot_tokens(rv, lo, &e, &p0, &n);
-    const int within = w0 - __ldcg(rv.woff + lo);
-    cur.slot = lo;
-    cur.chunk = within / spe;
-    cur.stage = within % spe;
-    cur.nchunks = chunks_of(n, ntc);
-  }
-  auto advance = [&](Cursor& c) {
-    if (++c.stage == spe) {
-      c.stage = 0;
-      if (++c.chunk == c.nchunks) {
-        c.chunk = 0;
-        ++c.slot;
-        if (c.slot < nslots) {
-          int e, p0, n;
-          slot_tokens(rv, c.slot, &e, &p0, &n);
-          c.nchunks = chunks_of(n, ntc);
-        }
-      }
-    }
-  };
+  cur.rv = &rv;
+  cur.nslots = nslots;
+  cur.spe = a.rows / Gm::RPS;
+  cur.ntc = ntc;
+  cur.init(w0);
 
   if (producer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = 0;
-      for (int w = w0; w < w1; ++w, advance(cur)) {
+      for (; cur.valid(w1); cur.advance()) {
         const int slot = issued % kStages;
         if (*abort_flag) break;
         if (issued >= kStages && !mbar_wait(&empty[slot], ((issued / kStages) - 1) & 1, abort_flag)) {
@@ -185,10 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
           report_error(a.status, MOE_ERR_TIMEOUT, 1);
           break;
         }
-        const int e = __ldcg(rv.ulist + cur.slot);
-        const bool sh = e >= rv.E;
-        const uint8_t* cb = sh ? a.sh_codes : a.codes + size_t(e) * a.expert_code_bytes;
-        const uint16_t* sb = sh ? a.sh_scales : a.scales + size_t(e) * a.expert_scale_count;
+        const bool sh = cur.e >= rv.E;
+        const uint8_t* cb = sh ? a.sh_codes : a.codes + size_t(cur.e) * a.expert_code_bytes;
+        const uint16_t* sb = sh ? a.sh_scales : a.scales + size_t(cur.e) * a.expert_scale_count;
         const size_t row0 = size_t(cur.stage) * Gm::RPS;
         unsigned char* dst = ring + slot * Gm::STAGE_BYTES;
         mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + Gm::SCALE_BYTES);
@@ -206,17 +346,17 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
   // -------------------------------------------------------------- consumers
   const int grp = lane / LPR, lr = lane % LPR;
   const int rl0 = (warp * Gm::RW + grp) * 2;     // local rows rl0, rl0+1 of each stage
-  int e = 0, p0 = 0, n = 0, nc = 0;
-  for (int w = w0, i = 0; w < w1; ++w, ++i, advance(cur)) {
-    if (w == w0 || cur.stage == 0) {
+  bool first = true;
+  for (int i = 0; cur.valid(w1); ++i, cur.advance()) {
+    const int nc = cur.nc;
+    if (first || cur.stage == 0) {
+      first = false;
       // (re)stage the activations of this slot's token chunk
-      slot_tokens(rv, cur.slot, &e, &p0, &n);
-      const bool is_shared = e >= rv.E;
+      const bool is_shared = cur.e >= rv.E;
       const int tbase = cur.chunk * ntc;
-      nc = min(ntc, n - tbase);
       named_bar_sync(1, kNCW * 32);
       for (int tl = warp; tl < nc; tl += kNCW) {
-        const int p = p0 + tbase + tl;
+        const int p = cur.p0 + tbase + tl;
         const int row = (MODE == GATEUP) ? (is_shared ? p - rv.T * rv.k : __ldcg(rv.pairs + p) / rv.k) : p;
         float vmax = 0.f;
         if (MODE == GATEUP) {
@@ -295,113 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
     }
     if (ok) {
       const unsigned char* st = ring + slot * Gm::STAGE_BYTES;
-      const unsigned char* crow0 = st + rl0 * Gm::RB;
-      const unsigned char* srow0 = st + Gm::CODE_BYTES + rl0 * Gm::SPR * 2;
-      const int r0 = cur.stage * Gm::RPS + rl0;    // row of the expert matrix
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * Gm::SPR * 2,
+                      cur.stage * Gm::RPS + rl0};
 #pragma unroll 1
-      for (int tp = 0; tp < nc; tp += 2) {
-        const bool two = tp + 1 < nc;
-        float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int s = 0; s < CPL; ++s) {
-          const int c = s * LPR + lr;
-          uint4 cw[2];
-          cw[0] = *reinterpret_cast<const uint4*>(crow0 + c * 16);
-          cw[1] = *reinterpret_cast<const uint4*>(crow0 + Gm::RB + c * 16);
-          const uint32_t wd[2][4] = {{cw[0].x, cw[0].y, cw[0].z, cw[0].w}, {cw[1].x, cw[1].y, cw[1].z, cw[1].w}};
-          if (BITS == 4) {
-            float sc[2];
-#pragma unroll
-            for (int rho = 0; rho < 2; ++rho)
-              sc[rho] = __half2float(*reinterpret_cast<const __half*>(srow0 + rho * Gm::SPR * 2 + c * 2));
-            __half2 hacc[2][2];
-#pragma unroll
-            for (int rho = 0; rho < 2; ++rho) hacc[rho][0] = hacc[rho][1] = __float2half2_rn(0.f);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              __half2 q[2][4];
-              decode_q4x8(wd[0][m], q[0]);
-              decode_q4x8(wd[1][m], q[1]);
-              const int off = ((s * 4 + m) * LPR + lr) * 8;
-#pragma unroll
-              for (int t = 0; t < 2; ++t) {
-                if (t == 0 || two) {
-                  const uint4 xv = *reinterpret_cast<const uint4*>(xs + size_t(tp + t) * K + off);
-                  const __half2 x2[4] = {u32_as_h2(xv.x), u32_as_h2(xv.y), u32_as_h2(xv.z), u32_as_h2(xv.w)};
-#pragma unroll
-                  for (int rho = 0; rho < 2; ++rho)
-#pragma unroll
-                    for (int z = 0; z < 4; ++z) hacc[rho][t] = __hfma2(q[rho][z], x2[z], hacc[rho][t]);
-                }
-              }
-            }
-#pragma unroll
-            for (int rho = 0; rho < 2; ++rho)
-#pragma unroll
-              for (int t = 0; t < 2; ++t) {
-                const float2 f = __half22float2(hacc[rho][t]);
-                acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
-              }
-          } else {
-            uint2 scp[2];
-#pragma unroll
-            for (int rho = 0; rho < 2; ++rho)
-              scp[rho] = *reinterpret_cast<const uint2*>(srow0 + rho * Gm::SPR * 2 + c * 8);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              __half2 q[2][8];
-              decode_q2x16(wd[0][m], q[0]);
-              decode_q2x16(wd[1][m], q[1]);
-              const int off = ((s * 4 + m) * 2 * LPR + lr) * 8;
-              float sc[2];
-#pragma unroll
-              for (int rho = 0; rho < 2; ++rho) {
-                const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
-                sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
-              }
-#pragma unroll
-              for (int t = 0; t < 2; ++t) {
-                if (t == 0 || two) {
-                  const __half* xr = xs + size_t(tp + t) * K + off;
-                  const uint4 xa = *reinterpret_cast<const uint4*>(xr);
-                  const uint4 xb = *reinterpret_cast<const uint4*>(xr + LPR * 8);
-                  const __half2 x2[8] = {u32_as_h2(xa.x), u32_as_h2(xa.y), u32_as_h2(xa.z), u32_as_h2(xa.w),
-                                         u32_as_h2(xb.x), u32_as_h2(xb.y), u32_as_h2(xb.z), u32_as_h2(xb.w)};
-#pragma unroll
-                  for (int rho = 0; rho < 2; ++rho) {
-                    __half2 h2 = __float2half2_rn(0.f);
-#pragma unroll
-                    for (int z = 0; z < 8; ++z) h2 = __hfma2(q[rho][z], x2[z], h2);
-                    const float2 f = __half22float2(h2);
-                    acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
-                  }
-                }
-              }
-            }
-          }
-        }
-        // reduce across the LPR lanes of each row
-#pragma unroll
-        for (int rho = 0; rho < 2; ++rho)
-#pragma unroll
-          for (int t = 0; t < 2; ++t)
-#pragma unroll
-            for (int o = LPR / 2; o > 0; o >>= 1) acc[rho][t] += __shfl_xor_sync(0xffffffffu, acc[rho][t], o);
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int tl = tp + t;
-          if (tl < nc && lr == (t % LPR)) {
-            const float inv = tok_inv[tl];
-            const int p = tok_pos[tl];
-            if (MODE == GATEUP) {
-              const float g = acc[0][t] * inv, u = acc[1][t] * inv;
-              a.out[size_t(p) * a.out_cols + (r0 >> 1)] = g / (1.f + expf(-g)) * u;
-            } else {
-              const float wgt = tok_w[tl] * inv;
-              *reinterpret_cast<float2*>(a.out + size_t(p) * a.out_cols + r0) = make_float2(acc[0][t] * wgt, acc[1][t] * wgt);
-            }
-          }
-        }
+      for (int tb = 0; tb < nc; tb += NTB) {
+        const int nt = min(NTB, nc - tb);          // warp-uniform
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(a, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(a, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos);
+        else rows_dot<MODE, BITS, LPR, CPL, 4>(a, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
       }
     }
     __syncwarp();
@@ -459,7 +500,7 @@ cudaError_t launch_one(FfnArgs fa, int num_sms, cudaStream_t s) {
 // 16-byte pieces per row C -> lanes per row (largest power of two <= 32
 // dividing C) and pieces per lane.
 #define MOE_C_CASES(X) X(2, 2, 1) X(4, 4, 1) X(8, 8, 1) X(12, 4, 3) X(16, 16, 1) X(24, 8, 3) \
-                       X(32, 32, 1) X(48, 16, 3) X(64, 32, 2) X(96, 32, 3) X(128, 32, 4)
+                       X(32, 32, 1) X(48, 16, 3) X(64, 16, 4) X(96, 32, 3) X(128, 32, 4)
 
 template <int MODE, int BITS>
 cudaError_t dispatch(int K, FfnArgs fa, int num_sms, cudaStream_t s) {

@@ -13,6 +13,9 @@ using namespace moe;
 
 namespace {
 
+// Batches of up to this many tokens take the decode path (grouped GEMV on CUDA
+// cores); larger batches the tensor-core prefill path.
+constexpr int kDecodeMaxTokens = 64;
 
 int num_sms_current() {
   static int cached[64] = {0};
@@ -86,7 +89,12 @@ int run_layer(const LayerArgs& a) {
                                     nullptr, nullptr, a.stream);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   prof_mark(call, 1, a.stream);
-  e = launch_decode_ffn(a, call >= 0 ? g_prof.ev[call * 5 + 2] : nullptr);
+  if (a.T > kDecodeMaxTokens && prefill_supported(a.cfg)) {
+    e = launch_prefill_ffn(a);
+    if (call >= 0) cudaEventRecord(g_prof.ev[call * 5 + 2], a.stream);
+  } else {
+    e = launch_decode_ffn(a, call >= 0 ? g_prof.ev[call * 5 + 2] : nullptr);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   prof_mark(call, 3, a.stream);
   e = launch_combine(a);

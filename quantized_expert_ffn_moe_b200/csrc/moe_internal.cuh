@@ -24,8 +24,8 @@ enum StatusSlot {
 };
 
 struct Layout {
-  size_t status, logits, topk_idx, topk_w, counts, offsets, pairs, inv, ulist, woff_gu, woff_dn, xhat, h, y, xs,
-      total;
+  size_t status, logits, topk_idx, topk_w, counts, offsets, pairs, inv, ulist, woff_gu, woff_dn, ntoff, xhat, h,
+      y, xs, xscale, total;
   int P;
 };
 
@@ -48,10 +48,12 @@ inline Layout make_layout(const moe_config& c, int T) {
   L.ulist = take(size_t(c.num_experts + 1) * 4);
   L.woff_gu = take(size_t(c.num_experts + 2) * 4);
   L.woff_dn = take(size_t(c.num_experts + 2) * 4);
+  L.ntoff = take(size_t(c.num_experts + 2) * 4);
   L.xhat = take(size_t(T) * c.hidden * 2);
   L.h = take(size_t(P) * c.inter * 4);
   L.y = take(size_t(P) * c.hidden * 4);
   L.xs = take(size_t(P) * c.hidden * 2);
+  L.xscale = take(size_t(P) * 4);
   L.total = o;
   L.P = P;
   return L;
@@ -69,12 +71,34 @@ struct RouteView {
   const int* woff;                  // [nslots+1] work-unit prefix of one GEMV pass
 };
 
+// Token range of a slot of the touched-expert list: a routed expert e -> its
+// sorted positions; the shared expert (id E) -> positions T*k .. T*k+T-1.
+__device__ __forceinline__ void slot_range(const RouteView& rv, int slot, int* e_out, int* p0, int* n) {
+  const int e = __ldcg(rv.ulist + slot);
+  *e_out = e;
+  if (e >= rv.E) {
+    *p0 = rv.T * rv.k;
+    *n = rv.T;
+  } else {
+    *p0 = __ldcg(rv.offsets + e);
+    *n = __ldcg(rv.offsets + e + 1) - *p0;
+  }
+}
+
+// Tokens per tensor-core tile of the prefill path.
+constexpr int kPrefillTileN = 128;
+
 // Work decomposition of one decode GEMV pass, shared by the grouping kernel
 // (which writes the per-slot work prefix) and the GEMV kernel.
 struct PassPlan {
   int ntc;    // tokens staged per chunk
   int spe;    // stages (row groups) per expert
 };
+// Work of one stage in balancing units: streaming its bytes costs about
+// kStageCostMem units and every token it is multiplied with about one more,
+// so CTAs get equal time, not only equal bytes.
+constexpr int kStageCostMem = 1;
+__host__ __device__ inline int stage_cost(int tokens) { return kStageCostMem + tokens; }
 
 // -------------------------------------------------------------- device ---
 __device__ __forceinline__ void pdl_wait() {
@@ -257,6 +281,8 @@ cudaError_t launch_route(const moe_config& c, const uint16_t* router_w, const fl
 cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between = nullptr);
 void decode_plans(const moe_config& c, PassPlan* gu, PassPlan* dn);
 cudaError_t launch_combine(const LayerArgs& a);
+cudaError_t launch_prefill_ffn(const LayerArgs& a);
+bool prefill_supported(const moe_config& c);
 cudaError_t launch_dequant_rows(int bits, int block, const uint8_t* codes, const uint16_t* scales,
                                 int row0, int rows, int cols, float* out, cudaStream_t s);
 bool decode_shape_supported(int bits, int H, int I);

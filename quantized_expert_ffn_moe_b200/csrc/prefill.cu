@@ -1,0 +1,568 @@
+// Prefill path (many tokens per expert): grouped GEMMs on the tcgen05 tensor
+// cores with the packed weights dequantized into shared memory.
+//
+// Same operation as the decode path (the expert FFN that replaces the dense
+// FFN, "Running a 125B Model on a Single RTX 5090: Strata Benchmarks Qwen3.8
+// Flash Next", section "Layer 1: On-Demand MoE Expert Scheduling"); with tens
+// of tokens per expert every weight byte feeds enough multiply-adds for the
+// work to be a dense contraction, so it runs on the tensor cores.
+//
+// Per tile (expert e, 128 weight rows, up to 128 of e's tokens):
+//   D[128 x N] (fp32, TMEM) = W_e[rows, :] (fp16, dequantized) . X_e^T (fp16)
+// with the weights as the UMMA A operand (M = 128) and the tokens as B (N =
+// the tile's token count rounded up to 16), K in steps of 64.
+// Warp roles of the persistent CTA (one per SM):
+//   warp 0      TMA of packed codes + fp16 scales (2-D tensor maps, swizzled)
+//   warp 1      TMA of the token tile (SWIZZLE_128B, the UMMA K-major layout)
+//   warp 2      TMEM allocation; one thread issues tcgen05.mma + commits
+//   warps 3-10  dequantize codes into the fp16 A tile (same swizzled layout)
+//   warps 11-14 epilogue: tcgen05.ld from TMEM, SwiGLU (gate/up) or gate
+//               weight (down), stores
+// Operands are fp16: a weight is q * s rounded once (q exact, s the block's
+// fp16 scale); token rows are converted exactly after a per-token power of
+// two brings their largest element into [2^13, 2^14); h is kept in fp16
+// between the passes.  Within a group of 8 (4-bit) or 16 (2-bit) consecutive
+// k the dequantizer emits elements in the pair order of its integer decode, so
+// the token operand is stored with the same permutation of k (the contraction
+// is unchanged).  Every wait is bounded.
+#include "moe_internal.cuh"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+namespace moe {
+
+namespace {
+
+constexpr int PBM = 128;       // weight rows per tile
+constexpr int PBN = kPrefillTileN;   // tokens per tile (max)
+static_assert(PBN == 128, "the grouping kernel's tile prefix assumes 128 tokens per tile");
+constexpr int PBK = 64;        // k per A/B stage: one 128-byte swizzle row of fp16
+constexpr int RAWK = 256;      // k per packed stage
+constexpr int PNK = 4;         // A/B stages
+constexpr int PNR = 2;         // packed stages
+constexpr int kWarpRaw = 0, kWarpB = 1, kWarpMma = 2, kWarpDq0 = 3, kNumDq = 8, kWarpEp0 = 11, kNumEp = 4;
+constexpr int kPThreads = (kWarpEp0 + kNumEp) * 32;
+constexpr uint32_t kTmemCols = 2 * PBN;
+constexpr int kAStageBytes = PBM * 128;           // 16 KB
+constexpr int kBStageBytes = PBN * 128;           // 16 KB
+
+template <int BITS>
+struct PGeom {
+  static constexpr int BLOCK = BITS == 4 ? 32 : 16;
+  static constexpr int IB = RAWK * BITS / 8;              // packed bytes of a row per packed stage
+  static constexpr int SB = RAWK / BLOCK * 2;             // scale bytes of a row per packed stage
+  static constexpr int CODE_BYTES = PBM * IB;
+  static constexpr int SCALE_BYTES = PBM * SB;
+  static constexpr int SCALE_OFF = (CODE_BYTES + 1023) / 1024 * 1024;   // swizzled scales need alignment
+  static constexpr int RAW_BYTES = SCALE_OFF + SCALE_BYTES;
+  static constexpr int G = BITS == 4 ? 8 : 16;            // k group of the pair order
+};
+
+struct PrefillArgs {
+  int K;                  // reduction length (H gate/up, I down)
+  int rows_pe;            // weight rows per expert (2I gate/up, H down)
+  int out_cols;           // I (h) or H (Y)
+  RouteView rv;
+  const int* ntoff;       // [nslots+1] prefix of token tiles per slot
+  uint16_t* hout;         // gate/up: h [P][I] fp16 bits, k permuted for the down pass
+  const float* xinv;      // gate/up: [P] inverse power-of-two scale of each token row
+  float* yout;            // down: Y [P][H] fp32
+  int* status;
+};
+
+// ------------------------------------------------------------ primitives
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// UMMA shared-memory descriptor of a K-major SWIZZLE_128B tile: rows of 128 B,
+// 8-row atoms 1024 B apart (SBO), version 1, layout type 2.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return uint64_t((saddr & 0x3FFFF) >> 4) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// Instruction descriptor: D fp32, A and B fp16, both K-major, M = 128, N.
+__device__ __forceinline__ uint32_t idesc_f16(int n) {
+  return (1u << 4) | (uint32_t(n >> 3) << 17) | (uint32_t(PBM >> 4) << 24);
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t v[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Packed word -> fp16 pairs q * s (q exact from the magic-number decode, one
+// rounding in the multiply).  Pair order as in the decode path: 4-bit
+// (q_j, q_{j+4}), 2-bit (q_j, q_{j+8}).
+__device__ __forceinline__ void dq4_f16(uint32_t v, __half2 s, uint32_t out[4]) {
+  __half2 q[4];
+  decode_q4x8(v, q);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) out[j] = h2_as_u32(__hmul2(q[j], s));
+}
+__device__ __forceinline__ void dq2_f16(uint32_t v, __half2 s, uint32_t out[8]) {
+  __half2 q[8];
+  decode_q2x16(v, q);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) out[j] = h2_as_u32(__hmul2(q[j], s));
+}
+
+struct TileInfo {
+  int slot, e, p0, n, nvalid, m, j;
+};
+
+__device__ __forceinline__ void tile_info(const PrefillArgs& a, int nslots, int mt, int t, TileInfo* ti) {
+  const int g = t / mt;
+  ti->m = t % mt;
+  int lo = 0, hi = nslots - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldcg(a.ntoff + mid) <= g) lo = mid; else hi = mid - 1;
+  }
+  ti->slot = lo;
+  ti->j = g - __ldcg(a.ntoff + lo);
+  slot_range(a.rv, lo, &ti->e, &ti->p0, &ti->n);
+  ti->nvalid = min(PBN, ti->n - ti->j * PBN);
+}
+
+template <int MODE, int BITS>
+__global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
+    PrefillArgs a, const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
+    const __grid_constant__ CUtensorMap tm_sh_codes, const __grid_constant__ CUtensorMap tm_sh_scales,
+    const __grid_constant__ CUtensorMap tm_b) {
+  using Gm = PGeom<BITS>;
+  extern __shared__ __align__(1024) unsigned char psmem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(psmem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base;                                   // PNK x 16 KB
+  unsigned char* sB = sA + PNK * kAStageBytes;                // PNK x 16 KB
+  unsigned char* sRaw = sB + PNK * kBStageBytes;              // PNR x RAW_BYTES (1024-aligned each)
+  constexpr int RAW_STRIDE = (Gm::RAW_BYTES + 1023) / 1024 * 1024;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + PNR * RAW_STRIDE);
+  uint64_t* full_raw = bars;
+  uint64_t* empty_raw = full_raw + PNR;
+  uint64_t* full_a = empty_raw + PNR;
+  uint64_t* full_b = full_a + PNK;
+  uint64_t* empty_ab = full_b + PNK;
+  uint64_t* acc_full = empty_ab + PNK;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < PNR; ++i) { mbar_init(&full_raw[i], 1); mbar_init(&empty_raw[i], kNumDq); }
+    for (int i = 0; i < PNK; ++i) { mbar_init(&full_a[i], kNumDq / 2); mbar_init(&full_b[i], 1); mbar_init(&empty_ab[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], kNumEp); }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kWarpMma) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  pdl_wait();                     // tokens (and routing) come from earlier kernels
+  pdl_launch_dependents();
+
+  const RouteView& rv = a.rv;
+  const int nslots = __ldcg(rv.status + ST_UCOUNT) + rv.shared;
+  const int mt = a.rows_pe / PBM;
+  const int ntiles = __ldcg(a.ntoff + nslots) * mt;
+  const int KB = a.K / PBK, KR = a.K / RAWK;
+
+  if (warp == kWarpRaw && lane == 0) {
+    // ------------------------------------------------ packed weight producer
+    int rc = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      TileInfo ti;
+      tile_info(a, nslots, mt, t, &ti);
+      const bool sh = ti.e >= rv.E;
+      const CUtensorMap* mc = sh ? &tm_sh_codes : &tm_codes;
+      const CUtensorMap* ms = sh ? &tm_sh_scales : &tm_scales;
+      const int row = (sh ? 0 : ti.e * a.rows_pe) + ti.m * PBM;
+      for (int r = 0; r < KR; ++r, ++rc) {
+        const int s = rc % PNR;
+        if (rc >= PNR && !mbar_wait(&empty_raw[s], ((rc / PNR) - 1) & 1, abort_flag)) {
+          *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 10); break;
+        }
+        unsigned char* dst = sRaw + s * RAW_STRIDE;
+        mbar_arrive_expect_tx(&full_raw[s], Gm::CODE_BYTES + Gm::SCALE_BYTES);
+        tma_load_2d(dst, mc, r * Gm::IB, row, &full_raw[s]);
+        tma_load_2d(dst + Gm::SCALE_OFF, ms, r * (RAWK / Gm::BLOCK), row, &full_raw[s]);
+      }
+    }
+    for (int i = max(0, rc - PNR); i < rc; ++i)
+      if (!mbar_wait(&full_raw[i % PNR], (i / PNR) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 11);
+  } else if (warp == kWarpB && lane == 0) {
+    // ------------------------------------------------------ token producer
+    int kc = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      TileInfo ti;
+      tile_info(a, nslots, mt, t, &ti);
+      const int prow = ti.p0 + ti.j * PBN;
+      for (int kb = 0; kb < KB; ++kb, ++kc) {
+        const int s = kc % PNK;
+        if (kc >= PNK && !mbar_wait(&empty_ab[s], ((kc / PNK) - 1) & 1, abort_flag)) {
+          *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 12); break;
+        }
+        mbar_arrive_expect_tx(&full_b[s], kBStageBytes);
+        tma_load_2d(sB + s * kBStageBytes, &tm_b, kb * PBK, prow, &full_b[s]);
+      }
+    }
+    for (int i = max(0, kc - PNK); i < kc; ++i)
+      if (!mbar_wait(&full_b[i % PNK], (i / PNK) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 13);
+  } else if (warp == kWarpMma && lane == 0) {
+    // ---------------------------------------------------------------- MMA
+    int kc = 0, tc = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x, ++tc) {
+      TileInfo ti;
+      tile_info(a, nslots, mt, t, &ti);
+      const int buf = tc & 1;
+      if (tc >= 2 && !mbar_wait(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag)) {
+        *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 14); break;
+      }
+      tc_fence_after();
+      const int n16 = (ti.nvalid + 15) & ~15;
+      const uint32_t idesc = idesc_f16(n16);
+      const uint32_t d_tmem = tmem_base + uint32_t(buf * PBN);
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++kc) {
+        const int s = kc % PNK;
+        if (!mbar_wait(&full_a[s], (kc / PNK) & 1, abort_flag) || !mbar_wait(&full_b[s], (kc / PNK) & 1, abort_flag)) {
+          *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 15); ok = false; break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kAStageBytes), b0 = smem_u32(sB + s * kBStageBytes);
+#pragma unroll
+        for (int k = 0; k < PBK / 16; ++k)
+          tc_mma(d_tmem, sw128_desc(a0 + k * 32), sw128_desc(b0 + k * 32), idesc, (kb | k) ? 1u : 0u);
+        tc_commit(&empty_ab[s]);
+      }
+      if (!ok) break;
+      tc_commit(&acc_full[buf]);
+    }
+    // wait for this thread's last MMAs before the CTA tears down TMEM
+    if (kc > 0 && !mbar_wait(&empty_ab[(kc - 1) % PNK], ((kc - 1) / PNK) & 1, nullptr))
+      report_error(a.status, MOE_ERR_TIMEOUT, 16);
+  } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kNumDq) {
+    // ----------------------------------------------------------- dequant
+    const int dt = threadIdx.x - kWarpDq0 * 32;    // 0..255
+    const int r = dt & (PBM - 1);                  // tile row
+    const int half = dt >> 7;                      // which two of the four k-blocks of a packed stage
+    int rc = 0, kc = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      for (int rs = 0; rs < KR; ++rs, ++rc) {
+        const int s = rc % PNR;
+        bool ok = !*abort_flag && mbar_wait(&full_raw[s], (rc / PNR) & 1, abort_flag);
+        const unsigned char* raw = sRaw + s * RAW_STRIDE;
+        const unsigned char* sc = raw + Gm::SCALE_OFF;
+        for (int jj = 0; jj < 2; ++jj) {
+          const int kbl = half * 2 + jj;            // k-block within the packed stage (0..3)
+          const int kglob = kc + kbl;               // global k-block counter of this A/B stage
+          const int as = kglob % PNK;
+          if (ok && kglob >= PNK) ok = mbar_wait(&empty_ab[as], ((kglob / PNK) - 1) & 1, abort_flag);
+          if (ok) {
+            unsigned char* arow = sA + as * kAStageBytes + r * 128;
+            if (BITS == 4) {
+              // row r: 2 x 16 bytes of codes = 64 weights, 2 scales
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const int lc = kbl * 2 + cc;                     // logical 16-B chunk in the 128-B row
+                const uint4 w = *reinterpret_cast<const uint4*>(raw + r * Gm::IB + ((lc ^ (r & 7)) << 4));
+                const __half hs = *reinterpret_cast<const __half*>(sc + r * Gm::SB + lc * 2);
+                const __half2 s2 = __half2half2(hs);
+                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  uint32_t o[4];
+                  dq4_f16(wd[q], s2, o);
+                  const int oc = cc * 4 + q;                     // output chunk 0..7
+                  *reinterpret_cast<uint4*>(arow + ((oc ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+              }
+            } else {
+              // row r: 16 bytes of codes = 64 weights in 4 words, 4 scales
+              const int lc = kbl;                                // logical 16-B chunk in the 64-B row
+              const uint4 w = *reinterpret_cast<const uint4*>(raw + r * Gm::IB + ((lc ^ ((r >> 1) & 3)) << 4));
+              const int sci = kbl * 4;                           // first scale of this k-block (of 16 per row)
+              const int schunk = sci >> 3;                       // logical 16-B chunk of the 32-B scale row
+              const uint4 sv = *reinterpret_cast<const uint4*>(sc + r * Gm::SB + ((schunk ^ ((r >> 2) & 1)) << 4));
+              const uint32_t svw[4] = {sv.x, sv.y, sv.z, sv.w};
+              const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int si = (sci & 7) + q;                    // scale index within the 16-B chunk
+                const uint32_t pr = svw[si >> 1];
+                const __half hs = __ushort_as_half((unsigned short)((si & 1) ? (pr >> 16) : (pr & 0xFFFFu)));
+                const __half2 s2 = __half2half2(hs);
+                uint32_t o[8];
+                dq2_f16(wd[q], s2, o);
+                *reinterpret_cast<uint4*>(arow + (((2 * q) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(arow + (((2 * q + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+              }
+            }
+            fence_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_a[as]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_raw[s]);
+        if (!ok && !*abort_flag) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 17); }
+        kc += 4;
+      }
+    }
+  } else if (warp >= kWarpEp0 && warp < kWarpEp0 + kNumEp) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                         // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;                    // tile row
+    int tc = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+      TileInfo ti;
+      tile_info(a, nslots, mt, t, &ti);
+      const int buf = tc & 1;
+      if (*abort_flag || !mbar_wait(&acc_full[buf], (tc >> 1) & 1, abort_flag)) {
+        if (!*abort_flag) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 18); }
+        break;
+      }
+      tc_fence_after();
+      const bool sh = ti.e >= rv.E;
+      const int R = ti.m * PBM + r;                 // row of the expert matrix
+      const int prow = ti.p0 + ti.j * PBN;
+      for (int n0 = 0; n0 < ti.nvalid; n0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
+        if (MODE == 0) {
+          // rows alternate gate / up: lane pairs (2i, 2i+1) hold g and u of row pair i
+          const int i = R >> 1;
+          const int G = Gm::G;
+          const int ip = (i & ~(G - 1)) | decode_slot(BITS, i & (G - 1));
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[c]), 1);
+            if (((lane & 1) == 0) && n0 + c < ti.nvalid) {
+              const int p = prow + n0 + c;
+              const float xi = __ldg(a.xinv + p);
+              const float g = __uint_as_float(v[c]) * xi, u = other * xi;
+              const float hval = g / (1.f + expf(-g)) * u;
+              a.hout[size_t(p) * a.out_cols + ip] = __half_as_ushort(__float2half_rn(hval));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int n = n0 + c;
+            if (n < ti.nvalid) {
+              const int p = prow + n;
+              const float w = sh ? 1.f : __ldg(rv.topk_w + __ldg(rv.pairs + p));
+              a.yout[size_t(p) * a.out_cols + R] = __uint_as_float(v[c]) * w;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  // ----------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+  }
+}
+
+// Token rows gathered into expert order as fp16, k permuted within each group
+// of G as the dequantized weights are, each row scaled by the power of two
+// that brings its largest magnitude into [2^13, 2^14) (exact conversion of the
+// bf16 values; xinv[p] undoes it).  One warp per pair position.
+template <int BITS>
+__global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __restrict__ x, RouteView rv, int H,
+                                                            uint16_t* __restrict__ xs, float* __restrict__ xinv) {
+  pdl_wait();
+  pdl_launch_dependents();
+  constexpr int G = BITS == 4 ? 8 : 16;
+  const int P = rv.T * rv.k + (rv.shared ? rv.T : 0);
+  const int lane = threadIdx.x & 31;
+  for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < P; p += gridDim.x * 8) {
+    const int tok = p < rv.T * rv.k ? __ldg(rv.pairs + p) / rv.k : p - rv.T * rv.k;
+    const uint16_t* src = x + size_t(tok) * H;
+    uint16_t* dst = xs + size_t(p) * H;
+    float vmax = 0.f;
+    for (int h0 = lane * 8; h0 < H; h0 += 256) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + h0));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int z = 0; z < 4; ++z)
+        vmax = fmaxf(vmax, fmaxf(fabsf(__uint_as_float(w[z] << 16)), fabsf(__uint_as_float(w[z] & 0xFFFF0000u))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+    int sh = 0;
+    if (vmax > 0.f) {
+      int ex;
+      frexpf(vmax, &ex);
+      sh = min(max(14 - ex, -100), 100);
+    }
+    const float mul = ldexpf(1.f, sh);
+    if (lane == 0) xinv[p] = ldexpf(1.f, -sh);
+    for (int h0 = lane * G; h0 < H; h0 += 32 * G) {
+      float in[G];
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + h0 + 8 * q));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int z = 0; z < 4; ++z) {
+          in[8 * q + 2 * z] = __uint_as_float(w[z] << 16);
+          in[8 * q + 2 * z + 1] = __uint_as_float(w[z] & 0xFFFF0000u);
+        }
+      }
+      __align__(16) __half out[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) out[decode_slot(BITS, j)] = __float2half_rn(in[j] * mul);
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q)
+        *reinterpret_cast<uint4*>(dst + h0 + 8 * q) = *reinterpret_cast<const uint4*>(out + 8 * q);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
+              uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE, int BITS>
+cudaError_t launch_gemm(const PrefillArgs& pa, const uint8_t* codes, const uint16_t* scales, const uint8_t* sh_codes,
+                        const uint16_t* sh_scales, int E, bool has_shared, const uint16_t* bmat, int P, int num_sms,
+                        cudaStream_t s) {
+  using Gm = PGeom<BITS>;
+  CUtensorMap mc, ms, msc, mss, mb;
+  const uint64_t rb = uint64_t(pa.K) * BITS / 8, spr = uint64_t(pa.K) / Gm::BLOCK;
+  const CUtensorMapSwizzle cswz = BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle sswz = BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_32B;
+  bool ok = make_map(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, codes, rb, uint64_t(E) * pa.rows_pe, Gm::IB, PBM, cswz) &&
+            make_map(&ms, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, spr, uint64_t(E) * pa.rows_pe, Gm::SB / 2, PBM, sswz) &&
+            make_map(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, bmat, uint64_t(pa.K), uint64_t(P), PBK, PBN,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+  if (has_shared) {
+    ok = ok && make_map(&msc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, sh_codes, rb, uint64_t(pa.rows_pe), Gm::IB, PBM, cswz) &&
+         make_map(&mss, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, sh_scales, spr, uint64_t(pa.rows_pe), Gm::SB / 2, PBM, sswz);
+  } else {
+    msc = mc;
+    mss = ms;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  constexpr int RAW_STRIDE = (Gm::RAW_BYTES + 1023) / 1024 * 1024;
+  const size_t smem = 1024 + PNK * (kAStageBytes + kBStageBytes) + PNR * RAW_STRIDE + 256;
+  auto kern = prefill_gemm_kernel<MODE, BITS>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, dim3(num_sms), dim3(kPThreads), smem, s, pa, mc, ms, msc, mss, mb);
+}
+
+}  // namespace
+
+bool prefill_supported(const moe_config& c) {
+  const int H = c.hidden, I = c.inter;
+  const int bs = c.block;
+  if (H % RAWK || I % RAWK) return false;
+  if ((2 * I) % PBM || H % PBM) return false;
+  if ((H / bs * 2) % 16 || (I / bs * 2) % 16) return false;      // TMA row strides
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_prefill_ffn(const LayerArgs& a) {
+  const moe_config& c = a.cfg;
+  const int H = c.hidden, I = c.inter, bits = c.bits;
+  RouteView rv;
+  rv.T = a.T; rv.k = c.top_k; rv.E = c.num_experts; rv.shared = c.shared_inter > 0 ? 1 : 0;
+  rv.status = reinterpret_cast<const int*>(a.ws + a.L.status);
+  rv.ulist = reinterpret_cast<const int*>(a.ws + a.L.ulist);
+  rv.offsets = reinterpret_cast<const int*>(a.ws + a.L.offsets);
+  rv.pairs = reinterpret_cast<const int*>(a.ws + a.L.pairs);
+  rv.inv = reinterpret_cast<const int*>(a.ws + a.L.inv);
+  rv.topk_w = reinterpret_cast<const float*>(a.ws + a.L.topk_w);
+  rv.woff = nullptr;
+  const int P = a.L.P;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(a.ws + a.L.xs);
+  uint16_t* hs = reinterpret_cast<uint16_t*>(a.ws + a.L.h);
+  float* xinv = reinterpret_cast<float*>(a.ws + a.L.xscale);
+  cudaError_t err = bits == 4
+      ? launch_pdl(gather_tokens_kernel<4>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv)
+      : launch_pdl(gather_tokens_kernel<2>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv);
+  if (err != cudaSuccess) return err;
+
+  PrefillArgs g{};
+  g.K = H; g.rows_pe = 2 * I; g.out_cols = I; g.rv = rv;
+  g.ntoff = reinterpret_cast<const int*>(a.ws + a.L.ntoff);
+  g.hout = hs; g.yout = nullptr; g.xinv = xinv;
+  g.status = reinterpret_cast<int*>(a.ws + a.L.status);
+  const bool sh = c.shared_inter > 0;
+  err = bits == 4 ? launch_gemm<0, 4>(g, a.w.gate_up_codes, a.w.gate_up_scales, a.w.shared_gate_up_codes,
+                                      a.w.shared_gate_up_scales, c.num_experts, sh, xs, P, a.num_sms, a.stream)
+                  : launch_gemm<0, 2>(g, a.w.gate_up_codes, a.w.gate_up_scales, a.w.shared_gate_up_codes,
+                                      a.w.shared_gate_up_scales, c.num_experts, sh, xs, P, a.num_sms, a.stream);
+  if (err != cudaSuccess) return err;
+
+  PrefillArgs d = g;
+  d.K = I; d.rows_pe = H; d.out_cols = H;
+  d.hout = nullptr; d.yout = reinterpret_cast<float*>(a.ws + a.L.y);
+  return bits == 4 ? launch_gemm<1, 4>(d, a.w.down_codes, a.w.down_scales, a.w.shared_down_codes,
+                                       a.w.shared_down_scales, c.num_experts, sh, hs, P, a.num_sms, a.stream)
+                   : launch_gemm<1, 2>(d, a.w.down_codes, a.w.down_scales, a.w.shared_down_codes,
+                                       a.w.shared_down_scales, c.num_experts, sh, hs, P, a.num_sms, a.stream);
+}
+
+}  // namespace moe

@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict
 template <int H>
 __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(
     const uint16_t* __restrict__ wr, const float* __restrict__ bias,
-    const uint16_t* __restrict__ x, int T, int E, float* __restrict__ logits) {
+    const uint16_t* __restrict__ x, int T, int E, int tokens_per_cta, float* __restrict__ logits) {
   constexpr int PER_LANE = H / 256;   // 16-byte pieces per lane
   extern __shared__ __align__(16) uint16_t xs[];   // [kRouterTokTile][H]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -71,12 +71,27 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(
   }
   const float b = (e < E && bias) ? bias[e] : 0.f;
   pdl_wait();   // x may be produced by the previous kernel
-  const int t_lo = blockIdx.y * kRouterTokBlock, t_hi = min(T, t_lo + kRouterTokBlock);
+  pdl_launch_dependents();
+  const int t_lo = blockIdx.y * tokens_per_cta, t_hi = min(T, t_lo + tokens_per_cta);
   for (int t0 = t_lo; t0 < t_hi; t0 += kRouterTokTile) {
     const int nt = min(kRouterTokTile, t_hi - t0);
     __syncthreads();
-    for (int i = threadIdx.x; i < nt * H / 8; i += blockDim.x)
-      reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(x + size_t(t0) * H)[i];
+    // stage nt token rows; loads are issued in batches of 8 per thread
+    const int n16 = nt * H / 8;
+    const uint4* src = reinterpret_cast<const uint4*>(x + size_t(t0) * H);
+    for (int base = threadIdx.x; base < n16; base += kRouterWarps * 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kRouterWarps * 32;
+        if (i < n16) v[j] = __ldg(src + i);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kRouterWarps * 32;
+        if (i < n16) reinterpret_cast<uint4*>(xs)[i] = v[j];
+      }
+    }
     __syncthreads();
     if (e < E) {
       for (int t = 0; t < nt; ++t) {
@@ -98,7 +113,6 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(
       }
     }
   }
-  pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------ top-k
@@ -170,7 +184,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
     int* __restrict__ offsets_out, int* __restrict__ pairs_out, int* __restrict__ inv_out,
     int* __restrict__ ulist_out, int* __restrict__ api_counts, int* __restrict__ api_offsets,
     int* __restrict__ api_pairs, PassPlan pg, PassPlan pd, int* __restrict__ woff_gu,
-    int* __restrict__ woff_dn) {
+    int* __restrict__ woff_dn, int* __restrict__ ntoff) {
   extern __shared__ int sm[];
   constexpr int NW = kGroupThreads / 32;
   int* hist = sm;                       // [NW][E]
@@ -275,11 +289,11 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
   }
   __syncthreads();
   // work prefix of the two GEMV passes over the slots (touched experts, then
-  // the shared expert): each slot contributes ceil(n / ntc) * stages units.
+  // the shared expert), in balancing cost units.
   if (warp == 0) {
     const int U = scan[NW - 1];
     const int nslots = U + shared;
-    int run_g = 0, run_d = 0;
+    int run_g = 0, run_d = 0, run_t = 0;
     for (int base = 0; base < nslots; base += 32) {
       const int u = base + lane;
       int n = 0;
@@ -289,24 +303,35 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
       } else if (u < nslots) {
         n = T;
       }
-      int g = u < nslots ? (n + pg.ntc - 1) / pg.ntc * pg.spe : 0;
-      int d = u < nslots ? (n + pd.ntc - 1) / pd.ntc * pd.spe : 0;
+      // cost of a slot = sum over its token chunks of stages * stage_cost(chunk tokens)
+      auto slot_cost = [&](const PassPlan& pp) {
+        if (u >= nslots) return 0;
+        const int full = n / pp.ntc, rest = n % pp.ntc;
+        return pp.spe * (full * stage_cost(pp.ntc) + (rest ? stage_cost(rest) : 0));
+      };
+      int g = slot_cost(pg);
+      int d = slot_cost(pd);
+      int nt = u < nslots ? (n + kPrefillTileN - 1) / kPrefillTileN : 0;   // token tiles (prefill)
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int ng = __shfl_up_sync(0xffffffffu, g, o);
         const int nd = __shfl_up_sync(0xffffffffu, d, o);
-        if (lane >= o) { g += ng; d += nd; }
+        const int nn = __shfl_up_sync(0xffffffffu, nt, o);
+        if (lane >= o) { g += ng; d += nd; nt += nn; }
       }
       if (u < nslots) {
         woff_gu[u + 1] = run_g + g;
         woff_dn[u + 1] = run_d + d;
+        ntoff[u + 1] = run_t + nt;
       }
       run_g += __shfl_sync(0xffffffffu, g, 31);
       run_d += __shfl_sync(0xffffffffu, d, 31);
+      run_t += __shfl_sync(0xffffffffu, nt, 31);
     }
     if (lane == 0) {
       woff_gu[0] = 0;
       woff_dn[0] = 0;
+      ntoff[0] = 0;
     }
   }
   // stable scatter: each warp walks its tokens in order
@@ -350,7 +375,7 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
                     reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
                     reinterpret_cast<int*>(ws + L.inv), reinterpret_cast<int*>(ws + L.ulist), api_counts,
                     api_offsets, api_pairs, pg, pd, reinterpret_cast<int*>(ws + L.woff_gu),
-                    reinterpret_cast<int*>(ws + L.woff_dn));
+                    reinterpret_cast<int*>(ws + L.woff_dn), reinterpret_cast<int*>(ws + L.ntoff));
 }
 
 }  // namespace
@@ -361,10 +386,12 @@ cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* xhat, int T, int H, cuda
 
 cudaError_t launch_router_logits(const moe_config& c, const uint16_t* router_w, const float* bias,
                                  const uint16_t* x, int T, float* logits, cudaStream_t s) {
-  const dim3 grid((c.num_experts + kRouterWarps - 1) / kRouterWarps, (T + kRouterTokBlock - 1) / kRouterTokBlock);
+  // decode batches: 4 tokens per CTA so each CTA stages little; prefill: 256
+  const int tpc = T <= 64 ? 4 : kRouterTokBlock;
+  const dim3 grid((c.num_experts + kRouterWarps - 1) / kRouterWarps, (T + tpc - 1) / tpc);
   const dim3 block(kRouterWarps * 32);
   const size_t smem = size_t(kRouterTokTile) * c.hidden * 2;
-  void (*kern)(const uint16_t*, const float*, const uint16_t*, int, int, float*) = nullptr;
+  void (*kern)(const uint16_t*, const float*, const uint16_t*, int, int, int, float*) = nullptr;
   switch (c.hidden) {
     case 256: kern = router_logits_kernel<256>; break;
     case 512: kern = router_logits_kernel<512>; break;
@@ -375,7 +402,7 @@ cudaError_t launch_router_logits(const moe_config& c, const uint16_t* router_w, 
   }
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(kern, grid, block, smem, s, router_w, bias, x, T, c.num_experts, logits);
+  return launch_pdl(kern, grid, block, smem, s, router_w, bias, x, T, c.num_experts, tpc, logits);
 }
 
 cudaError_t launch_topk_group_any(const moe_config& c, int T, char* ws, const Layout& L, bool fused,

@@ -108,6 +108,9 @@ def compute(name: str, procs: int):
                                      for l in range(L)])
         out["trace_logits"] = np.stack([np.concatenate([r[1]["trace"][l]["logits"] for r in res])[order]
                                         for l in range(L)])
+        # residual stream after each layer (bf16 values, stored exactly as fp32)
+        out["trace_x"] = np.stack([np.concatenate([r[1]["trace"][l]["x"] for r in res])[order]
+                                   for l in range(L)]).astype(np.float32)
     path = os.path.join(HERE, f"oracle_{name}.npz")
     np.savez_compressed(path, **out)
     print(f"{name}: {len(toks)} tokens in {time.time() - t0:.1f} s -> {path}", flush=True)

@@ -115,6 +115,26 @@ def assert_close(got: np.ndarray, ref: np.ndarray, rel=REL_TOL):
     return err / rms
 
 
+# The stack's residual stream is rounded to bf16 after every layer on both
+# sides; where the two sums differ in their last bits the rounding flips by one
+# bf16 ulp (2^-8 relative).  Over d layers the flips add like a random walk,
+# about sqrt(d) * 2^-9 * |x| per element; elements reach ~4 RMS, so d = 48 gives
+# about 0.05 RMS.  Stack checks use that bound on the largest element error and
+# 1e-2 on the root-mean-square error.
+STACK_MAX_TOL = 5e-2
+STACK_RMS_TOL = 1e-2
+
+
+def assert_close_stack(got: np.ndarray, ref: np.ndarray):
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    diff = got - ref
+    err = float(np.max(np.abs(diff)))
+    rerr = float(np.sqrt(np.mean(diff * diff)))
+    assert err <= STACK_MAX_TOL * rms, f"max|err| {err:.3e} > {STACK_MAX_TOL} * rms {rms:.3e}"
+    assert rerr <= STACK_RMS_TOL * rms, f"rms err {rerr:.3e} > {STACK_RMS_TOL} * rms {rms:.3e}"
+    return err / rms, rerr / rms
+
+
 def load_case(name):
     path = os.path.join(GOLDEN, f"oracle_{name}.npz")
     if not os.path.exists(path):

@@ -251,10 +251,17 @@ def test_stack_tiny_live_oracle():
                 over[t] = trace[l, t]
         return over
     r = orc.stack_forward(lays, x, choose_topk=choose)
-    gc.assert_close(got, r["x"])
+    gc.assert_close_stack(got, r["x"])
 
 
 def test_stack_full48_decode_stored_oracle():
+    """48 resident layers.  For each token the GPU's selections must equal the
+    oracle's up to the first layer l* where they differ, and that difference
+    must be a valid choice inside the tie band.  After l* the two residual
+    streams differ by a whole expert, so the comparison point is the stream
+    entering layer l*: the GPU stack is re-run on the first l* layers and
+    compared with the oracle's stream after those layers.  Tokens that never
+    diverge are compared after all 48 layers."""
     case = gc.load_case("full4_stack48_decode")
     shape = mi.FULL4
     L = int(case["layers"])
@@ -262,12 +269,53 @@ def test_stack_full48_decode_stored_oracle():
     x = mi.hidden_states_bf16(int(case["T"]), shape.hidden, 0, int(case["batch"]))
     got, trace = _gpu_stack(shape, ws, x)
     toks = case["tokens"]
-    compared = 0
+    depth = {}
     for i, t in enumerate(toks):
-        same = all(np.array_equal(trace[l, t], case["trace_idx"][l, i]) for l in range(L))
-        for l in range(L):
-            assert orc.tie_band_ok(case["trace_logits"][l, i], trace[l, t], shape.top_k, STACK_BAND)
-        if same:
-            gc.assert_close(got[t], case["x_final"][i].astype(np.float64))
-            compared += 1
-    assert compared >= len(toks) // 2
+        first = next((l for l in range(L) if not np.array_equal(trace[l, t], case["trace_idx"][l, i])), None)
+        if first is not None:
+            assert orc.tie_band_ok(case["trace_logits"][first, i], trace[first, t], shape.top_k, STACK_BAND), \
+                (t, first)
+        depth[i] = L if first is None else first
+    for d in sorted(set(depth.values())):
+        if d == 0:
+            continue
+        xd = got if d == L else _gpu_stack(shape, ws[:d], x, trace=False)[0]
+        for i, t in enumerate(toks):
+            if depth[i] == d:
+                gc.assert_close_stack(xd[t], case["trace_x"][d - 1, i].astype(np.float64))
+    assert max(depth.values()) >= 8, depth
+
+
+# --------------------------------------------------- tensor-core prefill ---
+# Shapes small enough for the live oracle that still take the tcgen05 path
+# (H and I multiples of 256): several expert groups per tile row, ragged tiles.
+MID4 = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=4, block=32)
+MID2 = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=2, block=16)
+
+
+@pytest.mark.parametrize("shape", [MID4, MID2], ids=["mid4", "mid2"])
+@pytest.mark.parametrize("T", [65, 129, 300])
+def test_prefill_path_live_oracle(shape, T):
+    x = mi.hidden_states_bf16(T, shape.hidden, 0, 21)
+    w = gc.device_layer(shape, 4, 0)
+    y = gc.run_layer(shape, w, x)
+    lay = gc.host_oracle_layer(shape, 4, 0, cache_size=shape.experts + 1)
+    idx = gc.run_route(shape, w, x)[0]
+    r = orc.layer_forward(lay, x)
+    differ = gc.check_selection(r["logits"], r["idx"], idx, shape.top_k)
+    if differ:
+        r = _oracle_given(lay, x, idx, differ)
+    gc.assert_close(y, r["out"])
+
+
+def test_prefill_path_without_shared_expert():
+    shape = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=2, shared=False, bits=4, block=32)
+    x = mi.hidden_states_bf16(200, shape.hidden, 0, 8)
+    w = gc.device_layer(shape, 6, 0)
+    y = gc.run_layer(shape, w, x)
+    r = orc.layer_forward(gc.host_oracle_layer(shape, 6, 0, cache_size=40), x)
+    idx = gc.run_route(shape, w, x)[0]
+    differ = gc.check_selection(r["logits"], r["idx"], idx, shape.top_k)
+    if differ:
+        r = _oracle_given(gc.host_oracle_layer(shape, 6, 0, cache_size=40), x, idx, differ)
+    gc.assert_close(y, r["out"])
