@@ -20,13 +20,14 @@ __all__ = [
     "MoeConfig", "LayerWeights", "MoeError", "load_library", "EXPORTS", "LIB_PATH",
     "moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
     "moe_device_status", "moe_dequant_rows", "moe_status_str", "config_of", "moe_profile_begin",
-    "moe_profile_end",
+    "moe_profile_end", "moe_layer_forward_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
-           "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end")
+           "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end",
+           "moe_layer_forward_noalloc")
 
 MOE_OK = 0
 
@@ -97,6 +98,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_device_status.restype = ctypes.c_int
     lib.moe_dequant_rows.argtypes = [cfgp, P, P, I32, I32, I32, P, P]
     lib.moe_dequant_rows.restype = ctypes.c_int
+    lib.moe_layer_forward_noalloc.argtypes = [cfgp, ctypes.POINTER(_Weights), P, I32, P, P]
+    lib.moe_layer_forward_noalloc.restype = ctypes.c_int
     lib.moe_profile_begin.argtypes = [I32]
     lib.moe_profile_begin.restype = ctypes.c_int
     lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)]
@@ -161,6 +164,22 @@ def moe_layer_forward(cfg: MoeConfig, w: LayerWeights, x, y, workspace, *, strea
     if check:
         _check(st, "moe_layer_forward")
     return st
+
+
+def moe_layer_forward_noalloc(cfg: MoeConfig, w: LayerWeights, x, y, *, stream=None, check=True,
+                              tokens: Optional[int] = None) -> int:
+    """moe_layer_forward without a workspace argument: the library's fixed
+    scratch array is used (see include/moe_capi.h for the size limit)."""
+    T = int(x.shape[0]) if tokens is None else tokens
+    cw = w.to_c()
+    st = load_library().moe_layer_forward_noalloc(ctypes.byref(cfg), ctypes.byref(cw), _ptr(x), T, _ptr(y),
+                                                  _stream(stream))
+    if check:
+        _check(st, "moe_layer_forward_noalloc")
+    return st
+
+
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 def moe_stack_forward(cfg: MoeConfig, layers: Sequence[LayerWeights], x_inout, workspace, *, topk_trace=None,
