@@ -314,14 +314,25 @@ def main():
     for i in range(n_prof):
         step(i)
     phase_ms, calls = q.moe_profile_end()
-    gu_ms = phase_ms[1] / calls
-    gu_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * GU_BYTES[4]
-    roofline = {"bound": "hbm", "kernel": "ffn_tma_kernel<gate/up>", "achieved": gu_bytes / (gu_ms * 1e-3) / 1e9,
+    fused = phase_ms[4] > 0
+    if fused:
+        # one cooperative kernel per layer: the dominant (only) kernel moves all touched bytes
+        k_ms = phase_ms[4] / calls
+        k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * EXPERT_BYTES[4] + ROUTER_BYTES
+        kname = "fused_decode_kernel (whole layer, one launch)"
+    else:
+        k_ms = phase_ms[1] / calls
+        k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * GU_BYTES[4]
+        kname = "ffn_tma_kernel<gate/up>"
+    roofline = {"bound": "hbm", "kernel": kname, "achieved": k_bytes / (k_ms * 1e-3) / 1e9,
                 "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": None,
                 "peak_source": f"{peak_src} (copy bandwidth)",
+                "algorithmic_bytes_per_launch": k_bytes, "launch_us": 1000 * k_ms,
                 "phase_us": {"route": 1000 * phase_ms[0] / calls, "gate_up": 1000 * phase_ms[1] / calls,
-                             "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls}}
+                             "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls,
+                             "fused": 1000 * phase_ms[4] / calls}}
     roofline["frac"] = roofline["achieved"] / hbm_peak
+    launches_per_step = 1 if fused else 5
 
     if args.quick:
         print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "steps": K, "ms_per_step": ms_step,
@@ -360,7 +371,7 @@ def main():
                     "achieved_gbs": touched_bytes / (ms_step * 1e-3) / 1e9,
                     "frac_of_measured": touched_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak,
                     "frac_of_8tbs": touched_bytes / (ms_step * 1e-3) / 8e12},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": 5 * K, "clocks": clocks}
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches_per_step * K, "clocks": clocks}
 
     # ---- secondary workloads of the same layer family
     if not args.no_detail:

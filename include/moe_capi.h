@@ -154,11 +154,16 @@ int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t
 /* Measurement hook.  moe_profile_begin(n) makes the next n layer calls
  * record CUDA events around their four phases on the call's stream (route,
  * gate/up + SwiGLU, down, combine); moe_profile_end() waits for those events
- * and returns the summed milliseconds per phase in ms_out[4] and the number of
- * recorded calls in *calls.  Events are host-side driver objects; no device
+ * and returns the summed milliseconds per phase in ms_out[0..3] -- and in
+ * ms_out[4] the time of calls that ran as one fused decode kernel -- and the
+ * number of recorded calls in *calls.  Events are host-side driver objects; no device
  * memory is allocated.  Not thread-safe; meant for benchmarks. */
 int moe_profile_begin(int32_t max_calls);
 int moe_profile_end(float* ms_out, int32_t* calls);
+
+/* The cudaError_t value behind the calling thread's most recent
+ * MOE_ERR_CUDA (0 if none). */
+int moe_last_cuda_error(void);
 
 /* Static description of a status code. */
 const char* moe_status_str(int status);

@@ -27,14 +27,15 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
            "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end",
-           "moe_layer_forward_noalloc")
+           "moe_layer_forward_noalloc", "moe_last_cuda_error")
 
 MOE_OK = 0
 
 
 class MoeError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: status {status} ({moe_status_str(status)})")
+        detail = f", cudaError {load_library().moe_last_cuda_error()}" if status == -4 else ""
+        super().__init__(f"{what}: status {status} ({moe_status_str(status)}{detail})")
         self.status = status
 
 
@@ -104,6 +105,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_profile_begin.restype = ctypes.c_int
     lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)]
     lib.moe_profile_end.restype = ctypes.c_int
+    lib.moe_last_cuda_error.argtypes = []
+    lib.moe_last_cuda_error.restype = ctypes.c_int
     lib.moe_status_str.argtypes = [ctypes.c_int]
     lib.moe_status_str.restype = ctypes.c_char_p
     _lib = lib
@@ -214,8 +217,8 @@ def moe_profile_begin(max_calls: int):
 
 
 def moe_profile_end():
-    """Returns ([route, gate_up, down, combine] summed ms, number of calls)."""
-    ms = (ctypes.c_float * 4)()
+    """Returns ([route, gate_up, down, combine, fused] summed ms, number of calls)."""
+    ms = (ctypes.c_float * 5)()
     n = ctypes.c_int32(0)
     _check(load_library().moe_profile_end(ms, ctypes.byref(n)), "moe_profile_end")
     return [float(v) for v in ms], int(n.value)

@@ -67,13 +67,20 @@ int check_ws(const moe_config* c, int T, void* ws, size_t ws_bytes) {
   return MOE_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  g_last_cuda_error = int(e);
+  return MOE_ERR_CUDA;
+}
 
 // Optional per-phase event recording (moe_profile_begin / moe_profile_end).
 struct Profile {
   bool on = false;
   int cap = 0, used = 0;
   cudaEvent_t* ev = nullptr;    // [cap][5]
+  unsigned char* fused = nullptr;  // [cap] call ran as one fused kernel
 };
 Profile g_prof;
 
@@ -87,7 +94,7 @@ int run_layer(const LayerArgs& a) {
   prof_mark(call, 0, a.stream);
   cudaError_t e = launch_route_full(a.cfg, a.w.router_w, a.w.router_bias, a.x, a.T, a.ws, a.L, nullptr,
                                     nullptr, nullptr, a.stream);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   prof_mark(call, 1, a.stream);
   if (a.T > kDecodeMaxTokens && prefill_supported(a.cfg)) {
     e = launch_prefill_ffn(a);
@@ -95,7 +102,7 @@ int run_layer(const LayerArgs& a) {
   } else {
     e = launch_decode_ffn(a, call >= 0 ? g_prof.ev[call * 5 + 2] : nullptr);
   }
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   prof_mark(call, 3, a.stream);
   e = launch_combine(a);
   prof_mark(call, 4, a.stream);
@@ -157,6 +164,19 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
   a.num_sms = num_sms_current();
   a.stream = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T)) {
+    const int call = (g_prof.on && g_prof.used < g_prof.cap) ? g_prof.used++ : -1;
+    prof_mark(call, 0, a.stream);
+    const cudaError_t e = launch_fused_decode(*cfg, w, 1, x, y, false, T, nullptr, a.ws, a.L, a.num_sms, a.stream);
+    if (e == cudaSuccess) {
+      for (int ph = 1; ph <= 4; ++ph) prof_mark(call, ph, a.stream);
+      if (call >= 0) g_prof.fused[call] = 1;
+      return MOE_OK;
+    }
+    if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
+    (void)cudaGetLastError();        // cannot co-schedule one CTA per SM here: separate kernels
+    if (call >= 0) g_prof.used--;
+  }
   return run_layer(a);
 }
 
@@ -179,6 +199,13 @@ int moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, in
   a.stream = static_cast<cudaStream_t>(stream);
   uint16_t* xhat = reinterpret_cast<uint16_t*>(a.ws + a.L.xhat);
   if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T)) {
+    const cudaError_t e = launch_fused_decode(*cfg, layers, L, x_inout, x_inout, true, T, topk_trace, a.ws, a.L,
+                                              a.num_sms, a.stream);
+    if (e == cudaSuccess) return MOE_OK;
+    if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
+    (void)cudaGetLastError();
+  }
   if (launch_rmsnorm(x_inout, xhat, T, cfg->hidden, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
   for (int l = 0; l < L; ++l) {
     a.w = layers[l];
@@ -219,6 +246,7 @@ int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t
 int moe_profile_begin(int32_t max_calls) {
   if (max_calls <= 0 || g_prof.on) return MOE_ERR_INVALID_ARG;
   g_prof.ev = new cudaEvent_t[size_t(max_calls) * 5];
+  g_prof.fused = new unsigned char[max_calls]();
   for (int i = 0; i < max_calls * 5; ++i)
     if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
   g_prof.cap = max_calls;
@@ -230,22 +258,25 @@ int moe_profile_begin(int32_t max_calls) {
 int moe_profile_end(float* ms_out, int32_t* calls) {
   if (!g_prof.on || !ms_out || !calls) return MOE_ERR_INVALID_ARG;
   int st = MOE_OK;
-  for (int p = 0; p < 4; ++p) ms_out[p] = 0.f;
+  for (int p = 0; p < 5; ++p) ms_out[p] = 0.f;
   for (int c = 0; c < g_prof.used; ++c) {
     for (int p = 0; p < 4; ++p) {
       float ms = 0.f;
       if (cudaEventSynchronize(g_prof.ev[c * 5 + p + 1]) != cudaSuccess ||
           cudaEventElapsedTime(&ms, g_prof.ev[c * 5 + p], g_prof.ev[c * 5 + p + 1]) != cudaSuccess)
         st = MOE_ERR_CUDA;
-      ms_out[p] += ms;
+      ms_out[g_prof.fused[c] ? 4 : p] += ms;
     }
   }
   *calls = g_prof.used;
   for (int i = 0; i < g_prof.cap * 5; ++i) cudaEventDestroy(g_prof.ev[i]);
   delete[] g_prof.ev;
+  delete[] g_prof.fused;
   g_prof = Profile{};
   return st;
 }
+
+int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* moe_status_str(int status) {
   switch (status) {

@@ -20,6 +20,8 @@ enum StatusSlot {
   ST_ERROR = 0,      // first failed device check (0 = none)
   ST_ERROR_AUX = 1,  // detail of that check
   ST_UCOUNT = 2,     // number of distinct routed experts selected
+  ST_GRID_COUNT = 4, // fused decode: grid barrier arrivals
+  ST_GRID_GEN = 5,   // fused decode: grid barrier generation
   ST_COUNT = 16
 };
 
@@ -282,7 +284,14 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between = nullptr)
 void decode_plans(const moe_config& c, PassPlan* gu, PassPlan* dn);
 cudaError_t launch_combine(const LayerArgs& a);
 cudaError_t launch_prefill_ffn(const LayerArgs& a);
+bool fused_supported(const moe_config& c, int T);
+cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x,
+                                uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
+                                cudaStream_t s);
 bool prefill_supported(const moe_config& c);
+bool router_gemm_supported(const moe_config& c, int T);
+cudaError_t launch_router_gemm(const moe_config& c, const uint16_t* router_w, const float* bias, const uint16_t* x,
+                               int T, float* logits, int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_dequant_rows(int bits, int block, const uint8_t* codes, const uint16_t* scales,
                                 int row0, int rows, int cols, float* out, cudaStream_t s);
 bool decode_shape_supported(int bits, int H, int I);

@@ -359,6 +359,13 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
       for (int n0 = 0; n0 < ti.nvalid; n0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
+        // per-column factor, loaded once by lane c and broadcast by shuffle:
+        // gate/up the token row's inverse scale, down the gate weight
+        float colf = 1.f;
+        if (lane < 16 && n0 + lane < ti.nvalid) {
+          const int pc = prow + n0 + lane;
+          colf = MODE == 0 ? __ldg(a.xinv + pc) : (sh ? 1.f : __ldg(rv.topk_w + __ldg(rv.pairs + pc)));
+        }
         if (MODE == 0) {
           // rows alternate gate / up: lane pairs (2i, 2i+1) hold g and u of row pair i
           const int i = R >> 1;
@@ -366,24 +373,19 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
           const int ip = (i & ~(G - 1)) | decode_slot(BITS, i & (G - 1));
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
+            const float xi = __shfl_sync(0xffffffffu, colf, c);
             const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[c]), 1);
             if (((lane & 1) == 0) && n0 + c < ti.nvalid) {
-              const int p = prow + n0 + c;
-              const float xi = __ldg(a.xinv + p);
               const float g = __uint_as_float(v[c]) * xi, u = other * xi;
               const float hval = g / (1.f + expf(-g)) * u;
-              a.hout[size_t(p) * a.out_cols + ip] = __half_as_ushort(__float2half_rn(hval));
+              a.hout[size_t(prow + n0 + c) * a.out_cols + ip] = __half_as_ushort(__float2half_rn(hval));
             }
           }
         } else {
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const int n = n0 + c;
-            if (n < ti.nvalid) {
-              const int p = prow + n;
-              const float w = sh ? 1.f : __ldg(rv.topk_w + __ldg(rv.pairs + p));
-              a.yout[size_t(p) * a.out_cols + R] = __uint_as_float(v[c]) * w;
-            }
+            const float w = __shfl_sync(0xffffffffu, colf, c);
+            if (n0 + c < ti.nvalid) a.yout[size_t(prow + n0 + c) * a.out_cols + R] = __uint_as_float(v[c]) * w;
           }
         }
       }
@@ -458,6 +460,129 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
   }
 }
 
+// Router logits of a large batch on the tensor cores:
+//   logits[t][e] = sum_h x[t][h] Wr[e][h] (+ b[e])
+// D[128 experts x N tokens] in TMEM from bf16 A = router rows and B = token
+// rows (both by TMA, SWIZZLE_128B), fp32 accumulation; bf16 x bf16 products
+// are exact in fp32.  Warp 0: TMA; warp 1: TMEM + MMA; warps 2-5: epilogue.
+constexpr int kRWarps = 6;
+constexpr int kRStages = 4;
+
+__global__ void __launch_bounds__(kRWarps * 32, 1) router_gemm_kernel(
+    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x, const float* __restrict__ bias,
+    int T, int E, int H, float* __restrict__ logits, int* status) {
+  extern __shared__ __align__(1024) unsigned char rsm_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(rsm_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sA = base;                                  // kRStages x 16 KB
+  unsigned char* sB = sA + kRStages * kAStageBytes;          // kRStages x 16 KB
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kRStages * kBStageBytes);
+  uint64_t* empty = full + kRStages;
+  uint64_t* acc_full = empty + kRStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int mt = E / PBM, ntn = (T + PBN - 1) / PBN, ntiles = mt * ntn, KB = H / PBK;
+
+  if (warp == 0 && lane == 0) {
+    int kc = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      const int m = t % mt, n = t / mt;
+      for (int kb = 0; kb < KB; ++kb, ++kc) {
+        const int s = kc % kRStages;
+        if (kc >= kRStages && !mbar_wait(&empty[s], ((kc / kRStages) - 1) & 1, abort_flag)) {
+          *abort_flag = 1; report_error(status, MOE_ERR_TIMEOUT, 30); break;
+        }
+        mbar_arrive_expect_tx(&full[s], kAStageBytes + kBStageBytes);
+        tma_load_2d(sA + s * kAStageBytes, &tm_w, kb * PBK, m * PBM, &full[s]);
+        tma_load_2d(sB + s * kBStageBytes, &tm_x, kb * PBK, n * PBN, &full[s]);
+      }
+    }
+    for (int i = max(0, kc - kRStages); i < kc; ++i)
+      if (!mbar_wait(&full[i % kRStages], (i / kRStages) & 1, nullptr)) report_error(status, MOE_ERR_TIMEOUT, 31);
+  } else if (warp == 1 && lane == 0) {
+    int kc = 0, tc = 0;
+    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x, ++tc) {
+      const int n = t / mt;
+      const int buf = tc & 1;
+      if (tc >= 2 && !mbar_wait(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag)) {
+        *abort_flag = 1; report_error(status, MOE_ERR_TIMEOUT, 32); break;
+      }
+      tc_fence_after();
+      const int nvalid = min(PBN, T - n * PBN);
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(((nvalid + 15) & ~15) >> 3) << 17) |
+                             (uint32_t(PBM >> 4) << 24);   // D fp32, A/B bf16, K-major
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++kc) {
+        const int s = kc % kRStages;
+        if (!mbar_wait(&full[s], (kc / kRStages) & 1, abort_flag)) {
+          *abort_flag = 1; report_error(status, MOE_ERR_TIMEOUT, 33); ok = false; break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kAStageBytes), b0 = smem_u32(sB + s * kBStageBytes);
+#pragma unroll
+        for (int k = 0; k < PBK / 16; ++k)
+          tc_mma(tmem_base + uint32_t(buf * PBN), sw128_desc(a0 + k * 32), sw128_desc(b0 + k * 32), idesc,
+                 (kb | k) ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      if (!ok) break;
+      tc_commit(&acc_full[buf]);
+    }
+    if (kc > 0 && !mbar_wait(&empty[(kc - 1) % kRStages], ((kc - 1) / kRStages) & 1, nullptr))
+      report_error(status, MOE_ERR_TIMEOUT, 34);
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int tc = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+      const int m = t % mt, n = t / mt;
+      const int buf = tc & 1;
+      if (*abort_flag || !mbar_wait(&acc_full[buf], (tc >> 1) & 1, abort_flag)) {
+        if (!*abort_flag) { *abort_flag = 1; report_error(status, MOE_ERR_TIMEOUT, 35); }
+        break;
+      }
+      tc_fence_after();
+      const int e = m * PBM + r;
+      const float b = bias ? __ldg(bias + e) : 0.f;
+      const int nvalid = min(PBN, T - n * PBN);
+      for (int n0 = 0; n0 < nvalid; n0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if (n0 + c < nvalid) logits[size_t(n * PBN + n0 + c) * E + e] = __uint_as_float(v[c]) + b;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ host
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -513,6 +638,26 @@ cudaError_t launch_gemm(const PrefillArgs& pa, const uint8_t* codes, const uint1
 }
 
 }  // namespace
+
+bool router_gemm_supported(const moe_config& c, int T) {
+  return T > 64 && c.num_experts % PBM == 0 && c.hidden % PBK == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_router_gemm(const moe_config& c, const uint16_t* router_w, const float* bias, const uint16_t* x,
+                               int T, float* logits, int* status, int num_sms, cudaStream_t s) {
+  CUtensorMap mw, mx;
+  if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, router_w, uint64_t(c.hidden), uint64_t(c.num_experts), PBK,
+                PBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, uint64_t(c.hidden), uint64_t(T), PBK, PBN,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const size_t smem = 1024 + kRStages * (kAStageBytes + kBStageBytes) + 256;
+  cudaError_t err = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const int tiles = (c.num_experts / PBM) * ((T + PBN - 1) / PBN);
+  return launch_pdl(router_gemm_kernel, dim3(min(num_sms, tiles)), dim3(kRWarps * 32), smem, s, mw, mx, bias, T,
+                    c.num_experts, c.hidden, logits, status);
+}
 
 bool prefill_supported(const moe_config& c) {
   const int H = c.hidden, I = c.inter;

@@ -421,7 +421,15 @@ cudaError_t launch_topk_group_any(const moe_config& c, int T, char* ws, const La
 cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
                               const uint16_t* x, int T, char* ws, const Layout& L, int* api_counts,
                               int* api_offsets, int* api_pairs, cudaStream_t s) {
-  cudaError_t err = launch_router_logits(c, router_w, bias, x, T, reinterpret_cast<float*>(ws + L.logits), s);
+  int nsm = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  }
+  cudaError_t err = router_gemm_supported(c, T)
+      ? launch_router_gemm(c, router_w, bias, x, T, reinterpret_cast<float*>(ws + L.logits),
+                           reinterpret_cast<int*>(ws + L.status), nsm, s)
+      : launch_router_logits(c, router_w, bias, x, T, reinterpret_cast<float*>(ws + L.logits), s);
   if (err != cudaSuccess) return err;
   const bool fused = T <= 64;
   return launch_topk_group_any(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
