@@ -161,6 +161,11 @@ int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t
 int moe_profile_begin(int32_t max_calls);
 int moe_profile_end(float* ms_out, int32_t* calls);
 
+/* Measurement hook: while device_buf is non-null, fused decode launches write
+ * %globaltimer stamps of each CTA's phase boundaries in their first layer to
+ * device_buf[cta][9] (the caller owns the buffer; null switches it off). */
+void moe_debug_fused_timing(unsigned long long* device_buf);
+
 /* The cudaError_t value behind the calling thread's most recent
  * MOE_ERR_CUDA (0 if none). */
 int moe_last_cuda_error(void);

@@ -274,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += NTB) {
         const int nt = min(NTB, nc - tb);          // warp-uniform
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos);
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 1);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 2);
         else rows_dot<MODE, BITS, LPR, CPL, 4>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
       }
     }

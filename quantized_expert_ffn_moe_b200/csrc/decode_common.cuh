@@ -61,9 +61,19 @@ struct Rows {
 template <int MODE, int BITS, int LPR, int CPL, int NT>
 __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& rw, const __half* xs, int tb, int lr,
                                          const float* tok_inv, const float* tok_w, const int* tok_pos,
-                                         int nt = NT) {
+                                         int nt = NT, const int* xrow = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
+  // staged activation row of each token of the block: consecutive rows after
+  // xs, or the rows listed in xrow (activations staged once per token).  Token
+  // slots past nt repeat the first token, so the inner loops run branch-free
+  // and only the epilogue skips them.
+  int xr0[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int tt = t < nt ? t : 0;
+    xr0[t] = (xrow ? xrow[tb + tt] : tt) * K;
+  }
   float acc[2][NT];
 #pragma unroll
   for (int rho = 0; rho < 2; ++rho)
@@ -90,11 +100,10 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
         __half2 q[2][4];
         decode_q4x8(wd[0][m], q[0]);
         decode_q4x8(wd[1][m], q[1]);
-        const __half* xcol = xs + ((s * 4 + m) * LPR + lr) * 8;
+        const int xoff = ((s * 4 + m) * LPR + lr) * 8;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          if (NT == 4 && t >= nt) continue;
-          const uint4 xv = *reinterpret_cast<const uint4*>(xcol + size_t(t) * K);
+          const uint4 xv = *reinterpret_cast<const uint4*>(xs + xr0[t] + xoff);
           const __half2 x2[4] = {u32_as_h2(xv.x), u32_as_h2(xv.y), u32_as_h2(xv.z), u32_as_h2(xv.w)};
 #pragma unroll
           for (int rho = 0; rho < 2; ++rho)
@@ -106,7 +115,6 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
       for (int rho = 0; rho < 2; ++rho)
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          if (NT == 4 && t >= nt) continue;
           const float2 f = __half22float2(__hadd2(hacc[rho][t][0], hacc[rho][t][1]));
           acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
         }
@@ -119,7 +127,7 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
         __half2 q[2][8];
         decode_q2x16(wd[0][m], q[0]);
         decode_q2x16(wd[1][m], q[1]);
-        const __half* xcol = xs + ((s * 4 + m) * 2 * LPR + lr) * 8;
+        const int xoff = ((s * 4 + m) * 2 * LPR + lr) * 8;
         float sc[2];
 #pragma unroll
         for (int rho = 0; rho < 2; ++rho) {
@@ -128,8 +136,7 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          if (NT == 4 && t >= nt) continue;
-          const __half* xr = xcol + size_t(t) * K;
+          const __half* xr = xs + xr0[t] + xoff;
           const uint4 xa = *reinterpret_cast<const uint4*>(xr);
           const uint4 xb = *reinterpret_cast<const uint4*>(xr + LPR * 8);
           const __half2 x2[8] = {u32_as_h2(xa.x), u32_as_h2(xa.y), u32_as_h2(xa.z), u32_as_h2(xa.w),
@@ -152,7 +159,6 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
   // reduce across the LPR lanes of each row
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    if (NT == 4 && t >= nt) continue;
 #pragma unroll
     for (int rho = 0; rho < 2; ++rho)
 #pragma unroll

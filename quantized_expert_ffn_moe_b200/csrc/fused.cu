@@ -35,6 +35,7 @@ constexpr int kFStages = 3;
 constexpr int kFMaxTokens = 64;
 constexpr int kFMaxPairs = kFMaxTokens * 16;
 constexpr int kMaxFusedLayers = 64;
+constexpr int kTimePoints = 9;
 
 struct FusedParams {
   moe_config cfg;
@@ -43,6 +44,7 @@ struct FusedParams {
   const uint16_t* x;             // layer mode input
   uint16_t* y;                   // layer mode output, or the residual stream (stack)
   int* trace;                    // stack: [L][T][k] selections, or null
+  unsigned long long* timing;    // null, or [gridDim][9] %globaltimer stamps of layer 0
   char* ws;
   Layout L_;
   int ntc_gu, ntc_dn;
@@ -52,6 +54,12 @@ struct FusedParams {
 
 // ------------------------------------------------------------ grid barrier
 // One thread per CTA.  Returns false when the wait gave up.
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 __device__ bool grid_barrier(unsigned* count, unsigned* gen, unsigned nblocks, unsigned* passed, int* status) {
   __threadfence();
   const unsigned target = *passed + 1;
@@ -61,9 +69,8 @@ __device__ bool grid_barrier(unsigned* count, unsigned* gen, unsigned nblocks, u
     atomicAdd(gen, 1u);
   } else {
     const unsigned long long t0 = global_ns();
-    while (true) {
-      const unsigned g = *reinterpret_cast<volatile unsigned*>(gen);
-      if (int(g - target) >= 0) break;
+    while (int(ld_acquire_u32(gen) - target) < 0) {
+      __nanosleep(64);
       if (global_ns() - t0 > kWaitLimitNs) {
         report_error(status, MOE_ERR_TIMEOUT, 40);
         return false;
@@ -140,46 +147,6 @@ struct FCursor {
   __device__ bool valid(long long w1) const { return slot < nslots && pos < w1; }
   __device__ void advance() { pos += stage_cost(nc); if (++stage == spe) next_chunk(); }
 };
-
-// Warp-per-token top-k of one token's logits (global, written by other CTAs:
-// read around L1).
-template <int NPL>
-__device__ void warp_topk_g(const float* lrow, int k, int E, int* idx_out, float* w_out) {
-  const int lane = threadIdx.x & 31;
-  float v[NPL];
-#pragma unroll
-  for (int m = 0; m < NPL; ++m) {
-    const int e = lane + 32 * m;
-    v[m] = e < E ? __ldcg(lrow + e) : -INFINITY;
-  }
-  uint32_t taken = 0;
-  float my_logit = -INFINITY;
-  int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int m = 0; m < NPL; ++m) {
-      const int e = lane + 32 * m;
-      const bool ok = !((taken >> m) & 1u) && e < E;
-      if (ok && (v[m] > bv || (v[m] == bv && e < be))) { bv = v[m]; be = e; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
-    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == j) { my_logit = bv; my_idx = be; }
-  }
-  const float top = __shfl_sync(0xffffffffu, my_logit, 0);
-  float ex = lane < k ? expf(my_logit - top) : 0.f;
-  float sum = ex;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < k) { idx_out[lane] = my_idx; w_out[lane] = ex / sum; }
-}
 
 __device__ __forceinline__ float round_bf16f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
@@ -262,25 +229,182 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
   }
 }
 
+// Stages token t once for the whole layer: one L2 round trip for the row
+// (each lane holds whole groups of G elements), RMSNorm factor (stack),
+// xhat = bf16(x * r), and the power-of-two scale that puts max |xhat| in
+// [128, 256); stored as fp16 in the gate/up operand order.
+template <int BITS, int LPR, int CPL>
+__device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, float* rnorm_out, float* inv_out,
+                                int lane) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);       // groups per lane
+  uint4 v[NG][G / 8];
+#pragma unroll
+  for (int q = 0; q < NG; ++q)
+#pragma unroll
+    for (int z = 0; z < G / 8; ++z)
+      v[q][z] = __ldcg(reinterpret_cast<const uint4*>(row + (q * 32 + lane) * G + 8 * z));
+  float r = 1.f;
+  if (stack) {
+    float ss = 0.f;
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+#pragma unroll
+      for (int z = 0; z < G / 8; ++z) {
+        const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const float a = __uint_as_float(w[y] << 16), b = __uint_as_float(w[y] & 0xFFFF0000u);
+          ss = fmaf(a, a, ss);
+          ss = fmaf(b, b, ss);
+        }
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    r = 1.0f / sqrtf(ss / float(K) + 1e-6f);
+  }
+  float vmax = 0.f;
+#pragma unroll
+  for (int q = 0; q < NG; ++q)
+#pragma unroll
+    for (int z = 0; z < G / 8; ++z) {
+      const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(w[y] << 16) * r)));
+        vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r)));
+      }
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  int sh = 0;
+  if (vmax > 0.f) {
+    int ex;
+    frexpf(vmax, &ex);
+    sh = min(max(8 - ex, -100), 100);
+  }
+  const float mul = ldexpf(1.f, sh);
+#pragma unroll
+  for (int q = 0; q < NG; ++q) {
+    __align__(16) __half hv[G];
+#pragma unroll
+    for (int z = 0; z < G / 8; ++z) {
+      const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int j = 8 * z + 2 * y;
+        hv[decode_slot(BITS, j)] = __float2half_rn(round_bf16f(__uint_as_float(w[y] << 16) * r) * mul);
+        hv[decode_slot(BITS, j + 1)] = __float2half_rn(round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r) * mul);
+      }
+    }
+    const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
+#pragma unroll
+    for (int part = 0; part < Gm::NPART; ++part)
+      *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+  }
+  if (lane == 0) {
+    *rnorm_out = r;
+    *inv_out = ldexpf(1.f, -sh);
+  }
+}
+
+// Router logits of expert e for all T tokens from the staged activations:
+// sum_j Wr[e][g0+j] * xs[slot(j)] (exact products), times the token's 2^-sh.
+template <int BITS, int LPR, int CPL>
+__device__ void router_from_staged(const uint16_t* wrow, float bias, const __half* xs, const float* inv_all, int T,
+                                   float* logit_col, int E, int lane) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);
+  uint4 wv[NG][G / 8];
+#pragma unroll
+  for (int q = 0; q < NG; ++q)
+#pragma unroll
+    for (int z = 0; z < G / 8; ++z) wv[q][z] = ld_stream16(wrow + (q * 32 + lane) * G + 8 * z);
+  for (int t = 0; t < T; ++t) {
+    const __half* xt = xs + size_t(t) * K;
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < NG; ++q) {
+      const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
+      __align__(16) __half xv[G];
+#pragma unroll
+      for (int part = 0; part < Gm::NPART; ++part)
+        *reinterpret_cast<uint4*>(xv + 8 * part) = *reinterpret_cast<const uint4*>(xt + base + part * LPR * 8);
+#pragma unroll
+      for (int z = 0; z < G / 8; ++z) {
+        const uint32_t w[4] = {wv[q][z].x, wv[q][z].y, wv[q][z].z, wv[q][z].w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const int j = 8 * z + 2 * y;
+          acc = fmaf(__uint_as_float(w[y] << 16), __half2float(xv[decode_slot(BITS, j)]), acc);
+          acc = fmaf(__uint_as_float(w[y] & 0xFFFF0000u), __half2float(xv[decode_slot(BITS, j + 1)]), acc);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) logit_col[size_t(t) * E] = acc * inv_all[t] + bias;
+  }
+}
+
+// Exclusive scan of one value per consumer thread (256 threads); also
+// returns the total.  Uses 8 ints of shared scratch.
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += n;
+  }
+  if (lane == 31) scratch[warp] = x;
+  named_bar_sync(1, kNCW * 32);
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kNCW; ++w) {
+    const int s = scratch[w];
+    if (w < warp) before += s;
+    all += s;
+  }
+  named_bar_sync(1, kNCW * 32);
+  *total = all;
+  return before + x - v;
+}
+
 // Consumer side of one pass over this CTA's stages.
 template <int MODE, int BITS, int LPR, int CPL>
 __device__ void consume_pass(const FusedParams& p, const SRoute& rt, const moe_layer_weights& lw, FCursor cur,
                              long long w1, unsigned char* ring, int ring_stride, uint64_t* full, uint64_t* empty,
                              int* consumed, const uint16_t* xsrc, const float* rnorm, const float* hin, float* out,
                              int out_cols, __half* xs, float* tok_inv, float* tok_w, int* tok_pos,
-                             volatile int* abort_flag, int* status) {
+                             volatile int* abort_flag, int* status, const float* inv_all = nullptr,
+                             int* tok_xrow = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane / LPR, lr = lane % LPR;
   const int rl0 = (warp * Gm::RW + grp) * 2;
+  const bool pre = inv_all != nullptr;      // every token already staged (gate/up)
   bool first = true;
   for (; cur.valid(w1); cur.advance()) {
     const int i = (*consumed)++;
     if (first || cur.stage == 0) {
       first = false;
       named_bar_sync(1, kNCW * 32);
-      stage_chunk<MODE, BITS, LPR, CPL>(p, rt, cur, xsrc, rnorm, hin, xs, tok_inv, tok_w, tok_pos, warp, lane);
+      if (pre) {
+        const int tbase = cur.chunk * cur.ntc;
+        const bool is_shared = cur.e >= p.cfg.num_experts;
+        for (int tl = threadIdx.x; tl < cur.nc; tl += kNCW * 32) {
+          const int pos = cur.p0 + tbase + tl;
+          const int tok = is_shared ? pos - p.T * p.cfg.top_k : rt.pairs[pos] / p.cfg.top_k;
+          tok_pos[tl] = pos;
+          tok_xrow[tl] = tok;
+          tok_inv[tl] = inv_all[tok];
+          tok_w[tl] = 1.f;
+        }
+      } else {
+        stage_chunk<MODE, BITS, LPR, CPL>(p, rt, cur, xsrc, rnorm, hin, xs, tok_inv, tok_w, tok_pos, warp, lane);
+      }
       named_bar_sync(1, kNCW * 32);
     }
     const int slot = i % kFStages;
@@ -297,9 +421,11 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, const moe_l
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
         const int nt = min(4, nc - tb);
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(out, out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(out, out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos);
-        else rows_dot<MODE, BITS, LPR, CPL, 4>(out, out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
+        const __half* xb = pre ? xs : xs + size_t(tb) * K;
+        const int* xr = pre ? tok_xrow : nullptr;
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(out, out_cols, rows, xb, tb, lr, tok_inv, tok_w, tok_pos, 1, xr);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(out, out_cols, rows, xb, tb, lr, tok_inv, tok_w, tok_pos, 2, xr);
+        else rows_dot<MODE, BITS, LPR, CPL, 4>(out, out_cols, rows, xb, tb, lr, tok_inv, tok_w, tok_pos, nt, xr);
       }
     }
     __syncwarp();
@@ -349,7 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kFStages);
   float* rnorm = reinterpret_cast<float*>(smem + 64);                    // [64]
   int* snslots = reinterpret_cast<int*>(smem + 320);
-  unsigned char* ring = smem + 512;
+  float* inv_all = reinterpret_cast<float*>(smem + 384);                 // [64]
+  int* tok_xrow = reinterpret_cast<int*>(smem + 640);                    // [64]
+  int* scan_scratch = reinterpret_cast<int*>(smem + 896);                // [8]
+  unsigned char* ring = smem + 1024;
   int* ri = reinterpret_cast<int*>(smem + p.smem_route_off);
   SRoute rt;
   rt.idx = ri;
@@ -389,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
 
   for (int l = 0; l < p.L; ++l) {
     const moe_layer_weights& lw = p.w[l];
+    if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 8] = global_ns();
     // ------------------------------------------------------------ phase R
     if (producer) {
       if (lane == 0 && S) {
@@ -400,24 +530,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
         if (b1 > b0) bulk_prefetch_l2(lw.shared_down_codes + b0, uint32_t(b1 - b0));
       }
     } else {
-      // RMSNorm factors (stack) of all tokens, identical in every CTA
-      for (int t = warp; t < T; t += kNCW) {
-        float ss = 0.f;
-        if (p.stack) {
-          for (int hh = lane * 8; hh < H; hh += 256) {
-            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(t) * H + hh));
-            const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+      // tokens: RMSNorm factors (stack), identical in every CTA; when all T
+      // fit, each token is staged once here for the router and gate/up
+      const bool xall = p.ntc_gu >= T;
+      if (xall) {
+        for (int t = warp; t < T; t += kNCW)
+          stage_token_all<BITS, LG, CG>(xsrc + size_t(t) * H, p.stack != 0, xs + size_t(t) * H, &rnorm[t],
+                                        &inv_all[t], lane);
+      } else {
+        for (int t = warp; t < T; t += kNCW) {
+          float ss = 0.f;
+          if (p.stack) {
+            for (int hh = lane * 8; hh < H; hh += 256) {
+              const uint4 v = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(t) * H + hh));
+              const uint32_t q[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              const float a = __uint_as_float(q[z] << 16), b = __uint_as_float(q[z] & 0xFFFF0000u);
-              ss = fmaf(a, a, ss);
-              ss = fmaf(b, b, ss);
+              for (int z = 0; z < 4; ++z) {
+                const float a = __uint_as_float(q[z] << 16), b = __uint_as_float(q[z] & 0xFFFF0000u);
+                ss = fmaf(a, a, ss);
+                ss = fmaf(b, b, ss);
+              }
             }
-          }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          }
+          if (lane == 0) rnorm[t] = p.stack ? 1.0f / sqrtf(ss / float(H) + 1e-6f) : 1.f;
         }
-        if (lane == 0) rnorm[t] = p.stack ? 1.0f / sqrtf(ss / float(H) + 1e-6f) : 1.f;
       }
       named_bar_sync(1, kNCW * 32);
       // router logits of this CTA's experts: one warp per expert row
@@ -425,6 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
       for (int e = e0 + warp; e < e1; e += kNCW) {
         const uint16_t* wr = lw.router_w + size_t(e) * H;
         const float b = lw.router_bias ? lw.router_bias[e] : 0.f;
+        if (xall) {
+          router_from_staged<BITS, LG, CG>(wr, b, xs, inv_all, T, logits + e, E, lane);
+          continue;
+        }
         constexpr int RPL = 2048 / 256;      // 16-byte pieces of the row per lane (H = 2048)
         uint4 wv[RPL];
 #pragma unroll
@@ -449,87 +591,105 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
         }
       }
       named_bar_sync(1, kNCW * 32);
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 0] = global_ns();
       if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
       named_bar_sync(1, kNCW * 32);
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 1] = global_ns();
       // ---------------------------------------------------------- phase S
-      for (int t = warp; t < T; t += kNCW) warp_topk_g<NPL>(logits + size_t(t) * E, k, E, rt.idx + t * k, rt.w + t * k);
       for (int e = threadIdx.x; e < E; e += kNCW * 32) rt.cnt[e] = 0;
+      for (int t = warp; t < T; t += kNCW) warp_topk_fast<NPL, true>(logits + size_t(t) * E, k, E, rt.idx + t * k, rt.w + t * k);
       named_bar_sync(1, kNCW * 32);
       for (int q = threadIdx.x; q < T * k; q += kNCW * 32) atomicAdd(&rt.cnt[rt.idx[q]], 1);
       named_bar_sync(1, kNCW * 32);
-      if (warp == 0) {
-        // exclusive scan of counts and the touched-expert list
-        int run = 0, urun = 0;
-        for (int base = 0; base < E; base += 32) {
-          const int e = base + lane;
+      {
+        // exclusive scan of the counts and the ascending touched-expert list;
+        // cnt becomes each expert's fill cursor
+        const int EPT = (E + kNCW * 32 - 1) / (kNCW * 32);      // experts per thread (<= 4)
+        const int eb = threadIdx.x * EPT;
+        int csum = 0, fsum = 0;
+        for (int z = 0; z < EPT; ++z) {
+          const int e = eb + z;
           const int cc = e < E ? rt.cnt[e] : 0;
-          int v = cc, f = cc > 0 ? 1 : 0;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int nv = __shfl_up_sync(0xffffffffu, v, o), nf = __shfl_up_sync(0xffffffffu, f, o);
-            if (lane >= o) { v += nv; f += nf; }
-          }
+          csum += cc;
+          fsum += cc > 0 ? 1 : 0;
+        }
+        int ctot, ftot;
+        int crun = block_excl_scan(csum, scan_scratch, &ctot);
+        int frun = block_excl_scan(fsum, scan_scratch, &ftot);
+        for (int z = 0; z < EPT; ++z) {
+          const int e = eb + z;
           if (e < E) {
-            rt.offsets[e] = run + v - cc;
-            if (cc > 0) rt.ulist[urun + f - 1] = e;
+            const int cc = rt.cnt[e];
+            rt.offsets[e] = crun;
+            rt.cnt[e] = crun;
+            crun += cc;
+            if (cc > 0) rt.ulist[frun++] = e;
           }
-          run += __shfl_sync(0xffffffffu, v, 31);
-          urun += __shfl_sync(0xffffffffu, f, 31);
         }
-        if (lane == 0) {
-          rt.offsets[E] = run;
-          if (S) rt.ulist[urun] = E;
-          *snslots = urun + S;
+        if (threadIdx.x == 0) {
+          rt.offsets[E] = ctot;
+          if (S) rt.ulist[ftot] = E;
+          *snslots = ftot + S;
         }
-        __syncwarp();
-        // stable positions: tokens in order, slots of one token in parallel
-        for (int e = lane; e < E; e += 32) rt.cnt[e] = rt.offsets[e];
-        __syncwarp();
-        for (int t = 0; t < T; ++t) {
-          if (lane < k) {
-            const int q = t * k + lane;
-            const int e = rt.idx[q];
-            const int pos = rt.cnt[e]++;
+      }
+      named_bar_sync(1, kNCW * 32);
+      // stable positions inside each expert's list (pairs in token order), by
+      // warp 0 over 32 pairs at a time: every CTA derives the same positions,
+      // which the passes of different CTAs rely on.  Meanwhile the
+      // cost-weighted work prefix of the slots for the two passes.
+      if (warp == 0) {
+        for (int base = 0; base < T * k; base += 32) {
+          const int q = base + lane;
+          const int e = q < T * k ? rt.idx[q] : -1 - lane;
+          const unsigned same = __match_any_sync(0xffffffffu, e);
+          const int rank = __popc(same & ((1u << lane) - 1u));
+          const int start = q < T * k ? rt.cnt[e] : 0;
+          __syncwarp();
+          if (q < T * k) {
+            const int pos = start + rank;
             rt.pairs[pos] = q;
             rt.inv[q] = pos;
+            if ((same >> lane) == 1u) rt.cnt[e] = start + rank + 1;     // last of its expert in this group
           }
           __syncwarp();
         }
-      } else if (warp == 1 && p.trace) {
-        // selections of this layer (CTA 0 only)
-        if (blockIdx.x == 0) for (int q = lane; q < T * k; q += 32) p.trace[size_t(l) * T * k + q] = rt.idx[q];
+      } else if (warp == 1 && p.trace && blockIdx.x == 0) {
+        for (int q = lane; q < T * k; q += 32) p.trace[size_t(l) * T * k + q] = rt.idx[q];
       }
-      named_bar_sync(1, kNCW * 32);
-      if (warp == 0) {
+      {
         const PassPlan pg{p.ntc_gu, 2 * I / GU::RPS}, pd{p.ntc_dn, H / DN::RPS};
-        int rg = 0, rd = 0;
         const int ns = *snslots;
-        for (int base = 0; base < ns; base += 32) {
-          const int u = base + lane;
-          int n = 0;
+        const int SPT = (ns + kNCW * 32 - 1) / (kNCW * 32);     // slots per thread
+        const int u0 = threadIdx.x * SPT;
+        int g = 0, d = 0;
+        for (int z = 0; z < SPT; ++z) {
+          const int u = u0 + z;
           if (u < ns) {
             const int e = rt.ulist[u];
-            n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+            const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+            g += pass_cost(pg, n);
+            d += pass_cost(pd, n);
           }
-          auto cost = [&](const PassPlan& pp) {
-            if (u >= ns) return 0;
-            const int fl = n / pp.ntc, rest = n % pp.ntc;
-            return pp.spe * (fl * stage_cost(pp.ntc) + (rest ? stage_cost(rest) : 0));
-          };
-          int g = cost(pg), d = cost(pd);
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int ng = __shfl_up_sync(0xffffffffu, g, o), nd = __shfl_up_sync(0xffffffffu, d, o);
-            if (lane >= o) { g += ng; d += nd; }
-          }
-          if (u < ns) { rt.woff_gu[u + 1] = rg + g; rt.woff_dn[u + 1] = rd + d; }
-          rg += __shfl_sync(0xffffffffu, g, 31);
-          rd += __shfl_sync(0xffffffffu, d, 31);
         }
-        if (lane == 0) { rt.woff_gu[0] = 0; rt.woff_dn[0] = 0; }
+        int gt, dt;
+        int grun = block_excl_scan(g, scan_scratch, &gt);
+        int drun = block_excl_scan(d, scan_scratch, &dt);
+        for (int z = 0; z < SPT; ++z) {
+          const int u = u0 + z;
+          if (u < ns) {
+            const int e = rt.ulist[u];
+            const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+            rt.woff_gu[u] = grun;
+            rt.woff_dn[u] = drun;
+            grun += pass_cost(pg, n);
+            drun += pass_cost(pd, n);
+          }
+        }
+        if (threadIdx.x == 0) { rt.woff_gu[ns] = gt; rt.woff_dn[ns] = dt; }
       }
     }
     __syncthreads();                 // routing of this layer ready for all warps
+    if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 2] = global_ns();
 
     const int ns = *snslots;
     FCursor cg{};
@@ -562,12 +722,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
       // ---------------------------------------------------------- phase G
       if (g0 < g1) {
         cg.init(g0);
+        const bool xall = p.ntc_gu >= T;
         consume_pass<GATEUP, BITS, LG, CG>(p, rt, lw, cg, g1, ring, RING_STRIDE, full, empty, &consumed, xsrc,
-                                           rnorm, nullptr, hbuf, I, xs, tok_inv, tok_w, tok_pos, abort_flag, status);
+                                           rnorm, nullptr, hbuf, I, xs, tok_inv, tok_w, tok_pos, abort_flag, status,
+                                           xall ? inv_all : nullptr, tok_xrow);
       }
       named_bar_sync(1, kNCW * 32);
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 3] = global_ns();
       if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
       named_bar_sync(1, kNCW * 32);
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 4] = global_ns();
       // ---------------------------------------------------------- phase D
       if (d0 < d1) {
         cd.init(d0);
@@ -575,8 +739,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
                                          rnorm, hbuf, ybuf, H, xs, tok_inv, tok_w, tok_pos, abort_flag, status);
       }
       named_bar_sync(1, kNCW * 32);
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 5] = global_ns();
       if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
       named_bar_sync(1, kNCW * 32);
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 6] = global_ns();
       // ---------------------------------------------------------- phase C
       const int units = T * (H / 8);
       const int u0 = int((long long)units * blockIdx.x / G), u1 = int((long long)units * (blockIdx.x + 1) / G);
@@ -612,6 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
         for (int z = 0; z < 8; ++z) ob[z] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[z]));
         *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob);
       }
+      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 7] = global_ns();
       if (p.stack && l + 1 < p.L) {
         named_bar_sync(1, kNCW * 32);
         if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
@@ -631,7 +798,7 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   constexpr int RING_STRIDE = GU::STAGE_BYTES > DN::STAGE_BYTES ? GU::STAGE_BYTES : DN::STAGE_BYTES;
   const int E = p.cfg.num_experts;
   const int route_bytes = (4 * kFMaxPairs + 2 * (E + 1) + 2 * (E + 2) + E) * 4;
-  q.smem_route_off = 512 + kFStages * RING_STRIDE;
+  q.smem_route_off = 1024 + kFStages * RING_STRIDE;
   q.smem_tok_off = q.smem_route_off + ((route_bytes + 127) & ~127);
   q.smem_xs_off = q.smem_tok_off + kMaxNTC * 12 + 128;
   q.smem_xs_off = (q.smem_xs_off + 127) & ~127;
@@ -658,6 +825,10 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
 
 }  // namespace
 
+unsigned long long* g_fused_timing = nullptr;
+
+void set_fused_timing(unsigned long long* buf) { g_fused_timing = buf; }
+
 bool fused_supported(const moe_config& c, int T) {
   if (T < 1 || T > kFMaxTokens || T * c.top_k > kFMaxPairs) return false;
   return c.hidden == 2048 && c.inter == 768 && (c.num_experts % 32) == 0 && c.num_experts <= 1024;
@@ -675,6 +846,7 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
     p.x = x;
     p.y = y;
     p.trace = trace ? trace + size_t(l0) * T * c.top_k : nullptr;
+    p.timing = l0 == 0 ? g_fused_timing : nullptr;
     p.ws = ws;
     p.L_ = Lw;
     for (int l = 0; l < p.L; ++l) p.w[l] = layers[l0 + l];

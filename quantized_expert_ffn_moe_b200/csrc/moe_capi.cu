@@ -278,6 +278,8 @@ int moe_profile_end(float* ms_out, int32_t* calls) {
 
 int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
+void moe_debug_fused_timing(unsigned long long* device_buf) { set_fused_timing(device_buf); }
+
 const char* moe_status_str(int status) {
   switch (status) {
     case MOE_OK: return "ok";

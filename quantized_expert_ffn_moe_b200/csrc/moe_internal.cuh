@@ -20,14 +20,17 @@ enum StatusSlot {
   ST_ERROR = 0,      // first failed device check (0 = none)
   ST_ERROR_AUX = 1,  // detail of that check
   ST_UCOUNT = 2,     // number of distinct routed experts selected
-  ST_GRID_COUNT = 4, // fused decode: grid barrier arrivals
-  ST_GRID_GEN = 5,   // fused decode: grid barrier generation
-  ST_COUNT = 16
+  ST_GRID_COUNT = 32,  // fused decode: grid barrier arrivals (own 128-byte line)
+  ST_GRID_GEN = 64,    // fused decode: grid barrier generation (own 128-byte line)
+  ST_COUNT = 96
 };
+
+// Tokens per chunk of the parallel grouping used for large batches.
+constexpr int kGroupChunk = 64;
 
 struct Layout {
   size_t status, logits, topk_idx, topk_w, counts, offsets, pairs, inv, ulist, woff_gu, woff_dn, ntoff, xhat, h,
-      y, xs, xscale, total;
+      y, xs, xscale, chunk_hist, total;
   int P;
 };
 
@@ -56,6 +59,7 @@ inline Layout make_layout(const moe_config& c, int T) {
   L.y = take(size_t(P) * c.hidden * 4);
   L.xs = take(size_t(P) * c.hidden * 2);
   L.xscale = take(size_t(P) * 4);
+  L.chunk_hist = take(size_t((T + kGroupChunk - 1) / kGroupChunk) * c.num_experts * 4);
   L.total = o;
   L.P = P;
   return L;
@@ -96,11 +100,20 @@ struct PassPlan {
   int ntc;    // tokens staged per chunk
   int spe;    // stages (row groups) per expert
 };
-// Work of one stage in balancing units: streaming its bytes costs about
-// kStageCostMem units and every token it is multiplied with about one more,
-// so CTAs get equal time, not only equal bytes.
-constexpr int kStageCostMem = 1;
-__host__ __device__ inline int stage_cost(int tokens) { return kStageCostMem + tokens; }
+// Work of one stage in balancing units, so that CTAs get equal time, not
+// only equal bytes.  A stage's tokens are multiplied in groups of at most 4
+// (1, 2 or 4 token slots, a group of 3 runs as 4); each group pays about
+// 4 units for decoding the stage's codes and 3 per token slot.
+__host__ __device__ inline int stage_cost(int tokens) {
+  const int full = tokens >> 2, rest = tokens & 3;
+  return full * (4 + 4 * 3) + (rest == 0 ? 0 : rest == 1 ? 4 + 3 : rest == 2 ? 4 + 2 * 3 : 4 + 4 * 3);
+}
+// Work of one expert slot of n tokens in a pass: its chunks of at most ntc
+// tokens, each over the pass's spe stages.
+__host__ __device__ inline int pass_cost(const PassPlan& pp, int n) {
+  const int full = n / pp.ntc, rest = n % pp.ntc;
+  return pp.spe * (full * stage_cost(pp.ntc) + (rest ? stage_cost(rest) : 0));
+}
 
 // -------------------------------------------------------------- device ---
 __device__ __forceinline__ void pdl_wait() {
@@ -210,6 +223,78 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t b, uint32_t 
   return d;
 }
 
+// ---------------------------------------------------------------- top-k ---
+// Unsigned key with the order of the float (for non-NaN values); 0 is below
+// every real key and marks a taken or absent logit.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Largest of a lane's NPL keys and its slot, the lower slot on equal keys
+// (a balanced tree, so the dependency chain is log2(NPL) deep).
+template <int NPL>
+__device__ __forceinline__ void lane_best(const uint32_t (&key)[NPL], uint32_t& bk, int& bm) {
+  uint32_t kk[NPL];
+  int mm[NPL];
+#pragma unroll
+  for (int m = 0; m < NPL; ++m) { kk[m] = key[m]; mm[m] = m; }
+#pragma unroll
+  for (int w = 1; w < NPL; w <<= 1)
+#pragma unroll
+    for (int m = 0; m + w < NPL; m += 2 * w)
+      if (kk[m + w] > kk[m]) { kk[m] = kk[m + w]; mm[m] = mm[m + w]; }
+  bk = kk[0];
+  bm = mm[0];
+}
+
+// Top-k of one token's E logits by one warp: the k largest in descending
+// order, equal logits by ascending expert id, then their softmax weights
+// renormalised over the selection (the softmax maximum is the first pick).
+// Lane l holds experts l, l+32, ...; each round takes the warp maximum of the
+// lanes' best keys with one redux, the lowest expert id among equal keys with
+// a second, and only the winning lane rescans its keys.  CG reads the logits
+// around L1 (they were written by other CTAs of the same launch).
+template <int NPL, bool CG>
+__device__ __forceinline__ void warp_topk_fast(const float* lrow, int k, int E, int* idx_out, float* w_out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[NPL];
+#pragma unroll
+  for (int m = 0; m < NPL; ++m) {
+    const int e = lane + 32 * m;
+    key[m] = e < E ? order_key(CG ? __ldcg(lrow + e) : lrow[e]) : 0u;
+  }
+  uint32_t bk;
+  int bm;
+  lane_best<NPL>(key, bk, bm);
+  uint32_t my_key = 0;
+  int my_idx = 0;
+  for (int j = 0; j < k; ++j) {
+    const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t we = __reduce_min_sync(0xffffffffu, bk == mx ? uint32_t(lane + 32 * bm) : 0xffffffffu);
+    if (lane == j) { my_key = mx; my_idx = int(we); }
+    if (int(we & 31u) == lane) {
+#pragma unroll
+      for (int m = 0; m < NPL; ++m)
+        if (m == bm) key[m] = 0u;
+      lane_best<NPL>(key, bk, bm);
+    }
+  }
+  const float my_logit = key_value(my_key);
+  const float top = __shfl_sync(0xffffffffu, my_logit, 0);
+  const float ex = lane < k ? expf(my_logit - top) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < k) {
+    idx_out[lane] = my_idx;
+    w_out[lane] = ex / sum;
+  }
+}
+
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
@@ -285,6 +370,7 @@ void decode_plans(const moe_config& c, PassPlan* gu, PassPlan* dn);
 cudaError_t launch_combine(const LayerArgs& a);
 cudaError_t launch_prefill_ffn(const LayerArgs& a);
 bool fused_supported(const moe_config& c, int T);
+void set_fused_timing(unsigned long long* buf);
 cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x,
                                 uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
                                 cudaStream_t s);

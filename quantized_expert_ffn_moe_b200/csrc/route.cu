@@ -120,53 +120,11 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(
 // Each round takes the warp-wide maximum (ties to the smaller expert), the
 // owner marks it taken.  Gates are a softmax over the k selected logits.
 template <int NPL>
-__device__ void warp_topk(const float* __restrict__ lrow, int k, int E,
-                          int* __restrict__ idx_out, float* __restrict__ w_out) {
-  const int lane = threadIdx.x & 31;
-  float v[NPL];
-#pragma unroll
-  for (int m = 0; m < NPL; ++m) {
-    const int e = lane + 32 * m;
-    v[m] = e < E ? lrow[e] : -INFINITY;
-  }
-  uint32_t taken = 0;
-  float my_logit = -INFINITY;
-  int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int m = 0; m < NPL; ++m) {
-      const int e = lane + 32 * m;
-      const bool ok = !((taken >> m) & 1u) && e < E;
-      if (ok && (v[m] > bv || (v[m] == bv && e < be))) { bv = v[m]; be = e; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
-    if (be != 0x7fffffff && (be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == j) { my_logit = bv; my_idx = be; }
-  }
-  const float top = __shfl_sync(0xffffffffu, my_logit, 0);
-  float ex = lane < k ? expf(my_logit - top) : 0.f;
-  float sum = ex;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < k) {
-    idx_out[lane] = my_idx;
-    w_out[lane] = ex / sum;
-  }
-}
-
-template <int NPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int* __restrict__ idx, float* __restrict__ w) {
   pdl_wait();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t < T) warp_topk<NPL>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
+  if (t < T) warp_topk_fast<NPL, false>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
   pdl_launch_dependents();
 }
 
@@ -194,7 +152,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
   pdl_wait();
   if (fused_topk) {
     for (int t = warp; t < T; t += NW)
-      warp_topk<NPL>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
+      warp_topk_fast<NPL, false>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
     __syncthreads();
     __threadfence_block();
   }
@@ -303,14 +261,8 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
       } else if (u < nslots) {
         n = T;
       }
-      // cost of a slot = sum over its token chunks of stages * stage_cost(chunk tokens)
-      auto slot_cost = [&](const PassPlan& pp) {
-        if (u >= nslots) return 0;
-        const int full = n / pp.ntc, rest = n % pp.ntc;
-        return pp.spe * (full * stage_cost(pp.ntc) + (rest ? stage_cost(rest) : 0));
-      };
-      int g = slot_cost(pg);
-      int d = slot_cost(pd);
+      int g = u < nslots ? pass_cost(pg, n) : 0;
+      int d = u < nslots ? pass_cost(pd, n) : 0;
       int nt = u < nslots ? (n + kPrefillTileN - 1) / kPrefillTileN : 0;   // token tiles (prefill)
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -352,6 +304,147 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
   pdl_launch_dependents();
 }
 
+// ------------------------------------------------- parallel grouping (large T)
+// The same stable counting sort as group_kernel, spread over CTAs: each
+// chunk of kGroupChunk tokens counts its pairs per expert; one CTA turns the
+// counts into per-chunk bases, offsets, the touched-expert list and the work
+// prefixes; each chunk then writes its pairs in token order.
+__global__ void __launch_bounds__(256) chunk_hist_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                                         int* __restrict__ chunk_hist, int* __restrict__ status) {
+  extern __shared__ int hs[];
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hs[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
+  for (int q = t0 * k + threadIdx.x; q < t1 * k; q += blockDim.x) {
+    const int e = idx[q];
+    if (e < 0 || e >= E) { atomicCAS(status + ST_ERROR, 0, 2); continue; }
+    atomicAdd(&hs[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[size_t(blockIdx.x) * E + e] = hs[e];
+}
+
+__global__ void __launch_bounds__(kGroupThreads) chunk_scan_kernel(
+    int nchunks, int T, int E, int shared, int* __restrict__ chunk_hist, int* __restrict__ status,
+    int* __restrict__ counts_out, int* __restrict__ offsets_out, int* __restrict__ ulist_out,
+    int* __restrict__ api_counts, int* __restrict__ api_offsets, PassPlan pg, PassPlan pd,
+    int* __restrict__ woff_gu, int* __restrict__ woff_dn, int* __restrict__ ntoff) {
+  __shared__ int offs[1025];
+  __shared__ int scan[32];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = threadIdx.x;
+  int c = 0;
+  if (e < E) {
+    // per-chunk base of expert e = exclusive prefix over chunks
+    int run = 0;
+    for (int ch0 = 0; ch0 < nchunks; ch0 += 16) {      // loads issued 16 at a time
+      int v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = ch0 + j < nchunks ? chunk_hist[size_t(ch0 + j) * E + e] : 0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (ch0 + j < nchunks) chunk_hist[size_t(ch0 + j) * E + e] = run;
+        run += v[j];
+      }
+    }
+    c = run;
+  }
+  // exclusive scan over experts
+  int v = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, v, o); if (lane >= o) v += n; }
+  if (lane == 31) scan[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int s2 = scan[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, s2, o); if (lane >= o) s2 += n; }
+    scan[lane] = s2;
+  }
+  __syncthreads();
+  const int excl = v - c + (warp > 0 ? scan[warp - 1] : 0);
+  __syncthreads();
+  if (e < E) {
+    counts_out[e] = c; offsets_out[e] = excl; offs[e] = excl;
+    if (api_counts) api_counts[e] = c;
+    if (api_offsets) api_offsets[e] = excl;
+  }
+  if (e == E - 1) { offsets_out[E] = excl + c; offs[E] = excl + c; if (api_offsets) api_offsets[E] = excl + c; }
+  // touched-expert list
+  const int f = (e < E && c > 0) ? 1 : 0;
+  int fv = f;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, fv, o); if (lane >= o) fv += n; }
+  __syncthreads();
+  if (lane == 31) scan[warp] = fv;
+  __syncthreads();
+  if (warp == 0) {
+    int s2 = scan[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, s2, o); if (lane >= o) s2 += n; }
+    scan[lane] = s2;
+  }
+  __syncthreads();
+  const int fpos = fv - f + (warp > 0 ? scan[warp - 1] : 0);
+  if (f) ulist_out[fpos] = e;
+  const int U = scan[31];
+  if (threadIdx.x == 0) { status[ST_UCOUNT] = U; if (shared) ulist_out[U] = E; }
+  __syncthreads();
+  if (warp == 0) {
+    const int nslots = U + shared;
+    int run_g = 0, run_d = 0, run_t = 0;
+    for (int base = 0; base < nslots; base += 32) {
+      const int u = base + lane;
+      int n = 0;
+      if (u < U) { const int ee = ulist_out[u]; n = offs[ee + 1] - offs[ee]; }
+      else if (u < nslots) n = T;
+      int g = u < nslots ? pass_cost(pg, n) : 0, d = u < nslots ? pass_cost(pd, n) : 0;
+      int nt = u < nslots ? (n + kPrefillTileN - 1) / kPrefillTileN : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ng = __shfl_up_sync(0xffffffffu, g, o), nd = __shfl_up_sync(0xffffffffu, d, o);
+        const int nn = __shfl_up_sync(0xffffffffu, nt, o);
+        if (lane >= o) { g += ng; d += nd; nt += nn; }
+      }
+      if (u < nslots) { woff_gu[u + 1] = run_g + g; woff_dn[u + 1] = run_d + d; ntoff[u + 1] = run_t + nt; }
+      run_g += __shfl_sync(0xffffffffu, g, 31);
+      run_d += __shfl_sync(0xffffffffu, d, 31);
+      run_t += __shfl_sync(0xffffffffu, nt, 31);
+    }
+    if (lane == 0) { woff_gu[0] = 0; woff_dn[0] = 0; ntoff[0] = 0; }
+  }
+}
+
+__global__ void __launch_bounds__(32) chunk_scatter_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                                           const int* __restrict__ chunk_base,
+                                                           const int* __restrict__ offsets, int* __restrict__ pairs,
+                                                           int* __restrict__ inv, int* __restrict__ api_pairs) {
+  extern __shared__ int cur[];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) cur[e] = offsets[e] + chunk_base[size_t(blockIdx.x) * E + e];
+  __syncwarp();
+  const int t0 = blockIdx.x * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
+  for (int t = t0; t < t1; ++t) {
+    if (lane < k) {
+      const int q = t * k + lane;
+      const int e = idx[q];
+      if (e >= 0 && e < E) {
+        const int pos = cur[e]++;     // distinct experts within one token
+        pairs[pos] = q;
+        inv[q] = pos;
+        if (api_pairs) api_pairs[pos] = q;
+      }
+    }
+    __syncwarp();
+  }
+}
+
 template <int NPL>
 cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout& L, bool fused,
                               int* api_counts, int* api_offsets, int* api_pairs, cudaStream_t s) {
@@ -368,6 +461,24 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
     err = launch_pdl(topk_kernel<NPL>, dim3((T + 7) / 8), dim3(256), 0, s, logits, T, c.num_experts,
                      c.top_k, idx, w);
     if (err != cudaSuccess) return err;
+    if (T > 4 * kGroupChunk) {
+      // large batch: parallel stable counting sort
+      const int nch = (T + kGroupChunk - 1) / kGroupChunk, E = c.num_experts;
+      int* hist = reinterpret_cast<int*>(ws + L.chunk_hist);
+      int* status = reinterpret_cast<int*>(ws + L.status);
+      err = launch_pdl(chunk_hist_kernel, dim3(nch), dim3(256), size_t(E) * 4, s, (const int*)idx, T, c.top_k, E,
+                       hist, status);
+      if (err != cudaSuccess) return err;
+      err = launch_pdl(chunk_scan_kernel, dim3(1), dim3(kGroupThreads), 0, s, nch, T, E, c.shared_inter > 0 ? 1 : 0,
+                       hist, status, reinterpret_cast<int*>(ws + L.counts), reinterpret_cast<int*>(ws + L.offsets),
+                       reinterpret_cast<int*>(ws + L.ulist), api_counts, api_offsets, pg, pd,
+                       reinterpret_cast<int*>(ws + L.woff_gu), reinterpret_cast<int*>(ws + L.woff_dn),
+                       reinterpret_cast<int*>(ws + L.ntoff));
+      if (err != cudaSuccess) return err;
+      return launch_pdl(chunk_scatter_kernel, dim3(nch), dim3(32), size_t(E) * 4, s, (const int*)idx, T, c.top_k, E,
+                        (const int*)hist, (const int*)(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
+                        reinterpret_cast<int*>(ws + L.inv), api_pairs);
+    }
   }
   return launch_pdl(kern, dim3(1), dim3(kGroupThreads), smem, s, logits, fused ? 1 : 0, idx, w, T,
                     c.num_experts, c.top_k, c.shared_inter > 0 ? 1 : 0,
