@@ -162,8 +162,16 @@ int moe_profile_begin(int32_t max_calls);
 int moe_profile_end(float* ms_out, int32_t* calls);
 
 /* Measurement hook: while device_buf is non-null, fused decode launches write
- * %globaltimer stamps of each CTA's phase boundaries in their first layer to
- * device_buf[cta][9] (the caller owns the buffer; null switches it off). */
+ * %globaltimer readings (ns) of each CTA's first layer to device_buf[cta][20]
+ * (zero it first; the caller owns the buffer; null switches it off):
+ *   [8] layer start, [0] router logits done, [1] after the first grid barrier,
+ *   [9] top-k done, [10] grouping scan done, [2] work lists ready,
+ *   [3] gate/up done, [4] after the second barrier, [5] down done,
+ *   [6] after the third barrier, [7] combine done;
+ *   [11..13] gate/up and [16..18] down, consumer group 0: ns spent waiting for
+ *   stage data, ns spent staging tokens, stages taken.
+ * Calls made while it is set are not reentrant-safe measurements of a
+ * production run; they only observe one. */
 void moe_debug_fused_timing(unsigned long long* device_buf);
 
 /* The cudaError_t value behind the calling thread's most recent

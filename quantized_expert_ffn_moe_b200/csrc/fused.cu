@@ -6,19 +6,26 @@
 // with the shared expert; in the stack RMSNorm before and the bf16 residual
 // after each layer), reorganised so that a decode step pays one launch:
 //
-//   R  every CTA: RMSNorm factors of the T tokens (stack), router logits of
-//      its slice of experts -> global; the producer thread prefetches this
-//      CTA's share of the shared expert's bytes into L2          | grid barrier
+//   R  every CTA: stages the T tokens (RMSNorm factor in the stack, xhat in
+//      fp16 with a power-of-two scale) and computes the router logits of its
+//      slice of experts -> global; the producer thread prefetches this CTA's
+//      share of the shared expert's bytes into L2                 | grid barrier
 //   S  every CTA (the same deterministic computation): top-k, gates, stable
 //      grouping and the cost-balanced work lists, in shared memory
 //   G  gate/up + SwiGLU over the CTA's share of the stages; the producer warp
-//      streams them (1-D TMA bulk copies into a 3-deep ring) and runs straight
+//      streams them (1-D TMA bulk copies into a 4-slot ring) and runs straight
 //      on into the CTA's down-pass stages                        | grid barrier
 //   D  down x gate weight -> Y                                   | grid barrier
 //   C  combine of the CTA's slice of (token, 8 columns) units    | grid barrier
 //                                                                  (stack only)
-// Grid barriers: a global counter and generation word; every spin is bounded
-// (1 s, then MOE_ERR_TIMEOUT in the status word and the CTA skips the rest).
+// The consumers are two groups of 8 warps that take the stages alternately
+// (group = stage index mod 2), so one group decodes while the other waits for
+// its next stage.  A ring slot always belongs to the same group: with slots
+// shared between groups a group could wait on a slot's barrier two phases
+// ahead, where the parity test passes on the stale phase.
+// Grid barriers: one word per launch, flipped by the last arrival; every spin
+// is bounded (1 s, then MOE_ERR_TIMEOUT in the status word and the CTA skips
+// the rest).
 // Decode is bound by moving expert weights ("125 billion parameters on one
 // gaming GPU -- first impressions of Strata + Qwen 3.8 Flash Next", section "In
 // brief": compute isn't the blocker); with one launch the HBM stream is not
@@ -31,11 +38,17 @@ namespace {
 
 using namespace gemv;
 
-constexpr int kFStages = 3;
+constexpr int kFGroups = 2;                       // consumer groups of kNCW warps
+constexpr int kFCons = kFGroups * kNCW;           // consumer warps
+constexpr int kFThreads = (kFCons + 1) * 32;      // + the producer warp
+constexpr int kFStages = 4;                       // ring slots; slot s belongs to group s % kFGroups
+static_assert(kFStages % kFGroups == 0, "a ring slot must belong to one consumer group");
+constexpr int kBarAll = 1;                        // named barrier of all consumer warps (group g: 2 + g)
+constexpr int kFRingOff = 3584;                   // shared-memory offset of the ring
 constexpr int kFMaxTokens = 64;
 constexpr int kFMaxPairs = kFMaxTokens * 16;
 constexpr int kMaxFusedLayers = 64;
-constexpr int kTimePoints = 9;
+constexpr int kTimePoints = 20;
 
 struct FusedParams {
   moe_config cfg;
@@ -44,40 +57,47 @@ struct FusedParams {
   const uint16_t* x;             // layer mode input
   uint16_t* y;                   // layer mode output, or the residual stream (stack)
   int* trace;                    // stack: [L][T][k] selections, or null
-  unsigned long long* timing;    // null, or [gridDim][9] %globaltimer stamps of layer 0
+  unsigned long long* timing;    // null, or [gridDim][20] %globaltimer stamps of layer 0
   char* ws;
   Layout L_;
-  int ntc_gu, ntc_dn;
-  int smem_route_off, smem_xs_off, smem_tok_off;
+  int ntc_gu, ntc_dn;             // tokens per chunk (gate/up: T when every token is pre-staged)
+  int pre;                        // 1: all T tokens staged once per layer for the router and gate/up
+  int rtc;                        // router: tokens staged at a time
+  int grp_xs;                     // halves of one group's chunk buffer
+  long long xs_halves;            // halves of the whole token region
+  int smem_route_off, smem_xs_off;
   moe_layer_weights w[kMaxFusedLayers];
 };
 
 // ------------------------------------------------------------ grid barrier
-// One thread per CTA.  Returns false when the wait gave up.
+// One thread per CTA, after a CTA-wide barrier.  CTA 0 adds 2^31 - (G - 1),
+// the others 1, so the word's top bit flips exactly when the last CTA
+// arrives and the low bits return to zero (the word starts at zero in every
+// launch); each CTA waits for the flip of the value its own add returned.
+// Returns false when the wait gave up.
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
-__device__ bool grid_barrier(unsigned* count, unsigned* gen, unsigned nblocks, unsigned* passed, int* status) {
+__device__ __forceinline__ unsigned atom_add_release_u32(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ bool grid_barrier(unsigned* word, unsigned nblocks, int* status) {
+  const unsigned inc = blockIdx.x == 0 ? 0x80000000u - (nblocks - 1u) : 1u;
   __threadfence();
-  const unsigned target = *passed + 1;
-  if (atomicAdd(count, 1u) == nblocks - 1) {
-    atomicExch(count, 0u);
-    __threadfence();
-    atomicAdd(gen, 1u);
-  } else {
-    const unsigned long long t0 = global_ns();
-    while (int(ld_acquire_u32(gen) - target) < 0) {
-      __nanosleep(64);
-      if (global_ns() - t0 > kWaitLimitNs) {
-        report_error(status, MOE_ERR_TIMEOUT, 40);
-        return false;
-      }
+  const unsigned old = atom_add_release_u32(word, inc);
+  const unsigned long long t0 = global_ns();
+  while (((ld_acquire_u32(word) ^ old) & 0x80000000u) == 0u) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      report_error(status, MOE_ERR_TIMEOUT, 40);
+      return false;
     }
   }
-  *passed = target;
   __threadfence();
   return true;
 }
@@ -150,6 +170,47 @@ struct FCursor {
 
 __device__ __forceinline__ float round_bf16f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
+// Stages one row of h (fp32, K values) as fp16 in the down decoder's order,
+// with the power-of-two scale that puts its max |h| in [128, 256); returns
+// 2^-sh through inv_out (lane 0).
+template <int BITS, int LPR, int CPL>
+__device__ void stage_h_row(const float* hrow, __half* dst, float* inv_out, int lane) {
+  using Gm = Geom<BITS, LPR, CPL>;
+  constexpr int K = Gm::K;
+  float vmax = 0.f;
+  for (int hh = lane * 8; hh < K; hh += 256) {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(hrow + hh));
+    const float4 b = __ldcg(reinterpret_cast<const float4*>(hrow + hh + 4));
+    vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  int sh = 0;
+  if (vmax > 0.f) {
+    int ex;
+    frexpf(vmax, &ex);
+    sh = min(max(8 - ex, -100), 100);
+  }
+  const float mul = ldexpf(1.f, sh);
+  for (int g0 = lane * Gm::G; g0 < K; g0 += 32 * Gm::G) {
+    float v[Gm::G];
+#pragma unroll
+    for (int q = 0; q < Gm::G / 4; ++q) {
+      const float4 u = __ldcg(reinterpret_cast<const float4*>(hrow + g0 + 4 * q));
+      v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+    }
+    __align__(16) __half hv[Gm::G];
+#pragma unroll
+    for (int j = 0; j < Gm::G; ++j) hv[decode_slot(BITS, j)] = __float2half_rn(v[j] * mul);
+    const int base = staged_offset<BITS, LPR, CPL>(g0);
+#pragma unroll
+    for (int part = 0; part < Gm::NPART; ++part)
+      *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+  }
+  if (lane == 0) *inv_out = ldexpf(1.f, -sh);
+}
+
 // Stages the activations of one slot chunk (gate/up: x rows, normalised and
 // rounded to bf16 in the stack; down: h rows) as fp16 in the decoder's order.
 template <int MODE, int BITS, int LPR, int CPL>
@@ -163,24 +224,24 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
   const int tbase = cur.chunk * cur.ntc;
   for (int tl = warp; tl < cur.nc; tl += kNCW) {
     const int pos = cur.p0 + tbase + tl;
-    const int row = (MODE == GATEUP) ? (is_shared ? pos - T * k : rt.pairs[pos] / k) : pos;
-    const float rn = (MODE == GATEUP) ? rnorm[row] : 1.f;
+    if (lane == 0) {
+      tok_pos[tl] = pos;
+      tok_w[tl] = (MODE == DOWN && !is_shared) ? rt.w[rt.pairs[pos]] : 1.f;
+    }
+    if (MODE == DOWN) {
+      stage_h_row<BITS, LPR, CPL>(h + size_t(pos) * K, xs + size_t(tl) * K, &tok_inv[tl], lane);
+      continue;
+    }
+    const int row = is_shared ? pos - T * k : rt.pairs[pos] / k;
+    const float rn = rnorm[row];
     float vmax = 0.f;
     for (int hh = lane * 8; hh < K; hh += 256) {
-      if (MODE == GATEUP) {
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(row) * K + hh));
-        const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(row) * K + hh));
+      const uint32_t q[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int z = 0; z < 4; ++z) {
-          vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(q[z] << 16) * rn)));
-          vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(q[z] & 0xFFFF0000u) * rn)));
-        }
-      } else {
-        const float* src = h + size_t(row) * K + hh;
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(src));
-        const float4 b = __ldcg(reinterpret_cast<const float4*>(src + 4));
-        vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
-        vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+      for (int z = 0; z < 4; ++z) {
+        vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(q[z] << 16) * rn)));
+        vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(q[z] & 0xFFFF0000u) * rn)));
       }
     }
 #pragma unroll
@@ -195,22 +256,14 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
     __half* dst = xs + size_t(tl) * K;
     for (int g0 = lane * Gm::G; g0 < K; g0 += 32 * Gm::G) {
       float v[Gm::G];
-      if (MODE == GATEUP) {
 #pragma unroll
-        for (int q = 0; q < Gm::G / 8; ++q) {
-          const uint4 u = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(row) * K + g0 + 8 * q));
-          const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+      for (int q = 0; q < Gm::G / 8; ++q) {
+        const uint4 u = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(row) * K + g0 + 8 * q));
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-          for (int z = 0; z < 4; ++z) {
-            v[8 * q + 2 * z] = round_bf16f(__uint_as_float(wd[z] << 16) * rn);
-            v[8 * q + 2 * z + 1] = round_bf16f(__uint_as_float(wd[z] & 0xFFFF0000u) * rn);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < Gm::G / 4; ++q) {
-          const float4 u = __ldcg(reinterpret_cast<const float4*>(h + size_t(row) * K + g0 + 4 * q));
-          v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+        for (int z = 0; z < 4; ++z) {
+          v[8 * q + 2 * z] = round_bf16f(__uint_as_float(wd[z] << 16) * rn);
+          v[8 * q + 2 * z + 1] = round_bf16f(__uint_as_float(wd[z] & 0xFFFF0000u) * rn);
         }
       }
       __align__(16) __half hv[Gm::G];
@@ -221,11 +274,7 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
       for (int part = 0; part < Gm::NPART; ++part)
         *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
     }
-    if (lane == 0) {
-      tok_inv[tl] = ldexpf(1.f, -sh);
-      tok_pos[tl] = pos;
-      tok_w[tl] = (MODE == DOWN && !is_shared) ? rt.w[rt.pairs[pos]] : 1.f;
-    }
+    if (lane == 0) tok_inv[tl] = ldexpf(1.f, -sh);
   }
 }
 
@@ -308,19 +357,21 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
   }
 }
 
-// Router logits of expert e for all T tokens from the staged activations:
-// sum_j Wr[e][g0+j] * xs[slot(j)] (exact products), times the token's 2^-sh.
+// Router logits of expert e for tokens t0 .. t0+nt-1 from their staged
+// activations (xs holds token t0 first) and the expert's router row already
+// in shared memory: sum_j Wr[e][j] * xs[slot(j)] (exact products), times the
+// token's 2^-sh.
 template <int BITS, int LPR, int CPL>
-__device__ void router_from_staged(const uint16_t* wrow, float bias, const __half* xs, const float* inv_all, int T,
-                                   float* logit_col, int E, int lane) {
+__device__ void router_from_staged(const uint16_t* wrow, float bias, const __half* xs, const float* inv_all, int t0,
+                                   int nt, float* logit_col, int E, int lane) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);
   uint4 wv[NG][G / 8];
 #pragma unroll
   for (int q = 0; q < NG; ++q)
 #pragma unroll
-    for (int z = 0; z < G / 8; ++z) wv[q][z] = ld_stream16(wrow + (q * 32 + lane) * G + 8 * z);
-  for (int t = 0; t < T; ++t) {
+    for (int z = 0; z < G / 8; ++z) wv[q][z] = *reinterpret_cast<const uint4*>(wrow + (q * 32 + lane) * G + 8 * z);
+  for (int t = 0; t < nt; ++t) {
     const __half* xt = xs + size_t(t) * K;
     float acc = 0.f;
 #pragma unroll
@@ -343,77 +394,102 @@ __device__ void router_from_staged(const uint16_t* wrow, float bias, const __hal
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) logit_col[size_t(t) * E] = acc * inv_all[t] + bias;
+    if (lane == 0) logit_col[size_t(t0 + t) * E] = acc * inv_all[t0 + t] + bias;
   }
 }
 
-// Exclusive scan of one value per consumer thread (256 threads); also
-// returns the total.  Uses 8 ints of shared scratch.
-__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+// Exclusive scans of two values per consumer thread (all kFCons warps), with
+// their totals.  Uses 2 * kFCons ints of shared scratch.
+__device__ __forceinline__ int2 block_excl_scan2(int a, int b, int* scratch, int2* total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int x = v;
+  int x = a, y = b;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int n = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += n;
+    const int nx = __shfl_up_sync(0xffffffffu, x, o), ny = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) { x += nx; y += ny; }
   }
-  if (lane == 31) scratch[warp] = x;
-  named_bar_sync(1, kNCW * 32);
-  int before = 0, all = 0;
+  if (lane == 31) { scratch[warp] = x; scratch[kFCons + warp] = y; }
+  named_bar_sync(kBarAll, kFCons * 32);
+  int bx = 0, by = 0, ax = 0, ay = 0;
 #pragma unroll
-  for (int w = 0; w < kNCW; ++w) {
-    const int s = scratch[w];
-    if (w < warp) before += s;
-    all += s;
+  for (int w = 0; w < kFCons; ++w) {
+    const int sx = scratch[w], sy = scratch[kFCons + w];
+    if (w < warp) { bx += sx; by += sy; }
+    ax += sx;
+    ay += sy;
   }
-  named_bar_sync(1, kNCW * 32);
-  *total = all;
-  return before + x - v;
+  named_bar_sync(kBarAll, kFCons * 32);
+  *total = make_int2(ax, ay);
+  return make_int2(bx + x - a, by + y - b);
 }
 
-// Consumer side of one pass over this CTA's stages.
+// Per-group token metadata of the chunk being multiplied.
+struct GroupTok {
+  float* inv;     // 2^-sh of each staged token
+  float* w;       // gate weight (down pass) or 1
+  int* pos;       // routed position of each token
+  int* xrow;      // pre-staged row of each token (gate/up with every token staged)
+};
+
+// Consumer side of one pass over this CTA's stages, for consumer group `grp`
+// (warps grp*kNCW ...): walks the same stage sequence as the producer and
+// takes the stages whose index has the group's parity.  A group stages the
+// tokens of a (slot, chunk) itself when it meets its first stage of it.
 template <int MODE, int BITS, int LPR, int CPL>
-__device__ void consume_pass(const FusedParams& p, const SRoute& rt, const moe_layer_weights& lw, FCursor cur,
-                             long long w1, unsigned char* ring, int ring_stride, uint64_t* full, uint64_t* empty,
-                             int* consumed, const uint16_t* xsrc, const float* rnorm, const float* hin, float* out,
-                             int out_cols, __half* xs, float* tok_inv, float* tok_w, int* tok_pos,
-                             volatile int* abort_flag, int* status, const float* inv_all = nullptr,
-                             int* tok_xrow = nullptr) {
+__device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur, long long w1, unsigned char* ring,
+                             int ring_stride, uint64_t* full, uint64_t* empty, int* consumed, int grp,
+                             const uint16_t* xsrc, const float* rnorm, const float* hin, float* out, int out_cols,
+                             const __half* xs_pre, const float* pre_inv, const float* pre_w, int pre_base,
+                             __half* xs_grp, const GroupTok& tk, volatile int* abort_flag, int* status,
+                             unsigned long long* tacc = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane / LPR, lr = lane % LPR;
-  const int rl0 = (warp * Gm::RW + grp) * 2;
-  const bool pre = inv_all != nullptr;      // every token already staged (gate/up)
-  bool first = true;
+  const bool timed = tacc != nullptr && threadIdx.x == 0;
+  const int wg = warp - grp * kNCW;                 // warp inside the group
+  const int gtid = threadIdx.x - grp * kNCW * 32;   // thread inside the group
+  const int lg = lane / LPR, lr = lane % LPR;
+  const int rl0 = (wg * Gm::RW + lg) * 2;
+  // pre: every row already staged in xs_pre -- gate/up: token t at row t,
+  // pre_inv[t]; down: routed position q at row q - pre_base with
+  // pre_inv / pre_w of that row
+  const bool pre = xs_pre != nullptr;
+  int staged_slot = -1, staged_chunk = -1;
   for (; cur.valid(w1); cur.advance()) {
     const int i = (*consumed)++;
-    if (first || cur.stage == 0) {
-      first = false;
-      named_bar_sync(1, kNCW * 32);
+    if (i % kFGroups != grp) continue;
+    if (cur.slot != staged_slot || cur.chunk != staged_chunk) {
+      staged_slot = cur.slot;
+      staged_chunk = cur.chunk;
+      const unsigned long long ts = timed ? global_ns() : 0;
+      named_bar_sync(2 + grp, kNCW * 32);
       if (pre) {
         const int tbase = cur.chunk * cur.ntc;
         const bool is_shared = cur.e >= p.cfg.num_experts;
-        for (int tl = threadIdx.x; tl < cur.nc; tl += kNCW * 32) {
+        for (int tl = gtid; tl < cur.nc; tl += kNCW * 32) {
           const int pos = cur.p0 + tbase + tl;
-          const int tok = is_shared ? pos - p.T * p.cfg.top_k : rt.pairs[pos] / p.cfg.top_k;
-          tok_pos[tl] = pos;
-          tok_xrow[tl] = tok;
-          tok_inv[tl] = inv_all[tok];
-          tok_w[tl] = 1.f;
+          const int row = MODE == GATEUP ? (is_shared ? pos - p.T * p.cfg.top_k : rt.pairs[pos] / p.cfg.top_k)
+                                         : pos - pre_base;
+          tk.pos[tl] = pos;
+          tk.xrow[tl] = row;
+          tk.inv[tl] = pre_inv[row];
+          tk.w[tl] = MODE == GATEUP ? 1.f : pre_w[row];
         }
       } else {
-        stage_chunk<MODE, BITS, LPR, CPL>(p, rt, cur, xsrc, rnorm, hin, xs, tok_inv, tok_w, tok_pos, warp, lane);
+        stage_chunk<MODE, BITS, LPR, CPL>(p, rt, cur, xsrc, rnorm, hin, xs_grp, tk.inv, tk.w, tk.pos, wg, lane);
       }
-      named_bar_sync(1, kNCW * 32);
+      named_bar_sync(2 + grp, kNCW * 32);
+      if (timed) tacc[1] += global_ns() - ts;
     }
     const int slot = i % kFStages;
     bool ok = !*abort_flag;
+    const unsigned long long tw = timed ? global_ns() : 0;
     if (ok && !mbar_wait(&full[slot], (i / kFStages) & 1, abort_flag)) {
       ok = false;
       *abort_flag = 1;
       report_error(status, MOE_ERR_TIMEOUT, 41);
     }
+    if (timed) { tacc[0] += global_ns() - tw; tacc[2] += 1; }
     if (ok) {
       const unsigned char* st = ring + slot * ring_stride;
       const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * Gm::SPR * 2, cur.stage * Gm::RPS + rl0};
@@ -421,11 +497,11 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, const moe_l
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
         const int nt = min(4, nc - tb);
-        const __half* xb = pre ? xs : xs + size_t(tb) * K;
-        const int* xr = pre ? tok_xrow : nullptr;
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(out, out_cols, rows, xb, tb, lr, tok_inv, tok_w, tok_pos, 1, xr);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(out, out_cols, rows, xb, tb, lr, tok_inv, tok_w, tok_pos, 2, xr);
-        else rows_dot<MODE, BITS, LPR, CPL, 4>(out, out_cols, rows, xb, tb, lr, tok_inv, tok_w, tok_pos, nt, xr);
+        const __half* xb = pre ? xs_pre : xs_grp + size_t(tb) * K;
+        const int* xr = pre ? tk.xrow : nullptr;
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 1, xr);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 2, xr);
+        else rows_dot<MODE, BITS, LPR, CPL, 4>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, nt, xr);
       }
     }
     __syncwarp();
@@ -461,8 +537,10 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
   }
 }
 
+constexpr int kRouterTB = 4;          // tokens per router work item
+
 template <int BITS, int LG, int CG, int LD, int CD, int NPL>
-__global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
+__global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
   using GU = Geom<BITS, LG, CG>;
   using DN = Geom<BITS, LD, CD>;
   constexpr int RING_STRIDE = GU::STAGE_BYTES > DN::STAGE_BYTES ? GU::STAGE_BYTES : DN::STAGE_BYTES;
@@ -473,138 +551,133 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kFStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kFStages);
-  float* rnorm = reinterpret_cast<float*>(smem + 64);                    // [64]
-  int* snslots = reinterpret_cast<int*>(smem + 320);
+  uint64_t* rbar = full + 2 * kFStages + 1;                                // router rows landed
+  float* rnorm = reinterpret_cast<float*>(smem + 128);                   // [64]
   float* inv_all = reinterpret_cast<float*>(smem + 384);                 // [64]
-  int* tok_xrow = reinterpret_cast<int*>(smem + 640);                    // [64]
-  int* scan_scratch = reinterpret_cast<int*>(smem + 896);                // [8]
-  unsigned char* ring = smem + 1024;
+  int* snslots = reinterpret_cast<int*>(smem + 640);
+  int* scan_scratch = reinterpret_cast<int*>(smem + 768);                // [2 * kFCons]
+  // [1024, 3072): per-group token metadata, 4 arrays of kMaxNTC each
+  float* dinv = reinterpret_cast<float*>(smem + 3072);                   // [64] down rows staged at once
+  float* dwt = dinv + kMaxNTC;                                           // [64]
+  unsigned char* ring = smem + kFRingOff;
+  const int P = T * k;
   int* ri = reinterpret_cast<int*>(smem + p.smem_route_off);
   SRoute rt;
   rt.idx = ri;
-  rt.w = reinterpret_cast<float*>(ri + kFMaxPairs);
-  rt.pairs = ri + 2 * kFMaxPairs;
-  rt.inv = ri + 3 * kFMaxPairs;
-  rt.offsets = ri + 4 * kFMaxPairs;
+  rt.w = reinterpret_cast<float*>(ri + P);
+  rt.pairs = ri + 2 * P;
+  rt.inv = ri + 3 * P;
+  rt.offsets = ri + 4 * P;
   rt.ulist = rt.offsets + (E + 1);
   rt.woff_gu = rt.ulist + (E + 1);
   rt.woff_dn = rt.woff_gu + (E + 2);
   rt.cnt = rt.woff_dn + (E + 2);
+  // tokens: every token (pre-staged) or router chunks in R and G; the two
+  // groups' chunk buffers in G (not pre-staged) and D
   __half* xs = reinterpret_cast<__half*>(smem + p.smem_xs_off);
-  float* tok_inv = reinterpret_cast<float*>(smem + p.smem_tok_off);
-  float* tok_w = tok_inv + kMaxNTC;
-  int* tok_pos = reinterpret_cast<int*>(tok_w + kMaxNTC);
 
   char* ws = p.ws;
   int* status = reinterpret_cast<int*>(ws + p.L_.status);
-  unsigned* gcount = reinterpret_cast<unsigned*>(status + ST_GRID_COUNT);
-  unsigned* ggen = reinterpret_cast<unsigned*>(status + ST_GRID_GEN);
+  unsigned* gword = reinterpret_cast<unsigned*>(status + ST_GRID_COUNT);
   float* logits = reinterpret_cast<float*>(ws + p.L_.logits);
   float* hbuf = reinterpret_cast<float*>(ws + p.L_.h);
   float* ybuf = reinterpret_cast<float*>(ws + p.L_.y);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool producer = warp == kNCW;
+  const bool producer = warp == kFCons;
+  const int grp = producer ? 0 : warp / kNCW;
+  float* tkb = reinterpret_cast<float*>(smem + 1024 + grp * 4 * kMaxNTC * 4);
+  const GroupTok tk{tkb, tkb + kMaxNTC, reinterpret_cast<int*>(tkb + 2 * kMaxNTC),
+                    reinterpret_cast<int*>(tkb + 3 * kMaxNTC)};
+  __half* xs_grp = xs + size_t(grp) * p.grp_xs;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kFStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kNCW); }
+    mbar_init(rbar, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
   __syncthreads();
-  unsigned passed = 0;                 // grid barriers passed (thread 0 only)
   int issued = 0, consumed = 0;
   const unsigned G = gridDim.x;
   const uint16_t* xsrc = p.stack ? p.y : p.x;
+  auto all_sync = [&]() { named_bar_sync(kBarAll, kFCons * 32); };
+  auto grid_sync = [&]() {
+    all_sync();
+    if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gword, G, status)) *abort_flag = 1;
+    all_sync();
+  };
+  auto stamp = [&](int l, int i) {
+    if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + i] = global_ns();
+  };
 
   for (int l = 0; l < p.L; ++l) {
     const moe_layer_weights& lw = p.w[l];
-    if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 8] = global_ns();
+    stamp(l, 8);
     // ------------------------------------------------------------ phase R
+    // (the ring is idle until the routing is done: slot 0 takes this CTA's
+    // router rows, slot 3 the top-k scratch)
+    const int e0 = int((long long)E * blockIdx.x / G), e1 = int((long long)E * (blockIdx.x + 1) / G);
     if (producer) {
-      if (lane == 0 && S) {
-        // this CTA's share of the shared expert, into L2 for whoever streams it
-        const size_t gu = size_t(2 * I) * H * c.bits / 8, dn = size_t(H) * I * c.bits / 8;
-        const size_t a0 = (gu * blockIdx.x / G) & ~size_t(15), a1 = (gu * (blockIdx.x + 1) / G) & ~size_t(15);
-        if (a1 > a0) bulk_prefetch_l2(lw.shared_gate_up_codes + a0, uint32_t(a1 - a0));
-        const size_t b0 = (dn * blockIdx.x / G) & ~size_t(15), b1 = (dn * (blockIdx.x + 1) / G) & ~size_t(15);
-        if (b1 > b0) bulk_prefetch_l2(lw.shared_down_codes + b0, uint32_t(b1 - b0));
+      if (lane == 0) {
+        if (e1 > e0) {
+          mbar_arrive_expect_tx(rbar, uint32_t(e1 - e0) * H * 2);
+          bulk_g2s(ring, lw.router_w + size_t(e0) * H, uint32_t(e1 - e0) * H * 2, rbar);
+        }
+        if (S) {
+          // this CTA's share of the shared expert, into L2 for whoever streams it
+          const size_t gu = size_t(2 * I) * H * c.bits / 8, dn = size_t(H) * I * c.bits / 8;
+          const size_t a0 = (gu * blockIdx.x / G) & ~size_t(15), a1 = (gu * (blockIdx.x + 1) / G) & ~size_t(15);
+          if (a1 > a0) bulk_prefetch_l2(lw.shared_gate_up_codes + a0, uint32_t(a1 - a0));
+          const size_t b0 = (dn * blockIdx.x / G) & ~size_t(15), b1 = (dn * (blockIdx.x + 1) / G) & ~size_t(15);
+          if (b1 > b0) bulk_prefetch_l2(lw.shared_down_codes + b0, uint32_t(b1 - b0));
+        }
       }
     } else {
-      // tokens: RMSNorm factors (stack), identical in every CTA; when all T
-      // fit, each token is staged once here for the router and gate/up
-      const bool xall = p.ntc_gu >= T;
-      if (xall) {
-        for (int t = warp; t < T; t += kNCW)
-          stage_token_all<BITS, LG, CG>(xsrc + size_t(t) * H, p.stack != 0, xs + size_t(t) * H, &rnorm[t],
-                                        &inv_all[t], lane);
-      } else {
-        for (int t = warp; t < T; t += kNCW) {
-          float ss = 0.f;
-          if (p.stack) {
-            for (int hh = lane * 8; hh < H; hh += 256) {
-              const uint4 v = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(t) * H + hh));
-              const uint32_t q[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int z = 0; z < 4; ++z) {
-                const float a = __uint_as_float(q[z] << 16), b = __uint_as_float(q[z] & 0xFFFF0000u);
-                ss = fmaf(a, a, ss);
-                ss = fmaf(b, b, ss);
-              }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          }
-          if (lane == 0) rnorm[t] = p.stack ? 1.0f / sqrtf(ss / float(H) + 1e-6f) : 1.f;
-        }
-      }
-      named_bar_sync(1, kNCW * 32);
-      // router logits of this CTA's experts: one warp per expert row
-      const int e0 = int((long long)E * blockIdx.x / G), e1 = int((long long)E * (blockIdx.x + 1) / G);
-      for (int e = e0 + warp; e < e1; e += kNCW) {
-        const uint16_t* wr = lw.router_w + size_t(e) * H;
-        const float b = lw.router_bias ? lw.router_bias[e] : 0.f;
-        if (xall) {
-          router_from_staged<BITS, LG, CG>(wr, b, xs, inv_all, T, logits + e, E, lane);
-          continue;
-        }
-        constexpr int RPL = 2048 / 256;      // 16-byte pieces of the row per lane (H = 2048)
-        uint4 wv[RPL];
-#pragma unroll
-        for (int q = 0; q < RPL; ++q) wv[q] = ld_stream16(wr + (q * 32 + lane) * 8);
-        for (int t = 0; t < T; ++t) {
-          const float rn = rnorm[t];
-          float acc = 0.f;
-#pragma unroll
-          for (int q = 0; q < RPL; ++q) {
-            const uint4 xv = __ldcg(reinterpret_cast<const uint4*>(xsrc + size_t(t) * H + (q * 32 + lane) * 8));
-            const uint32_t wa[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
-            const uint32_t xa[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              acc = fmaf(__uint_as_float(wa[z] << 16), round_bf16f(__uint_as_float(xa[z] << 16) * rn), acc);
-              acc = fmaf(__uint_as_float(wa[z] & 0xFFFF0000u), round_bf16f(__uint_as_float(xa[z] & 0xFFFF0000u) * rn), acc);
+      // tokens staged (RMSNorm factor in the stack, fp16 xhat with its
+      // power-of-two scale) in chunks of rtc, identical in every CTA, and
+      // the router logits of this CTA's experts over each chunk: work items
+      // of (expert, kRouterTB tokens) spread over all consumer warps
+      for (int e = threadIdx.x; e < E; e += kFCons * 32) rt.cnt[e] = 0;
+      bool have_rows = false;
+      for (int t0 = 0; t0 < T; t0 += p.rtc) {
+        const int nt = min(p.rtc, T - t0);
+        if (t0 > 0) all_sync();
+        for (int t = warp; t < nt; t += kFCons)
+          stage_token_all<BITS, LG, CG>(xsrc + size_t(t0 + t) * H, p.stack != 0, xs + size_t(t) * H, &rnorm[t0 + t],
+                                        &inv_all[t0 + t], lane);
+        all_sync();
+        const int nb = (nt + kRouterTB - 1) / kRouterTB;
+        for (int it = warp; it < (e1 - e0) * nb; it += kFCons) {
+          if (!have_rows) {
+            have_rows = true;
+            if (!*abort_flag && !mbar_wait(rbar, l & 1, abort_flag)) {
+              *abort_flag = 1;
+              report_error(status, MOE_ERR_TIMEOUT, 43);
             }
           }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-          if (lane == 0) logits[size_t(t) * E + e] = acc + b;
+          const int e = e0 + it / nb, b = it % nb;
+          const float bias = lw.router_bias ? lw.router_bias[e] : 0.f;
+          router_from_staged<BITS, LG, CG>(reinterpret_cast<const uint16_t*>(ring) + size_t(e - e0) * H, bias,
+                                           xs + size_t(b) * kRouterTB * H, inv_all, t0 + b * kRouterTB,
+                                           min(kRouterTB, nt - b * kRouterTB), logits + e, E, lane);
         }
       }
-      named_bar_sync(1, kNCW * 32);
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 0] = global_ns();
-      if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
-      named_bar_sync(1, kNCW * 32);
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 1] = global_ns();
+      all_sync();
+      stamp(l, 0);
+      grid_sync();
+      stamp(l, 1);
       // ---------------------------------------------------------- phase S
-      for (int e = threadIdx.x; e < E; e += kNCW * 32) rt.cnt[e] = 0;
-      for (int t = warp; t < T; t += kNCW) warp_topk_fast<NPL, true>(logits + size_t(t) * E, k, E, rt.idx + t * k, rt.w + t * k);
-      named_bar_sync(1, kNCW * 32);
-      for (int q = threadIdx.x; q < T * k; q += kNCW * 32) atomicAdd(&rt.cnt[rt.idx[q]], 1);
-      named_bar_sync(1, kNCW * 32);
+      {
+        uint2* tscr = reinterpret_cast<uint2*>(ring + 3 * RING_STRIDE) + warp * 32;
+        for (int t = warp; t < T; t += kFCons)
+          warp_topk<NPL, true>(logits + size_t(t) * E, k, E, rt.idx + t * k, rt.w + t * k, tscr, rt.cnt);
+      }
+      all_sync();
+      stamp(l, 9);
       {
         // exclusive scan of the counts and the ascending touched-expert list;
         // cnt becomes each expert's fill cursor
-        const int EPT = (E + kNCW * 32 - 1) / (kNCW * 32);      // experts per thread (<= 4)
+        const int EPT = (E + kFCons * 32 - 1) / (kFCons * 32);     // experts per thread
         const int eb = threadIdx.x * EPT;
         int csum = 0, fsum = 0;
         for (int z = 0; z < EPT; ++z) {
@@ -613,9 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
           csum += cc;
           fsum += cc > 0 ? 1 : 0;
         }
-        int ctot, ftot;
-        int crun = block_excl_scan(csum, scan_scratch, &ctot);
-        int frun = block_excl_scan(fsum, scan_scratch, &ftot);
+        int2 tot;
+        const int2 run = block_excl_scan2(csum, fsum, scan_scratch, &tot);
+        int crun = run.x, frun = run.y;
         for (int z = 0; z < EPT; ++z) {
           const int e = eb + z;
           if (e < E) {
@@ -627,25 +700,26 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
           }
         }
         if (threadIdx.x == 0) {
-          rt.offsets[E] = ctot;
-          if (S) rt.ulist[ftot] = E;
-          *snslots = ftot + S;
+          rt.offsets[E] = tot.x;
+          if (S) rt.ulist[tot.y] = E;
+          *snslots = tot.y + S;
         }
       }
-      named_bar_sync(1, kNCW * 32);
+      all_sync();
+      stamp(l, 10);
       // stable positions inside each expert's list (pairs in token order), by
       // warp 0 over 32 pairs at a time: every CTA derives the same positions,
       // which the passes of different CTAs rely on.  Meanwhile the
       // cost-weighted work prefix of the slots for the two passes.
       if (warp == 0) {
-        for (int base = 0; base < T * k; base += 32) {
+        for (int base = 0; base < P; base += 32) {
           const int q = base + lane;
-          const int e = q < T * k ? rt.idx[q] : -1 - lane;
+          const int e = q < P ? rt.idx[q] : -1 - lane;
           const unsigned same = __match_any_sync(0xffffffffu, e);
           const int rank = __popc(same & ((1u << lane) - 1u));
-          const int start = q < T * k ? rt.cnt[e] : 0;
+          const int start = q < P ? rt.cnt[e] : 0;
           __syncwarp();
-          if (q < T * k) {
+          if (q < P) {
             const int pos = start + rank;
             rt.pairs[pos] = q;
             rt.inv[q] = pos;
@@ -654,12 +728,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
           __syncwarp();
         }
       } else if (warp == 1 && p.trace && blockIdx.x == 0) {
-        for (int q = lane; q < T * k; q += 32) p.trace[size_t(l) * T * k + q] = rt.idx[q];
+        for (int q = lane; q < P; q += 32) p.trace[size_t(l) * P + q] = rt.idx[q];
       }
       {
         const PassPlan pg{p.ntc_gu, 2 * I / GU::RPS}, pd{p.ntc_dn, H / DN::RPS};
         const int ns = *snslots;
-        const int SPT = (ns + kNCW * 32 - 1) / (kNCW * 32);     // slots per thread
+        const int SPT = (ns + kFCons * 32 - 1) / (kFCons * 32);    // slots per thread
         const int u0 = threadIdx.x * SPT;
         int g = 0, d = 0;
         for (int z = 0; z < SPT; ++z) {
@@ -671,9 +745,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
             d += pass_cost(pd, n);
           }
         }
-        int gt, dt;
-        int grun = block_excl_scan(g, scan_scratch, &gt);
-        int drun = block_excl_scan(d, scan_scratch, &dt);
+        int2 tot;
+        const int2 run = block_excl_scan2(g, d, scan_scratch, &tot);
+        int grun = run.x, drun = run.y;
+        const int gt = tot.x, dt = tot.y;
         for (int z = 0; z < SPT; ++z) {
           const int u = u0 + z;
           if (u < ns) {
@@ -689,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
       }
     }
     __syncthreads();                 // routing of this layer ready for all warps
-    if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 2] = global_ns();
+    stamp(l, 2);
 
     const int ns = *snslots;
     FCursor cg{};
@@ -722,35 +797,50 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
       // ---------------------------------------------------------- phase G
       if (g0 < g1) {
         cg.init(g0);
-        const bool xall = p.ntc_gu >= T;
-        consume_pass<GATEUP, BITS, LG, CG>(p, rt, lw, cg, g1, ring, RING_STRIDE, full, empty, &consumed, xsrc,
-                                           rnorm, nullptr, hbuf, I, xs, tok_inv, tok_w, tok_pos, abort_flag, status,
-                                           xall ? inv_all : nullptr, tok_xrow);
+        consume_pass<GATEUP, BITS, LG, CG>(p, rt, cg, g1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
+                                           rnorm, nullptr, hbuf, I, p.pre ? xs : nullptr, inv_all, nullptr, 0, xs_grp,
+                                           tk, abort_flag, status,
+                                           p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 11 : nullptr);
       }
-      named_bar_sync(1, kNCW * 32);
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 3] = global_ns();
-      if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
-      named_bar_sync(1, kNCW * 32);
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 4] = global_ns();
+      all_sync();
+      stamp(l, 3);
+      grid_sync();
+      stamp(l, 4);
       // ---------------------------------------------------------- phase D
       if (d0 < d1) {
         cd.init(d0);
-        consume_pass<DOWN, BITS, LD, CD>(p, rt, lw, cd, d1, ring, RING_STRIDE, full, empty, &consumed, xsrc,
-                                         rnorm, hbuf, ybuf, H, xs, tok_inv, tok_w, tok_pos, abort_flag, status);
+        // the CTA's stages cover one contiguous range of routed positions:
+        // when it fits, all its h rows are staged at once by every warp
+        FCursor cw = cd;
+        const int lo = cw.p0 + cw.chunk * cw.ntc;
+        int hi = lo;
+        for (; cw.valid(d1); cw.advance()) hi = max(hi, cw.p0 + cw.chunk * cw.ntc + cw.nc);
+        const bool dpre = hi - lo <= kMaxNTC && size_t(hi - lo) * DN::K <= p.xs_halves;
+        if (dpre) {
+          for (int r = warp; r < hi - lo; r += kFCons) {
+            const int pos = lo + r;
+            stage_h_row<BITS, LD, CD>(hbuf + size_t(pos) * I, xs + size_t(r) * DN::K, &dinv[r], lane);
+            if (lane == 0) dwt[r] = pos < P ? rt.w[rt.pairs[pos]] : 1.f;
+          }
+          all_sync();
+        }
+        consume_pass<DOWN, BITS, LD, CD>(p, rt, cd, d1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
+                                         rnorm, hbuf, ybuf, H, dpre ? xs : nullptr, dinv, dwt, lo, xs_grp, tk,
+                                         abort_flag, status,
+                                         p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 16 : nullptr);
       }
-      named_bar_sync(1, kNCW * 32);
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 5] = global_ns();
-      if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
-      named_bar_sync(1, kNCW * 32);
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 6] = global_ns();
+      all_sync();
+      stamp(l, 5);
+      grid_sync();
+      stamp(l, 6);
       // ---------------------------------------------------------- phase C
       const int units = T * (H / 8);
       const int u0 = int((long long)units * blockIdx.x / G), u1 = int((long long)units * (blockIdx.x + 1) / G);
-      for (int u = u0 + threadIdx.x; u < u1; u += kNCW * 32) {
+      for (int u = u0 + threadIdx.x; u < u1; u += kFCons * 32) {
         const int t = u / (H / 8), h0 = (u % (H / 8)) * 8;
         float acc[8];
         if (S) {
-          const float* r = ybuf + size_t(T * k + t) * H + h0;
+          const float* r = ybuf + size_t(P + t) * H + h0;
           const float4 a = __ldcg(reinterpret_cast<const float4*>(r)), b = __ldcg(reinterpret_cast<const float4*>(r + 4));
           acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w; acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
         } else {
@@ -778,12 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_decode_kernel(const __grid_
         for (int z = 0; z < 8; ++z) ob[z] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[z]));
         *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob);
       }
-      if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + 7] = global_ns();
-      if (p.stack && l + 1 < p.L) {
-        named_bar_sync(1, kNCW * 32);
-        if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gcount, ggen, G, &passed, status)) *abort_flag = 1;
-        named_bar_sync(1, kNCW * 32);
-      }
+      stamp(l, 7);
+      if (p.stack && l + 1 < p.L) grid_sync();
     }
     __syncthreads();                 // the next layer's routing overwrites this one's
   }
@@ -796,23 +882,41 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   using DN = Geom<BITS, LD, CD>;
   FusedParams q = p;
   constexpr int RING_STRIDE = GU::STAGE_BYTES > DN::STAGE_BYTES ? GU::STAGE_BYTES : DN::STAGE_BYTES;
-  const int E = p.cfg.num_experts;
-  const int route_bytes = (4 * kFMaxPairs + 2 * (E + 1) + 2 * (E + 2) + E) * 4;
-  q.smem_route_off = 1024 + kFStages * RING_STRIDE;
-  q.smem_tok_off = q.smem_route_off + ((route_bytes + 127) & ~127);
-  q.smem_xs_off = q.smem_tok_off + kMaxNTC * 12 + 128;
-  q.smem_xs_off = (q.smem_xs_off + 127) & ~127;
-  const int avail = 227 * 1024 - q.smem_xs_off - 256;
-  q.ntc_gu = min(p.T, min(kMaxNTC, (avail / (GU::K * 2)) & ~1));
-  q.ntc_dn = min(p.T * (p.cfg.top_k + 1), min(kMaxNTC, (avail / (DN::K * 2)) & ~1));
-  if (q.ntc_gu < 1 || q.ntc_dn < 1) return cudaErrorInvalidValue;
-  const size_t smem = q.smem_xs_off + size_t(max(q.ntc_gu * GU::K, q.ntc_dn * DN::K)) * 2;
+  constexpr int kSmemMax = 227 * 1024;
+  const int E = p.cfg.num_experts, T = p.T, k = p.cfg.top_k;
+  const int route_bytes = (4 * T * k + 2 * (E + 1) + 2 * (E + 2) + E) * 4;
+  if (size_t((E + num_sms - 1) / num_sms) * p.cfg.hidden * 2 > size_t(RING_STRIDE)) return cudaErrorCooperativeLaunchTooLarge;
+  q.smem_route_off = kFRingOff + kFStages * RING_STRIDE;
+  q.smem_xs_off = (q.smem_route_off + route_bytes + 127) & ~127;
+  const int avail = kSmemMax - q.smem_xs_off;
+  if (avail <= 0) return cudaErrorInvalidValue;
+  size_t xs_halves;
+  if (size_t(T) * GU::K * 2 <= size_t(avail)) {
+    // every token staged once per layer for the router and gate/up
+    q.pre = 1;
+    q.rtc = T;
+    q.ntc_gu = T;
+    q.ntc_dn = min(T * (k + 1), min(kMaxNTC, avail / (kFGroups * DN::K * 2)));
+    q.grp_xs = q.ntc_dn * DN::K;
+    xs_halves = max(size_t(T) * GU::K, size_t(kFGroups) * q.grp_xs);
+  } else {
+    q.pre = 0;
+    q.rtc = avail / (GU::K * 2);
+    q.ntc_gu = min(T, min(kMaxNTC, avail / (kFGroups * GU::K * 2)));
+    q.ntc_dn = min(T * (k + 1), min(kMaxNTC, avail / (kFGroups * DN::K * 2)));
+    q.grp_xs = max(q.ntc_gu * GU::K, q.ntc_dn * DN::K);
+    xs_halves = max(size_t(q.rtc) * GU::K, size_t(kFGroups) * q.grp_xs);
+  }
+  if (q.rtc < 1 || q.ntc_gu < 1 || q.ntc_dn < 1) return cudaErrorInvalidValue;
+  q.xs_halves = (long long)xs_halves;
+  const size_t smem = q.smem_xs_off + xs_halves * 2;
+  if (smem > size_t(kSmemMax)) return cudaErrorInvalidValue;
   auto kern = fused_decode_kernel<BITS, LG, CG, LD, CD, NPL>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(num_sms);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kFThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

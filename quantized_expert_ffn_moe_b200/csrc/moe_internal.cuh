@@ -254,12 +254,16 @@ __device__ __forceinline__ void lane_best(const uint32_t (&key)[NPL], uint32_t& 
 // Top-k of one token's E logits by one warp: the k largest in descending
 // order, equal logits by ascending expert id, then their softmax weights
 // renormalised over the selection (the softmax maximum is the first pick).
-// Lane l holds experts l, l+32, ...; each round takes the warp maximum of the
-// lanes' best keys with one redux, the lowest expert id among equal keys with
-// a second, and only the winning lane rescans its keys.  CG reads the logits
-// around L1 (they were written by other CTAs of the same launch).
+// Lane l holds experts l, l+32, ...  The k-th largest of the 32 lane maxima,
+// theta, bounds the selection from below (those k lanes already hold k values
+// >= theta), so only the logits >= theta are candidates; when there are at
+// most 32 of them they are ranked all at once through `scratch` (32 uint2 of
+// shared memory for this warp), otherwise k rounds of warp maxima decide.
+// CG reads the logits around L1 (they were written by other CTAs of the same
+// launch).  Optionally counts each pick into cnt[expert] (shared memory).
 template <int NPL, bool CG>
-__device__ __forceinline__ void warp_topk_fast(const float* lrow, int k, int E, int* idx_out, float* w_out) {
+__device__ __forceinline__ void warp_topk(const float* lrow, int k, int E, int* idx_out, float* w_out,
+                                          uint2* scratch, int* cnt = nullptr) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NPL];
 #pragma unroll
@@ -267,20 +271,70 @@ __device__ __forceinline__ void warp_topk_fast(const float* lrow, int k, int E, 
     const int e = lane + 32 * m;
     key[m] = e < E ? order_key(CG ? __ldcg(lrow + e) : lrow[e]) : 0u;
   }
-  uint32_t bk;
-  int bm;
-  lane_best<NPL>(key, bk, bm);
+  uint32_t lb = key[0];
+#pragma unroll
+  for (int m = 1; m < NPL; ++m) lb = max(lb, key[m]);
+  int r = 0;                       // rank of this lane's maximum among the 32
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t o = __shfl_sync(0xffffffffu, lb, j);
+    r += (o > lb) || (o == lb && j < lane);
+  }
+  const unsigned sel = __ballot_sync(0xffffffffu, r == k - 1);
+  const uint32_t theta = __shfl_sync(0xffffffffu, lb, __ffs(sel) - 1);
+  int nc = 0;
+#pragma unroll
+  for (int m = 0; m < NPL; ++m) nc += key[m] >= theta ? 1 : 0;
+  int inc = nc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  const int C = __shfl_sync(0xffffffffu, inc, 31);
   uint32_t my_key = 0;
   int my_idx = 0;
-  for (int j = 0; j < k; ++j) {
-    const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
-    const uint32_t we = __reduce_min_sync(0xffffffffu, bk == mx ? uint32_t(lane + 32 * bm) : 0xffffffffu);
-    if (lane == j) { my_key = mx; my_idx = int(we); }
-    if (int(we & 31u) == lane) {
+  if (C <= 32) {
+    int w = inc - nc;
 #pragma unroll
-      for (int m = 0; m < NPL; ++m)
-        if (m == bm) key[m] = 0u;
-      lane_best<NPL>(key, bk, bm);
+    for (int m = 0; m < NPL; ++m)
+      if (key[m] >= theta) scratch[w++] = make_uint2(key[m], uint32_t(lane + 32 * m));
+    __syncwarp();
+    uint32_t ck = 0, ce = 0;
+    int rank = 32;
+    if (lane < C) {
+      const uint2 cc = scratch[lane];
+      ck = cc.x;
+      ce = cc.y;
+      rank = 0;
+      for (int j = 0; j < C; ++j) {
+        const uint2 o = scratch[j];
+        rank += (o.x > ck) || (o.x == ck && o.y < ce);
+      }
+    }
+    __syncwarp();
+    if (rank < k) scratch[rank] = make_uint2(ck, ce);
+    __syncwarp();
+    if (lane < k) {
+      const uint2 cc = scratch[lane];
+      my_key = cc.x;
+      my_idx = int(cc.y);
+    }
+    __syncwarp();
+  } else {
+    uint32_t bk;
+    int bm;
+    lane_best<NPL>(key, bk, bm);
+    for (int j = 0; j < k; ++j) {
+      const uint32_t mx = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t we = __reduce_min_sync(0xffffffffu, bk == mx ? uint32_t(lane + 32 * bm) : 0xffffffffu);
+      if (lane == j) { my_key = mx; my_idx = int(we); }
+      if (int(we & 31u) == lane) {
+#pragma unroll
+        for (int m = 0; m < NPL; ++m)
+          if (m == bm) key[m] = 0u;
+        lane_best<NPL>(key, bk, bm);
+      }
     }
   }
   const float my_logit = key_value(my_key);
@@ -292,6 +346,7 @@ __device__ __forceinline__ void warp_topk_fast(const float* lrow, int k, int E, 
   if (lane < k) {
     idx_out[lane] = my_idx;
     w_out[lane] = ex / sum;
+    if (cnt) atomicAdd(&cnt[my_idx], 1);
   }
 }
 

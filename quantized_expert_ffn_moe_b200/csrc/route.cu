@@ -122,9 +122,11 @@ __global__ void __launch_bounds__(kRouterWarps * 32) router_logits_kernel(
 template <int NPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int* __restrict__ idx, float* __restrict__ w) {
+  __shared__ uint2 scratch[8][32];
   pdl_wait();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t < T) warp_topk_fast<NPL, false>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
+  if (t < T)
+    warp_topk<NPL, false>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k, scratch[threadIdx.x >> 5]);
   pdl_launch_dependents();
 }
 
@@ -151,8 +153,9 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
   if (fused_topk) {
+    __shared__ uint2 topk_scratch[kGroupThreads / 32][32];
     for (int t = warp; t < T; t += NW)
-      warp_topk_fast<NPL, false>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k);
+      warp_topk<NPL, false>(logits + size_t(t) * E, k, E, idx + size_t(t) * k, w + size_t(t) * k, topk_scratch[warp]);
     __syncthreads();
     __threadfence_block();
   }
