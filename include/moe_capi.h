@@ -174,6 +174,20 @@ int moe_profile_end(float* ms_out, int32_t* calls);
  * production run; they only observe one. */
 void moe_debug_fused_timing(unsigned long long* device_buf);
 
+/* Measurement hook: while device_buf is non-null, the prefill grouped GEMMs
+ * write per-CTA totals to device_buf[pass][cta][16] (pass 0 gate/up, 1 down;
+ * cta < the SM count; zero it first; the caller owns it).  Waits are in SM
+ * clock cycles:
+ *   [0] packed-weight producer waiting for a free stage, [1] token producer
+ *   waiting for a free stage, [2] MMA waiting for the A and B operands,
+ *   [4] MMA waiting for a free accumulator, [5] dequantizer (first thread)
+ *   waiting for packed weights, [6] dequantizer waiting for a free A stage,
+ *   [7] epilogue (first thread) waiting for an accumulator, [12] cycles in the
+ *   MMA issue blocks, [13] cycles in tile lookups; %globaltimer (ns): [8]
+ *   start and [9] end of the MMA thread, [11] end of the epilogue; counts:
+ *   [10] tiles, [14] k-blocks. */
+void moe_debug_prefill_timing(unsigned long long* device_buf);
+
 /* The cudaError_t value behind the calling thread's most recent
  * MOE_ERR_CUDA (0 if none). */
 int moe_last_cuda_error(void);

@@ -24,8 +24,8 @@
 // shared between groups a group could wait on a slot's barrier two phases
 // ahead, where the parity test passes on the stale phase.
 // Grid barriers: one word per launch, flipped by the last arrival; every spin
-// is bounded (1 s, then MOE_ERR_TIMEOUT in the status word and the CTA skips
-// the rest).
+// is bounded (kWaitLimitCycles, then MOE_ERR_TIMEOUT in the status word and
+// the CTA skips the rest).
 // Decode is bound by moving expert weights ("125 billion parameters on one
 // gaming GPU -- first impressions of Strata + Qwen 3.8 Flash Next", section "In
 // brief": compute isn't the blocker); with one launch the HBM stream is not
@@ -91,9 +91,9 @@ __device__ bool grid_barrier(unsigned* word, unsigned nblocks, int* status) {
   const unsigned inc = blockIdx.x == 0 ? 0x80000000u - (nblocks - 1u) : 1u;
   __threadfence();
   const unsigned old = atom_add_release_u32(word, inc);
-  const unsigned long long t0 = global_ns();
+  const long long t0 = clock64();
   while (((ld_acquire_u32(word) ^ old) & 0x80000000u) == 0u) {
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       report_error(status, MOE_ERR_TIMEOUT, 40);
       return false;
     }

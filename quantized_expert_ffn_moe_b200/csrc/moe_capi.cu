@@ -280,6 +280,8 @@ int moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 void moe_debug_fused_timing(unsigned long long* device_buf) { set_fused_timing(device_buf); }
 
+void moe_debug_prefill_timing(unsigned long long* device_buf) { set_prefill_timing(device_buf); }
+
 const char* moe_status_str(int status) {
   switch (status) {
     case MOE_OK: return "ok";

@@ -151,10 +151,12 @@ __device__ __forceinline__ uint16_t ld_stream2(const void* p) {
 }
 
 // ------------------------------------------------ mbarrier / bulk copy ---
-// Every wait is bounded: after kWaitLimitNs of wall time (or when the CTA's
-// abort flag is raised) it gives up and returns false; the caller records
+// Every wait is bounded: after kWaitLimitCycles SM clock cycles (1-3 s at the
+// B200's clocks; the SM cycle counter is read, as it costs a few cycles where
+// %globaltimer costs tens of nanoseconds inside a spin) or when the CTA's
+// abort flag is raised it gives up and returns false; the caller records
 // MOE_ERR_TIMEOUT in the status word and skips the remaining work.
-constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s
+constexpr long long kWaitLimitCycles = 3000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -191,11 +193,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase of `bar` with the given parity; false on timeout/abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
+  const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag && *abort_flag) return false;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (clock64() - t0 > kWaitLimitCycles) return false;
   }
 }
 // 1-D TMA: `bytes` (multiple of 16, both addresses 16-byte aligned) from
@@ -426,6 +428,8 @@ cudaError_t launch_combine(const LayerArgs& a);
 cudaError_t launch_prefill_ffn(const LayerArgs& a);
 bool fused_supported(const moe_config& c, int T);
 void set_fused_timing(unsigned long long* buf);
+void set_prefill_timing(unsigned long long* buf);
+extern unsigned long long* g_prefill_timing;
 cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x,
                                 uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
                                 cudaStream_t s);

@@ -15,7 +15,9 @@
 //   warp 0      TMA of packed codes + fp16 scales (2-D tensor maps, swizzled)
 //   warp 1      TMA of the token tile (SWIZZLE_128B, the UMMA K-major layout)
 //   warp 2      TMEM allocation; one thread issues tcgen05.mma + commits
-//   warps 3-10  dequantize codes into the fp16 A tile (same swizzled layout)
+//   warps 3-10  dequantize codes into the fp16 A operand, written straight
+//               into tensor memory (tcgen05.st, one row per TMEM lane), so
+//               the dequantized tile never passes through shared memory
 //   warps 11-14 epilogue: tcgen05.ld from TMEM, SwiGLU (gate/up) or gate
 //               weight (down), stores
 // Operands are fp16: a weight is q * s rounded once (q exact, s the block's
@@ -39,11 +41,21 @@ constexpr int PBN = kPrefillTileN;   // tokens per tile (max)
 static_assert(PBN == 128, "the grouping kernel's tile prefix assumes 128 tokens per tile");
 constexpr int PBK = 64;        // k per A/B stage: one 128-byte swizzle row of fp16
 constexpr int RAWK = 256;      // k per packed stage
-constexpr int PNK = 4;         // A/B stages
-constexpr int PNR = 2;         // packed stages
+constexpr int PNK = 8;         // A (tensor memory) / B (shared memory) stages
+constexpr int PNR = 4;         // packed stages
 constexpr int kWarpRaw = 0, kWarpB = 1, kWarpMma = 2, kWarpDq0 = 3, kNumDq = 8, kWarpEp0 = 11, kNumEp = 4;
 constexpr int kPThreads = (kWarpEp0 + kNumEp) * 32;
-constexpr uint32_t kTmemCols = 2 * PBN;
+constexpr uint32_t kTmemCols = 2 * PBN;          // router GEMM: two accumulators
+// Grouped GEMM tensor memory: two accumulators of PBN columns, then PNK
+// dequantized A stages of PBK / 2 columns (128 lanes = the tile's rows, two
+// fp16 per 32-bit column in k order).
+constexpr uint32_t kAColBase = 2 * PBN;
+constexpr uint32_t kAStageCols = PBK / 2;
+constexpr uint32_t kPTmemCols = 512;
+static_assert(kAColBase + PNK * kAStageCols <= kPTmemCols, "tensor memory budget");
+// barriers (2 PNR + 2 PNK + 4 of 8 bytes), the TMEM address and the abort flag
+constexpr int kBarBytes = 512;
+static_assert((2 * PNR + 2 * PNK + 4) * 8 + 8 <= kBarBytes, "barrier area");
 constexpr int kAStageBytes = PBM * 128;           // 16 KB
 constexpr int kBStageBytes = PBN * 128;           // 16 KB
 
@@ -69,7 +81,10 @@ struct PrefillArgs {
   const float* xinv;      // gate/up: [P] inverse power-of-two scale of each token row
   float* yout;            // down: Y [P][H] fp32
   int* status;
+  unsigned long long* timing;   // null, or [gridDim][16] per-role wait times (ns) of this launch
 };
+
+constexpr int kPTime = 16;
 
 // ------------------------------------------------------------ primitives
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
@@ -80,7 +95,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -94,6 +108,29 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Same with the A operand in tensor memory (lane = row, two fp16 per column).
+__device__ __forceinline__ void tc_mma_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive columns of this thread's tensor-memory lane (warp-wide; the
+// warp's lane quarter is fixed by its rank within the warpgroup).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t v[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // UMMA shared-memory descriptor of a K-major SWIZZLE_128B tile: rows of 128 B,
 // 8-row atoms 1024 B apart (SBO), version 1, layout type 2.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -129,21 +166,42 @@ __device__ __forceinline__ void dq2_f16(uint32_t v, __half2 s, uint32_t out[8]) 
   for (int j = 0; j < 8; ++j) out[j] = h2_as_u32(__hmul2(q[j], s));
 }
 
+// mbar_wait that adds the SM cycles it waited to *acc when acc is non-null.
+__device__ __forceinline__ bool mbar_wait_t(uint64_t* bar, uint32_t parity, const volatile int* abort_flag,
+                                            unsigned long long* acc) {
+  if (!acc) return mbar_wait(bar, parity, abort_flag);
+  const long long t0 = clock64();
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  *acc += clock64() - t0;
+  return ok;
+}
+
 struct TileInfo {
   int slot, e, p0, n, nvalid, m, j;
 };
 
-__device__ __forceinline__ void tile_info(const PrefillArgs& a, int nslots, int mt, int t, TileInfo* ti) {
+// Slot table of the pass in shared memory (read once per CTA): token-tile
+// prefix, expert, first routed position and token count of every slot.
+struct SlotTab {
+  int* ntoff;   // [nslots + 1]
+  int* e;       // [nslots]
+  int* p0;      // [nslots]
+  int* n;       // [nslots]
+};
+
+__device__ __forceinline__ void tile_info(const SlotTab& st, int nslots, int mt, int t, TileInfo* ti) {
   const int g = t / mt;
   ti->m = t % mt;
   int lo = 0, hi = nslots - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldcg(a.ntoff + mid) <= g) lo = mid; else hi = mid - 1;
+    if (st.ntoff[mid] <= g) lo = mid; else hi = mid - 1;
   }
   ti->slot = lo;
-  ti->j = g - __ldcg(a.ntoff + lo);
-  slot_range(a.rv, lo, &ti->e, &ti->p0, &ti->n);
+  ti->j = g - st.ntoff[lo];
+  ti->e = st.e[lo];
+  ti->p0 = st.p0[lo];
+  ti->n = st.n[lo];
   ti->nvalid = min(PBN, ti->n - ti->j * PBN);
 }
 
@@ -155,16 +213,14 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   using Gm = PGeom<BITS>;
   extern __shared__ __align__(1024) unsigned char psmem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(psmem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sA = base;                                   // PNK x 16 KB
-  unsigned char* sB = sA + PNK * kAStageBytes;                // PNK x 16 KB
+  unsigned char* sB = base;                                   // PNK x 16 KB
   unsigned char* sRaw = sB + PNK * kBStageBytes;              // PNR x RAW_BYTES (1024-aligned each)
   constexpr int RAW_STRIDE = (Gm::RAW_BYTES + 1023) / 1024 * 1024;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + PNR * RAW_STRIDE);
   uint64_t* full_raw = bars;
   uint64_t* empty_raw = full_raw + PNR;
   uint64_t* full_a = empty_raw + PNR;
-  uint64_t* full_b = full_a + PNK;
-  uint64_t* empty_ab = full_b + PNK;
+  uint64_t* empty_ab = full_a + PNK;
   uint64_t* acc_full = empty_ab + PNK;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
@@ -173,14 +229,15 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < PNR; ++i) { mbar_init(&full_raw[i], 1); mbar_init(&empty_raw[i], kNumDq); }
-    for (int i = 0; i < PNK; ++i) { mbar_init(&full_a[i], kNumDq / 2); mbar_init(&full_b[i], 1); mbar_init(&empty_ab[i], 1); }
+    // full_a: the four dequant warps of the k-block's half + the token tile's bytes
+    for (int i = 0; i < PNK; ++i) { mbar_init(&full_a[i], kNumDq / 2 + 1); mbar_init(&empty_ab[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], kNumEp); }
     *abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(kTmemCols) : "memory");
+                 "r"(kPTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
@@ -190,11 +247,26 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
 
   pdl_wait();                     // tokens (and routing) come from earlier kernels
   pdl_launch_dependents();
+  unsigned long long* tm = a.timing ? a.timing + size_t(blockIdx.x) * kPTime : nullptr;
+  unsigned long long tw0 = 0, tw1 = 0, tw2 = 0, tw3 = 0, tw4 = 0;   // this thread's totals (timed roles only)
+  const unsigned long long t_start = tm ? global_ns() : 0;
 
   const RouteView& rv = a.rv;
   const int nslots = __ldcg(rv.status + ST_UCOUNT) + rv.shared;
   const int mt = a.rows_pe / PBM;
-  const int ntiles = __ldcg(a.ntoff + nslots) * mt;
+  // slot table into shared memory (nslots <= E + 1): one L2 round trip here
+  // instead of a dependent binary search through global memory per tile
+  SlotTab stab;
+  stab.ntoff = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(bars) + kBarBytes);
+  stab.e = stab.ntoff + (rv.E + 2);
+  stab.p0 = stab.e + (rv.E + 1);
+  stab.n = stab.p0 + (rv.E + 1);
+  for (int i = threadIdx.x; i <= nslots; i += blockDim.x) {
+    stab.ntoff[i] = __ldcg(a.ntoff + i);
+    if (i < nslots) slot_range(rv, i, &stab.e[i], &stab.p0[i], &stab.n[i]);
+  }
+  __syncthreads();
+  const int ntiles = stab.ntoff[nslots] * mt;
   const int KB = a.K / PBK, KR = a.K / RAWK;
 
   if (warp == kWarpRaw && lane == 0) {
@@ -202,14 +274,14 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     int rc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       TileInfo ti;
-      tile_info(a, nslots, mt, t, &ti);
+      tile_info(stab, nslots, mt, t, &ti);
       const bool sh = ti.e >= rv.E;
       const CUtensorMap* mc = sh ? &tm_sh_codes : &tm_codes;
       const CUtensorMap* ms = sh ? &tm_sh_scales : &tm_scales;
       const int row = (sh ? 0 : ti.e * a.rows_pe) + ti.m * PBM;
       for (int r = 0; r < KR; ++r, ++rc) {
         const int s = rc % PNR;
-        if (rc >= PNR && !mbar_wait(&empty_raw[s], ((rc / PNR) - 1) & 1, abort_flag)) {
+        if (rc >= PNR && !mbar_wait_t(&empty_raw[s], ((rc / PNR) - 1) & 1, abort_flag, tm ? &tw0 : nullptr)) {
           *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 10); break;
         }
         unsigned char* dst = sRaw + s * RAW_STRIDE;
@@ -220,32 +292,36 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     }
     for (int i = max(0, rc - PNR); i < rc; ++i)
       if (!mbar_wait(&full_raw[i % PNR], (i / PNR) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 11);
+    if (tm) tm[0] = tw0;
   } else if (warp == kWarpB && lane == 0) {
     // ------------------------------------------------------ token producer
     int kc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       TileInfo ti;
-      tile_info(a, nslots, mt, t, &ti);
+      tile_info(stab, nslots, mt, t, &ti);
       const int prow = ti.p0 + ti.j * PBN;
       for (int kb = 0; kb < KB; ++kb, ++kc) {
         const int s = kc % PNK;
-        if (kc >= PNK && !mbar_wait(&empty_ab[s], ((kc / PNK) - 1) & 1, abort_flag)) {
+        if (kc >= PNK && !mbar_wait_t(&empty_ab[s], ((kc / PNK) - 1) & 1, abort_flag, tm ? &tw0 : nullptr)) {
           *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 12); break;
         }
-        mbar_arrive_expect_tx(&full_b[s], kBStageBytes);
-        tma_load_2d(sB + s * kBStageBytes, &tm_b, kb * PBK, prow, &full_b[s]);
+        mbar_arrive_expect_tx(&full_a[s], kBStageBytes);
+        tma_load_2d(sB + s * kBStageBytes, &tm_b, kb * PBK, prow, &full_a[s]);
       }
     }
     for (int i = max(0, kc - PNK); i < kc; ++i)
-      if (!mbar_wait(&full_b[i % PNK], (i / PNK) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 13);
+      if (!mbar_wait(&full_a[i % PNK], (i / PNK) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 13);
+    if (tm) tm[1] = tw0;
   } else if (warp == kWarpMma && lane == 0) {
     // ---------------------------------------------------------------- MMA
     int kc = 0, tc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x, ++tc) {
+      const long long cti = tm ? clock64() : 0;
       TileInfo ti;
-      tile_info(a, nslots, mt, t, &ti);
+      tile_info(stab, nslots, mt, t, &ti);
+      if (tm) tw4 += clock64() - cti;
       const int buf = tc & 1;
-      if (tc >= 2 && !mbar_wait(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag)) {
+      if (tc >= 2 && !mbar_wait_t(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag, tm ? &tw2 : nullptr)) {
         *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 14); break;
       }
       tc_fence_after();
@@ -255,15 +331,17 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++kc) {
         const int s = kc % PNK;
-        if (!mbar_wait(&full_a[s], (kc / PNK) & 1, abort_flag) || !mbar_wait(&full_b[s], (kc / PNK) & 1, abort_flag)) {
+        if (!mbar_wait_t(&full_a[s], (kc / PNK) & 1, abort_flag, tm ? &tw0 : nullptr)) {
           *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 15); ok = false; break;
         }
+        const long long ci = tm ? clock64() : 0;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * kAStageBytes), b0 = smem_u32(sB + s * kBStageBytes);
+        const uint32_t a0 = tmem_base + kAColBase + uint32_t(s) * kAStageCols, b0 = smem_u32(sB + s * kBStageBytes);
 #pragma unroll
         for (int k = 0; k < PBK / 16; ++k)
-          tc_mma(d_tmem, sw128_desc(a0 + k * 32), sw128_desc(b0 + k * 32), idesc, (kb | k) ? 1u : 0u);
+          tc_mma_ta(d_tmem, a0 + uint32_t(k * 8), sw128_desc(b0 + k * 32), idesc, (kb | k) ? 1u : 0u);
         tc_commit(&empty_ab[s]);
+        if (tm) tw3 += clock64() - ci;
       }
       if (!ok) break;
       tc_commit(&acc_full[buf]);
@@ -271,25 +349,31 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     // wait for this thread's last MMAs before the CTA tears down TMEM
     if (kc > 0 && !mbar_wait(&empty_ab[(kc - 1) % PNK], ((kc - 1) / PNK) & 1, nullptr))
       report_error(a.status, MOE_ERR_TIMEOUT, 16);
+    if (tm) { tm[2] = tw0; tm[3] = tw1; tm[4] = tw2; tm[8] = t_start; tm[9] = global_ns(); tm[10] = tc; tm[12] = tw3; tm[13] = tw4; tm[14] = kc; }
   } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kNumDq) {
     // ----------------------------------------------------------- dequant
-    const int dt = threadIdx.x - kWarpDq0 * 32;    // 0..255
-    const int r = dt & (PBM - 1);                  // tile row
-    const int half = dt >> 7;                      // which two of the four k-blocks of a packed stage
+    // warp w writes rows of its tensor-memory lane quarter (w % 4); the two
+    // warps of a quarter take the first and second half of a packed stage
+    const int r = (warp & 3) * 32 + lane;          // tile row
+    const int half = (warp - kWarpDq0) >> 2;       // which two of the four k-blocks of a packed stage
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     int rc = 0, kc = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       for (int rs = 0; rs < KR; ++rs, ++rc) {
         const int s = rc % PNR;
-        bool ok = !*abort_flag && mbar_wait(&full_raw[s], (rc / PNR) & 1, abort_flag);
+        const bool timed = tm && threadIdx.x == kWarpDq0 * 32;
+        bool ok = !*abort_flag && mbar_wait_t(&full_raw[s], (rc / PNR) & 1, abort_flag, timed ? &tw0 : nullptr);
         const unsigned char* raw = sRaw + s * RAW_STRIDE;
         const unsigned char* sc = raw + Gm::SCALE_OFF;
         for (int jj = 0; jj < 2; ++jj) {
           const int kbl = half * 2 + jj;            // k-block within the packed stage (0..3)
           const int kglob = kc + kbl;               // global k-block counter of this A/B stage
           const int as = kglob % PNK;
-          if (ok && kglob >= PNK) ok = mbar_wait(&empty_ab[as], ((kglob / PNK) - 1) & 1, abort_flag);
+          if (ok && kglob >= PNK) ok = mbar_wait_t(&empty_ab[as], ((kglob / PNK) - 1) & 1, abort_flag, timed ? &tw1 : nullptr);
+          ok = __all_sync(0xffffffffu, ok);         // the tensor-memory store is warp-wide
           if (ok) {
-            unsigned char* arow = sA + as * kAStageBytes + r * 128;
+            tc_fence_after();
+            uint32_t o32[32];                       // the row's 64 fp16 of this k-block, in k order
             if (BITS == 4) {
               // row r: 2 x 16 bytes of codes = 64 weights, 2 scales
 #pragma unroll
@@ -300,12 +384,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
                 const __half2 s2 = __half2half2(hs);
                 const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  uint32_t o[4];
-                  dq4_f16(wd[q], s2, o);
-                  const int oc = cc * 4 + q;                     // output chunk 0..7
-                  *reinterpret_cast<uint4*>(arow + ((oc ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                }
+                for (int q = 0; q < 4; ++q) dq4_f16(wd[q], s2, o32 + (cc * 4 + q) * 4);
               }
             } else {
               // row r: 16 bytes of codes = 64 weights in 4 words, 4 scales
@@ -322,13 +401,12 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
                 const uint32_t pr = svw[si >> 1];
                 const __half hs = __ushort_as_half((unsigned short)((si & 1) ? (pr >> 16) : (pr & 0xFFFFu)));
                 const __half2 s2 = __half2half2(hs);
-                uint32_t o[8];
-                dq2_f16(wd[q], s2, o);
-                *reinterpret_cast<uint4*>(arow + (((2 * q) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4*>(arow + (((2 * q + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                dq2_f16(wd[q], s2, o32 + q * 8);
               }
             }
-            fence_async_smem();
+            tmem_st32(tmem_base + lane_base + kAColBase + uint32_t(as) * kAStageCols, o32);
+            tmem_st_wait();
+            tc_fence_before();
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&full_a[as]);
@@ -339,6 +417,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
         kc += 4;
       }
     }
+    if (tm && threadIdx.x == kWarpDq0 * 32) { tm[5] = tw0; tm[6] = tw1; }
   } else if (warp >= kWarpEp0 && warp < kWarpEp0 + kNumEp) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                         // TMEM lane quarter of this warp
@@ -346,26 +425,42 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     int tc = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
       TileInfo ti;
-      tile_info(a, nslots, mt, t, &ti);
+      tile_info(stab, nslots, mt, t, &ti);
       const int buf = tc & 1;
-      if (*abort_flag || !mbar_wait(&acc_full[buf], (tc >> 1) & 1, abort_flag)) {
+      const bool sh = ti.e >= rv.E;
+      const int R = ti.m * PBM + r;                 // row of the expert matrix
+      const int prow = ti.p0 + ti.j * PBN;
+      // per-column factors of the tile (gate/up: the token row's inverse
+      // scale, down: the gate weight), column u*32 + lane in f[u], loaded
+      // before the accumulator wait so the latency overlaps it
+      float f[PBN / 32];
+      int pr[PBN / 32];
+#pragma unroll
+      for (int u = 0; u < PBN / 32; ++u) {
+        const int c = u * 32 + lane;
+        f[u] = 1.f;
+        pr[u] = -1;
+        if (c < ti.nvalid) {
+          if (MODE == 0) f[u] = __ldg(a.xinv + prow + c);
+          else if (!sh) pr[u] = __ldg(rv.pairs + prow + c);
+        }
+      }
+      if (MODE == 1) {
+#pragma unroll
+        for (int u = 0; u < PBN / 32; ++u)
+          if (pr[u] >= 0) f[u] = __ldg(rv.topk_w + pr[u]);
+      }
+      const bool timed = tm && threadIdx.x == kWarpEp0 * 32;
+      if (*abort_flag || !mbar_wait_t(&acc_full[buf], (tc >> 1) & 1, abort_flag, timed ? &tw0 : nullptr)) {
         if (!*abort_flag) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 18); }
         break;
       }
       tc_fence_after();
-      const bool sh = ti.e >= rv.E;
-      const int R = ti.m * PBM + r;                 // row of the expert matrix
-      const int prow = ti.p0 + ti.j * PBN;
       for (int n0 = 0; n0 < ti.nvalid; n0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
-        // per-column factor, loaded once by lane c and broadcast by shuffle:
-        // gate/up the token row's inverse scale, down the gate weight
-        float colf = 1.f;
-        if (lane < 16 && n0 + lane < ti.nvalid) {
-          const int pc = prow + n0 + lane;
-          colf = MODE == 0 ? __ldg(a.xinv + pc) : (sh ? 1.f : __ldg(rv.topk_w + __ldg(rv.pairs + pc)));
-        }
+        const int u0 = n0 >> 5;
+        const float colf = u0 == 0 ? f[0] : u0 == 1 ? f[1] : u0 == 2 ? f[2] : f[3];
         if (MODE == 0) {
           // rows alternate gate / up: lane pairs (2i, 2i+1) hold g and u of row pair i
           const int i = R >> 1;
@@ -373,7 +468,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
           const int ip = (i & ~(G - 1)) | decode_slot(BITS, i & (G - 1));
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float xi = __shfl_sync(0xffffffffu, colf, c);
+            const float xi = __shfl_sync(0xffffffffu, colf, (n0 & 31) + c);
             const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[c]), 1);
             if (((lane & 1) == 0) && n0 + c < ti.nvalid) {
               const float g = __uint_as_float(v[c]) * xi, u = other * xi;
@@ -384,7 +479,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
         } else {
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float w = __shfl_sync(0xffffffffu, colf, c);
+            const float w = __shfl_sync(0xffffffffu, colf, (n0 & 31) + c);
             if (n0 + c < ti.nvalid) a.yout[size_t(prow + n0 + c) * a.out_cols + R] = __uint_as_float(v[c]) * w;
           }
         }
@@ -393,6 +488,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
+    if (tm && threadIdx.x == kWarpEp0 * 32) { tm[7] = tw0; tm[11] = global_ns(); }
   }
 
   // ----------------------------------------------------------- teardown
@@ -400,7 +496,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   __syncthreads();
   if (warp == kWarpMma) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kPTmemCols) : "memory");
   }
 }
 
@@ -630,7 +726,7 @@ cudaError_t launch_gemm(const PrefillArgs& pa, const uint8_t* codes, const uint1
   }
   if (!ok) return cudaErrorInvalidValue;
   constexpr int RAW_STRIDE = (Gm::RAW_BYTES + 1023) / 1024 * 1024;
-  const size_t smem = 1024 + PNK * (kAStageBytes + kBStageBytes) + PNR * RAW_STRIDE + 256;
+  const size_t smem = 1024 + PNK * kBStageBytes + PNR * RAW_STRIDE + kBarBytes + size_t(4 * E + 5) * 4;
   auto kern = prefill_gemm_kernel<MODE, BITS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -638,6 +734,9 @@ cudaError_t launch_gemm(const PrefillArgs& pa, const uint8_t* codes, const uint1
 }
 
 }  // namespace
+
+unsigned long long* g_prefill_timing = nullptr;
+void set_prefill_timing(unsigned long long* buf) { g_prefill_timing = buf; }
 
 bool router_gemm_supported(const moe_config& c, int T) {
   return T > 64 && c.num_experts % PBM == 0 && c.hidden % PBK == 0 && encode_fn() != nullptr;
@@ -694,6 +793,7 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   g.ntoff = reinterpret_cast<const int*>(a.ws + a.L.ntoff);
   g.hout = hs; g.yout = nullptr; g.xinv = xinv;
   g.status = reinterpret_cast<int*>(a.ws + a.L.status);
+  g.timing = g_prefill_timing;
   const bool sh = c.shared_inter > 0;
   err = bits == 4 ? launch_gemm<0, 4>(g, a.w.gate_up_codes, a.w.gate_up_scales, a.w.shared_gate_up_codes,
                                       a.w.shared_gate_up_scales, c.num_experts, sh, xs, P, a.num_sms, a.stream)
@@ -704,6 +804,7 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   PrefillArgs d = g;
   d.K = I; d.rows_pe = H; d.out_cols = H;
   d.hout = nullptr; d.yout = reinterpret_cast<float*>(a.ws + a.L.y);
+  d.timing = g_prefill_timing ? g_prefill_timing + size_t(a.num_sms) * kPTime : nullptr;
   return bits == 4 ? launch_gemm<1, 4>(d, a.w.down_codes, a.w.down_scales, a.w.shared_down_codes,
                                        a.w.shared_down_scales, c.num_experts, sh, hs, P, a.num_sms, a.stream)
                    : launch_gemm<1, 2>(d, a.w.down_codes, a.w.down_scales, a.w.shared_down_codes,
