@@ -52,6 +52,27 @@ def parse():
 
 # ------------------------------------------------------------------ utils ---
 
+def profiled_traffic(profile: str, sources) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or
+    None when the kernel's sources changed since that capture (the summary
+    records the sha256 of the sources it was taken with)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for ln in open(path):
+        if ":" in ln and not ln.startswith(" "):
+            k, v = ln.split(":", 1)
+            fields[k.strip()] = v.strip().split()[0] if v.strip() else ""
+    h = hashlib.sha256()
+    for f in sources:
+        h.update(open(os.path.join(ROOT, "quantized_expert_ffn_moe_b200", "csrc", f), "rb").read())
+    if fields.get("source_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return float(fields["traffic_bytes_per_launch"])
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -324,8 +345,12 @@ def main():
         k_ms = phase_ms[1] / calls
         k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * GU_BYTES[4]
         kname = "ffn_tma_kernel<gate/up>"
+    traffic = profiled_traffic("fused_decode_kernel_decode4_t16.txt",
+                               ["fused.cu", "decode_common.cuh", "moe_internal.cuh"]) if fused else None
     roofline = {"bound": "hbm", "kernel": kname, "achieved": k_bytes / (k_ms * 1e-3) / 1e9,
-                "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": None,
+                "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": traffic,
+                "traffic_source": "profiles/fused_decode_kernel_decode4_t16.txt (ncu dram__bytes_read.sum + "
+                                  "dram__bytes_write.sum, one launch of the same workload)" if traffic else None,
                 "peak_source": f"{peak_src} (copy bandwidth)",
                 "algorithmic_bytes_per_launch": k_bytes, "launch_us": 1000 * k_ms,
                 "phase_us": {"route": 1000 * phase_ms[0] / calls, "gate_up": 1000 * phase_ms[1] / calls,
