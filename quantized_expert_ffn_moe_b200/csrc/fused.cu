@@ -295,7 +295,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
       v[q][z] = __ldcg(reinterpret_cast<const uint4*>(row + (q * 32 + lane) * G + 8 * z));
   float r = 1.f;
   if (stack) {
-    float ss = 0.f;
+    float ss[4] = {0.f, 0.f, 0.f, 0.f};        // four partial sums: short dependency chains
 #pragma unroll
     for (int q = 0; q < NG; ++q)
 #pragma unroll
@@ -304,15 +304,16 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
           const float a = __uint_as_float(w[y] << 16), b = __uint_as_float(w[y] & 0xFFFF0000u);
-          ss = fmaf(a, a, ss);
-          ss = fmaf(b, b, ss);
+          ss[y] = fmaf(a, a, ss[y]);
+          ss[y] = fmaf(b, b, ss[y]);
         }
       }
+    float st = (ss[0] + ss[1]) + (ss[2] + ss[3]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    r = 1.0f / sqrtf(ss / float(K) + 1e-6f);
+    for (int o = 16; o > 0; o >>= 1) st += __shfl_xor_sync(0xffffffffu, st, o);
+    r = 1.0f / sqrtf(st / float(K) + 1e-6f);
   }
-  float vmax = 0.f;
+  float vm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int q = 0; q < NG; ++q)
 #pragma unroll
@@ -320,10 +321,11 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
       const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
-        vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(w[y] << 16) * r)));
-        vmax = fmaxf(vmax, fabsf(round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r)));
+        vm[y] = fmaxf(vm[y], fabsf(round_bf16f(__uint_as_float(w[y] << 16) * r)));
+        vm[y] = fmaxf(vm[y], fabsf(round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r)));
       }
     }
+  float vmax = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
   int sh = 0;
@@ -357,44 +359,52 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
   }
 }
 
-// Router logits of expert e for tokens t0 .. t0+nt-1 from their staged
-// activations (xs holds token t0 first) and the expert's router row already
-// in shared memory: sum_j Wr[e][j] * xs[slot(j)] (exact products), times the
-// token's 2^-sh.
+// Router logits of expert e for tokens t0 .. t0+nt-1 (nt <= kRTok) from their
+// staged activations (xs holds token t0 first) and the expert's router row
+// already in shared memory: sum_j Wr[e][j] * xs[slot(j)] (exact products),
+// times the token's 2^-sh.  The item's tokens run together, each with two
+// partial sums, so the multiply-add chains overlap.
+constexpr int kRTok = 4;
 template <int BITS, int LPR, int CPL>
 __device__ void router_from_staged(const uint16_t* wrow, float bias, const __half* xs, const float* inv_all, int t0,
                                    int nt, float* logit_col, int E, int lane) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);
-  uint4 wv[NG][G / 8];
+  float acc[kRTok][2];
 #pragma unroll
-  for (int q = 0; q < NG; ++q)
+  for (int t = 0; t < kRTok; ++t) acc[t][0] = acc[t][1] = 0.f;
 #pragma unroll
-    for (int z = 0; z < G / 8; ++z) wv[q][z] = *reinterpret_cast<const uint4*>(wrow + (q * 32 + lane) * G + 8 * z);
-  for (int t = 0; t < nt; ++t) {
-    const __half* xt = xs + size_t(t) * K;
-    float acc = 0.f;
+  for (int q = 0; q < NG; ++q) {
+    const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
+    uint4 wv[G / 8];
 #pragma unroll
-    for (int q = 0; q < NG; ++q) {
-      const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
+    for (int z = 0; z < G / 8; ++z) wv[z] = *reinterpret_cast<const uint4*>(wrow + (q * 32 + lane) * G + 8 * z);
+#pragma unroll
+    for (int t = 0; t < kRTok; ++t) {
+      const __half* xt = xs + size_t(t < nt ? t : 0) * K;
       __align__(16) __half xv[G];
 #pragma unroll
       for (int part = 0; part < Gm::NPART; ++part)
         *reinterpret_cast<uint4*>(xv + 8 * part) = *reinterpret_cast<const uint4*>(xt + base + part * LPR * 8);
 #pragma unroll
       for (int z = 0; z < G / 8; ++z) {
-        const uint32_t w[4] = {wv[q][z].x, wv[q][z].y, wv[q][z].z, wv[q][z].w};
+        const uint32_t w[4] = {wv[z].x, wv[z].y, wv[z].z, wv[z].w};
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
           const int j = 8 * z + 2 * y;
-          acc = fmaf(__uint_as_float(w[y] << 16), __half2float(xv[decode_slot(BITS, j)]), acc);
-          acc = fmaf(__uint_as_float(w[y] & 0xFFFF0000u), __half2float(xv[decode_slot(BITS, j + 1)]), acc);
+          acc[t][y & 1] = fmaf(__uint_as_float(w[y] << 16), __half2float(xv[decode_slot(BITS, j)]), acc[t][y & 1]);
+          acc[t][y & 1] = fmaf(__uint_as_float(w[y] & 0xFFFF0000u), __half2float(xv[decode_slot(BITS, j + 1)]),
+                               acc[t][y & 1]);
         }
       }
     }
+  }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) logit_col[size_t(t0 + t) * E] = acc * inv_all[t0 + t] + bias;
+  for (int t = 0; t < kRTok; ++t) {
+    float v = acc[t][0] + acc[t][1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0 && t < nt) logit_col[size_t(t0 + t) * E] = v * inv_all[t0 + t] + bias;
   }
 }
 
@@ -537,7 +547,7 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
   }
 }
 
-constexpr int kRouterTB = 4;          // tokens per router work item
+constexpr int kRouterTB = kRTok;      // tokens per router work item
 
 template <int BITS, int LG, int CG, int LD, int CD, int NPL>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
@@ -646,6 +656,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
           stage_token_all<BITS, LG, CG>(xsrc + size_t(t0 + t) * H, p.stack != 0, xs + size_t(t) * H, &rnorm[t0 + t],
                                         &inv_all[t0 + t], lane);
         all_sync();
+        if (t0 == 0) stamp(l, 14);
         const int nb = (nt + kRouterTB - 1) / kRouterTB;
         for (int it = warp; it < (e1 - e0) * nb; it += kFCons) {
           if (!have_rows) {
@@ -654,6 +665,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
               *abort_flag = 1;
               report_error(status, MOE_ERR_TIMEOUT, 43);
             }
+            stamp(l, 19);
           }
           const int e = e0 + it / nb, b = it % nb;
           const float bias = lw.router_bias ? lw.router_bias[e] : 0.f;
@@ -662,6 +674,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
                                            min(kRouterTB, nt - b * kRouterTB), logits + e, E, lane);
         }
       }
+      stamp(l, 15);
       all_sync();
       stamp(l, 0);
       grid_sync();

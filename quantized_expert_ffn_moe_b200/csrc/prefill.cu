@@ -39,25 +39,28 @@ namespace {
 constexpr int PBM = 128;       // weight rows per tile
 constexpr int PBN = kPrefillTileN;   // tokens per tile (max)
 static_assert(PBN == 128, "the grouping kernel's tile prefix assumes 128 tokens per tile");
-constexpr int PBK = 64;        // k per A/B stage: one 128-byte swizzle row of fp16
+constexpr int PBK = 64;        // k of one 128-byte swizzle row of fp16 (a TMA box; the router GEMM's stage)
+constexpr int PSK = 128;       // grouped GEMM: k per A/B stage (two swizzle atoms, 8 MMAs per barrier)
 constexpr int RAWK = 256;      // k per packed stage
-constexpr int PNK = 8;         // A (tensor memory) / B (shared memory) stages
+constexpr int PNK = 4;         // A (tensor memory) / B (shared memory) stages
 constexpr int PNR = 4;         // packed stages
 constexpr int kWarpRaw = 0, kWarpB = 1, kWarpMma = 2, kWarpDq0 = 3, kNumDq = 8, kWarpEp0 = 11, kNumEp = 4;
 constexpr int kPThreads = (kWarpEp0 + kNumEp) * 32;
 constexpr uint32_t kTmemCols = 2 * PBN;          // router GEMM: two accumulators
 // Grouped GEMM tensor memory: two accumulators of PBN columns, then PNK
-// dequantized A stages of PBK / 2 columns (128 lanes = the tile's rows, two
+// dequantized A stages of PSK / 2 columns (128 lanes = the tile's rows, two
 // fp16 per 32-bit column in k order).
 constexpr uint32_t kAColBase = 2 * PBN;
-constexpr uint32_t kAStageCols = PBK / 2;
+constexpr uint32_t kAStageCols = PSK / 2;
 constexpr uint32_t kPTmemCols = 512;
 static_assert(kAColBase + PNK * kAStageCols <= kPTmemCols, "tensor memory budget");
 // barriers (2 PNR + 2 PNK + 4 of 8 bytes), the TMEM address and the abort flag
 constexpr int kBarBytes = 512;
 static_assert((2 * PNR + 2 * PNK + 4) * 8 + 8 <= kBarBytes, "barrier area");
-constexpr int kAStageBytes = PBM * 128;           // 16 KB
-constexpr int kBStageBytes = PBN * 128;           // 16 KB
+constexpr int kTileTab = 512;      // per-CTA tile table entries (16 B each)
+constexpr int kAStageBytes = PBM * 128;           // 16 KB (router GEMM)
+constexpr int kBStageBytes = PBN * 128;           // 16 KB: one swizzle atom column of the token tile
+constexpr int kGBStageBytes = kBStageBytes * (PSK / PBK);   // grouped GEMM token stage
 
 template <int BITS>
 struct PGeom {
@@ -150,6 +153,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t v[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t v[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // Packed word -> fp16 pairs q * s (q exact from the magic-number decode, one
 // rounding in the multiply).  Pair order as in the decode path: 4-bit
 // (q_j, q_{j+4}), 2-bit (q_j, q_{j+8}).
@@ -213,8 +228,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   using Gm = PGeom<BITS>;
   extern __shared__ __align__(1024) unsigned char psmem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(psmem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* sB = base;                                   // PNK x 16 KB
-  unsigned char* sRaw = sB + PNK * kBStageBytes;              // PNR x RAW_BYTES (1024-aligned each)
+  unsigned char* sB = base;                                   // PNK x 32 KB
+  unsigned char* sRaw = sB + PNK * kGBStageBytes;             // PNR x RAW_BYTES (1024-aligned each)
   constexpr int RAW_STRIDE = (Gm::RAW_BYTES + 1023) / 1024 * 1024;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + PNR * RAW_STRIDE);
   uint64_t* full_raw = bars;
@@ -267,14 +282,39 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   }
   __syncthreads();
   const int ntiles = stab.ntoff[nslots] * mt;
-  const int KB = a.K / PBK, KR = a.K / RAWK;
+  const int KB = a.K / PSK, KR = a.K / RAWK;
+  // this CTA's tiles (t = blockIdx.x + i * gridDim.x) decoded once into a
+  // shared table, read by every role; beyond kTileTab tiles the lookup is redone
+  int4* ttab = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(stab.n + rv.E + 1) + 15) & ~uintptr_t(15));
+  {
+    const int my_tiles = ntiles > int(blockIdx.x) ? (ntiles - int(blockIdx.x) + int(gridDim.x) - 1) / int(gridDim.x) : 0;
+    for (int i = threadIdx.x; i < min(my_tiles, kTileTab); i += blockDim.x) {
+      TileInfo ti;
+      tile_info(stab, nslots, mt, blockIdx.x + i * gridDim.x, &ti);
+      ttab[i] = make_int4(ti.e, ti.p0, (ti.j << 16) | ti.m, ti.nvalid);
+    }
+  }
+  __syncthreads();
+  auto get_tile = [&](int t, TileInfo* ti) {
+    const int i = (t - int(blockIdx.x)) / int(gridDim.x);
+    if (i < kTileTab) {
+      const int4 v = ttab[i];
+      ti->e = v.x;
+      ti->p0 = v.y;
+      ti->j = v.z >> 16;
+      ti->m = v.z & 0xFFFF;
+      ti->nvalid = v.w;
+    } else {
+      tile_info(stab, nslots, mt, t, ti);
+    }
+  };
 
   if (warp == kWarpRaw && lane == 0) {
     // ------------------------------------------------ packed weight producer
     int rc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       TileInfo ti;
-      tile_info(stab, nslots, mt, t, &ti);
+      get_tile(t, &ti);
       const bool sh = ti.e >= rv.E;
       const CUtensorMap* mc = sh ? &tm_sh_codes : &tm_codes;
       const CUtensorMap* ms = sh ? &tm_sh_scales : &tm_scales;
@@ -298,15 +338,17 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     int kc = 0;
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
       TileInfo ti;
-      tile_info(stab, nslots, mt, t, &ti);
+      get_tile(t, &ti);
       const int prow = ti.p0 + ti.j * PBN;
       for (int kb = 0; kb < KB; ++kb, ++kc) {
         const int s = kc % PNK;
         if (kc >= PNK && !mbar_wait_t(&empty_ab[s], ((kc / PNK) - 1) & 1, abort_flag, tm ? &tw0 : nullptr)) {
           *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 12); break;
         }
-        mbar_arrive_expect_tx(&full_a[s], kBStageBytes);
-        tma_load_2d(sB + s * kBStageBytes, &tm_b, kb * PBK, prow, &full_a[s]);
+        mbar_arrive_expect_tx(&full_a[s], kGBStageBytes);
+#pragma unroll
+        for (int h = 0; h < PSK / PBK; ++h)
+          tma_load_2d(sB + s * kGBStageBytes + h * kBStageBytes, &tm_b, kb * PSK + h * PBK, prow, &full_a[s]);
       }
     }
     for (int i = max(0, kc - PNK); i < kc; ++i)
@@ -318,7 +360,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x, ++tc) {
       const long long cti = tm ? clock64() : 0;
       TileInfo ti;
-      tile_info(stab, nslots, mt, t, &ti);
+      get_tile(t, &ti);
       if (tm) tw4 += clock64() - cti;
       const int buf = tc & 1;
       if (tc >= 2 && !mbar_wait_t(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag, tm ? &tw2 : nullptr)) {
@@ -336,10 +378,11 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
         }
         const long long ci = tm ? clock64() : 0;
         tc_fence_after();
-        const uint32_t a0 = tmem_base + kAColBase + uint32_t(s) * kAStageCols, b0 = smem_u32(sB + s * kBStageBytes);
+        const uint32_t a0 = tmem_base + kAColBase + uint32_t(s) * kAStageCols, b0 = smem_u32(sB + s * kGBStageBytes);
 #pragma unroll
-        for (int k = 0; k < PBK / 16; ++k)
-          tc_mma_ta(d_tmem, a0 + uint32_t(k * 8), sw128_desc(b0 + k * 32), idesc, (kb | k) ? 1u : 0u);
+        for (int k = 0; k < PSK / 16; ++k)
+          tc_mma_ta(d_tmem, a0 + uint32_t(k * 8), sw128_desc(b0 + (k >> 2) * kBStageBytes + (k & 3) * 32), idesc,
+                    (kb | k) ? 1u : 0u);
         tc_commit(&empty_ab[s]);
         if (tm) tw3 += clock64() - ci;
       }
@@ -355,8 +398,9 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     // warp w writes rows of its tensor-memory lane quarter (w % 4); the two
     // warps of a quarter take the first and second half of a packed stage
     const int r = (warp & 3) * 32 + lane;          // tile row
-    const int half = (warp - kWarpDq0) >> 2;       // which two of the four k-blocks of a packed stage
+    const int half = (warp - kWarpDq0) >> 2;       // which of the two A stages of a packed stage
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    static_assert(RAWK == 2 * PSK, "a packed stage feeds two A stages, one per dequant half");
     int rc = 0, kc = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
       for (int rs = 0; rs < KR; ++rs, ++rc) {
@@ -365,17 +409,19 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
         bool ok = !*abort_flag && mbar_wait_t(&full_raw[s], (rc / PNR) & 1, abort_flag, timed ? &tw0 : nullptr);
         const unsigned char* raw = sRaw + s * RAW_STRIDE;
         const unsigned char* sc = raw + Gm::SCALE_OFF;
-        for (int jj = 0; jj < 2; ++jj) {
-          const int kbl = half * 2 + jj;            // k-block within the packed stage (0..3)
-          const int kglob = kc + kbl;               // global k-block counter of this A/B stage
-          const int as = kglob % PNK;
-          if (ok && kglob >= PNK) ok = mbar_wait_t(&empty_ab[as], ((kglob / PNK) - 1) & 1, abort_flag, timed ? &tw1 : nullptr);
-          ok = __all_sync(0xffffffffu, ok);         // the tensor-memory store is warp-wide
-          if (ok) {
-            tc_fence_after();
-            uint32_t o32[32];                       // the row's 64 fp16 of this k-block, in k order
+        const int kglob = kc + half;                // global counter of this thread's A/B stage
+        const int as = kglob % PNK;
+        if (ok && kglob >= PNK) ok = mbar_wait_t(&empty_ab[as], ((kglob / PNK) - 1) & 1, abort_flag, timed ? &tw1 : nullptr);
+        ok = __all_sync(0xffffffffu, ok);           // the tensor-memory store is warp-wide
+        if (ok) {
+          tc_fence_after();
+          // the row's 128 fp16 of this A stage, in k order, in two 64-column halves
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            const int kbl = half * 2 + hb;          // 64-k block within the packed stage (0..3)
+            uint32_t o32[32];
             if (BITS == 4) {
-              // row r: 2 x 16 bytes of codes = 64 weights, 2 scales
+              // 2 x 16 bytes of codes = 64 weights, 2 scales
 #pragma unroll
               for (int cc = 0; cc < 2; ++cc) {
                 const int lc = kbl * 2 + cc;                     // logical 16-B chunk in the 128-B row
@@ -387,10 +433,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
                 for (int q = 0; q < 4; ++q) dq4_f16(wd[q], s2, o32 + (cc * 4 + q) * 4);
               }
             } else {
-              // row r: 16 bytes of codes = 64 weights in 4 words, 4 scales
+              // 16 bytes of codes = 64 weights in 4 words, 4 scales
               const int lc = kbl;                                // logical 16-B chunk in the 64-B row
               const uint4 w = *reinterpret_cast<const uint4*>(raw + r * Gm::IB + ((lc ^ ((r >> 1) & 3)) << 4));
-              const int sci = kbl * 4;                           // first scale of this k-block (of 16 per row)
+              const int sci = kbl * 4;                           // first scale of this block (of 16 per row)
               const int schunk = sci >> 3;                       // logical 16-B chunk of the 32-B scale row
               const uint4 sv = *reinterpret_cast<const uint4*>(sc + r * Gm::SB + ((schunk ^ ((r >> 2) & 1)) << 4));
               const uint32_t svw[4] = {sv.x, sv.y, sv.z, sv.w};
@@ -404,17 +450,17 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
                 dq2_f16(wd[q], s2, o32 + q * 8);
               }
             }
-            tmem_st32(tmem_base + lane_base + kAColBase + uint32_t(as) * kAStageCols, o32);
-            tmem_st_wait();
-            tc_fence_before();
+            tmem_st32(tmem_base + lane_base + kAColBase + uint32_t(as) * kAStageCols + uint32_t(hb * 32), o32);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_a[as]);
+          tmem_st_wait();
+          tc_fence_before();
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full_a[as]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_raw[s]);
         if (!ok && !*abort_flag) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 17); }
-        kc += 4;
+        kc += 2;
       }
     }
     if (tm && threadIdx.x == kWarpDq0 * 32) { tm[5] = tw0; tm[6] = tw1; }
@@ -422,68 +468,93 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                         // TMEM lane quarter of this warp
     const int r = q * 32 + lane;                    // tile row
-    int tc = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
-      TileInfo ti;
-      tile_info(stab, nslots, mt, t, &ti);
-      const int buf = tc & 1;
-      const bool sh = ti.e >= rv.E;
-      const int R = ti.m * PBM + r;                 // row of the expert matrix
-      const int prow = ti.p0 + ti.j * PBN;
-      // per-column factors of the tile (gate/up: the token row's inverse
-      // scale, down: the gate weight), column u*32 + lane in f[u], loaded
-      // before the accumulator wait so the latency overlaps it
-      float f[PBN / 32];
-      int pr[PBN / 32];
+    // per-column factors of a tile (gate/up: the token row's inverse scale,
+    // down: the gate weight), column u*32 + lane in f[u].  They are fetched
+    // one tile ahead (down: the pair ids while the current tile's columns are
+    // written, the gate weights after), so their latency overlaps the work.
+    auto first_level = [&](const TileInfo& tn, float fo[PBN / 32], int po[PBN / 32]) {
+      const int prn = tn.p0 + tn.j * PBN;
+      const bool shn = tn.e >= rv.E;
 #pragma unroll
       for (int u = 0; u < PBN / 32; ++u) {
         const int c = u * 32 + lane;
-        f[u] = 1.f;
-        pr[u] = -1;
-        if (c < ti.nvalid) {
-          if (MODE == 0) f[u] = __ldg(a.xinv + prow + c);
-          else if (!sh) pr[u] = __ldg(rv.pairs + prow + c);
+        fo[u] = 1.f;
+        po[u] = -1;
+        if (c < tn.nvalid) {
+          if (MODE == 0) fo[u] = __ldg(a.xinv + prn + c);
+          else if (!shn) po[u] = __ldg(rv.pairs + prn + c);
         }
       }
+    };
+    auto second_level = [&](float fo[PBN / 32], const int po[PBN / 32]) {
       if (MODE == 1) {
 #pragma unroll
         for (int u = 0; u < PBN / 32; ++u)
-          if (pr[u] >= 0) f[u] = __ldg(rv.topk_w + pr[u]);
+          if (po[u] >= 0) fo[u] = __ldg(rv.topk_w + po[u]);
       }
+    };
+    int tc = 0;
+    TileInfo ti_n;
+    float f_n[PBN / 32];
+    int pr_n[PBN / 32];
+    if (blockIdx.x < ntiles) {
+      get_tile(blockIdx.x, &ti_n);
+      first_level(ti_n, f_n, pr_n);
+      second_level(f_n, pr_n);
+    }
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+      const TileInfo ti = ti_n;
+      float f[PBN / 32];
+#pragma unroll
+      for (int u = 0; u < PBN / 32; ++u) f[u] = f_n[u];
+      const int buf = tc & 1;
+      const int R = ti.m * PBM + r;                 // row of the expert matrix
+      const int prow = ti.p0 + ti.j * PBN;
       const bool timed = tm && threadIdx.x == kWarpEp0 * 32;
       if (*abort_flag || !mbar_wait_t(&acc_full[buf], (tc >> 1) & 1, abort_flag, timed ? &tw0 : nullptr)) {
         if (!*abort_flag) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 18); }
         break;
       }
+      const bool more = t + int(gridDim.x) < ntiles;
+      if (more) {
+        get_tile(t + gridDim.x, &ti_n);
+        first_level(ti_n, f_n, pr_n);
+      }
       tc_fence_after();
-      for (int n0 = 0; n0 < ti.nvalid; n0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
+      for (int n0 = 0; n0 < ti.nvalid; n0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
         const int u0 = n0 >> 5;
         const float colf = u0 == 0 ? f[0] : u0 == 1 ? f[1] : u0 == 2 ? f[2] : f[3];
         if (MODE == 0) {
-          // rows alternate gate / up: lane pairs (2i, 2i+1) hold g and u of row pair i
+          // rows alternate gate / up: lane pairs (2i, 2i+1) hold g and u of row
+          // pair i.  For columns (c, c+1) the even lane takes column c and the
+          // odd lane column c+1 (one exchange), so both lanes do the SwiGLU.
           const int i = R >> 1;
           const int G = Gm::G;
           const int ip = (i & ~(G - 1)) | decode_slot(BITS, i & (G - 1));
+          const int odd = lane & 1;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float xi = __shfl_sync(0xffffffffu, colf, (n0 & 31) + c);
-            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[c]), 1);
-            if (((lane & 1) == 0) && n0 + c < ti.nvalid) {
-              const float g = __uint_as_float(v[c]) * xi, u = other * xi;
-              const float hval = g / (1.f + expf(-g)) * u;
-              a.hout[size_t(prow + n0 + c) * a.out_cols + ip] = __half_as_ushort(__float2half_rn(hval));
+          for (int c = 0; c < 32; c += 2) {
+            const float mine = __uint_as_float(v[c + odd]);
+            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(v[c + 1 - odd]), 1);
+            const int col = c + odd;
+            const float xi = __shfl_sync(0xffffffffu, colf, col);
+            if (n0 + col < ti.nvalid) {
+              const float g = (odd ? other : mine) * xi, u = (odd ? mine : other) * xi;
+              const float hval = __fdividef(g * u, 1.f + __expf(-g));
+              a.hout[size_t(prow + n0 + col) * a.out_cols + ip] = __half_as_ushort(__float2half_rn(hval));
             }
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float w = __shfl_sync(0xffffffffu, colf, (n0 & 31) + c);
+          for (int c = 0; c < 32; ++c) {
+            const float w = __shfl_sync(0xffffffffu, colf, c);
             if (n0 + c < ti.nvalid) a.yout[size_t(prow + n0 + c) * a.out_cols + R] = __uint_as_float(v[c]) * w;
           }
         }
       }
+      if (more) second_level(f_n, pr_n);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -726,7 +797,8 @@ cudaError_t launch_gemm(const PrefillArgs& pa, const uint8_t* codes, const uint1
   }
   if (!ok) return cudaErrorInvalidValue;
   constexpr int RAW_STRIDE = (Gm::RAW_BYTES + 1023) / 1024 * 1024;
-  const size_t smem = 1024 + PNK * kBStageBytes + PNR * RAW_STRIDE + kBarBytes + size_t(4 * E + 5) * 4;
+  const size_t smem = 1024 + PNK * kGBStageBytes + PNR * RAW_STRIDE + kBarBytes + size_t(4 * E + 5) * 4 + 16 +
+                      size_t(kTileTab) * 16;
   auto kern = prefill_gemm_kernel<MODE, BITS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
