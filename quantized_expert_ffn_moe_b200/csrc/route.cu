@@ -426,17 +426,21 @@ __global__ void __launch_bounds__(32) chunk_scatter_kernel(const int* __restrict
                                                            const int* __restrict__ chunk_base,
                                                            const int* __restrict__ offsets, int* __restrict__ pairs,
                                                            int* __restrict__ inv, int* __restrict__ api_pairs) {
-  extern __shared__ int cur[];
+  extern __shared__ int cur[];                 // [E] fill cursors, then the chunk's ids
+  int* cidx = cur + E;                         // [kGroupChunk * k]
   pdl_wait();
   pdl_launch_dependents();
   const int lane = threadIdx.x;
+  const int t0 = blockIdx.x * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
+  // the chunk's selections in one coalesced pass, so the ordered walk below
+  // reads shared memory instead of waiting on a global load per token
+  for (int q = t0 * k + lane; q < t1 * k; q += 32) cidx[q - t0 * k] = idx[q];
   for (int e = lane; e < E; e += 32) cur[e] = offsets[e] + chunk_base[size_t(blockIdx.x) * E + e];
   __syncwarp();
-  const int t0 = blockIdx.x * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
   for (int t = t0; t < t1; ++t) {
     if (lane < k) {
       const int q = t * k + lane;
-      const int e = idx[q];
+      const int e = cidx[q - t0 * k];
       if (e >= 0 && e < E) {
         const int pos = cur[e]++;     // distinct experts within one token
         pairs[pos] = q;
@@ -478,7 +482,8 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
                        reinterpret_cast<int*>(ws + L.woff_gu), reinterpret_cast<int*>(ws + L.woff_dn),
                        reinterpret_cast<int*>(ws + L.ntoff));
       if (err != cudaSuccess) return err;
-      return launch_pdl(chunk_scatter_kernel, dim3(nch), dim3(32), size_t(E) * 4, s, (const int*)idx, T, c.top_k, E,
+      return launch_pdl(chunk_scatter_kernel, dim3(nch), dim3(32), size_t(E + kGroupChunk * c.top_k) * 4, s,
+                        (const int*)idx, T, c.top_k, E,
                         (const int*)hist, (const int*)(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
                         reinterpret_cast<int*>(ws + L.inv), api_pairs);
     }
