@@ -319,3 +319,32 @@ def test_prefill_path_without_shared_expert():
     if differ:
         r = _oracle_given(gc.host_oracle_layer(shape, 6, 0, cache_size=40), x, idx, differ)
     gc.assert_close(y, r["out"])
+
+
+def _sampled_full_case(shape, T, batch, seed, n_sample, sample_seed):
+    """Full-shape layer at T tokens, checked on a seeded sample of tokens
+    against the live oracle (tokens are independent in one layer)."""
+    x = mi.hidden_states_bf16(T, shape.hidden, seed, batch)
+    w = gc.device_layer(shape, seed, 0)
+    y = gc.run_layer(shape, w, x)
+    idx = gc.run_route(shape, w, x)[0]
+    sel = np.sort(np.random.default_rng(sample_seed).choice(T, size=n_sample, replace=False))
+    lay = gc.host_oracle_layer(shape, seed, 0, cache_size=8)
+    r = orc.layer_forward(lay, x[sel])
+    differ = gc.check_selection(r["logits"], r["idx"], idx[sel], shape.top_k)
+    ref = r["out"].copy()
+    for i in differ:
+        ref[i] = orc.layer_forward(lay, x[sel[i]:sel[i] + 1], topk_override={0: idx[sel[i]]})["out"][0]
+    gc.assert_close(y[sel], ref)
+
+
+def test_layer_full4_decode_unstaged_chunks():
+    # 40 tokens do not fit the fused decode kernel's once-per-layer token
+    # staging, so gate/up stages its tokens per slot chunk and per consumer group
+    _sampled_full_case(mi.FULL4, 40, 3, 0, 4, 40)
+
+
+def test_prefill_full4_large_batch_tile_lookup():
+    # 60,000 tokens: more tiles per CTA than the per-CTA tile table holds (the
+    # down pass falls back to the per-tile lookup) and the chunked grouping at scale
+    _sampled_full_case(mi.FULL4, 60000, 4, 0, 4, 60000)
