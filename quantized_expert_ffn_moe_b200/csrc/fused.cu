@@ -519,21 +519,69 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
   }
 }
 
+// Completion publishing of gate/up stages, run by the producer thread: it
+// learns that a stage was consumed when it waits for the stage's ring slot
+// (the consumers' mbarrier arrivals release their h stores to it), and adds
+// the finished stages of each expert slot to gdone[slot] after a gpu-scope
+// fence, batched per slot, so no consumer warp stalls on a fence.
+// The last slot is flushed as soon as the CTA's last gate/up stage is
+// confirmed: holding it until the end would wait on down stages whose
+// consumers wait for this very count.
+struct Publisher {
+  int* gdone;
+  int rslot[kFStages];     // expert slot of the stage in each ring slot, -1 = not a gate/up stage
+  int acc_slot, acc_cnt;
+  int pending;             // gate/up stages issued, not yet confirmed
+  bool all_issued;         // the gate/up pass has issued its last stage
+
+  __device__ void reset() {
+    for (int r = 0; r < kFStages; ++r) rslot[r] = -1;
+    acc_slot = -1;
+    acc_cnt = 0;
+    pending = 0;
+    all_issued = false;
+  }
+  __device__ void issued_all() {
+    all_issued = true;
+    if (pending == 0) flush();
+  }
+  __device__ void flush() {
+    if (acc_cnt > 0) {
+      __threadfence();
+      atomicAdd(&gdone[acc_slot], acc_cnt);
+    }
+    acc_cnt = 0;
+  }
+  // the stage that occupied ring slot r has been consumed
+  __device__ void consumed(int r) {
+    const int u = rslot[r];
+    rslot[r] = -1;
+    if (u < 0) return;
+    if (u != acc_slot) { flush(); acc_slot = u; }
+    ++acc_cnt;
+    if (--pending == 0 && all_issued) flush();
+  }
+};
+
 // Producer side of one pass: issues this CTA's stages into the ring.
 template <int BITS, int LPR, int CPL>
 __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, const uint16_t* scales,
                              const uint8_t* sh_codes, const uint16_t* sh_scales, size_t expert_code_bytes,
                              size_t expert_scale_count, unsigned char* ring, int ring_stride, uint64_t* full,
-                             uint64_t* empty, int* issued, volatile int* abort_flag, int* status) {
+                             uint64_t* empty, int* issued, volatile int* abort_flag, int* status, Publisher& pub,
+                             bool gate_up) {
   using Gm = Geom<BITS, LPR, CPL>;
   for (; cur.valid(w1); cur.advance()) {
     const int i = *issued;
     const int slot = i % kFStages;
     if (*abort_flag) return;
-    if (i >= kFStages && !mbar_wait(&empty[slot], ((i / kFStages) - 1) & 1, abort_flag)) {
-      *abort_flag = 1;
-      report_error(status, MOE_ERR_TIMEOUT, 42);
-      return;
+    if (i >= kFStages) {
+      if (!mbar_wait(&empty[slot], ((i / kFStages) - 1) & 1, abort_flag)) {
+        *abort_flag = 1;
+        report_error(status, MOE_ERR_TIMEOUT, 42);
+        return;
+      }
+      pub.consumed(slot);
     }
     const bool sh = cur.e >= cur.E;
     const uint8_t* cb = sh ? sh_codes : codes + size_t(cur.e) * expert_code_bytes;
@@ -543,8 +591,25 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
     mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + Gm::SCALE_BYTES);
     bulk_g2s(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot]);
     bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * Gm::SPR, Gm::SCALE_BYTES, &full[slot]);
+    pub.rslot[slot] = gate_up ? cur.slot : -1;
+    if (gate_up) ++pub.pending;
     *issued = i + 1;
   }
+}
+
+// After the CTA's last stage is issued: waits (bounded) for the stages still
+// in the ring and publishes the gate/up ones.
+__device__ void drain_publish(int issued, uint64_t* empty, volatile int* abort_flag, int* status, Publisher& pub) {
+  for (int j = max(0, issued - kFStages); j < issued; ++j) {
+    const int slot = j % kFStages;
+    if (pub.rslot[slot] < 0) continue;
+    if (*abort_flag || !mbar_wait(&empty[slot], (j / kFStages) & 1, abort_flag)) {
+      if (!*abort_flag) { *abort_flag = 1; report_error(status, MOE_ERR_TIMEOUT, 45); }
+      return;
+    }
+    pub.consumed(slot);
+  }
+  pub.flush();
 }
 
 constexpr int kRouterTB = kRTok;      // tokens per router work item
@@ -592,6 +657,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   float* logits = reinterpret_cast<float*>(ws + p.L_.logits);
   float* hbuf = reinterpret_cast<float*>(ws + p.L_.h);
   float* ybuf = reinterpret_cast<float*>(ws + p.L_.y);
+  int* gdone = reinterpret_cast<int*>(ws + p.L_.gdone);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool producer = warp == kFCons;
@@ -648,6 +714,11 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       // the router logits of this CTA's experts over each chunk: work items
       // of (expert, kRouterTB tokens) spread over all consumer warps
       for (int e = threadIdx.x; e < E; e += kFCons * 32) rt.cnt[e] = 0;
+      {
+        // this CTA's share of the per-slot gate/up completion counters
+        const int z0 = int((long long)(E + 2) * blockIdx.x / G), z1 = int((long long)(E + 2) * (blockIdx.x + 1) / G);
+        for (int u = z0 + threadIdx.x; u < z1; u += kFCons * 32) gdone[u] = 0;
+      }
       bool have_rows = false;
       for (int t0 = 0; t0 < T; t0 += p.rtc) {
         const int nt = min(p.rtc, T - t0);
@@ -792,19 +863,24 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
 
     if (producer) {
       if (lane == 0) {
+        Publisher pub;
+        pub.gdone = gdone;
+        pub.reset();
         if (g0 < g1) {
           cg.init(g0);
           produce_pass<BITS, LG, CG>(cg, g1, lw.gate_up_codes, lw.gate_up_scales, lw.shared_gate_up_codes,
                                       lw.shared_gate_up_scales, size_t(2 * I) * H * c.bits / 8,
                                       size_t(2 * I) * (H / c.block), ring, RING_STRIDE, full, empty, &issued,
-                                      abort_flag, status);
+                                      abort_flag, status, pub, true);
         }
+        pub.issued_all();
         if (d0 < d1) {
           cd.init(d0);
           produce_pass<BITS, LD, CD>(cd, d1, lw.down_codes, lw.down_scales, lw.shared_down_codes,
                                       lw.shared_down_scales, size_t(H) * I * c.bits / 8, size_t(H) * (I / c.block),
-                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status);
+                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false);
         }
+        drain_publish(issued, empty, abort_flag, status, pub);
       }
     } else {
       // ---------------------------------------------------------- phase G
@@ -817,17 +893,35 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       }
       all_sync();
       stamp(l, 3);
-      grid_sync();
-      stamp(l, 4);
       // ---------------------------------------------------------- phase D
+      // no grid barrier: the CTA waits only until every slot of its down range
+      // has all its gate/up stages published (any CTA may have computed them)
       if (d0 < d1) {
         cd.init(d0);
         // the CTA's stages cover one contiguous range of routed positions:
         // when it fits, all its h rows are staged at once by every warp
         FCursor cw = cd;
         const int lo = cw.p0 + cw.chunk * cw.ntc;
-        int hi = lo;
-        for (; cw.valid(d1); cw.advance()) hi = max(hi, cw.p0 + cw.chunk * cw.ntc + cw.nc);
+        const int s_first = cw.slot;
+        int hi = lo, s_last = cw.slot;
+        for (; cw.valid(d1); cw.advance()) {
+          hi = max(hi, cw.p0 + cw.chunk * cw.ntc + cw.nc);
+          s_last = cw.slot;
+        }
+        for (int u = s_first + threadIdx.x; u <= s_last; u += kFCons * 32) {
+          const int e = rt.ulist[u];
+          const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+          const unsigned need = unsigned((2 * I / GU::RPS) * ((n + p.ntc_gu - 1) / p.ntc_gu));
+          const long long t0 = clock64();
+          while (ld_acquire_u32(reinterpret_cast<const unsigned*>(gdone + u)) < need) {
+            if (*abort_flag || clock64() - t0 > kWaitLimitCycles) {
+              if (!*abort_flag) { *abort_flag = 1; report_error(status, MOE_ERR_TIMEOUT, 44); }
+              break;
+            }
+          }
+        }
+        all_sync();
+        stamp(l, 4);
         const bool dpre = hi - lo <= kMaxNTC && size_t(hi - lo) * DN::K <= p.xs_halves;
         if (dpre) {
           for (int r = warp; r < hi - lo; r += kFCons) {

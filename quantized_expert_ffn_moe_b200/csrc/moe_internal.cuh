@@ -30,7 +30,7 @@ constexpr int kGroupChunk = 64;
 
 struct Layout {
   size_t status, logits, topk_idx, topk_w, counts, offsets, pairs, inv, ulist, woff_gu, woff_dn, ntoff, xhat, h,
-      y, xs, xscale, chunk_hist, total;
+      y, xs, xscale, chunk_hist, gdone, total;
   int P;
 };
 
@@ -60,6 +60,7 @@ inline Layout make_layout(const moe_config& c, int T) {
   L.xs = take(size_t(P) * c.hidden * 2);
   L.xscale = take(size_t(P) * 4);
   L.chunk_hist = take(size_t((T + kGroupChunk - 1) / kGroupChunk) * c.num_experts * 4);
+  L.gdone = take(size_t(c.num_experts + 2) * 4);   // fused decode: gate/up stages finished per slot
   L.total = o;
   L.P = P;
   return L;
