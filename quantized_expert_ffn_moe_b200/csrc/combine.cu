@@ -19,8 +19,9 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
   pdl_wait();
   const int t = blockIdx.x;
   const int P_routed = T * k;
-  int pos[16];
-  for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+  __shared__ int pos[16];
+  if (threadIdx.x < k) pos[threadIdx.x] = inv[t * k + threadIdx.x];
+  __syncthreads();
   float ss = 0.f;
   constexpr int VPT = 8;                      // elements per thread per step
   for (int h0 = threadIdx.x * VPT; h0 < H; h0 += kCombThreads * VPT) {
@@ -42,7 +43,6 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
     uint16_t* dst = out + size_t(t) * H + h0;
-    uint16_t ob[VPT];
     if (residual) {
       const uint4 xv = *reinterpret_cast<const uint4*>(dst);
       const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -52,14 +52,15 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
         acc[2 * i + 1] += __uint_as_float(xw[i] & 0xFFFF0000u);
       }
     }
+    const uint4 ov = pack_bf16x8(acc);
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const __nv_bfloat16 b = __float2bfloat16_rn(acc[i]);
-      ob[i] = *reinterpret_cast<const uint16_t*>(&b);
-      const float r = __bfloat162float(b);
-      ss = fmaf(r, r, ss);
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(ow[i] << 16), hi = __uint_as_float(ow[i] & 0xFFFF0000u);
+      ss = fmaf(lo, lo, ss);
+      ss = fmaf(hi, hi, ss);
     }
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob);
+    *reinterpret_cast<uint4*>(dst) = ov;
   }
   if (xhat_next) {
     __shared__ float red[kCombThreads / 32];
@@ -73,15 +74,13 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     for (int h0 = threadIdx.x * VPT; h0 < H; h0 += kCombThreads * VPT) {
       const uint4 xv = *reinterpret_cast<const uint4*>(out + size_t(t) * H + h0);
       const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-      uint16_t hb[VPT];
+      float hv[VPT];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat16 lo = __float2bfloat16_rn(__uint_as_float(xw[i] << 16) * r);
-        const __nv_bfloat16 hi = __float2bfloat16_rn(__uint_as_float(xw[i] & 0xFFFF0000u) * r);
-        hb[2 * i] = *reinterpret_cast<const uint16_t*>(&lo);
-        hb[2 * i + 1] = *reinterpret_cast<const uint16_t*>(&hi);
+        hv[2 * i] = __uint_as_float(xw[i] << 16) * r;
+        hv[2 * i + 1] = __uint_as_float(xw[i] & 0xFFFF0000u) * r;
       }
-      *reinterpret_cast<uint4*>(xhat_next + size_t(t) * H + h0) = *reinterpret_cast<const uint4*>(hb);
+      *reinterpret_cast<uint4*>(xhat_next + size_t(t) * H + h0) = pack_bf16x8(hv);
     }
   }
   pdl_launch_dependents();

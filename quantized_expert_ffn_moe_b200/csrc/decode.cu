@@ -243,13 +243,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
               v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
             }
           }
-          __align__(16) __half hv[Gm::G];
-#pragma unroll
-          for (int j = 0; j < Gm::G; ++j) hv[decode_slot(BITS, j)] = __float2half_rn(v[j] * mul);
+          uint4 parts[Gm::NPART];
+          pack_pair_order<Gm::G>(v, mul, parts);
           const int base = staged_offset<BITS, LPR, CPL>(g0);
 #pragma unroll
-          for (int part = 0; part < Gm::NPART; ++part)
-            *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+          for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
         }
         if (lane == 0) {
           tok_inv[tl] = ldexpf(1.f, -sh);

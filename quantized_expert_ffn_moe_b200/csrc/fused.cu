@@ -200,13 +200,11 @@ __device__ void stage_h_row(const float* hrow, __half* dst, float* inv_out, int 
       const float4 u = __ldcg(reinterpret_cast<const float4*>(hrow + g0 + 4 * q));
       v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
     }
-    __align__(16) __half hv[Gm::G];
-#pragma unroll
-    for (int j = 0; j < Gm::G; ++j) hv[decode_slot(BITS, j)] = __float2half_rn(v[j] * mul);
+    uint4 parts[Gm::NPART];
+    pack_pair_order<Gm::G>(v, mul, parts);
     const int base = staged_offset<BITS, LPR, CPL>(g0);
 #pragma unroll
-    for (int part = 0; part < Gm::NPART; ++part)
-      *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+    for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
   }
   if (lane == 0) *inv_out = ldexpf(1.f, -sh);
 }
@@ -266,13 +264,11 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
           v[8 * q + 2 * z + 1] = round_bf16f(__uint_as_float(wd[z] & 0xFFFF0000u) * rn);
         }
       }
-      __align__(16) __half hv[Gm::G];
-#pragma unroll
-      for (int j = 0; j < Gm::G; ++j) hv[decode_slot(BITS, j)] = __float2half_rn(v[j] * mul);
+      uint4 parts[Gm::NPART];
+      pack_pair_order<Gm::G>(v, mul, parts);
       const int base = staged_offset<BITS, LPR, CPL>(g0);
 #pragma unroll
-      for (int part = 0; part < Gm::NPART; ++part)
-        *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+      for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
     }
     if (lane == 0) tok_inv[tl] = ldexpf(1.f, -sh);
   }
@@ -337,21 +333,21 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
   const float mul = ldexpf(1.f, sh);
 #pragma unroll
   for (int q = 0; q < NG; ++q) {
-    __align__(16) __half hv[G];
+    float vf[G];
 #pragma unroll
     for (int z = 0; z < G / 8; ++z) {
       const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
-        const int j = 8 * z + 2 * y;
-        hv[decode_slot(BITS, j)] = __float2half_rn(round_bf16f(__uint_as_float(w[y] << 16) * r) * mul);
-        hv[decode_slot(BITS, j + 1)] = __float2half_rn(round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r) * mul);
+        vf[8 * z + 2 * y] = round_bf16f(__uint_as_float(w[y] << 16) * r);
+        vf[8 * z + 2 * y + 1] = round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r);
       }
     }
+    uint4 parts[Gm::NPART];
+    pack_pair_order<G>(vf, mul, parts);
     const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
 #pragma unroll
-    for (int part = 0; part < Gm::NPART; ++part)
-      *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = *reinterpret_cast<const uint4*>(hv + 8 * part);
+    for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
   }
   if (lane == 0) {
     *rnorm_out = r;
@@ -362,10 +358,9 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
 // Router logits of expert e for tokens t0 .. t0+nt-1 (nt <= kRTok) from their
 // staged activations (xs holds token t0 first) and the expert's router row
 // already in shared memory: sum_j Wr[e][j] * xs[slot(j)] (exact products),
-// times the token's 2^-sh.  The item's tokens run together, each with two
-// partial sums, so the multiply-add chains overlap.
-constexpr int kRTok = 4;
-template <int BITS, int LPR, int CPL>
+// times the token's 2^-sh.  The tokens run together, each with two partial
+// sums, so the multiply-add chains overlap.
+template <int BITS, int LPR, int CPL, int kRTok>
 __device__ void router_from_staged(const uint16_t* wrow, float bias, const __half* xs, const float* inv_all, int t0,
                                    int nt, float* logit_col, int E, int lane) {
   using Gm = Geom<BITS, LPR, CPL>;
@@ -376,26 +371,33 @@ __device__ void router_from_staged(const uint16_t* wrow, float bias, const __hal
 #pragma unroll
   for (int q = 0; q < NG; ++q) {
     const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
-    uint4 wv[G / 8];
+    // router weights of the group (k order) as fp32
+    float wf[G];
 #pragma unroll
-    for (int z = 0; z < G / 8; ++z) wv[z] = *reinterpret_cast<const uint4*>(wrow + (q * 32 + lane) * G + 8 * z);
+    for (int z = 0; z < G / 8; ++z) {
+      const uint4 u = *reinterpret_cast<const uint4*>(wrow + (q * 32 + lane) * G + 8 * z);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        wf[8 * z + 2 * y] = __uint_as_float(w[y] << 16);
+        wf[8 * z + 2 * y + 1] = __uint_as_float(w[y] & 0xFFFF0000u);
+      }
+    }
 #pragma unroll
     for (int t = 0; t < kRTok; ++t) {
       const __half* xt = xs + size_t(t < nt ? t : 0) * K;
-      __align__(16) __half xv[G];
+      // staged word i holds elements (i, i + G/2) of the group
+      uint32_t xw[G / 2];
 #pragma unroll
-      for (int part = 0; part < Gm::NPART; ++part)
-        *reinterpret_cast<uint4*>(xv + 8 * part) = *reinterpret_cast<const uint4*>(xt + base + part * LPR * 8);
+      for (int part = 0; part < Gm::NPART; ++part) {
+        const uint4 u = *reinterpret_cast<const uint4*>(xt + base + part * LPR * 8);
+        xw[4 * part] = u.x; xw[4 * part + 1] = u.y; xw[4 * part + 2] = u.z; xw[4 * part + 3] = u.w;
+      }
 #pragma unroll
-      for (int z = 0; z < G / 8; ++z) {
-        const uint32_t w[4] = {wv[z].x, wv[z].y, wv[z].z, wv[z].w};
-#pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          const int j = 8 * z + 2 * y;
-          acc[t][y & 1] = fmaf(__uint_as_float(w[y] << 16), __half2float(xv[decode_slot(BITS, j)]), acc[t][y & 1]);
-          acc[t][y & 1] = fmaf(__uint_as_float(w[y] & 0xFFFF0000u), __half2float(xv[decode_slot(BITS, j + 1)]),
-                               acc[t][y & 1]);
-        }
+      for (int i = 0; i < G / 2; ++i) {
+        const float2 f = __half22float2(u32_as_h2(xw[i]));
+        acc[t][i & 1] = fmaf(wf[i], f.x, acc[t][i & 1]);
+        acc[t][i & 1] = fmaf(wf[i + G / 2], f.y, acc[t][i & 1]);
       }
     }
   }
@@ -612,8 +614,6 @@ __device__ void drain_publish(int issued, uint64_t* empty, volatile int* abort_f
   pub.flush();
 }
 
-constexpr int kRouterTB = kRTok;      // tokens per router work item
-
 template <int BITS, int LG, int CG, int LD, int CD, int NPL>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
   using GU = Geom<BITS, LG, CG>;
@@ -709,10 +709,11 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         }
       }
     } else {
-      // tokens staged (RMSNorm factor in the stack, fp16 xhat with its
-      // power-of-two scale) in chunks of rtc, identical in every CTA, and
-      // the router logits of this CTA's experts over each chunk: work items
-      // of (expert, kRouterTB tokens) spread over all consumer warps
+      // one warp per token: it stages the token (RMSNorm factor in the stack,
+      // fp16 xhat with its power-of-two scale) -- into the token region, where
+      // it stays for gate/up, or, when the tokens do not all fit, into its own
+      // row of the idle ring slots 1-2 -- and at once computes the token's
+      // router logits for this CTA's experts from their rows in ring slot 0
       for (int e = threadIdx.x; e < E; e += kFCons * 32) rt.cnt[e] = 0;
       {
         // this CTA's share of the per-slot gate/up completion counters
@@ -720,30 +721,25 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         for (int u = z0 + threadIdx.x; u < z1; u += kFCons * 32) gdone[u] = 0;
       }
       bool have_rows = false;
-      for (int t0 = 0; t0 < T; t0 += p.rtc) {
-        const int nt = min(p.rtc, T - t0);
-        if (t0 > 0) all_sync();
-        for (int t = warp; t < nt; t += kFCons)
-          stage_token_all<BITS, LG, CG>(xsrc + size_t(t0 + t) * H, p.stack != 0, xs + size_t(t) * H, &rnorm[t0 + t],
-                                        &inv_all[t0 + t], lane);
-        all_sync();
-        if (t0 == 0) stamp(l, 14);
-        const int nb = (nt + kRouterTB - 1) / kRouterTB;
-        for (int it = warp; it < (e1 - e0) * nb; it += kFCons) {
-          if (!have_rows) {
-            have_rows = true;
-            if (!*abort_flag && !mbar_wait(rbar, l & 1, abort_flag)) {
-              *abort_flag = 1;
-              report_error(status, MOE_ERR_TIMEOUT, 43);
-            }
-            stamp(l, 19);
+      for (int t = warp; t < T; t += kFCons) {
+        __half* dst = p.pre ? xs + size_t(t) * H : reinterpret_cast<__half*>(ring + RING_STRIDE) + size_t(warp) * H;
+        stage_token_all<BITS, LG, CG>(xsrc + size_t(t) * H, p.stack != 0, dst, &rnorm[t], &inv_all[t], lane);
+        __syncwarp();
+        if (t == 0) stamp(l, 14);
+        if (!have_rows && e1 > e0) {
+          have_rows = true;
+          if (!*abort_flag && !mbar_wait(rbar, l & 1, abort_flag)) {
+            *abort_flag = 1;
+            report_error(status, MOE_ERR_TIMEOUT, 43);
           }
-          const int e = e0 + it / nb, b = it % nb;
-          const float bias = lw.router_bias ? lw.router_bias[e] : 0.f;
-          router_from_staged<BITS, LG, CG>(reinterpret_cast<const uint16_t*>(ring) + size_t(e - e0) * H, bias,
-                                           xs + size_t(b) * kRouterTB * H, inv_all, t0 + b * kRouterTB,
-                                           min(kRouterTB, nt - b * kRouterTB), logits + e, E, lane);
+          if (t == 0) stamp(l, 19);
         }
+        for (int e = e0; e < e1; ++e) {
+          const float bias = lw.router_bias ? lw.router_bias[e] : 0.f;
+          router_from_staged<BITS, LG, CG, 1>(reinterpret_cast<const uint16_t*>(ring) + size_t(e - e0) * H, bias, dst,
+                                              inv_all, t, 1, logits + e, E, lane);
+        }
+        __syncwarp();
       }
       stamp(l, 15);
       all_sync();
@@ -970,10 +966,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
             acc[2 * z + 1] += __uint_as_float(xw[z] & 0xFFFF0000u);
           }
         }
-        __align__(16) uint16_t ob[8];
-#pragma unroll
-        for (int z = 0; z < 8; ++z) ob[z] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[z]));
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob);
+        *reinterpret_cast<uint4*>(dst) = pack_bf16x8(acc);
       }
       stamp(l, 7);
       if (p.stack && l + 1 < p.L) grid_sync();
@@ -1015,6 +1008,9 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
     xs_halves = max(size_t(q.rtc) * GU::K, size_t(kFGroups) * q.grp_xs);
   }
   if (q.rtc < 1 || q.ntc_gu < 1 || q.ntc_dn < 1) return cudaErrorInvalidValue;
+  // tokens that are not pre-staged use one row per consumer warp in ring slots 1-2
+  static_assert(kFCons * 2048 * 2 <= 2 * RING_STRIDE, "per-warp token rows exceed ring slots 1-2");
+  if (!q.pre && size_t(kFCons) * p.cfg.hidden * 2 > size_t(2) * RING_STRIDE) return cudaErrorCooperativeLaunchTooLarge;
   q.xs_halves = (long long)xs_halves;
   const size_t smem = q.smem_xs_off + xs_halves * 2;
   if (smem > size_t(kSmemMax)) return cudaErrorInvalidValue;

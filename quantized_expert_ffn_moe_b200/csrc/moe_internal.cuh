@@ -398,6 +398,35 @@ __device__ __forceinline__ void decode_q2x16(uint32_t v, __half2 out[8]) {
   }
 }
 
+// Eight fp32 values rounded to bf16 (round to nearest even) as one 16-byte
+// word group, element 2i in the low half of word i; in registers.
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&a)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Packs G fp32 values of one code group (k order), times mul, into the fp16
+// pair order of the integer decoders -- word w = (v[w], v[w + G/2]), i.e. the
+// element at position decode_slot(j) -- as G/8 16-byte parts, in registers
+// (no local array, one paired conversion per word).
+template <int G>
+__device__ __forceinline__ void pack_pair_order(const float (&v)[G], float mul, uint4 (&parts)[G / 8]) {
+  constexpr int HALF = G / 2;
+  uint32_t w[HALF];
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const __half2 h = __floats2half2_rn(v[i] * mul, v[i + HALF] * mul);
+    w[i] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+#pragma unroll
+  for (int q = 0; q < G / 8; ++q) parts[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
 // Position, inside a group of 8 (4-bit) or 16 (2-bit) consecutive elements,
 // of element j in the half2 order produced by the decoders above.
 __host__ __device__ inline int decode_slot(int bits, int j) {

@@ -617,12 +617,10 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
           in[8 * q + 2 * z + 1] = __uint_as_float(w[z] & 0xFFFF0000u);
         }
       }
-      __align__(16) __half out[G];
+      uint4 parts[G / 8];
+      pack_pair_order<G>(in, mul, parts);
 #pragma unroll
-      for (int j = 0; j < G; ++j) out[decode_slot(BITS, j)] = __float2half_rn(in[j] * mul);
-#pragma unroll
-      for (int q = 0; q < G / 8; ++q)
-        *reinterpret_cast<uint4*>(dst + h0 + 8 * q) = *reinterpret_cast<const uint4*>(out + 8 * q);
+      for (int q = 0; q < G / 8; ++q) *reinterpret_cast<uint4*>(dst + h0 + 8 * q) = parts[q];
     }
   }
 }
