@@ -112,7 +112,7 @@ struct SRoute {
   int* ulist;    // [E+1]
   int* woff_gu;  // [E+2]
   int* woff_dn;  // [E+2]
-  int* cnt;      // [E] scratch
+  unsigned* tmask;  // [ceil(T/32)][E] tokens that picked each expert (bit t % 32)
 };
 
 // Cursor over a CTA's stages in shared-memory routing (same walk as the
@@ -274,20 +274,30 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
   }
 }
 
+constexpr int kMaxRE = 8;        // router rows (experts) per CTA
+
 // Stages token t once for the whole layer: one L2 round trip for the row
 // (each lane holds whole groups of G elements), RMSNorm factor (stack),
 // xhat = bf16(x * r), and the power-of-two scale that puts max |xhat| in
-// [128, 256); stored as fp16 in the gate/up operand order.
+// [128, 256); stored as fp16 in the gate/up operand order.  Then, from the
+// same registers, the token's router logits for the ne <= kMaxRE experts
+// whose rows (bf16) are in shared memory at rrows once `rbar` completes
+// (rbar == nullptr: they already have): sum_h Wr[e][h] * xhat[h] in fp32
+// with exact products, plus the bias.  dst == nullptr skips the fp16 row;
+// xb_out (if set) receives xhat as bf16 in natural order.
 template <int BITS, int LPR, int CPL>
 __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, float* rnorm_out, float* inv_out,
-                                int lane) {
+                                uint16_t* xb_out, const uint16_t* rrows, int ne, const float* rbias,
+                                float* logit_row, uint64_t* rbar, uint32_t rpar, volatile int* abort_flag,
+                                int* status, int lane) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);       // groups per lane
-  uint4 v[NG][G / 8];
+  constexpr int NW = G / 8;                                     // 16-byte words per group
+  uint4 v[NG][NW];
 #pragma unroll
   for (int q = 0; q < NG; ++q)
 #pragma unroll
-    for (int z = 0; z < G / 8; ++z)
+    for (int z = 0; z < NW; ++z)
       v[q][z] = __ldcg(reinterpret_cast<const uint4*>(row + (q * 32 + lane) * G + 8 * z));
   float r = 1.f;
   if (stack) {
@@ -295,7 +305,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
 #pragma unroll
     for (int q = 0; q < NG; ++q)
 #pragma unroll
-      for (int z = 0; z < G / 8; ++z) {
+      for (int z = 0; z < NW; ++z) {
         const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
 #pragma unroll
         for (int y = 0; y < 4; ++y) {
@@ -308,17 +318,31 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) st += __shfl_xor_sync(0xffffffffu, st, o);
     r = 1.0f / sqrtf(st / float(K) + 1e-6f);
+    // xhat = bf16(x * r), in place (element 2y in the low half of word y)
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+#pragma unroll
+      for (int z = 0; z < NW; ++z) {
+        uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(w[y] << 16) * r,
+                                                          __uint_as_float(w[y] & 0xFFFF0000u) * r);
+          w[y] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        v[q][z] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
   }
   float vm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int q = 0; q < NG; ++q)
 #pragma unroll
-    for (int z = 0; z < G / 8; ++z) {
+    for (int z = 0; z < NW; ++z) {
       const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
-        vm[y] = fmaxf(vm[y], fabsf(round_bf16f(__uint_as_float(w[y] << 16) * r)));
-        vm[y] = fmaxf(vm[y], fabsf(round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r)));
+        vm[y] = fmaxf(vm[y], fabsf(__uint_as_float(w[y] << 16)));
+        vm[y] = fmaxf(vm[y], fabsf(__uint_as_float(w[y] & 0xFFFF0000u)));
       }
     }
   float vmax = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
@@ -332,15 +356,15 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
   }
   const float mul = ldexpf(1.f, sh);
 #pragma unroll
-  for (int q = 0; q < NG; ++q) {
+  for (int q = 0; q < NG && dst != nullptr; ++q) {
     float vf[G];
 #pragma unroll
-    for (int z = 0; z < G / 8; ++z) {
+    for (int z = 0; z < NW; ++z) {
       const uint32_t w[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
-        vf[8 * z + 2 * y] = round_bf16f(__uint_as_float(w[y] << 16) * r);
-        vf[8 * z + 2 * y + 1] = round_bf16f(__uint_as_float(w[y] & 0xFFFF0000u) * r);
+        vf[8 * z + 2 * y] = __uint_as_float(w[y] << 16);
+        vf[8 * z + 2 * y + 1] = __uint_as_float(w[y] & 0xFFFF0000u);
       }
     }
     uint4 parts[Gm::NPART];
@@ -349,65 +373,81 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
 #pragma unroll
     for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
   }
+  if (xb_out != nullptr) {
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+#pragma unroll
+      for (int z = 0; z < NW; ++z) *reinterpret_cast<uint4*>(xb_out + (q * 32 + lane) * G + 8 * z) = v[q][z];
+  }
   if (lane == 0) {
     *rnorm_out = r;
     *inv_out = ldexpf(1.f, -sh);
   }
+  if (ne <= 0) return;
+  if (rbar != nullptr) {
+    if (*abort_flag) return;
+    if (!mbar_wait(rbar, rpar, abort_flag)) {
+      *abort_flag = 1;
+      report_error(status, MOE_ERR_TIMEOUT, 43);
+      return;
+    }
+  }
+  // experts in groups of 4 (bounded register use)
+#pragma unroll 1
+  for (int e0 = 0; e0 < ne; e0 += 4) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int q = 0; q < NG; ++q)
+#pragma unroll
+      for (int z = 0; z < NW; ++z) {
+        const int h0 = (q * 32 + lane) * G + 8 * z;
+        const uint32_t xw[4] = {v[q][z].x, v[q][z].y, v[q][z].z, v[q][z].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (e0 + e < ne) {
+            const uint4 u = *reinterpret_cast<const uint4*>(rrows + size_t(e0 + e) * K + h0);
+            const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+              acc[e] = fmaf(__uint_as_float(ww[y] << 16), __uint_as_float(xw[y] << 16), acc[e]);
+              acc[e] = fmaf(__uint_as_float(ww[y] & 0xFFFF0000u), __uint_as_float(xw[y] & 0xFFFF0000u), acc[e]);
+            }
+          }
+        }
+      }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (e0 + e < ne) {
+        float a = acc[e];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        if (lane == 0) logit_row[e0 + e] = a + (rbias ? rbias[e0 + e] : 0.f);
+      }
+    }
+  }
 }
 
-// Router logits of expert e for tokens t0 .. t0+nt-1 (nt <= kRTok) from their
-// staged activations (xs holds token t0 first) and the expert's router row
-// already in shared memory: sum_j Wr[e][j] * xs[slot(j)] (exact products),
-// times the token's 2^-sh.  The tokens run together, each with two partial
-// sums, so the multiply-add chains overlap.
-template <int BITS, int LPR, int CPL, int kRTok>
-__device__ void router_from_staged(const uint16_t* wrow, float bias, const __half* xs, const float* inv_all, int t0,
-                                   int nt, float* logit_col, int E, int lane) {
-  using Gm = Geom<BITS, LPR, CPL>;
-  constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);
-  float acc[kRTok][2];
+// Router logit of one token and one expert from shared-memory rows (xhat and
+// the router row, both bf16 in natural order): fp32 sum of exact products,
+// reduced over the warp; lane 0 stores it plus the bias.
+template <int K>
+__device__ void router_dot(const uint16_t* xrow, const uint16_t* wrow, float bias, float* logit, int lane) {
+  float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-  for (int t = 0; t < kRTok; ++t) acc[t][0] = acc[t][1] = 0.f;
+  for (int h = lane * 8; h < K; h += 256) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(xrow + h);
+    const uint4 wv = *reinterpret_cast<const uint4*>(wrow + h);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-  for (int q = 0; q < NG; ++q) {
-    const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
-    // router weights of the group (k order) as fp32
-    float wf[G];
-#pragma unroll
-    for (int z = 0; z < G / 8; ++z) {
-      const uint4 u = *reinterpret_cast<const uint4*>(wrow + (q * 32 + lane) * G + 8 * z);
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        wf[8 * z + 2 * y] = __uint_as_float(w[y] << 16);
-        wf[8 * z + 2 * y + 1] = __uint_as_float(w[y] & 0xFFFF0000u);
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < kRTok; ++t) {
-      const __half* xt = xs + size_t(t < nt ? t : 0) * K;
-      // staged word i holds elements (i, i + G/2) of the group
-      uint32_t xw[G / 2];
-#pragma unroll
-      for (int part = 0; part < Gm::NPART; ++part) {
-        const uint4 u = *reinterpret_cast<const uint4*>(xt + base + part * LPR * 8);
-        xw[4 * part] = u.x; xw[4 * part + 1] = u.y; xw[4 * part + 2] = u.z; xw[4 * part + 3] = u.w;
-      }
-#pragma unroll
-      for (int i = 0; i < G / 2; ++i) {
-        const float2 f = __half22float2(u32_as_h2(xw[i]));
-        acc[t][i & 1] = fmaf(wf[i], f.x, acc[t][i & 1]);
-        acc[t][i & 1] = fmaf(wf[i + G / 2], f.y, acc[t][i & 1]);
-      }
+    for (int y = 0; y < 4; ++y) {
+      a0 = fmaf(__uint_as_float(ww[y] << 16), __uint_as_float(xw[y] << 16), a0);
+      a1 = fmaf(__uint_as_float(ww[y] & 0xFFFF0000u), __uint_as_float(xw[y] & 0xFFFF0000u), a1);
     }
   }
+  float a = a0 + a1;
 #pragma unroll
-  for (int t = 0; t < kRTok; ++t) {
-    float v = acc[t][0] + acc[t][1];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && t < nt) logit_col[size_t(t0 + t) * E] = v * inv_all[t0 + t] + bias;
-  }
+  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  if (lane == 0) *logit = a + bias;
 }
 
 // Exclusive scans of two values per consumer thread (all kFCons warps), with
@@ -646,7 +686,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   rt.ulist = rt.offsets + (E + 1);
   rt.woff_gu = rt.ulist + (E + 1);
   rt.woff_dn = rt.woff_gu + (E + 2);
-  rt.cnt = rt.woff_dn + (E + 2);
+  rt.tmask = reinterpret_cast<unsigned*>(rt.woff_dn + (E + 2));
+  const int NMW = (T + 31) >> 5;                                          // token mask words per expert
   // tokens: every token (pre-staged) or router chunks in R and G; the two
   // groups' chunk buffers in G (not pre-staged) and D
   __half* xs = reinterpret_cast<__half*>(smem + p.smem_xs_off);
@@ -714,32 +755,46 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       // it stays for gate/up, or, when the tokens do not all fit, into its own
       // row of the idle ring slots 1-2 -- and at once computes the token's
       // router logits for this CTA's experts from their rows in ring slot 0
-      for (int e = threadIdx.x; e < E; e += kFCons * 32) rt.cnt[e] = 0;
+      for (int e = threadIdx.x; e < NMW * E; e += kFCons * 32) rt.tmask[e] = 0u;
       {
         // this CTA's share of the per-slot gate/up completion counters
         const int z0 = int((long long)(E + 2) * blockIdx.x / G), z1 = int((long long)(E + 2) * (blockIdx.x + 1) / G);
         for (int u = z0 + threadIdx.x; u < z1; u += kFCons * 32) gdone[u] = 0;
       }
+      // one warp per token: staging and, from the same registers, the
+      // token's router logits for this CTA's experts; with fewer tokens than
+      // warps, the warps keep xhat (bf16) in the idle ring slots 1-2 instead
+      // and then all warps share the (token, expert) dots
+      const int ne = e1 - e0;
+      const bool few = T < kFCons;
+      uint16_t* xb = reinterpret_cast<uint16_t*>(ring + RING_STRIDE);
       bool have_rows = false;
       for (int t = warp; t < T; t += kFCons) {
-        __half* dst = p.pre ? xs + size_t(t) * H : reinterpret_cast<__half*>(ring + RING_STRIDE) + size_t(warp) * H;
-        stage_token_all<BITS, LG, CG>(xsrc + size_t(t) * H, p.stack != 0, dst, &rnorm[t], &inv_all[t], lane);
-        __syncwarp();
+        stage_token_all<BITS, LG, CG>(xsrc + size_t(t) * H, p.stack != 0, p.pre ? xs + size_t(t) * H : nullptr,
+                                      &rnorm[t], &inv_all[t], few ? xb + size_t(t) * H : nullptr,
+                                      reinterpret_cast<const uint16_t*>(ring), few ? 0 : ne,
+                                      lw.router_bias ? lw.router_bias + e0 : nullptr, logits + size_t(t) * E + e0,
+                                      have_rows ? nullptr : rbar, l & 1, abort_flag, status, lane);
+        have_rows = !few;
         if (t == 0) stamp(l, 14);
-        if (!have_rows && e1 > e0) {
-          have_rows = true;
-          if (!*abort_flag && !mbar_wait(rbar, l & 1, abort_flag)) {
-            *abort_flag = 1;
-            report_error(status, MOE_ERR_TIMEOUT, 43);
-          }
-          if (t == 0) stamp(l, 19);
-        }
-        for (int e = e0; e < e1; ++e) {
-          const float bias = lw.router_bias ? lw.router_bias[e] : 0.f;
-          router_from_staged<BITS, LG, CG, 1>(reinterpret_cast<const uint16_t*>(ring) + size_t(e - e0) * H, bias, dst,
-                                              inv_all, t, 1, logits + e, E, lane);
-        }
         __syncwarp();
+      }
+      if (few) {
+        all_sync();
+        for (int pr = warp; pr < T * ne; pr += kFCons) {
+          if (!have_rows) {
+            have_rows = true;
+            if (*abort_flag) break;
+            if (!mbar_wait(rbar, l & 1, abort_flag)) {
+              *abort_flag = 1;
+              report_error(status, MOE_ERR_TIMEOUT, 43);
+              break;
+            }
+          }
+          const int t = pr / ne, e = pr % ne;
+          router_dot<GU::K>(xb + size_t(t) * H, reinterpret_cast<const uint16_t*>(ring) + size_t(e) * H,
+                            lw.router_bias ? lw.router_bias[e0 + e] : 0.f, logits + size_t(t) * E + e0 + e, lane);
+        }
       }
       stamp(l, 15);
       all_sync();
@@ -749,20 +804,25 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       // ---------------------------------------------------------- phase S
       {
         uint2* tscr = reinterpret_cast<uint2*>(ring + 3 * RING_STRIDE) + warp * 32;
-        for (int t = warp; t < T; t += kFCons)
-          warp_topk<NPL, true>(logits + size_t(t) * E, k, E, rt.idx + t * k, rt.w + t * k, tscr, rt.cnt);
+        // CTAs start at different tokens, so their reads of the freshly
+        // written logits spread over the L2 lines of all tokens
+        for (int tt = warp; tt < T; tt += kFCons) {
+          const int t = (tt + int(blockIdx.x)) % T;
+          warp_topk<NPL, true>(logits + size_t(t) * E, k, E, rt.idx + t * k, rt.w + t * k, tscr, rt.tmask, t);
+        }
       }
       all_sync();
       stamp(l, 9);
       {
-        // exclusive scan of the counts and the ascending touched-expert list;
-        // cnt becomes each expert's fill cursor
+        // exclusive scan of the counts and the ascending touched-expert list
         const int EPT = (E + kFCons * 32 - 1) / (kFCons * 32);     // experts per thread
         const int eb = threadIdx.x * EPT;
         int csum = 0, fsum = 0;
         for (int z = 0; z < EPT; ++z) {
           const int e = eb + z;
-          const int cc = e < E ? rt.cnt[e] : 0;
+          int cc = 0;
+          if (e < E)
+            for (int m = 0; m < NMW; ++m) cc += __popc(rt.tmask[m * E + e]);
           csum += cc;
           fsum += cc > 0 ? 1 : 0;
         }
@@ -772,9 +832,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         for (int z = 0; z < EPT; ++z) {
           const int e = eb + z;
           if (e < E) {
-            const int cc = rt.cnt[e];
             rt.offsets[e] = crun;
-            rt.cnt[e] = crun;
+            int cc = 0;
+            for (int m = 0; m < NMW; ++m) cc += __popc(rt.tmask[m * E + e]);
             crun += cc;
             if (cc > 0) rt.ulist[frun++] = e;
           }
@@ -787,27 +847,25 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       }
       all_sync();
       stamp(l, 10);
-      // stable positions inside each expert's list (pairs in token order), by
-      // warp 0 over 32 pairs at a time: every CTA derives the same positions,
-      // which the passes of different CTAs rely on.  Meanwhile the
-      // cost-weighted work prefix of the slots for the two passes.
-      if (warp == 0) {
-        for (int base = 0; base < P; base += 32) {
-          const int q = base + lane;
-          const int e = q < P ? rt.idx[q] : -1 - lane;
-          const unsigned same = __match_any_sync(0xffffffffu, e);
-          const int rank = __popc(same & ((1u << lane) - 1u));
-          const int start = q < P ? rt.cnt[e] : 0;
-          __syncwarp();
-          if (q < P) {
-            const int pos = start + rank;
-            rt.pairs[pos] = q;
-            rt.inv[q] = pos;
-            if ((same >> lane) == 1u) rt.cnt[e] = start + rank + 1;     // last of its expert in this group
-          }
-          __syncwarp();
+      // stable positions inside each expert's list (pairs in token order): a
+      // pair of token t sits after the earlier tokens in its expert's mask, so
+      // every CTA derives the same positions, which the passes of different
+      // CTAs rely on.  Meanwhile the cost-weighted work prefix of the slots
+      // for the two passes.
+      for (int q = threadIdx.x; q < P; q += kFCons * 32) {
+        const int e = rt.idx[q], t = q / k;
+        int r = 0;
+        for (int m = 0; m < NMW; ++m) {
+          const int tb = t - 32 * m;
+          if (tb <= 0) break;
+          const unsigned below = tb >= 32 ? 0xFFFFFFFFu : ((1u << tb) - 1u);
+          r += __popc(rt.tmask[m * E + e] & below);
         }
-      } else if (warp == 1 && p.trace && blockIdx.x == 0) {
+        const int pos = rt.offsets[e] + r;
+        rt.pairs[pos] = q;
+        rt.inv[q] = pos;
+      }
+      if (warp == 1 && p.trace && blockIdx.x == 0) {
         for (int q = lane; q < P; q += 32) p.trace[size_t(l) * P + q] = rt.idx[q];
       }
       {
@@ -984,8 +1042,9 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   constexpr int RING_STRIDE = GU::STAGE_BYTES > DN::STAGE_BYTES ? GU::STAGE_BYTES : DN::STAGE_BYTES;
   constexpr int kSmemMax = 227 * 1024;
   const int E = p.cfg.num_experts, T = p.T, k = p.cfg.top_k;
-  const int route_bytes = (4 * T * k + 2 * (E + 1) + 2 * (E + 2) + E) * 4;
+  const int route_bytes = (4 * T * k + 2 * (E + 1) + 2 * (E + 2) + E * ((T + 31) / 32)) * 4;
   if (size_t((E + num_sms - 1) / num_sms) * p.cfg.hidden * 2 > size_t(RING_STRIDE)) return cudaErrorCooperativeLaunchTooLarge;
+  if ((E + num_sms - 1) / num_sms > kMaxRE) return cudaErrorCooperativeLaunchTooLarge;
   q.smem_route_off = kFRingOff + kFStages * RING_STRIDE;
   q.smem_xs_off = (q.smem_route_off + route_bytes + 127) & ~127;
   const int avail = kSmemMax - q.smem_xs_off;
@@ -1008,9 +1067,9 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
     xs_halves = max(size_t(q.rtc) * GU::K, size_t(kFGroups) * q.grp_xs);
   }
   if (q.rtc < 1 || q.ntc_gu < 1 || q.ntc_dn < 1) return cudaErrorInvalidValue;
-  // tokens that are not pre-staged use one row per consumer warp in ring slots 1-2
-  static_assert(kFCons * 2048 * 2 <= 2 * RING_STRIDE, "per-warp token rows exceed ring slots 1-2");
-  if (!q.pre && size_t(kFCons) * p.cfg.hidden * 2 > size_t(2) * RING_STRIDE) return cudaErrorCooperativeLaunchTooLarge;
+  // with fewer tokens than consumer warps, xhat rows (bf16) wait in ring slots 1-2
+  static_assert(kFCons * 2048 * 2 <= 2 * RING_STRIDE, "xhat rows exceed ring slots 1-2");
+  if (T < kFCons && size_t(T) * p.cfg.hidden * 2 > size_t(2) * RING_STRIDE) return cudaErrorCooperativeLaunchTooLarge;
   q.xs_halves = (long long)xs_halves;
   const size_t smem = q.smem_xs_off + xs_halves * 2;
   if (smem > size_t(kSmemMax)) return cudaErrorInvalidValue;

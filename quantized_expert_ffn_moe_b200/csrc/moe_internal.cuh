@@ -263,10 +263,11 @@ __device__ __forceinline__ void lane_best(const uint32_t (&key)[NPL], uint32_t& 
 // most 32 of them they are ranked all at once through `scratch` (32 uint2 of
 // shared memory for this warp), otherwise k rounds of warp maxima decide.
 // CG reads the logits around L1 (they were written by other CTAs of the same
-// launch).  Optionally counts each pick into cnt[expert] (shared memory).
+// launch).  Optionally marks the token in the picked experts' token masks
+// (shared memory, word tmask[(t / 32) * E + expert], bit t % 32).
 template <int NPL, bool CG>
 __device__ __forceinline__ void warp_topk(const float* lrow, int k, int E, int* idx_out, float* w_out,
-                                          uint2* scratch, int* cnt = nullptr) {
+                                          uint2* scratch, unsigned* tmask = nullptr, int t = 0) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NPL];
 #pragma unroll
@@ -349,7 +350,7 @@ __device__ __forceinline__ void warp_topk(const float* lrow, int k, int E, int* 
   if (lane < k) {
     idx_out[lane] = my_idx;
     w_out[lane] = ex / sum;
-    if (cnt) atomicAdd(&cnt[my_idx], 1);
+    if (tmask) atomicOr(&tmask[(t >> 5) * E + my_idx], 1u << (t & 31));
   }
 }
 
