@@ -282,22 +282,21 @@ def barrier(dist, world):
         dist.barrier()
 
 
-def max_over_ranks(dist, world, v: float) -> float:
-    if world <= 1:
-        return v
+def _reduce_scalar(dist, v: float, op) -> float:
     import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(dist, world, v: float) -> float:
+    """Step time of the whole job: the slowest rank's."""
+    return v if world <= 1 else _reduce_scalar(dist, v, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(dist, world, v: float) -> float:
-    if world <= 1:
-        return v
-    import torch
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return v if world <= 1 else _reduce_scalar(dist, v, dist.ReduceOp.SUM)
 
 
 def main():

@@ -110,6 +110,26 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w,
                       const uint16_t* x, int32_t T, uint16_t* y,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/* Expert-parallel share of one MoE layer (one rank of ep_size, experts
+ * sharded by e % ep_size == ep_rank).  The pages run every expert of a layer
+ * on one machine; splitting the routed experts over GPUs is the one exchange
+ * step the layer admits: each rank routes all T tokens (the router is
+ * replicated), computes only the pairs whose expert it owns, and the layer
+ * output is the sum of the ranks' partials (an all-reduce), rounded to bf16.
+ *   y_partial[t][h] (fp32, device, [T][H], owned by the caller) =
+ *       [ep_rank == 0] * FFN_shared(x_t)[h]
+ *     + sum over j with idx[t][j] % ep_size == ep_rank of w[t][j] * FFN_idx[t][j](x_t)[h]
+ * with idx, w and FFN as in moe_layer_forward.  w holds the full expert
+ * arrays; only the owned experts' rows (and the shared expert's on rank 0,
+ * which other ranks may pass as NULL) are read.  1 <= ep_size <= num_experts,
+ * 0 <= ep_rank < ep_size, else MOE_ERR_INVALID_ARG; x and y_partial may not
+ * overlap.  Runs the separate route / grouped GEMV or GEMM / combine kernels
+ * (not the single-launch decode kernel).  ep_size = 1 gives the whole layer
+ * output before its bf16 rounding. */
+int moe_layer_forward_ep(const moe_config* cfg, const moe_layer_weights* w,
+                         const uint16_t* x, int32_t T, int32_t ep_rank, int32_t ep_size,
+                         float* y_partial, void* workspace, size_t ws_bytes, void* stream);
+
 /* L layers in sequence on the residual stream, in place:
  *   for l in 0..L-1:  x <- bf16(x + moe_l(bf16(rmsnorm(x))))
  * rmsnorm(x) = x / sqrt(mean(x^2) + 1e-6) per token (weight 1).

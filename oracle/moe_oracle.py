@@ -53,7 +53,7 @@ import numpy as np
 __all__ = [
     "bf16_to_f64", "round_bf16", "unpack_codes", "dequantize", "router_logits",
     "select_topk", "gate_weights", "group_by_expert", "silu", "swiglu_ffn",
-    "rmsnorm_bf16", "OracleLayer", "layer_forward", "stack_forward",
+    "rmsnorm_bf16", "OracleLayer", "layer_forward", "layer_forward_ep", "stack_forward",
     "tie_band_ok", "RMS_EPS",
 ]
 
@@ -257,6 +257,35 @@ def layer_forward(layer: OracleLayer, x_bits: np.ndarray, *, rmsnorm: bool = Fal
             acc += w[t, j] * swiglu_ffn(*layer.expert_dense(int(idx[t, j])), xhat[t])
         out[t] = acc
     return {"xhat": xhat, "logits": logits, "idx": idx, "w": w, "out": out}
+
+
+def layer_forward_ep(layer: OracleLayer, x_bits: np.ndarray, ep_rank: int, ep_size: int) -> dict:
+    """One rank's share of the layer when its experts are split over ep_size
+    ranks by e % ep_size (expert parallelism; the pages run all experts of a
+    layer on one machine, so this split is a reading of how the layer shards).
+
+    Every rank routes all tokens over all experts exactly as layer_forward
+    does; rank r then adds only the pairs (t, j) whose expert idx[t, j]
+    satisfies idx % ep_size == r, weighted by w[t, j], and rank 0 alone adds
+    the shared expert.  Returns float64 ``partial`` [T, H] and the routing;
+    the sum of the partials over the ranks is layer_forward's ``out``."""
+    if not (1 <= ep_size <= layer.experts and 0 <= ep_rank < ep_size):
+        raise ValueError("need 1 <= ep_size <= experts and 0 <= ep_rank < ep_size")
+    x = bf16_to_f64(x_bits)
+    logits = router_logits(x, layer.router_w_bits, layer.router_bias)
+    idx = select_topk(logits, layer.top_k)
+    w = gate_weights(logits, idx)
+    T = x.shape[0]
+    partial = np.zeros((T, layer.hidden), dtype=np.float64)
+    shared = layer.shared_dense() if ep_rank == 0 else None
+    for t in range(T):
+        if shared is not None:
+            partial[t] += swiglu_ffn(*shared, x[t])
+        for j in range(layer.top_k):
+            e = int(idx[t, j])
+            if e % ep_size == ep_rank:
+                partial[t] += w[t, j] * swiglu_ffn(*layer.expert_dense(e), x[t])
+    return {"partial": partial, "idx": idx, "w": w}
 
 
 def stack_forward(layers, x_bits: np.ndarray, *, choose_topk=None) -> dict:

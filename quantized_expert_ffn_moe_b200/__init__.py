@@ -20,7 +20,8 @@ __all__ = [
     "MoeConfig", "LayerWeights", "MoeError", "load_library", "EXPORTS", "LIB_PATH",
     "moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
     "moe_device_status", "moe_dequant_rows", "moe_status_str", "config_of", "moe_profile_begin",
-    "moe_profile_end", "moe_layer_forward_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "moe_profile_end", "moe_layer_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "moe_layer_forward_ep",
+    "ep_all_reduce",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -28,7 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
            "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end",
            "moe_layer_forward_noalloc", "moe_last_cuda_error", "moe_debug_fused_timing",
-           "moe_debug_prefill_timing")
+           "moe_debug_prefill_timing", "moe_layer_forward_ep")
 
 MOE_OK = 0
 
@@ -94,6 +95,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_route.restype = ctypes.c_int
     lib.moe_layer_forward.argtypes = [cfgp, ctypes.POINTER(_Weights), P, I32, P, P, SZ, P]
     lib.moe_layer_forward.restype = ctypes.c_int
+    lib.moe_layer_forward_ep.argtypes = [cfgp, ctypes.POINTER(_Weights), P, I32, I32, I32, P, P, SZ, P]
+    lib.moe_layer_forward_ep.restype = ctypes.c_int
     lib.moe_stack_forward.argtypes = [cfgp, ctypes.POINTER(_Weights), I32, P, I32, P, P, SZ, P]
     lib.moe_stack_forward.restype = ctypes.c_int
     lib.moe_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
@@ -172,6 +175,29 @@ def moe_layer_forward(cfg: MoeConfig, w: LayerWeights, x, y, workspace, *, strea
     if check:
         _check(st, "moe_layer_forward")
     return st
+
+
+def moe_layer_forward_ep(cfg: MoeConfig, w: LayerWeights, x, y_partial, workspace, ep_rank: int, ep_size: int,
+                         *, stream=None, check=True, tokens: Optional[int] = None) -> int:
+    """This rank's fp32 partial [T, H] of the layer output: the routed experts
+    e with e % ep_size == ep_rank, plus the shared expert on rank 0."""
+    T = int(x.shape[0]) if tokens is None else tokens
+    cw = w.to_c()
+    st = load_library().moe_layer_forward_ep(ctypes.byref(cfg), ctypes.byref(cw), _ptr(x), T, ep_rank, ep_size,
+                                             _ptr(y_partial), _ptr(workspace), _nbytes(workspace), _stream(stream))
+    if check:
+        _check(st, "moe_layer_forward_ep")
+    return st
+
+
+def ep_all_reduce(y_partial, group=None):
+    """The exchange step of the expert-parallel layer: sums the ranks' fp32
+    partials in place over the torch.distributed process group (NCCL over
+    NVLink on GPUs).  Afterwards every rank holds the layer output before its
+    bf16 rounding."""
+    import torch.distributed as dist
+    dist.all_reduce(y_partial, op=dist.ReduceOp.SUM, group=group)
+    return y_partial
 
 
 def moe_layer_forward_noalloc(cfg: MoeConfig, w: LayerWeights, x, y, *, stream=None, check=True,

@@ -5,6 +5,9 @@
 // practice": 10 routed experts plus one shared expert are active per token).
 // In the stack the residual add and the next layer's RMSNorm are fused here:
 // x <- bf16(x + out), xhat <- bf16(x / sqrt(mean(x^2) + 1e-6)).
+// Expert-parallel share: pairs whose expert another rank owns carry position
+// -1 and are skipped, and the partial sum is written in fp32 (out_f32) for
+// the all-reduce over ranks.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -15,7 +18,7 @@ constexpr int kCombThreads = 256;
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const float* __restrict__ Y, const int* __restrict__ inv, int T, int k, int H, int shared,
-    uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next) {
+    uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next, float* __restrict__ out_f32) {
   pdl_wait();
   const int t = blockIdx.x;
   const int P_routed = T * k;
@@ -36,11 +39,18 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
       for (int i = 0; i < VPT; ++i) acc[i] = 0.f;
     }
     for (int j = 0; j < k; ++j) {
+      if (pos[j] < 0) continue;                 // expert owned by another rank
       const float* row = Y + size_t(pos[j]) * H + h0;
       const float4 a = *reinterpret_cast<const float4*>(row);
       const float4 b = *reinterpret_cast<const float4*>(row + 4);
       acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    if (out_f32) {
+      float* fd = out_f32 + size_t(t) * H + h0;
+      *reinterpret_cast<float4*>(fd) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float4*>(fd + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      continue;
     }
     uint16_t* dst = out + size_t(t) * H + h0;
     if (residual) {
@@ -62,7 +72,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     }
     *reinterpret_cast<uint4*>(dst) = ov;
   }
-  if (xhat_next) {
+  if (xhat_next && !out_f32) {
     __shared__ float red[kCombThreads / 32];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -92,7 +102,8 @@ cudaError_t launch_combine(const LayerArgs& a) {
   const moe_config& c = a.cfg;
   return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, a.stream,
                     reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
-                    a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next);
+                    a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next,
+                    a.y_f32);
 }
 
 }  // namespace moe

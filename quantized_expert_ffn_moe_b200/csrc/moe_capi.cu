@@ -6,7 +6,7 @@
 namespace moe {
 cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
                               const uint16_t* x, int T, char* ws, const Layout& L, int* api_counts,
-                              int* api_offsets, int* api_pairs, cudaStream_t s);
+                              int* api_offsets, int* api_pairs, cudaStream_t s, int ep_rank, int ep_size);
 }
 
 using namespace moe;
@@ -93,7 +93,7 @@ int run_layer(const LayerArgs& a) {
   const int call = (g_prof.on && g_prof.used < g_prof.cap) ? g_prof.used++ : -1;
   prof_mark(call, 0, a.stream);
   cudaError_t e = launch_route_full(a.cfg, a.w.router_w, a.w.router_bias, a.x, a.T, a.ws, a.L, nullptr,
-                                    nullptr, nullptr, a.stream);
+                                    nullptr, nullptr, a.stream, a.ep_rank, a.ep_size);
   if (e != cudaSuccess) return cuda_status(e);
   prof_mark(call, 1, a.stream);
   if (a.T > kDecodeMaxTokens && prefill_supported(a.cfg)) {
@@ -134,7 +134,7 @@ int moe_route(const moe_config* cfg, const uint16_t* router_w, const float* rout
   const Layout L = make_layout(*cfg, T);
   if (cudaMemsetAsync(ws + L.status, 0, ST_COUNT * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t e = launch_route_full(*cfg, router_w, router_bias, x, T, ws, L, expert_counts, expert_offsets,
-                                    pairs, s);
+                                    pairs, s, 0, 1);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const size_t n = size_t(T) * cfg->top_k;
   if (cudaMemcpyAsync(topk_idx, ws + L.topk_idx, n * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -177,6 +177,35 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
     (void)cudaGetLastError();        // cannot co-schedule one CTA per SM here: separate kernels
     if (call >= 0) g_prof.used--;
   }
+  return run_layer(a);
+}
+
+int moe_layer_forward_ep(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
+                         int32_t ep_rank, int32_t ep_size, float* y_partial, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  int st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0 || ep_size < 1 || ep_size > cfg->num_experts || ep_rank < 0 || ep_rank >= ep_size)
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  moe_config c = *cfg;
+  if (ep_rank != 0) c.shared_inter = 0;          // the shared expert belongs to rank 0
+  if ((st = validate_weights(&c, w)) != MOE_OK) return st;
+  if (!x || !y_partial || !aligned(x, 16) || !aligned(y_partial, 16)) return MOE_ERR_INVALID_ARG;
+  const char* xb = reinterpret_cast<const char*>(x);
+  const char* yb = reinterpret_cast<const char*>(y_partial);
+  if (xb < yb + size_t(T) * cfg->hidden * 4 && yb < xb + size_t(T) * cfg->hidden * 2) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(cfg, T, workspace, ws_bytes)) != MOE_OK) return st;
+  LayerArgs a{};
+  a.cfg = c; a.w = *w; a.T = T; a.x = x; a.y = nullptr; a.residual = false; a.xhat_next = nullptr;
+  a.ws = static_cast<char*>(workspace);
+  a.L = make_layout(*cfg, T);
+  a.num_sms = num_sms_current();
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.ep_rank = ep_rank;
+  a.ep_size = ep_size;
+  a.y_f32 = y_partial;
+  if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
   return run_layer(a);
 }
 

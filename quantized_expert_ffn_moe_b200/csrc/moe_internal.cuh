@@ -447,6 +447,8 @@ struct LayerArgs {
   Layout L;
   int num_sms;
   cudaStream_t stream;
+  int ep_rank = 0, ep_size = 1;   // expert-parallel share: experts e with e % ep_size == ep_rank
+  float* y_f32 = nullptr;         // [T][H] fp32 partial output (expert-parallel share) instead of y
 };
 
 cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* xhat, int T, int H, cudaStream_t s);

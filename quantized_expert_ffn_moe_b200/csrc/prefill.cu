@@ -582,8 +582,12 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
   pdl_launch_dependents();
   constexpr int G = BITS == 4 ? 8 : 16;
   const int P = rv.T * rv.k + (rv.shared ? rv.T : 0);
+  // routed positions in use: all T*k, or fewer when the experts are split
+  // over ranks (this rank's pairs only)
+  const int Pr = __ldcg(rv.offsets + rv.E);
   const int lane = threadIdx.x & 31;
   for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < P; p += gridDim.x * 8) {
+    if (p < rv.T * rv.k && p >= Pr) continue;
     const int tok = p < rv.T * rv.k ? __ldg(rv.pairs + p) / rv.k : p - rv.T * rv.k;
     const uint16_t* src = x + size_t(tok) * H;
     uint16_t* dst = xs + size_t(p) * H;

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
     int* __restrict__ offsets_out, int* __restrict__ pairs_out, int* __restrict__ inv_out,
     int* __restrict__ ulist_out, int* __restrict__ api_counts, int* __restrict__ api_offsets,
     int* __restrict__ api_pairs, PassPlan pg, PassPlan pd, int* __restrict__ woff_gu,
-    int* __restrict__ woff_dn, int* __restrict__ ntoff) {
+    int* __restrict__ woff_dn, int* __restrict__ ntoff, int ep_rank, int ep_size) {
   extern __shared__ int sm[];
   constexpr int NW = kGroupThreads / 32;
   int* hist = sm;                       // [NW][E]
@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
       atomicCAS(status + ST_ERROR, 0, 1);
       continue;
     }
+    if (e % ep_size != ep_rank) continue;   // expert of another rank
     atomicAdd(&hist[warp * E + e], 1);
   }
   __syncthreads();
@@ -294,12 +295,14 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
     if (lane < k) {
       const int q = t * k + lane;
       const int e = idx[q];
-      if (e >= 0 && e < E) {
+      if (e >= 0 && e < E && e % ep_size == ep_rank) {
         const int pos = offs[e] + hist[warp * E + e];
         hist[warp * E + e] += 1;        // distinct experts within one token
         pairs_out[pos] = q;
         inv_out[q] = pos;
         if (api_pairs) api_pairs[pos] = q;
+      } else {
+        inv_out[q] = -1;                // not computed on this rank
       }
     }
     __syncwarp();
@@ -313,7 +316,8 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
 // counts into per-chunk bases, offsets, the touched-expert list and the work
 // prefixes; each chunk then writes its pairs in token order.
 __global__ void __launch_bounds__(256) chunk_hist_kernel(const int* __restrict__ idx, int T, int k, int E,
-                                                         int* __restrict__ chunk_hist, int* __restrict__ status) {
+                                                         int* __restrict__ chunk_hist, int* __restrict__ status,
+                                                         int ep_rank, int ep_size) {
   extern __shared__ int hs[];
   pdl_wait();
   pdl_launch_dependents();
@@ -323,6 +327,7 @@ __global__ void __launch_bounds__(256) chunk_hist_kernel(const int* __restrict__
   for (int q = t0 * k + threadIdx.x; q < t1 * k; q += blockDim.x) {
     const int e = idx[q];
     if (e < 0 || e >= E) { atomicCAS(status + ST_ERROR, 0, 2); continue; }
+    if (e % ep_size != ep_rank) continue;     // expert of another rank
     atomicAdd(&hs[e], 1);
   }
   __syncthreads();
@@ -425,7 +430,8 @@ __global__ void __launch_bounds__(kGroupThreads) chunk_scan_kernel(
 __global__ void __launch_bounds__(32) chunk_scatter_kernel(const int* __restrict__ idx, int T, int k, int E,
                                                            const int* __restrict__ chunk_base,
                                                            const int* __restrict__ offsets, int* __restrict__ pairs,
-                                                           int* __restrict__ inv, int* __restrict__ api_pairs) {
+                                                           int* __restrict__ inv, int* __restrict__ api_pairs,
+                                                           int ep_rank, int ep_size) {
   extern __shared__ int cur[];                 // [E] fill cursors, then the chunk's ids
   int* cidx = cur + E;                         // [kGroupChunk * k]
   pdl_wait();
@@ -441,11 +447,13 @@ __global__ void __launch_bounds__(32) chunk_scatter_kernel(const int* __restrict
     if (lane < k) {
       const int q = t * k + lane;
       const int e = cidx[q - t0 * k];
-      if (e >= 0 && e < E) {
+      if (e >= 0 && e < E && e % ep_size == ep_rank) {
         const int pos = cur[e]++;     // distinct experts within one token
         pairs[pos] = q;
         inv[q] = pos;
         if (api_pairs) api_pairs[pos] = q;
+      } else {
+        inv[q] = -1;                  // not computed on this rank
       }
     }
     __syncwarp();
@@ -454,7 +462,8 @@ __global__ void __launch_bounds__(32) chunk_scatter_kernel(const int* __restrict
 
 template <int NPL>
 cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout& L, bool fused,
-                              int* api_counts, int* api_offsets, int* api_pairs, cudaStream_t s) {
+                              int* api_counts, int* api_offsets, int* api_pairs, int ep_rank, int ep_size,
+                              cudaStream_t s) {
   const size_t smem = (size_t(32) * c.num_experts + c.num_experts + 1 + kGroupThreads) * sizeof(int);
   auto kern = group_kernel<NPL>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -474,7 +483,7 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
       int* hist = reinterpret_cast<int*>(ws + L.chunk_hist);
       int* status = reinterpret_cast<int*>(ws + L.status);
       err = launch_pdl(chunk_hist_kernel, dim3(nch), dim3(256), size_t(E) * 4, s, (const int*)idx, T, c.top_k, E,
-                       hist, status);
+                       hist, status, ep_rank, ep_size);
       if (err != cudaSuccess) return err;
       err = launch_pdl(chunk_scan_kernel, dim3(1), dim3(kGroupThreads), 0, s, nch, T, E, c.shared_inter > 0 ? 1 : 0,
                        hist, status, reinterpret_cast<int*>(ws + L.counts), reinterpret_cast<int*>(ws + L.offsets),
@@ -485,7 +494,7 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
       return launch_pdl(chunk_scatter_kernel, dim3(nch), dim3(32), size_t(E + kGroupChunk * c.top_k) * 4, s,
                         (const int*)idx, T, c.top_k, E,
                         (const int*)hist, (const int*)(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
-                        reinterpret_cast<int*>(ws + L.inv), api_pairs);
+                        reinterpret_cast<int*>(ws + L.inv), api_pairs, ep_rank, ep_size);
     }
   }
   return launch_pdl(kern, dim3(1), dim3(kGroupThreads), smem, s, logits, fused ? 1 : 0, idx, w, T,
@@ -494,7 +503,7 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
                     reinterpret_cast<int*>(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
                     reinterpret_cast<int*>(ws + L.inv), reinterpret_cast<int*>(ws + L.ulist), api_counts,
                     api_offsets, api_pairs, pg, pd, reinterpret_cast<int*>(ws + L.woff_gu),
-                    reinterpret_cast<int*>(ws + L.woff_dn), reinterpret_cast<int*>(ws + L.ntoff));
+                    reinterpret_cast<int*>(ws + L.woff_dn), reinterpret_cast<int*>(ws + L.ntoff), ep_rank, ep_size);
 }
 
 }  // namespace
@@ -525,21 +534,22 @@ cudaError_t launch_router_logits(const moe_config& c, const uint16_t* router_w, 
 }
 
 cudaError_t launch_topk_group_any(const moe_config& c, int T, char* ws, const Layout& L, bool fused,
-                                  int* api_counts, int* api_offsets, int* api_pairs, cudaStream_t s) {
+                                  int* api_counts, int* api_offsets, int* api_pairs, int ep_rank, int ep_size,
+                                  cudaStream_t s) {
   switch (c.num_experts / 32) {
-    case 1: return launch_topk_group<1>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
-    case 2: return launch_topk_group<2>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
-    case 4: return launch_topk_group<4>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
-    case 8: return launch_topk_group<8>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
-    case 16: return launch_topk_group<16>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
-    case 32: return launch_topk_group<32>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+    case 1: return launch_topk_group<1>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
+    case 2: return launch_topk_group<2>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
+    case 4: return launch_topk_group<4>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
+    case 8: return launch_topk_group<8>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
+    case 16: return launch_topk_group<16>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
+    case 32: return launch_topk_group<32>(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
                               const uint16_t* x, int T, char* ws, const Layout& L, int* api_counts,
-                              int* api_offsets, int* api_pairs, cudaStream_t s) {
+                              int* api_offsets, int* api_pairs, cudaStream_t s, int ep_rank, int ep_size) {
   int nsm = 148;
   {
     int dev = 0;
@@ -551,12 +561,12 @@ cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, con
       : launch_router_logits(c, router_w, bias, x, T, reinterpret_cast<float*>(ws + L.logits), s);
   if (err != cudaSuccess) return err;
   const bool fused = T <= 64;
-  return launch_topk_group_any(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, s);
+  return launch_topk_group_any(c, T, ws, L, fused, api_counts, api_offsets, api_pairs, ep_rank, ep_size, s);
 }
 
 cudaError_t launch_route(const moe_config& c, const uint16_t* router_w, const float* bias,
                          const uint16_t* x, int T, char* ws, const Layout& L, int, cudaStream_t s) {
-  return launch_route_full(c, router_w, bias, x, T, ws, L, nullptr, nullptr, nullptr, s);
+  return launch_route_full(c, router_w, bias, x, T, ws, L, nullptr, nullptr, nullptr, s, 0, 1);
 }
 
 }  // namespace moe

@@ -111,6 +111,32 @@ def test_layer_forward_argument_errors(lib):
     assert lib.moe_layer_forward(None, ctypes.byref(w), 1 << 30, 4, 2 << 30, 3 << 30, 1 << 40, None) == -1
 
 
+def _layer_ep(lib, c, w, rank, size, x=1 << 30, T=4, y=2 << 30, ws=3 << 30, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.moe_workspace_bytes(ctypes.byref(c), T)
+    return lib.moe_layer_forward_ep(ctypes.byref(c), ctypes.byref(w), x, T, rank, size, y, ws, ws_bytes, None)
+
+
+def test_layer_forward_ep_argument_errors(lib):
+    """Rejections happen on the host, before any launch."""
+    c = cfg()
+    w = _fake_weights()
+    E = c.num_experts
+    assert _layer_ep(lib, c, w, 0, 2, T=0) == 0                  # empty batch: no-op
+    assert _layer_ep(lib, c, w, 0, 0) == -1                      # ep_size < 1
+    assert _layer_ep(lib, c, w, 2, 2) == -1                      # rank out of range
+    assert _layer_ep(lib, c, w, -1, 2) == -1
+    assert _layer_ep(lib, c, w, 0, E + 1) == -1                  # more ranks than experts
+    assert _layer_ep(lib, c, w, 0, 2, y=None) == -1
+    assert _layer_ep(lib, c, w, 0, 2, y=(2 << 30) + 8) == -1     # misaligned fp32 output
+    assert _layer_ep(lib, c, w, 0, 2, y=(1 << 30) + 4096) == -1  # output overlaps x
+    assert _layer_ep(lib, c, w, 0, 2, ws_bytes=100) == -3
+    # the shared expert is required on rank 0 only
+    assert _layer_ep(lib, c, _fake_weights(shared=False), 0, 2) == -1
+    assert _layer_ep(lib, c, _fake_weights(shared=False), 1, 2, ws_bytes=0) == -3
+    assert _layer_ep(lib, cfg(bits=3), w, 0, 2) == -2
+
+
 def test_route_and_stack_argument_errors(lib):
     c = cfg()
     n = lib.moe_workspace_bytes(ctypes.byref(c), 4)

@@ -348,3 +348,67 @@ def test_prefill_full4_large_batch_tile_lookup():
     # 60,000 tokens: more tiles per CTA than the per-CTA tile table holds (the
     # down pass falls back to the per-tile lookup) and the chunked grouping at scale
     _sampled_full_case(mi.FULL4, 60000, 4, 0, 4, 60000)
+
+
+# ------------------------------------------------------- expert parallel ---
+
+def _ep_partials(shape, w, x_bits, ep_size):
+    """Every rank's fp32 partial, computed one rank after the other on this GPU
+    (the ranks share nothing but the inputs)."""
+    t = gc.torch()
+    cfg = gc.cfg_of(shape)
+    T = x_bits.shape[0]
+    x = gc.to_dev_bits(x_bits)
+    ws = gc.workspace(cfg, T)
+    parts = []
+    for r in range(ep_size):
+        yp = t.full((T, shape.hidden), float("nan"), dtype=t.float32, device="cuda")
+        q.moe_layer_forward_ep(cfg, w, x, yp, ws, r, ep_size)
+        t.cuda.synchronize()
+        assert q.moe_device_status(ws) == 0
+        parts.append(yp.cpu().numpy().astype(np.float64))
+    return parts
+
+
+@pytest.mark.parametrize("shape,T", [(mi.TINY, 8), (mi.TINY, 100), (SHAPE_2BIT_TINY, 17), (MID4, 300)],
+                         ids=["tiny4_t8", "tiny4_t100", "tiny2_t17", "mid4_t300"])
+@pytest.mark.parametrize("ep_size", [1, 2, 3])
+def test_expert_parallel_partials_live_oracle(shape, T, ep_size):
+    """Each rank's partial against the oracle's share of that rank, and their
+    sum against the whole layer (decode GEMV, and for mid4_t300 the chunked
+    grouping and the tcgen05 path)."""
+    x = mi.hidden_states_bf16(T, shape.hidden, 0, 31)
+    w = gc.device_layer(shape, 0, 0)
+    lay = gc.host_oracle_layer(shape, 0, 0, cache_size=shape.experts + 1)
+    idx = gc.run_route(shape, w, x)[0]
+    full = orc.layer_forward(lay, x)
+    differ = gc.check_selection(full["logits"], full["idx"], idx, shape.top_k)
+    keep = np.setdiff1d(np.arange(T), differ)          # tie-band tokens: checked by the layer tests
+    parts = _ep_partials(shape, w, x, ep_size)
+    scale = float(np.sqrt(np.mean(full["out"] ** 2)))
+    for r, p in enumerate(parts):
+        ref = orc.layer_forward_ep(lay, x, r, ep_size)["partial"]
+        err = float(np.abs(p[keep] - ref[keep]).max())
+        assert err <= gc.REL_TOL * scale, (r, err / scale)
+    err = float(np.abs(sum(parts)[keep] - full["out"][keep]).max())
+    assert err <= gc.REL_TOL * scale, err / scale
+
+
+def test_expert_parallel_full4_decode_stored_oracle():
+    """Full shape, 16 tokens, 2 and 4 ranks: the partials' sum against the
+    stored oracle output."""
+    case = gc.load_case("full4_decode")
+    E, H, I, k, sh, bits, bs = case["shape"].tolist()
+    shape = mi.MoeShape(E, H, I, k, bool(sh), bits, bs)
+    w = gc.device_layer(shape, int(case["seed"]), 0)
+    x = mi.hidden_states_bf16(int(case["T"]), H, int(case["seed"]), int(case["batch"]))[:16]
+    idx = gc.run_route(shape, w, x)[0]
+    toks = case["tokens"]
+    sel = toks[toks < 16]
+    rows = np.searchsorted(toks, sel)
+    differ = gc.check_selection(case["logits"][rows], case["idx"][rows], idx[sel], k)
+    keep = np.setdiff1d(np.arange(len(sel)), differ)
+    ref = case["out_"][rows].astype(np.float64)
+    for ep_size in (2, 4):
+        tot = sum(_ep_partials(shape, w, x, ep_size))
+        gc.assert_close(tot[sel][keep], ref[keep])
