@@ -488,6 +488,21 @@ def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
     for T in (1, 4):
         layer_rate(cfg, shape, pool4, T, 4000, 4, f"decode4_t{T}")
     layer_rate(cfg, shape, pool4, 4096, 8, 4, "prefill4_t4096")
+
+    # expert-parallel share: one rank's partial of the 4096-token layer when
+    # the experts are split over n ranks (computed on this one GPU; the
+    # all-reduce of the fp32 partials is not included)
+    xs = R.xbatches(shape, 4096, 2, base=900)
+    yp = torch.empty((4096, shape.hidden), dtype=torch.float32, device="cuda")
+    ep = {}
+    for n in (1, 2, 4, 8):
+        def estep(i, n=n):
+            q.moe_layer_forward_ep(cfg, pool4[i % NI], xs[i % 2], yp, ws, 0, n)
+        graphs, full = R.timed_graph(estep, 4, 2, chunk=4)
+        barrier(dist, world)
+        ms = max_over_ranks(dist, world, R.replay(graphs, full))
+        ep[f"ep{n}_rank0_us"] = 1000 * ms / 4
+    out["expert_parallel_share_t4096"] = ep
     # 2-bit skewed routing
     s2 = mi.FULL2
     cfg2 = q.config_of(512, 2048, 768, 10, True, 2, 16)
