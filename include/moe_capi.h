@@ -105,7 +105,11 @@ int moe_route(const moe_config* cfg, const uint16_t* router_w, const float* rout
 
 /* One MoE layer: y[T][H] (bf16) = out as defined above for x[T][H] (bf16).
  * x and y may not overlap.  T <= 64 takes the decode path (grouped GEMV on
- * CUDA cores); larger T takes the prefill path. */
+ * CUDA cores); larger T takes the prefill path (grouped tcgen05 GEMMs).  At
+ * 32 <= T <= 64 the decode kernel, once it has routed the batch, hands the
+ * layer to the prefill kernels when its cost model predicts them faster for
+ * that routing (see moe_debug_decode_path); the result is within the same
+ * tolerance either way, and the same inputs still give the same output. */
 int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w,
                       const uint16_t* x, int32_t T, uint16_t* y,
                       void* workspace, size_t ws_bytes, void* stream);
@@ -207,6 +211,16 @@ void moe_debug_fused_timing(unsigned long long* device_buf);
  *   start and [9] end of the MMA thread, [11] end of the epilogue; counts:
  *   [10] tiles, [14] k-blocks. */
 void moe_debug_prefill_timing(unsigned long long* device_buf);
+
+/* Measurement and test hook for single-layer batches of 32..64 tokens, where
+ * the single-launch decode kernel routes the batch and then either finishes
+ * the layer on the CUDA cores or leaves it to the grouped tensor-core kernels
+ * queued behind it, whichever its cost model predicts to be faster (skewed
+ * routing puts tens of tokens on a few experts, where the tensor cores win).
+ * mode 0: that choice (default); 1: always the CUDA-core kernel; 2: always
+ * the tensor-core kernels.  Other values mean 0.  Process-wide, not
+ * thread-safe. */
+void moe_debug_decode_path(int32_t mode);
 
 /* The cudaError_t value behind the calling thread's most recent
  * MOE_ERR_CUDA (0 if none). */

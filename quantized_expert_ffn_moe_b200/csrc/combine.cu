@@ -18,8 +18,13 @@ constexpr int kCombThreads = 256;
 
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const float* __restrict__ Y, const int* __restrict__ inv, int T, int k, int H, int shared,
-    uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next, float* __restrict__ out_f32) {
+    uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next, float* __restrict__ out_f32,
+    const int* __restrict__ gate) {
   pdl_wait();
+  if (gate && __ldcg(gate) == 0) {                // the fused decode kernel kept (and combined) the layer
+    pdl_launch_dependents();
+    return;
+  }
   const int t = blockIdx.x;
   const int P_routed = T * k;
   __shared__ int pos[16];
@@ -103,7 +108,7 @@ cudaError_t launch_combine(const LayerArgs& a) {
   return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, a.stream,
                     reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
                     a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next,
-                    a.y_f32);
+                    a.y_f32, a.gated ? reinterpret_cast<const int*>(a.ws + a.L.status) + ST_PATH : nullptr);
 }
 
 }  // namespace moe

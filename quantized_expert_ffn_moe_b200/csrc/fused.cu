@@ -66,6 +66,12 @@ struct FusedParams {
   int grp_xs;                     // halves of one group's chunk buffer
   long long xs_halves;            // halves of the whole token region
   int smem_route_off, smem_xs_off;
+  // single layer, 32..64 tokens: after routing, hand the layer to the grouped
+  // tcgen05 kernels that follow in the stream when their predicted time is
+  // lower (hybrid 1 = choose, 2 = always hand over)
+  int hybrid;
+  float cost_f0, cost_f1;         // CUDA-core time model: f0 + f1 * cost units per CTA (us)
+  float cost_t0, cost_t1;         // tensor-core time model: t0 + t1 * k-blocks per CTA (us)
   moe_layer_weights w[kMaxFusedLayers];
 };
 
@@ -670,6 +676,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   float* rnorm = reinterpret_cast<float*>(smem + 128);                   // [64]
   float* inv_all = reinterpret_cast<float*>(smem + 384);                 // [64]
   int* snslots = reinterpret_cast<int*>(smem + 640);
+  int* s_handover = snslots + 1;                                         // 1: tensor-core kernels take the layer
   int* scan_scratch = reinterpret_cast<int*>(smem + 768);                // [2 * kFCons]
   // [1024, 3072): per-group token metadata, 4 arrays of kMaxNTC each
   float* dinv = reinterpret_cast<float*>(smem + 3072);                   // [64] down rows staged at once
@@ -899,10 +906,75 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
           }
         }
         if (threadIdx.x == 0) { rt.woff_gu[ns] = gt; rt.woff_dn[ns] = dt; }
+        if (p.hybrid) {
+          // tensor-core work of the same slots: 128-token tiles of each slot
+          // over the gate/up (2I/128 row tiles x H/128 k-blocks) and down
+          // (H/128 x I/128) matrices
+          const int kb_tile = (2 * I / 128) * (H / 128) + (H / 128) * (I / 128);
+          int tk = 0;
+          for (int z = 0; z < SPT; ++z) {
+            const int u = u0 + z;
+            if (u < ns) {
+              const int e = rt.ulist[u];
+              const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+              tk += (n + 127) / 128;
+            }
+          }
+          int2 ttot;
+          const int2 trun = block_excl_scan2(tk, 0, scan_scratch, &ttot);
+          const float per_f = float(gt + dt) / float(G), per_t = float(ttot.x) * kb_tile / float(G);
+          const bool tc = p.hybrid == 2 || p.cost_t0 + p.cost_t1 * per_t < p.cost_f0 + p.cost_f1 * per_f;
+          if (threadIdx.x == 0) *s_handover = tc ? 1 : 0;
+          if (blockIdx.x == 0) {
+            if (threadIdx.x == 0) {
+              status[ST_COST_F] = gt + dt;
+              status[ST_COST_T] = ttot.x * kb_tile;
+              status[ST_PATH] = tc ? 1 : 0;
+            }
+            if (tc) {
+              // the routing in the layout the grouped kernels read
+              int* g_counts = reinterpret_cast<int*>(ws + p.L_.counts);
+              int* g_offsets = reinterpret_cast<int*>(ws + p.L_.offsets);
+              int* g_pairs = reinterpret_cast<int*>(ws + p.L_.pairs);
+              int* g_inv = reinterpret_cast<int*>(ws + p.L_.inv);
+              int* g_ulist = reinterpret_cast<int*>(ws + p.L_.ulist);
+              int* g_ntoff = reinterpret_cast<int*>(ws + p.L_.ntoff);
+              int* g_idx = reinterpret_cast<int*>(ws + p.L_.topk_idx);
+              float* g_w = reinterpret_cast<float*>(ws + p.L_.topk_w);
+              for (int e = threadIdx.x; e <= E; e += kFCons * 32) {
+                g_offsets[e] = rt.offsets[e];
+                if (e < E) g_counts[e] = rt.offsets[e + 1] - rt.offsets[e];
+              }
+              for (int u = threadIdx.x; u < ns; u += kFCons * 32) g_ulist[u] = rt.ulist[u];
+              for (int q = threadIdx.x; q < P; q += kFCons * 32) {
+                g_pairs[q] = rt.pairs[q];
+                g_inv[q] = rt.inv[q];
+                g_idx[q] = rt.idx[q];
+                g_w[q] = rt.w[q];
+              }
+              // token-tile prefix over the slots, in this thread's SPT slots
+              int run = trun.x;
+              for (int z = 0; z < SPT; ++z) {
+                const int u = u0 + z;
+                if (u < ns) {
+                  const int e = rt.ulist[u];
+                  const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+                  g_ntoff[u] = run;
+                  run += (n + 127) / 128;
+                }
+              }
+              if (threadIdx.x == 0) {
+                g_ntoff[ns] = ttot.x;
+                status[ST_UCOUNT] = ns - S;
+              }
+            }
+          }
+        }
       }
     }
     __syncthreads();                 // routing of this layer ready for all warps
     stamp(l, 2);
+    if (p.hybrid && *s_handover) break;     // the grouped tensor-core kernels take the layer
 
     const int ns = *snslots;
     FCursor cg{};
@@ -1093,6 +1165,14 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
 
 unsigned long long* g_fused_timing = nullptr;
 
+// Hand-over time models, [0] 4-bit/32, [1] 2-bit/16: layer time in us as
+// f0 + f1 * (CUDA-core cost units per CTA) and t0 + t1 * (tensor-core
+// k-blocks per CTA), least-squares fits to 120 layer times measured on a B200
+// (32..64 tokens, near-uniform and Zipf-skewed routing; largest residual
+// 16 us); on those batches the comparison picked the faster path every time.
+constexpr float kHyF0[2] = {57.9f, 72.5f}, kHyF1[2] = {0.1655f, 0.1294f};
+constexpr float kHyT0[2] = {89.7f, 93.5f}, kHyT1[2] = {0.6231f, 0.5696f};
+
 void set_fused_timing(unsigned long long* buf) { g_fused_timing = buf; }
 
 bool fused_supported(const moe_config& c, int T) {
@@ -1100,9 +1180,14 @@ bool fused_supported(const moe_config& c, int T) {
   return c.hidden == 2048 && c.inter == 768 && (c.num_experts % 32) == 0 && c.num_experts <= 1024;
 }
 
+int g_decode_path_mode = 0;
+
+void set_decode_path_mode(int mode) { g_decode_path_mode = mode; }
+int decode_path_mode() { return g_decode_path_mode; }
+
 cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x,
                                 uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
-                                cudaStream_t s) {
+                                cudaStream_t s, int hybrid) {
   for (int l0 = 0; l0 < L; l0 += kMaxFusedLayers) {
     FusedParams p{};
     p.cfg = c;
@@ -1115,6 +1200,11 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
     p.timing = l0 == 0 ? g_fused_timing : nullptr;
     p.ws = ws;
     p.L_ = Lw;
+    p.hybrid = (hybrid && L == 1) ? hybrid : 0;
+    // time models of the layer (us) from per-CTA work: CUDA cores
+    // f0 + f1 * cost units, tensor cores t0 + t1 * k-blocks
+    if (c.bits == 4) { p.cost_f0 = kHyF0[0]; p.cost_f1 = kHyF1[0]; p.cost_t0 = kHyT0[0]; p.cost_t1 = kHyT1[0]; }
+    else { p.cost_f0 = kHyF0[1]; p.cost_f1 = kHyF1[1]; p.cost_t0 = kHyT0[1]; p.cost_t1 = kHyT1[1]; }
     for (int l = 0; l < p.L; ++l) p.w[l] = layers[l0 + l];
     cudaError_t err;
     const int npl = c.num_experts / 32;

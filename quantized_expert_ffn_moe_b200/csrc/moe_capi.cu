@@ -16,6 +16,8 @@ namespace {
 // Batches of up to this many tokens take the decode path (grouped GEMV on CUDA
 // cores); larger batches the tensor-core prefill path.
 constexpr int kDecodeMaxTokens = 64;
+// Single-layer batches from this size up may hand over to the tensor cores.
+constexpr int kHybridMinTokens = 32;
 
 int num_sms_current() {
   static int cached[64] = {0};
@@ -167,7 +169,17 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
   if (T <= kDecodeMaxTokens && fused_supported(*cfg, T)) {
     const int call = (g_prof.on && g_prof.used < g_prof.cap) ? g_prof.used++ : -1;
     prof_mark(call, 0, a.stream);
-    const cudaError_t e = launch_fused_decode(*cfg, w, 1, x, y, false, T, nullptr, a.ws, a.L, a.num_sms, a.stream);
+    // 32..64 tokens: the fused kernel routes and then either finishes the
+    // layer or, when its cost model favours them, leaves it to the grouped
+    // tensor-core kernels queued behind it (they do nothing otherwise)
+    const int mode = decode_path_mode();
+    const int hybrid = (T >= kHybridMinTokens && prefill_supported(*cfg) && mode != 1) ? (mode == 2 ? 2 : 1) : 0;
+    cudaError_t e = launch_fused_decode(*cfg, w, 1, x, y, false, T, nullptr, a.ws, a.L, a.num_sms, a.stream, hybrid);
+    if (e == cudaSuccess && hybrid) {
+      a.gated = 1;
+      e = launch_prefill_ffn(a);
+      if (e == cudaSuccess) e = launch_combine(a);
+    }
     if (e == cudaSuccess) {
       for (int ph = 1; ph <= 4; ++ph) prof_mark(call, ph, a.stream);
       if (call >= 0) g_prof.fused[call] = 1;
@@ -310,6 +322,8 @@ int moe_last_cuda_error(void) { return g_last_cuda_error; }
 void moe_debug_fused_timing(unsigned long long* device_buf) { set_fused_timing(device_buf); }
 
 void moe_debug_prefill_timing(unsigned long long* device_buf) { set_prefill_timing(device_buf); }
+
+void moe_debug_decode_path(int32_t mode) { set_decode_path_mode(mode >= 0 && mode <= 2 ? mode : 0); }
 
 const char* moe_status_str(int status) {
   switch (status) {

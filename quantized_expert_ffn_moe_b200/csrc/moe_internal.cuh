@@ -20,6 +20,9 @@ enum StatusSlot {
   ST_ERROR = 0,      // first failed device check (0 = none)
   ST_ERROR_AUX = 1,  // detail of that check
   ST_UCOUNT = 2,     // number of distinct routed experts selected
+  ST_PATH = 3,       // fused decode with a tensor-core alternative: 1 = the grouped tcgen05 kernels run this call
+  ST_COST_F = 4,     // that choice's inputs: CUDA-core cost units (gate/up + down) of the batch,
+  ST_COST_T = 5,     //   and tensor-core k-blocks (128 rows x 128 tokens x 128 deep) of the batch
   ST_GRID_COUNT = 32,  // fused decode: grid barrier arrivals (own 128-byte line)
   ST_GRID_GEN = 64,    // fused decode: grid barrier generation (own 128-byte line)
   ST_COUNT = 96
@@ -447,6 +450,7 @@ struct LayerArgs {
   Layout L;
   int num_sms;
   cudaStream_t stream;
+  int gated = 0;                  // run the tensor-core kernels only if the fused decode kernel handed over
   int ep_rank = 0, ep_size = 1;   // expert-parallel share: experts e with e % ep_size == ep_rank
   float* y_f32 = nullptr;         // [T][H] fp32 partial output (expert-parallel share) instead of y
 };
@@ -465,8 +469,13 @@ void set_prefill_timing(unsigned long long* buf);
 extern unsigned long long* g_prefill_timing;
 cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x,
                                 uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
-                                cudaStream_t s);
+                                cudaStream_t s, int hybrid = 0);
 bool prefill_supported(const moe_config& c);
+// Decode-path choice for single layers of 32..64 tokens: 0 = by the cost
+// model after routing, 1 = always the fused CUDA-core kernel, 2 = always the
+// grouped tensor-core kernels (measurement hook moe_debug_decode_path).
+void set_decode_path_mode(int mode);
+int decode_path_mode();
 bool router_gemm_supported(const moe_config& c, int T);
 cudaError_t launch_router_gemm(const moe_config& c, const uint16_t* router_w, const float* bias, const uint16_t* x,
                                int T, float* logits, int* status, int num_sms, cudaStream_t s);

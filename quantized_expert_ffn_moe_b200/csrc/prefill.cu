@@ -85,6 +85,7 @@ struct PrefillArgs {
   float* yout;            // down: Y [P][H] fp32
   int* status;
   unsigned long long* timing;   // null, or [gridDim][16] per-role wait times (ns) of this launch
+  int gated;                    // 1: no tiles unless the fused decode kernel handed the layer over
 };
 
 constexpr int kPTime = 16;
@@ -267,7 +268,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   const unsigned long long t_start = tm ? global_ns() : 0;
 
   const RouteView& rv = a.rv;
-  const int nslots = __ldcg(rv.status + ST_UCOUNT) + rv.shared;
+  const bool closed = a.gated && __ldcg(rv.status + ST_PATH) == 0;     // the fused decode kernel kept the layer
+  const int nslots = closed ? 0 : __ldcg(rv.status + ST_UCOUNT) + rv.shared;
   const int mt = a.rows_pe / PBM;
   // slot table into shared memory (nslots <= E + 1): one L2 round trip here
   // instead of a dependent binary search through global memory per tile
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     if (i < nslots) slot_range(rv, i, &stab.e[i], &stab.p0[i], &stab.n[i]);
   }
   __syncthreads();
-  const int ntiles = stab.ntoff[nslots] * mt;
+  const int ntiles = closed ? 0 : stab.ntoff[nslots] * mt;
   const int KB = a.K / PSK, KR = a.K / RAWK;
   // this CTA's tiles (t = blockIdx.x + i * gridDim.x) decoded once into a
   // shared table, read by every role; beyond kTileTab tiles the lookup is redone
@@ -577,9 +579,11 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
 // bf16 values; xinv[p] undoes it).  One warp per pair position.
 template <int BITS>
 __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __restrict__ x, RouteView rv, int H,
-                                                            uint16_t* __restrict__ xs, float* __restrict__ xinv) {
+                                                            uint16_t* __restrict__ xs, float* __restrict__ xinv,
+                                                            int gated) {
   pdl_wait();
   pdl_launch_dependents();
+  if (gated && __ldcg(rv.status + ST_PATH) == 0) return;     // the fused decode kernel kept the layer
   constexpr int G = BITS == 4 ? 8 : 16;
   const int P = rv.T * rv.k + (rv.shared ? rv.T : 0);
   // routed positions in use: all T*k, or fewer when the experts are split
@@ -858,8 +862,10 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   uint16_t* hs = reinterpret_cast<uint16_t*>(a.ws + a.L.h);
   float* xinv = reinterpret_cast<float*>(a.ws + a.L.xscale);
   cudaError_t err = bits == 4
-      ? launch_pdl(gather_tokens_kernel<4>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv)
-      : launch_pdl(gather_tokens_kernel<2>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv);
+      ? launch_pdl(gather_tokens_kernel<4>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv,
+                   a.gated)
+      : launch_pdl(gather_tokens_kernel<2>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv,
+                   a.gated);
   if (err != cudaSuccess) return err;
 
   PrefillArgs g{};
@@ -868,6 +874,7 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   g.hout = hs; g.yout = nullptr; g.xinv = xinv;
   g.status = reinterpret_cast<int*>(a.ws + a.L.status);
   g.timing = g_prefill_timing;
+  g.gated = a.gated;
   const bool sh = c.shared_inter > 0;
   err = bits == 4 ? launch_gemm<0, 4>(g, a.w.gate_up_codes, a.w.gate_up_scales, a.w.shared_gate_up_codes,
                                       a.w.shared_gate_up_scales, c.num_experts, sh, xs, P, a.num_sms, a.stream)

@@ -338,10 +338,33 @@ def _sampled_full_case(shape, T, batch, seed, n_sample, sample_seed):
     gc.assert_close(y[sel], ref)
 
 
+def _with_path(mode, fn):
+    """Runs fn with the 32..64-token decode path fixed (1 CUDA cores, 2 tensor
+    cores, 0 the cost model's choice)."""
+    lib = q.load_library()
+    lib.moe_debug_decode_path(mode)
+    try:
+        fn()
+    finally:
+        lib.moe_debug_decode_path(0)
+
+
 def test_layer_full4_decode_unstaged_chunks():
     # 40 tokens do not fit the fused decode kernel's once-per-layer token
     # staging, so gate/up stages its tokens per slot chunk and per consumer group
-    _sampled_full_case(mi.FULL4, 40, 3, 0, 4, 40)
+    _with_path(1, lambda: _sampled_full_case(mi.FULL4, 40, 3, 0, 4, 40))
+
+
+@pytest.mark.parametrize("mode", [1, 2, 0], ids=["cuda_cores", "tensor_cores", "cost_model"])
+def test_decode_handover_full2_zipf(mode):
+    """Skewed 2-bit batches of 33 and 64 tokens on each decode path: after the
+    fused kernel's routing, the grouped tcgen05 kernels read its exported
+    routing and finish the layer."""
+    _with_path(mode, lambda: _stored_layer_case("full2_zipf_decode", [33, 64]))
+
+
+def test_decode_handover_full4():
+    _with_path(2, lambda: _sampled_full_case(mi.FULL4, 48, 5, 0, 4, 48))
 
 
 def test_prefill_full4_large_batch_tile_lookup():
