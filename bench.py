@@ -29,7 +29,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-EXPERT_BYTES = {4: 2654208, 2: 1769472}     # packed gate/up + down of one expert (H=2048, I=768)
+EXPERT_BYTES = {4: 2654208, 2: 1769472,     # packed gate/up + down of one expert (H=2048, I=768)
+                "4g128": 2433024}            # 4-bit with one fp16 scale per 128 elements
 GU_BYTES = {4: 1769472, 2: 1179648}
 ROUTER_BYTES = 512 * 2048 * 2
 METRIC = "MoE-layer decode tokens/s (512 experts, top-10 + shared, H=2048, I=768, 4-bit/32, 16 tokens)"
@@ -487,6 +488,13 @@ def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
 
     for T in (1, 4):
         layer_rate(cfg, shape, pool4, T, 4000, 4, f"decode4_t{T}")
+    # 4-bit with GPTQ-style 128-element groups, 16 tokens (4 layer instances:
+    # 9.7 GB, far above L2)
+    sg = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=128)
+    cfg_g = q.config_of(512, 2048, 768, 10, True, 4, 128)
+    poolg = R.layers(sg, 4)
+    layer_rate(cfg_g, sg, poolg, 16, 2000, "4g128", "decode4g128_t16")
+    del poolg
     layer_rate(cfg, shape, pool4, 4096, 8, 4, "prefill4_t4096")
 
     # expert-parallel share: one rank's partial of the 4096-token layer when

@@ -83,7 +83,7 @@ __global__ void gen_pool_kernel(PoolArgs a) {
       K = a.I;
     }
     const uint64_t key = stream_key(a.seed, (uint64_t)a.layer, (uint64_t)role, (uint64_t)expert);
-    float w[32];
+    float w[128];                        // block <= 128 elements
     float amax = 0.f;
     for (int j = 0; j < a.block; ++j) {
       w[j] = normal_at(key, (uint64_t)row * K + col0 + j, a.c);
@@ -91,7 +91,7 @@ __global__ void gen_pool_kernel(PoolArgs a) {
     }
     const __half s16 = __float2half_rn(__fdiv_rn(amax, float(qmax)));
     const float sf = __half2float(s16);
-    uint32_t packed[4] = {0, 0, 0, 0};   // up to 16 bytes of codes per block
+    uint32_t packed[16] = {0};           // up to 64 bytes of codes per block
     for (int j = 0; j < a.block; ++j) {
       int q = 0;
       if (sf != 0.f) {
@@ -137,7 +137,7 @@ extern "C" {
 int moe_gen_pool(uint64_t seed, int layer, int E, int H, int I, int bits, int block, int e0, int ne, int shared,
                  float c, uint8_t* gu_codes, uint16_t* gu_scales, uint8_t* d_codes, uint16_t* d_scales,
                  void* stream) {
-  if (!((bits == 4 && block == 32) || (bits == 2 && block == 16))) return -2;
+  if (!((bits == 4 && (block == 32 || block == 128)) || (bits == 2 && block == 16))) return -2;
   if (ne <= 0 || (shared && ne != 1) || (!shared && (e0 < 0 || e0 + ne > E))) return -1;
   if (!gu_codes || !gu_scales || !d_codes || !d_scales) return -1;
   if (H % block || I % block) return -2;

@@ -35,6 +35,7 @@ struct FfnArgs {
   size_t expert_code_bytes;      // per routed expert
   size_t expert_scale_count;
   int rows;                      // rows per expert (2I gate/up, H down)
+  int block;                     // elements per scale
   int out_cols;                  // columns of the output buffer (I gate/up, H down)
   int ntc;                       // tokens staged per chunk
   const uint16_t* xin;           // GATEUP: [T][K] bf16 activations
@@ -165,9 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
         const uint16_t* sb = sh ? a.sh_scales : a.scales + size_t(cur.e) * a.expert_scale_count;
         const size_t row0 = size_t(cur.stage) * Gm::RPS;
         unsigned char* dst = ring + slot * Gm::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + Gm::SCALE_BYTES);
+        const int spr = scales_per_row(Gm::K, a.block);
+        const uint32_t sbytes = uint32_t(Gm::RPS) * spr * 2;
+        mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes);
         bulk_g2s(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot]);
-        bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * Gm::SPR, Gm::SCALE_BYTES, &full[slot]);
+        bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot]);
         ++issued;
       }
       // never leave with copies in flight
@@ -267,8 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
     }
     if (ok) {
       const unsigned char* st = ring + slot * Gm::STAGE_BYTES;
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * Gm::SPR * 2,
-                      cur.stage * Gm::RPS + rl0};
+      const int spr = scales_per_row(Gm::K, a.block);
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * spr * 2, cur.stage * Gm::RPS + rl0, spr,
+                      piece_shift(BITS, a.block)};
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += NTB) {
         const int nt = min(NTB, nc - tb);          // warp-uniform
@@ -287,9 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
 // same word decoders the GEMV uses (test hook, not on the timed path).
 template <int BITS>
 __global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
-                                    int row0, int rows, int cols, float* __restrict__ out) {
+                                    int row0, int rows, int cols, int BLOCK, float* __restrict__ out) {
   constexpr int G = BITS == 4 ? 8 : 16;
-  constexpr int BLOCK = BITS == 4 ? 32 : 16;
   const int words_per_row = cols / G;
   const long long total = (long long)rows * words_per_row;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -390,7 +393,7 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   g.sh_codes = a.w.shared_gate_up_codes; g.sh_scales = a.w.shared_gate_up_scales;
   g.expert_code_bytes = size_t(2 * I) * H * bits / 8;
   g.expert_scale_count = size_t(2 * I) * (H / c.block);
-  g.rows = 2 * I; g.out_cols = I; g.ntc = pg.ntc;
+  g.rows = 2 * I; g.out_cols = I; g.ntc = pg.ntc; g.block = c.block;
   g.xin = a.x; g.hin = nullptr;
   g.out = reinterpret_cast<float*>(a.ws + a.L.h);
   g.status = reinterpret_cast<int*>(a.ws + a.L.status);
@@ -406,7 +409,7 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   d.sh_codes = a.w.shared_down_codes; d.sh_scales = a.w.shared_down_scales;
   d.expert_code_bytes = size_t(H) * I * bits / 8;
   d.expert_scale_count = size_t(H) * (I / c.block);
-  d.rows = H; d.out_cols = H; d.ntc = pd.ntc;
+  d.rows = H; d.out_cols = H; d.ntc = pd.ntc; d.block = c.block;
   d.xin = nullptr; d.hin = reinterpret_cast<const float*>(a.ws + a.L.h);
   d.out = reinterpret_cast<float*>(a.ws + a.L.y);
   d.status = reinterpret_cast<int*>(a.ws + a.L.status);
@@ -415,14 +418,14 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   return bits == 4 ? dispatch<DOWN, 4>(I, d, a.num_sms, a.stream) : dispatch<DOWN, 2>(I, d, a.num_sms, a.stream);
 }
 
-cudaError_t launch_dequant_rows(int bits, int, const uint8_t* codes, const uint16_t* scales, int row0, int rows,
+cudaError_t launch_dequant_rows(int bits, int block, const uint8_t* codes, const uint16_t* scales, int row0, int rows,
                                 int cols, float* out, cudaStream_t s) {
   const int G = bits == 4 ? 8 : 16;
   const long long total = (long long)rows * (cols / G);
   const long long want = (total + 255) / 256;
   const int blocks = int(want < 4096 ? want : 4096);
-  if (bits == 4) dequant_rows_kernel<4><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, out);
-  else dequant_rows_kernel<2><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, out);
+  if (bits == 4) dequant_rows_kernel<4><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, out);
+  else dequant_rows_kernel<2><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, out);
   return cudaGetLastError();
 }
 

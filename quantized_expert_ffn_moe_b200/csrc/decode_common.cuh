@@ -22,8 +22,8 @@ struct Geom {
   static constexpr int K = LPR * CPL * W16;           // reduction length
   static constexpr int NPART = BITS == 4 ? 1 : 2;     // 16-byte activation slots per code word
   static constexpr int G = BITS == 4 ? 8 : 16;        // elements per code word
-  static constexpr int BLOCK = BITS == 4 ? 32 : 16;
-  static constexpr int SPR = K / BLOCK;               // scales per row
+  static constexpr int BLOCK = BITS == 4 ? 32 : 16;  // smallest block of the format (4-bit also runs 128)
+  static constexpr int SPR = K / BLOCK;               // scales per row at that block (stage upper bound)
   static constexpr int RB = K * BITS / 8;             // code bytes per row
   static constexpr int RPS = kNCW * RW * 2;           // rows per pipeline stage
   static constexpr int CODE_BYTES = RPS * RB;
@@ -47,12 +47,19 @@ __device__ __forceinline__ int staged_offset(int h) {
 }
 
 // Two rows of one stage (codes + scales in shared memory) and their row index
-// in the expert matrix.
+// in the expert matrix.  spr = scales per row (K / block); 4-bit: ps =
+// log2(block / 32), so the 32-element piece c takes scale c >> ps.
 struct Rows {
   const unsigned char* codes;     // row rl0; row rl0+1 follows at +RB
-  const unsigned char* scales;    // row rl0; row rl0+1 follows at +SPR*2
+  const unsigned char* scales;    // row rl0; row rl0+1 follows at +spr*2
   int r0;
+  int spr, ps;
 };
+
+// Scales per row and the piece-to-scale shift of a 4-bit block of 32 or 128
+// (2-bit: blocks of 16, four per 64-element piece).
+__host__ __device__ inline int scales_per_row(int K, int block) { return K / block; }
+__host__ __device__ inline int piece_shift(int bits, int block) { return bits == 4 && block == 128 ? 2 : 0; }
 
 // Dot products of the lane group's two rows with NT staged tokens, reduced
 // over the LPR lanes of the row, then the epilogue.  Each block's products
@@ -89,7 +96,7 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
       float sc[2];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
-        sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * Gm::SPR * 2 + c * 2));
+        sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * rw.spr * 2 + (c >> rw.ps) * 2));
       __half2 hacc[2][NT][2];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
@@ -121,7 +128,7 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
     } else {
       uint2 scp[2];
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
+      for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * rw.spr * 2 + c * 8);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         __half2 q[2][8];

@@ -550,7 +550,9 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
     if (timed) { tacc[0] += global_ns() - tw; tacc[2] += 1; }
     if (ok) {
       const unsigned char* st = ring + slot * ring_stride;
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * Gm::SPR * 2, cur.stage * Gm::RPS + rl0};
+      const int spr = scales_per_row(K, p.cfg.block);
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * spr * 2, cur.stage * Gm::RPS + rl0, spr,
+                      piece_shift(BITS, p.cfg.block)};
       const int nc = cur.nc;
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
@@ -617,7 +619,7 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
                              const uint8_t* sh_codes, const uint16_t* sh_scales, size_t expert_code_bytes,
                              size_t expert_scale_count, unsigned char* ring, int ring_stride, uint64_t* full,
                              uint64_t* empty, int* issued, volatile int* abort_flag, int* status, Publisher& pub,
-                             bool gate_up) {
+                             bool gate_up, int block) {
   using Gm = Geom<BITS, LPR, CPL>;
   for (; cur.valid(w1); cur.advance()) {
     const int i = *issued;
@@ -636,9 +638,11 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
     const uint16_t* sb = sh ? sh_scales : scales + size_t(cur.e) * expert_scale_count;
     const size_t row0 = size_t(cur.stage) * Gm::RPS;
     unsigned char* dst = ring + slot * ring_stride;
-    mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + Gm::SCALE_BYTES);
+    const int spr = scales_per_row(Gm::K, block);
+    const uint32_t sbytes = uint32_t(Gm::RPS) * spr * 2;
+    mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes);
     bulk_g2s(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot]);
-    bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * Gm::SPR, Gm::SCALE_BYTES, &full[slot]);
+    bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot]);
     pub.rslot[slot] = gate_up ? cur.slot : -1;
     if (gate_up) ++pub.pending;
     *issued = i + 1;
@@ -997,14 +1001,14 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
           produce_pass<BITS, LG, CG>(cg, g1, lw.gate_up_codes, lw.gate_up_scales, lw.shared_gate_up_codes,
                                       lw.shared_gate_up_scales, size_t(2 * I) * H * c.bits / 8,
                                       size_t(2 * I) * (H / c.block), ring, RING_STRIDE, full, empty, &issued,
-                                      abort_flag, status, pub, true);
+                                      abort_flag, status, pub, true, c.block);
         }
         pub.issued_all();
         if (d0 < d1) {
           cd.init(d0);
           produce_pass<BITS, LD, CD>(cd, d1, lw.down_codes, lw.down_scales, lw.shared_down_codes,
                                       lw.shared_down_scales, size_t(H) * I * c.bits / 8, size_t(H) * (I / c.block),
-                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false);
+                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false, c.block);
         }
         drain_publish(issued, empty, abort_flag, status, pub);
       }

@@ -39,7 +39,8 @@ int validate_config(const moe_config* c) {
     return MOE_ERR_INVALID_ARG;
   if (c->num_experts > 1024 || c->num_experts % 32 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->top_k > 16 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
-  if (!((c->bits == 4 && c->block == 32) || (c->bits == 2 && c->block == 16))) return MOE_ERR_UNSUPPORTED;
+  if (!((c->bits == 4 && (c->block == 32 || c->block == 128)) || (c->bits == 2 && c->block == 16)))
+    return MOE_ERR_UNSUPPORTED;
   const int H = c->hidden;
   if (!(H == 256 || H == 512 || H == 1024 || H == 2048 || H == 4096)) return MOE_ERR_UNSUPPORTED;
   if (c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
@@ -276,7 +277,8 @@ int moe_device_status(const void* workspace, int32_t* code_out) {
 int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t* scales, int32_t row0,
                      int32_t rows, int32_t cols, float* out, void* stream) {
   if (!cfg || !codes || !scales || !out || row0 < 0 || rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
-  if (!((cfg->bits == 4 && cfg->block == 32) || (cfg->bits == 2 && cfg->block == 16))) return MOE_ERR_UNSUPPORTED;
+  if (!((cfg->bits == 4 && (cfg->block == 32 || cfg->block == 128)) || (cfg->bits == 2 && cfg->block == 16)))
+    return MOE_ERR_UNSUPPORTED;
   if (cols % cfg->block != 0 || (cols * cfg->bits / 8) % 4 != 0) return MOE_ERR_UNSUPPORTED;
   if (!aligned(codes, 4) || !aligned(scales, 2) || !aligned(out, 4)) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;

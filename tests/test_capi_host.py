@@ -61,7 +61,8 @@ def test_workspace_bytes(lib):
     assert q.moe_workspace_bytes(cfg(), -1) == 0
 
 
-@pytest.mark.parametrize("kw", [dict(bits=3), dict(bits=4, block=16), dict(bits=2, block=32), dict(hidden=300),
+@pytest.mark.parametrize("kw", [dict(bits=3), dict(bits=4, block=16), dict(bits=4, block=64), dict(bits=2, block=32),
+                                dict(bits=2, block=128), dict(hidden=300),
                                 dict(experts=500), dict(top_k=17), dict(inter=100), dict(experts=2048)])
 def test_unsupported_configs_report_zero_workspace(lib, kw):
     assert q.moe_workspace_bytes(cfg(**kw), 16) == 0
@@ -71,6 +72,7 @@ def test_tiny_and_2bit_configs_supported(lib):
     assert q.moe_workspace_bytes(q.config_of(64, 256, 128, 4, True, 4, 32), 8) > 0
     assert q.moe_workspace_bytes(cfg(bits=2, block=16), 64) > 0
     assert q.moe_workspace_bytes(cfg(shared=False), 64) > 0
+    assert q.moe_workspace_bytes(cfg(bits=4, block=128), 64) > 0      # GPTQ-style 128-element groups
 
 
 def _fake_weights(shared=True, misalign=None):

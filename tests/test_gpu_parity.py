@@ -17,6 +17,9 @@ import quantized_expert_ffn_moe_b200 as q
 pytestmark = pytest.mark.gpu
 
 SHAPE_2BIT_TINY = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=2, block=16)
+# 4-bit with one scale per 128 elements (the GPTQ-style group size)
+TINY_G128 = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=4, block=128)
+FULL4_G128 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=128)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -33,7 +36,8 @@ def _cuda():
 
 # ------------------------------------------------------------ input bytes ---
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2], ids=["tiny4", "tiny2", "full4", "full2"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, TINY_G128],
+                         ids=["tiny4", "tiny2", "full4", "full2", "tiny4g128"])
 def test_device_generator_matches_host(shape):
     """The device generator writes the same bytes as the numpy generator."""
     w = gc.device_layer(shape, seed=3, layer=5)
@@ -51,7 +55,8 @@ def test_device_generator_matches_host(shape):
 
 # ----------------------------------------------------------- dequant hook ---
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2], ids=["tiny4", "tiny2", "full4", "full2"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, FULL4_G128],
+                         ids=["tiny4", "tiny2", "full4", "full2", "full4g128"])
 def test_device_decoder_bit_exact(shape):
     torch = gc.torch()
     w = gc.device_layer(shape, seed=1, layer=0)
@@ -128,7 +133,7 @@ def _oracle_given(lay, x_bits, gpu_idx, differ):
     return orc.layer_forward(lay, x_bits, topk_override=over)
 
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY], ids=["tiny4", "tiny2"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, TINY_G128], ids=["tiny4", "tiny2", "tiny4g128"])
 @pytest.mark.parametrize("T", [1, 2, 7, 8, 17, 64, 100])
 def test_layer_tiny_live_oracle(shape, T):
     x = mi.hidden_states_bf16(T, shape.hidden, 0, 0)
@@ -435,3 +440,13 @@ def test_expert_parallel_full4_decode_stored_oracle():
     for ep_size in (2, 4):
         tot = sum(_ep_partials(shape, w, x, ep_size))
         gc.assert_close(tot[sel][keep], ref[keep])
+
+
+# ------------------------------------------------- 4-bit, 128-element groups ---
+
+@pytest.mark.parametrize("T", [16, 48, 100])
+def test_layer_full4_g128_sampled(T):
+    """Full shape with one scale per 128 elements: the fused decode kernel at
+    16 and 48 tokens, the stand-alone GEMV kernels at 100 (no tensor-core path
+    for this group size)."""
+    _sampled_full_case(FULL4_G128, T, 7, 0, 4, 128 + T)

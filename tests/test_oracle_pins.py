@@ -45,7 +45,7 @@ def test_format_blocks_hand_decoded():
         np.testing.assert_array_equal(got, exp)
 
 
-@pytest.mark.parametrize("bits,block", [(4, 32), (2, 16)])
+@pytest.mark.parametrize("bits,block", [(4, 32), (4, 128), (2, 16)])
 def test_encoder_roundtrip_bound(bits, block):
     """|w - dequant(encode(w))| <= max(s/2, absmax - qmax*s) per element, where
     the second term covers an fp16 scale rounded below absmax/qmax.  A wrong
