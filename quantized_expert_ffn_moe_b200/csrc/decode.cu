@@ -103,7 +103,7 @@ struct Cursor {
   }
 };
 
-template <int MODE, int BITS, int LPR, int CPL>
+template <int MODE, int BITS, int LPR, int CPL, int PS>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
@@ -270,15 +270,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
     }
     if (ok) {
       const unsigned char* st = ring + slot * Gm::STAGE_BYTES;
-      const int spr = scales_per_row(Gm::K, a.block);
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * spr * 2, cur.stage * Gm::RPS + rl0, spr,
-                      piece_shift(BITS, a.block)};
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0};
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += NTB) {
         const int nt = min(NTB, nc - tb);          // warp-uniform
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 1);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 2);
-        else rows_dot<MODE, BITS, LPR, CPL, 4>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 1);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 2);
+        else rows_dot<MODE, BITS, LPR, CPL, 4, PS>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
       }
     }
     __syncwarp();
@@ -322,10 +320,10 @@ PassPlan plan_of(int rows, int K) {
   return p;
 }
 
-template <int MODE, int BITS, int LPR, int CPL>
+template <int MODE, int BITS, int LPR, int CPL, int PS>
 cudaError_t launch_one(FfnArgs fa, int num_sms, cudaStream_t s) {
   using Gm = Geom<BITS, LPR, CPL>;
-  auto kern = ffn_tma_kernel<MODE, BITS, LPR, CPL>;
+  auto kern = ffn_tma_kernel<MODE, BITS, LPR, CPL, PS>;
   const size_t smem = 256 + size_t(kStages) * Gm::STAGE_BYTES + size_t(fa.ntc) * Gm::K * 2 + kMaxNTC * 12;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -341,7 +339,12 @@ template <int MODE, int BITS>
 cudaError_t dispatch(int K, FfnArgs fa, int num_sms, cudaStream_t s) {
   const int C = K * BITS / 8 / 16;
   switch (C) {
-#define X(c, lpr, cpl) case c: return launch_one<MODE, BITS, lpr, cpl>(fa, num_sms, s);
+#define X(c, lpr, cpl)                                                              \
+  case c:                                                                           \
+    if constexpr (BITS == 4) {                                                      \
+      if (fa.block == 128) return launch_one<MODE, BITS, lpr, cpl, 2>(fa, num_sms, s); \
+    }                                                                               \
+    return launch_one<MODE, BITS, lpr, cpl, 0>(fa, num_sms, s);
     MOE_C_CASES(X)
 #undef X
     default: return cudaErrorInvalidValue;

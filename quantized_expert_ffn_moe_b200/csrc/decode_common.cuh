@@ -47,17 +47,16 @@ __device__ __forceinline__ int staged_offset(int h) {
 }
 
 // Two rows of one stage (codes + scales in shared memory) and their row index
-// in the expert matrix.  spr = scales per row (K / block); 4-bit: ps =
-// log2(block / 32), so the 32-element piece c takes scale c >> ps.
+// in the expert matrix.
 struct Rows {
   const unsigned char* codes;     // row rl0; row rl0+1 follows at +RB
-  const unsigned char* scales;    // row rl0; row rl0+1 follows at +spr*2
+  const unsigned char* scales;    // row rl0; row rl0+1 follows at +(SPR >> PS)*2
   int r0;
-  int spr, ps;
 };
 
-// Scales per row and the piece-to-scale shift of a 4-bit block of 32 or 128
-// (2-bit: blocks of 16, four per 64-element piece).
+// Scales per row, and the piece-to-scale shift PS of a 4-bit block of 32
+// (PS 0) or 128 (PS 2): the 32-element piece c takes scale c >> PS.  2-bit:
+// blocks of 16, four per 64-element piece, PS 0.
 __host__ __device__ inline int scales_per_row(int K, int block) { return K / block; }
 __host__ __device__ inline int piece_shift(int bits, int block) { return bits == 4 && block == 128 ? 2 : 0; }
 
@@ -65,7 +64,7 @@ __host__ __device__ inline int piece_shift(int bits, int block) { return bits ==
 // over the LPR lanes of the row, then the epilogue.  Each block's products
 // accumulate in two independent fp16x2 chains (even / odd code words) and
 // are folded into fp32 with the block scale.  `nt` <= NT tokens are valid.
-template <int MODE, int BITS, int LPR, int CPL, int NT>
+template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0>
 __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& rw, const __half* xs, int tb, int lr,
                                          const float* tok_inv, const float* tok_w, const int* tok_pos,
                                          int nt = NT, const int* xrow = nullptr) {
@@ -96,7 +95,7 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
       float sc[2];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
-        sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * rw.spr * 2 + (c >> rw.ps) * 2));
+        sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * (Gm::SPR >> PS) * 2 + (c >> PS) * 2));
       __half2 hacc[2][NT][2];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
@@ -128,7 +127,7 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
     } else {
       uint2 scp[2];
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * rw.spr * 2 + c * 8);
+      for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         __half2 q[2][8];

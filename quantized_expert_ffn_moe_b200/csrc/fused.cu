@@ -493,7 +493,7 @@ struct GroupTok {
 // (warps grp*kNCW ...): walks the same stage sequence as the producer and
 // takes the stages whose index has the group's parity.  A group stages the
 // tokens of a (slot, chunk) itself when it meets its first stage of it.
-template <int MODE, int BITS, int LPR, int CPL>
+template <int MODE, int BITS, int LPR, int CPL, int PS>
 __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur, long long w1, unsigned char* ring,
                              int ring_stride, uint64_t* full, uint64_t* empty, int* consumed, int grp,
                              const uint16_t* xsrc, const float* rnorm, const float* hin, float* out, int out_cols,
@@ -550,18 +550,16 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
     if (timed) { tacc[0] += global_ns() - tw; tacc[2] += 1; }
     if (ok) {
       const unsigned char* st = ring + slot * ring_stride;
-      const int spr = scales_per_row(K, p.cfg.block);
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * spr * 2, cur.stage * Gm::RPS + rl0, spr,
-                      piece_shift(BITS, p.cfg.block)};
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0};
       const int nc = cur.nc;
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
         const int nt = min(4, nc - tb);
         const __half* xb = pre ? xs_pre : xs_grp + size_t(tb) * K;
         const int* xr = pre ? tk.xrow : nullptr;
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 1, xr);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 2, xr);
-        else rows_dot<MODE, BITS, LPR, CPL, 4>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, nt, xr);
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 1, xr);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 2, xr);
+        else rows_dot<MODE, BITS, LPR, CPL, 4, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, nt, xr);
       }
     }
     __syncwarp();
@@ -664,7 +662,7 @@ __device__ void drain_publish(int issued, uint64_t* empty, volatile int* abort_f
   pub.flush();
 }
 
-template <int BITS, int LG, int CG, int LD, int CD, int NPL>
+template <int BITS, int LG, int CG, int LD, int CD, int NPL, int PS>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
   using GU = Geom<BITS, LG, CG>;
   using DN = Geom<BITS, LD, CD>;
@@ -1016,7 +1014,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       // ---------------------------------------------------------- phase G
       if (g0 < g1) {
         cg.init(g0);
-        consume_pass<GATEUP, BITS, LG, CG>(p, rt, cg, g1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
+        consume_pass<GATEUP, BITS, LG, CG, PS>(p, rt, cg, g1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
                                            rnorm, nullptr, hbuf, I, p.pre ? xs : nullptr, inv_all, nullptr, 0, xs_grp,
                                            tk, abort_flag, status,
                                            p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 11 : nullptr);
@@ -1061,7 +1059,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
           }
           all_sync();
         }
-        consume_pass<DOWN, BITS, LD, CD>(p, rt, cd, d1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
+        consume_pass<DOWN, BITS, LD, CD, PS>(p, rt, cd, d1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
                                          rnorm, hbuf, ybuf, H, dpre ? xs : nullptr, dinv, dwt, lo, xs_grp, tk,
                                          abort_flag, status,
                                          p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 16 : nullptr);
@@ -1110,7 +1108,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   // the ring is drained: every issued stage was waited on by the consumers
 }
 
-template <int BITS, int LG, int CG, int LD, int CD, int NPL>
+template <int BITS, int LG, int CG, int LD, int CD, int NPL, int PS = 0>
 cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   using GU = Geom<BITS, LG, CG>;
   using DN = Geom<BITS, LD, CD>;
@@ -1149,7 +1147,7 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   q.xs_halves = (long long)xs_halves;
   const size_t smem = q.smem_xs_off + xs_halves * 2;
   if (smem > size_t(kSmemMax)) return cudaErrorInvalidValue;
-  auto kern = fused_decode_kernel<BITS, LG, CG, LD, CD, NPL>;
+  auto kern = fused_decode_kernel<BITS, LG, CG, LD, CD, NPL, PS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
@@ -1216,9 +1214,12 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
     //                                  32 lanes x 1 piece,   4 lanes x 3 (2-bit)
     if (c.bits == 4) {
       switch (npl) {
-        case 16: err = launch_fused_t<4, 16, 4, 8, 3, 16>(p, num_sms, s); break;
-        case 32: err = launch_fused_t<4, 16, 4, 8, 3, 32>(p, num_sms, s); break;
-        case 8: err = launch_fused_t<4, 16, 4, 8, 3, 8>(p, num_sms, s); break;
+        case 16: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 16, 2>(p, num_sms, s)
+                                      : launch_fused_t<4, 16, 4, 8, 3, 16>(p, num_sms, s); break;
+        case 32: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 32, 2>(p, num_sms, s)
+                                      : launch_fused_t<4, 16, 4, 8, 3, 32>(p, num_sms, s); break;
+        case 8: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 8, 2>(p, num_sms, s)
+                                     : launch_fused_t<4, 16, 4, 8, 3, 8>(p, num_sms, s); break;
         default: return cudaErrorInvalidValue;
       }
     } else {
