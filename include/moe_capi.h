@@ -188,7 +188,9 @@ int moe_profile_end(float* ms_out, int32_t* calls);
 /* Measurement hook: while device_buf is non-null, fused decode launches write
  * %globaltimer readings (ns) of each CTA's first layer to device_buf[cta][20]
  * (zero it first; the caller owns the buffer; null switches it off):
- *   [8] layer start, [0] router logits done, [1] after the first grid barrier,
+ *   [8] layer start, [14] token 0 staged (with its router logits when each
+ *   warp stages one token), [15] this CTA's router logits written,
+ *   [0] router logits done (CTA barrier), [1] after the first grid barrier,
  *   [9] top-k done, [10] grouping scan done, [2] work lists ready,
  *   [3] gate/up done, [4] after the second barrier, [5] down done,
  *   [6] after the third barrier, [7] combine done;
