@@ -20,7 +20,8 @@
  *   S     = the k largest l_e, slots by descending logit, ties -> smaller e
  *   w_j   = softmax over the selected logits (= full softmax renormalised)
  *   FFN_e = W_down,e (silu(W_gate,e x) * (W_up,e x)),   W = (code - 2^(b-1)) * scale
- *   out   = FFN_shared(x) + sum_j w_j FFN_{S_j}(x)      slot order, fp32, -> bf16
+ *   out   = g(x) FFN_shared(x) + sum_j w_j FFN_{S_j}(x)  slot order, fp32, -> bf16
+ *   g(x)  = 1, or sigmoid(sum_h x_h Wg[h]) when a shared-expert gate vector Wg is given
  *
  * Packed weight format (all arrays row-major, dense, caller-owned, device
  * memory, 16-byte aligned):
@@ -84,6 +85,12 @@ typedef struct moe_layer_weights {
   const uint16_t* shared_down_scales;     /* [H][I/block]                       */
   const uint16_t* router_w;               /* [E][H] bf16 bits                   */
   const float*    router_bias;            /* [E] fp32, or NULL (no bias)        */
+  const uint16_t* shared_gate_w;          /* [H] bf16 bits: the shared expert's
+                                             output is scaled by sigmoid(x . w)
+                                             (fp32); NULL = weight 1.  Needs a
+                                             shared expert.  Layers with a gate
+                                             run on the separate kernels, not
+                                             the single-launch decode kernel.  */
 } moe_layer_weights;
 
 /* Bytes of device workspace needed by moe_route / moe_layer_forward /

@@ -58,10 +58,12 @@ def fill_normal_bf16(key: int, start: int, out, c=gen.C_SIGMA002):
         raise RuntimeError(f"moe_gen_normal_bf16 failed: {st}")
 
 
-def device_layer_tensors(shape: gen.MoeShape, seed: int, layer: int, zipf: bool = False, device: str = "cuda"):
+def device_layer_tensors(shape: gen.MoeShape, seed: int, layer: int, zipf: bool = False, device: str = "cuda",
+                         shared_gate: bool = False):
     """One layer's inputs generated on the device: a dict of torch tensors named
     like the fields of the C ABI's moe_layer_weights (shared_* absent when the
-    shape has no shared expert, router_bias only for the skewed workload)."""
+    shape has no shared expert, router_bias only for the skewed workload,
+    shared_gate_w only when asked for)."""
     import torch
     E, H, I, b, bs = shape.experts, shape.hidden, shape.inter, shape.bits, shape.block
     t = dict(
@@ -82,6 +84,9 @@ def device_layer_tensors(shape: gen.MoeShape, seed: int, layer: int, zipf: bool 
         )
         fill_pool(shape, seed, layer, t["shared_gate_up_codes"], t["shared_gate_up_scales"],
                   t["shared_down_codes"], t["shared_down_scales"], shared=True)
+    if shared_gate and shape.shared:
+        t["shared_gate_w"] = torch.empty(H, dtype=torch.int16, device=device)
+        fill_normal_bf16(gen.stream_key(seed, layer, gen.ROLE_SH_GATE_W, 0), 0, t["shared_gate_w"], gen.C_SIGMA002)
     if zipf:
         t["router_bias"] = torch.from_numpy(gen.zipf_router_bias(shape, seed, layer)).to(device)
     return t

@@ -37,10 +37,10 @@ import numpy as np
 
 __all__ = [
     "GOLDEN", "ROLE_ROUTER", "ROLE_GATE", "ROLE_UP", "ROLE_DOWN", "ROLE_SH_GATE",
-    "ROLE_SH_UP", "ROLE_SH_DOWN", "ROLE_X", "ROLE_PERM", "C_SIGMA1", "C_SIGMA002",
+    "ROLE_SH_UP", "ROLE_SH_DOWN", "ROLE_X", "ROLE_PERM", "ROLE_SH_GATE_W", "C_SIGMA1", "C_SIGMA002",
     "ZIPF_ALPHA", "MoeShape", "TINY", "FULL4", "FULL2", "mix64", "stream_key",
     "normal_f32", "bf16_bits_from_f32", "bf16_bits_to_f32", "quantize_blocks",
-    "masters", "expert_packed", "shared_packed", "router_weight_bf16",
+    "masters", "expert_packed", "shared_packed", "router_weight_bf16", "shared_gate_weight_bf16",
     "hidden_states_bf16", "zipf_router_bias", "layer_packed_pool",
     "packed_row_bytes", "scales_per_row",
 ]
@@ -53,6 +53,7 @@ _M2 = 0x94D049BB133111EB
 ROLE_ROUTER, ROLE_GATE, ROLE_UP, ROLE_DOWN = 0, 1, 2, 3
 ROLE_SH_GATE, ROLE_SH_UP, ROLE_SH_DOWN = 4, 5, 6
 ROLE_X, ROLE_PERM = 7, 8
+ROLE_SH_GATE_W = 9          # the shared expert's gate vector (format variant)
 
 # sigma / std(D) rounded to fp32 once; both sides receive these exact bits.
 _STD_D = math.sqrt(4.0 / 3.0 * (65536.0 ** 2 - 1.0))
@@ -217,6 +218,12 @@ def router_weight_bf16(shape: MoeShape, seed: int, layer: int) -> np.ndarray:
     n = shape.experts * shape.hidden
     f = normal_f32(stream_key(seed, layer, ROLE_ROUTER, 0), 0, n, C_SIGMA002)
     return bf16_bits_from_f32(f).reshape(shape.experts, shape.hidden)
+
+
+def shared_gate_weight_bf16(shape: MoeShape, seed: int, layer: int) -> np.ndarray:
+    """The shared expert's gate vector [H] as bf16 bits, N(0, 0.02)."""
+    f = normal_f32(stream_key(seed, layer, ROLE_SH_GATE_W, 0), 0, shape.hidden, C_SIGMA002)
+    return bf16_bits_from_f32(f)
 
 
 def hidden_states_bf16(tokens: int, hidden: int, seed: int, batch: int = 0) -> np.ndarray:

@@ -48,6 +48,8 @@ from __future__ import annotations
 import dataclasses
 from typing import Callable, Optional
 
+import math
+
 import numpy as np
 
 __all__ = [
@@ -204,6 +206,7 @@ class OracleLayer:
     expert: Callable[[int], tuple]
     shared: Callable[[], Optional[tuple]]
     cache_size: int = 48
+    shared_gate_w_bits: Optional[np.ndarray] = None   # [H] bf16 bits, or None (shared weight 1)
 
     def __post_init__(self):
         self._cache: dict = {}
@@ -229,6 +232,15 @@ class OracleLayer:
             return None
         return self._dense(("s",), self.shared)
 
+    def shared_weight(self, xhat_t: np.ndarray) -> float:
+        """Weight of the shared expert for one token: 1, or, for the gated
+        variant, the logistic function of the dot product of the token with
+        the gate vector (float64)."""
+        if self.shared_gate_w_bits is None:
+            return 1.0
+        z = float(np.dot(xhat_t, bf16_to_f64(self.shared_gate_w_bits)))
+        return 1.0 / (1.0 + math.exp(-z))
+
 
 def layer_forward(layer: OracleLayer, x_bits: np.ndarray, *, rmsnorm: bool = False,
                   topk_override: Optional[dict] = None) -> dict:
@@ -252,7 +264,7 @@ def layer_forward(layer: OracleLayer, x_bits: np.ndarray, *, rmsnorm: bool = Fal
     for t in range(T):
         acc = np.zeros(layer.hidden, dtype=np.float64)
         if shared is not None:
-            acc += swiglu_ffn(*shared, xhat[t])
+            acc += layer.shared_weight(xhat[t]) * swiglu_ffn(*shared, xhat[t])
         for j in range(layer.top_k):
             acc += w[t, j] * swiglu_ffn(*layer.expert_dense(int(idx[t, j])), xhat[t])
         out[t] = acc
@@ -280,7 +292,7 @@ def layer_forward_ep(layer: OracleLayer, x_bits: np.ndarray, ep_rank: int, ep_si
     shared = layer.shared_dense() if ep_rank == 0 else None
     for t in range(T):
         if shared is not None:
-            partial[t] += swiglu_ffn(*shared, x[t])
+            partial[t] += layer.shared_weight(x[t]) * swiglu_ffn(*shared, x[t])
         for j in range(layer.top_k):
             e = int(idx[t, j])
             if e % ep_size == ep_rank:

@@ -50,7 +50,8 @@ class MoeConfig(ctypes.Structure):
 class _Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "gate_up_codes", "gate_up_scales", "down_codes", "down_scales", "shared_gate_up_codes",
-        "shared_gate_up_scales", "shared_down_codes", "shared_down_scales", "router_w", "router_bias")]
+        "shared_gate_up_scales", "shared_down_codes", "shared_down_scales", "router_w", "router_bias",
+        "shared_gate_w")]
 
 
 @dataclasses.dataclass
@@ -67,6 +68,7 @@ class LayerWeights:
     shared_gate_up_scales: Optional[object] = None
     shared_down_codes: Optional[object] = None
     shared_down_scales: Optional[object] = None
+    shared_gate_w: Optional[object] = None      # [H] bf16: shared expert weighted by sigmoid(x . w)
 
     def to_c(self) -> _Weights:
         w = _Weights()

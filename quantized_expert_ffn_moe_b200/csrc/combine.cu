@@ -1,5 +1,6 @@
-// Gate-weighted combine: out[t] = Y[shared, t] + sum_j Y[(t, j)] in fixed slot
-// order (the gate weight is already inside Y), fp32, rounded once to bf16.
+// Gate-weighted combine: out[t] = g_t Y[shared, t] + sum_j Y[(t, j)] in fixed
+// slot order (the gate weight is already inside Y), fp32, rounded once to
+// bf16; g_t = 1, or sigmoid(x_t . w) when the layer has a shared-expert gate.
 // The shared expert is added with weight 1 ("How a 125B Model Reaches 100
 // Tok/s on an RTX 4090", section "The model is large on paper, sparse in
 // practice": 10 routed experts plus one shared expert are active per token).
@@ -19,7 +20,7 @@ constexpr int kCombThreads = 256;
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const float* __restrict__ Y, const int* __restrict__ inv, int T, int k, int H, int shared,
     uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next, float* __restrict__ out_f32,
-    const int* __restrict__ gate) {
+    const int* __restrict__ gate, const uint16_t* __restrict__ xin, const uint16_t* __restrict__ sgate_w) {
   pdl_wait();
   if (gate && __ldcg(gate) == 0) {                // the fused decode kernel kept (and combined) the layer
     pdl_launch_dependents();
@@ -28,7 +29,31 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
   const int t = blockIdx.x;
   const int P_routed = T * k;
   __shared__ int pos[16];
+  __shared__ float gred[kCombThreads / 32];
   if (threadIdx.x < k) pos[threadIdx.x] = inv[t * k + threadIdx.x];
+  // the shared expert's weight: 1, or sigmoid(x . w) with the layer input x
+  // (exact bf16 products, fp32 sum)
+  float gsh = 1.f;
+  if (shared && sgate_w) {
+    float a = 0.f;
+    for (int h0 = threadIdx.x * 8; h0 < H; h0 += kCombThreads * 8) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xin + size_t(t) * H + h0);
+      const uint4 wv = *reinterpret_cast<const uint4*>(sgate_w + h0);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a = fmaf(__uint_as_float(xw[i] << 16), __uint_as_float(ww[i] << 16), a);
+        a = fmaf(__uint_as_float(xw[i] & 0xFFFF0000u), __uint_as_float(ww[i] & 0xFFFF0000u), a);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if ((threadIdx.x & 31) == 0) gred[threadIdx.x >> 5] = a;
+    __syncthreads();
+    float z = 0.f;
+    for (int i = 0; i < kCombThreads / 32; ++i) z += gred[i];
+    gsh = 1.f / (1.f + expf(-z));
+  }
   __syncthreads();
   float ss = 0.f;
   constexpr int VPT = 8;                      // elements per thread per step
@@ -37,8 +62,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     if (shared) {
       const float4 a = *reinterpret_cast<const float4*>(Y + size_t(P_routed + t) * H + h0);
       const float4 b = *reinterpret_cast<const float4*>(Y + size_t(P_routed + t) * H + h0 + 4);
-      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
-      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+      acc[0] = gsh * a.x; acc[1] = gsh * a.y; acc[2] = gsh * a.z; acc[3] = gsh * a.w;
+      acc[4] = gsh * b.x; acc[5] = gsh * b.y; acc[6] = gsh * b.z; acc[7] = gsh * b.w;
     } else {
 #pragma unroll
       for (int i = 0; i < VPT; ++i) acc[i] = 0.f;
@@ -108,7 +133,8 @@ cudaError_t launch_combine(const LayerArgs& a) {
   return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, a.stream,
                     reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
                     a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next,
-                    a.y_f32, a.gated ? reinterpret_cast<const int*>(a.ws + a.L.status) + ST_PATH : nullptr);
+                    a.y_f32, a.gated ? reinterpret_cast<const int*>(a.ws + a.L.status) + ST_PATH : nullptr, a.x,
+                    a.w.shared_gate_w);
 }
 
 }  // namespace moe

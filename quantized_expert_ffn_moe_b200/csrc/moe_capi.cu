@@ -61,6 +61,7 @@ int validate_weights(const moe_config* c, const moe_layer_weights* w) {
       if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
   }
   if (w->router_bias && !aligned(w->router_bias, 4)) return MOE_ERR_INVALID_ARG;
+  if (w->shared_gate_w && (c->shared_inter == 0 || !aligned(w->shared_gate_w, 16))) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -167,7 +168,7 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
   a.num_sms = num_sms_current();
   a.stream = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T)) {
+  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T) && !w->shared_gate_w) {
     const int call = (g_prof.on && g_prof.used < g_prof.cap) ? g_prof.used++ : -1;
     prof_mark(call, 0, a.stream);
     // 32..64 tokens: the fused kernel routes and then either finishes the
@@ -202,15 +203,19 @@ int moe_layer_forward_ep(const moe_config* cfg, const moe_layer_weights* w, cons
     return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   moe_config c = *cfg;
-  if (ep_rank != 0) c.shared_inter = 0;          // the shared expert belongs to rank 0
-  if ((st = validate_weights(&c, w)) != MOE_OK) return st;
+  moe_layer_weights wl = *w;
+  if (ep_rank != 0) {                            // the shared expert (and its gate) belong to rank 0
+    c.shared_inter = 0;
+    wl.shared_gate_w = nullptr;
+  }
+  if ((st = validate_weights(&c, &wl)) != MOE_OK) return st;
   if (!x || !y_partial || !aligned(x, 16) || !aligned(y_partial, 16)) return MOE_ERR_INVALID_ARG;
   const char* xb = reinterpret_cast<const char*>(x);
   const char* yb = reinterpret_cast<const char*>(y_partial);
   if (xb < yb + size_t(T) * cfg->hidden * 4 && yb < xb + size_t(T) * cfg->hidden * 2) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(cfg, T, workspace, ws_bytes)) != MOE_OK) return st;
   LayerArgs a{};
-  a.cfg = c; a.w = *w; a.T = T; a.x = x; a.y = nullptr; a.residual = false; a.xhat_next = nullptr;
+  a.cfg = c; a.w = wl; a.T = T; a.x = x; a.y = nullptr; a.residual = false; a.xhat_next = nullptr;
   a.ws = static_cast<char*>(workspace);
   a.L = make_layout(*cfg, T);
   a.num_sms = num_sms_current();
@@ -241,7 +246,9 @@ int moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, in
   a.stream = static_cast<cudaStream_t>(stream);
   uint16_t* xhat = reinterpret_cast<uint16_t*>(a.ws + a.L.xhat);
   if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T)) {
+  bool gated = false;
+  for (int l = 0; l < L; ++l) gated = gated || layers[l].shared_gate_w != nullptr;
+  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T) && !gated) {
     const cudaError_t e = launch_fused_decode(*cfg, layers, L, x_inout, x_inout, true, T, topk_trace, a.ws, a.L,
                                               a.num_sms, a.stream);
     if (e == cudaSuccess) return MOE_OK;

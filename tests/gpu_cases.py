@@ -30,11 +30,12 @@ def cfg_of(shape: mi.MoeShape) -> q.MoeConfig:
                        shape.block)
 
 
-def device_layer(shape: mi.MoeShape, seed: int, layer: int, zipf: bool = False) -> q.LayerWeights:
+def device_layer(shape: mi.MoeShape, seed: int, layer: int, zipf: bool = False,
+                 shared_gate: bool = False) -> q.LayerWeights:
     """One layer's packed weights generated on the device (same bytes as the
     host generator), as LayerWeights."""
     import moe_inputs.device as md
-    return q.LayerWeights(**md.device_layer_tensors(shape, seed, layer, zipf=zipf))
+    return q.LayerWeights(**md.device_layer_tensors(shape, seed, layer, zipf=zipf, shared_gate=shared_gate))
 
 
 def to_dev_bits(a: np.ndarray):
@@ -83,14 +84,15 @@ def run_route(shape, w, x_bits: np.ndarray):
             pairs.cpu().numpy())
 
 
-def host_oracle_layer(shape, seed, layer, zipf=False, cache_size=16):
+def host_oracle_layer(shape, seed, layer, zipf=False, cache_size=16, shared_gate=False):
     return orc.OracleLayer(
         experts=shape.experts, hidden=shape.hidden, inter=shape.inter, top_k=shape.top_k, bits=shape.bits,
         block=shape.block, router_w_bits=mi.router_weight_bf16(shape, seed, layer),
         router_bias=mi.zipf_router_bias(shape, seed, layer) if zipf else None,
         expert=lambda e: mi.expert_packed(shape, seed, layer, e),
         shared=(lambda: mi.shared_packed(shape, seed, layer)) if shape.shared else (lambda: None),
-        cache_size=cache_size)
+        cache_size=cache_size,
+        shared_gate_w_bits=mi.shared_gate_weight_bf16(shape, seed, layer) if shared_gate else None)
 
 
 def check_selection(oracle_logits, oracle_idx, gpu_idx, k, band=TIE_BAND):

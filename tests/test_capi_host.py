@@ -85,6 +85,7 @@ def _fake_weights(shared=True, misalign=None):
         for n in ("shared_gate_up_codes", "shared_gate_up_scales", "shared_down_codes", "shared_down_scales"):
             setattr(w, n, None)
     w.router_bias = None
+    w.shared_gate_w = None
     if misalign:
         setattr(w, misalign, getattr(w, misalign) + 8)
     return w
@@ -110,6 +111,12 @@ def test_layer_forward_argument_errors(lib):
     assert _layer(lib, c, _fake_weights(shared=False)) == -1  # shared expert configured but missing
     assert _layer(lib, cfg(shared=False), _fake_weights(shared=False), ws_bytes=0) == -3
     assert _layer(lib, cfg(bits=3), w) == -2                  # MOE_ERR_UNSUPPORTED
+    g = _fake_weights()
+    g.shared_gate_w = 1 << 24
+    assert _layer(lib, cfg(), g, ws_bytes=0) == -3           # a gate with a shared expert is valid
+    assert _layer(lib, cfg(shared=False), g) == -1           # a gate needs a shared expert
+    g.shared_gate_w = (1 << 24) + 8
+    assert _layer(lib, cfg(), g) == -1                        # misaligned gate vector
     assert lib.moe_layer_forward(None, ctypes.byref(w), 1 << 30, 4, 2 << 30, 3 << 30, 1 << 40, None) == -1
 
 

@@ -450,3 +450,51 @@ def test_layer_full4_g128_sampled(T):
     16 and 48 tokens, the stand-alone GEMV kernels at 100 (no tensor-core path
     for this group size)."""
     _sampled_full_case(FULL4_G128, T, 7, 0, 4, 128 + T)
+
+
+# ----------------------------------------------------- gated shared expert ---
+
+def _gated_case(shape, T, seed, batch, sample=None):
+    x = mi.hidden_states_bf16(T, shape.hidden, seed, batch)
+    w = gc.device_layer(shape, seed, 0, shared_gate=True)
+    y = gc.run_layer(shape, w, x)
+    idx = gc.run_route(shape, w, x)[0]
+    sel = np.arange(T) if sample is None else np.sort(np.random.default_rng(batch).choice(T, sample, replace=False))
+    lay = gc.host_oracle_layer(shape, seed, 0, cache_size=min(shape.experts + 1, 24), shared_gate=True)
+    r = orc.layer_forward(lay, x[sel])
+    differ = gc.check_selection(r["logits"], r["idx"], idx[sel], shape.top_k)
+    if differ:
+        r = orc.layer_forward(lay, x[sel], topk_override={i: idx[sel[i]] for i in differ})
+    gc.assert_close(y[sel], r["out"])
+
+
+def test_device_generator_gate_vector():
+    w = gc.device_layer(mi.TINY, 3, 2, shared_gate=True)
+    np.testing.assert_array_equal(gc.bits_to_np(w.shared_gate_w), mi.shared_gate_weight_bf16(mi.TINY, 3, 2))
+
+
+@pytest.mark.parametrize("T", [8, 100])
+def test_gated_shared_expert_tiny(T):
+    _gated_case(mi.TINY, T, 0, 41)
+
+
+def test_gated_shared_expert_prefill_mid():
+    _gated_case(MID4, 129, 4, 42)
+
+
+def test_gated_shared_expert_full4_sampled():
+    # the gated layer leaves the single-launch decode kernel for the separate kernels
+    _gated_case(mi.FULL4, 16, 0, 43, sample=4)
+
+
+def test_gated_shared_expert_expert_parallel():
+    shape = mi.TINY
+    x = mi.hidden_states_bf16(8, shape.hidden, 0, 44)
+    w = gc.device_layer(shape, 0, 0, shared_gate=True)
+    lay = gc.host_oracle_layer(shape, 0, 0, cache_size=shape.experts + 1, shared_gate=True)
+    idx = gc.run_route(shape, w, x)[0]
+    full = orc.layer_forward(lay, x)
+    differ = gc.check_selection(full["logits"], full["idx"], idx, shape.top_k)
+    keep = np.setdiff1d(np.arange(8), differ)
+    parts = _ep_partials(shape, w, x, 2)
+    gc.assert_close(sum(parts)[keep], full["out"][keep])

@@ -332,3 +332,43 @@ def test_zipf_alpha_matches_calibration():
     idx = orc.select_topk(l, shape.top_k)
     rank = np.rint(np.exp(bias.astype(np.float64) / -mi.ZIPF_ALPHA)).astype(np.int64)
     assert abs(np.mean(rank[idx] <= 102) - 0.95) < 0.02
+
+
+# ----------------------------------------------- gated shared expert (variant)
+
+def test_shared_gate_weight_closed_form():
+    """sigmoid of an exactly representable dot product, evaluated by hand."""
+    shape = mi.MoeShape(experts=4, hidden=8, inter=4, top_k=1, shared=True, bits=4, block=4)
+    gate = mi.bf16_bits_from_f32(np.array([0.5, -0.25, 1.0, 0, 0, 0, 0, 2.0], dtype=np.float32))
+    lay = orc.OracleLayer(experts=4, hidden=8, inter=4, top_k=1, bits=4, block=4,
+                          router_w_bits=np.zeros((4, 8), np.uint16), router_bias=None,
+                          expert=lambda e: None, shared=lambda: None, shared_gate_w_bits=gate)
+    x = np.array([2.0, 4.0, -1.0, 7.0, 7.0, 7.0, 7.0, 0.5])
+    z = 0.5 * 2.0 - 0.25 * 4.0 + 1.0 * -1.0 + 2.0 * 0.5          # 1 - 1 - 1 + 1
+    assert z == 0.0
+    assert lay.shared_weight(x) == 0.5
+    x2 = x.copy()
+    x2[7] = 3.0                                                     # z = 1 - 1 - 1 + 6 = 5
+    assert abs(lay.shared_weight(x2) - 1.0 / (1.0 + math.exp(-5.0))) < 1e-15
+    assert _tiny_layer(shape=mi.TINY).shared_weight(x) == 1.0      # no gate: weight 1
+
+
+def test_zero_gate_halves_the_shared_expert():
+    shape = mi.TINY
+    x = mi.hidden_states_bf16(6, shape.hidden, seed=9)
+    with_sh = orc.layer_forward(_tiny_layer(shape), x)["out"]
+    no_sh = orc.layer_forward(_tiny_layer(shape, shared=False), x)["out"]
+    zero_gate = _tiny_layer(shape)
+    zero_gate.shared_gate_w_bits = np.zeros(shape.hidden, np.uint16)
+    half = orc.layer_forward(zero_gate, x)["out"]
+    np.testing.assert_allclose(half, no_sh + 0.5 * (with_sh - no_sh), rtol=0, atol=1e-12 * np.abs(with_sh).max())
+
+
+def test_gated_layer_partials_sum_to_the_layer():
+    shape = mi.TINY
+    lay = _tiny_layer(shape)
+    lay.shared_gate_w_bits = mi.shared_gate_weight_bf16(shape, 0, 0)
+    x = mi.hidden_states_bf16(6, shape.hidden, seed=10)
+    full = orc.layer_forward(lay, x)["out"]
+    parts = [orc.layer_forward_ep(lay, x, r, 3)["partial"] for r in range(3)]
+    np.testing.assert_allclose(sum(parts), full, rtol=0, atol=1e-12 * np.abs(full).max())
