@@ -231,6 +231,15 @@ void moe_debug_prefill_timing(unsigned long long* device_buf);
  * thread-safe. */
 void moe_debug_decode_path(int32_t mode);
 
+/* Failure-path test hook: launches one bounded wait, through the library's
+ * own mbarrier wait, on a barrier that never completes.  After the wait's
+ * cycle limit (about 1.5 s) the probe records MOE_ERR_TIMEOUT in the status
+ * word of `workspace` (device, 256-byte aligned, its first 8 bytes zeroed by
+ * the caller; read back with moe_device_status) and returns; the context
+ * stays usable.  Asynchronous on `stream`; MOE_ERR_INVALID_ARG for a null or
+ * misaligned workspace. */
+int moe_debug_wait_probe(void* workspace, void* stream);
+
 /* The cudaError_t value behind the calling thread's most recent
  * MOE_ERR_CUDA (0 if none). */
 int moe_last_cuda_error(void);

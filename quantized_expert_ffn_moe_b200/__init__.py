@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
            "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end",
            "moe_layer_forward_noalloc", "moe_last_cuda_error", "moe_debug_fused_timing",
-           "moe_debug_prefill_timing", "moe_layer_forward_ep", "moe_debug_decode_path")
+           "moe_debug_prefill_timing", "moe_layer_forward_ep", "moe_debug_decode_path", "moe_debug_wait_probe")
 
 MOE_OK = 0
 
@@ -116,6 +116,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_debug_prefill_timing.argtypes = [P]
     lib.moe_debug_decode_path.argtypes = [I32]
     lib.moe_debug_decode_path.restype = None
+    lib.moe_debug_wait_probe.argtypes = [P, P]
+    lib.moe_debug_wait_probe.restype = ctypes.c_int
     lib.moe_debug_prefill_timing.restype = None
     lib.moe_last_cuda_error.argtypes = []
     lib.moe_last_cuda_error.restype = ctypes.c_int

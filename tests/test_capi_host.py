@@ -146,6 +146,11 @@ def test_layer_forward_ep_argument_errors(lib):
     assert _layer_ep(lib, cfg(bits=3), w, 0, 2) == -2
 
 
+def test_wait_probe_argument_errors(lib):
+    assert lib.moe_debug_wait_probe(None, None) == -1
+    assert lib.moe_debug_wait_probe((1 << 30) + 16, None) == -1
+
+
 def test_route_and_stack_argument_errors(lib):
     c = cfg()
     n = lib.moe_workspace_bytes(ctypes.byref(c), 4)

@@ -498,3 +498,18 @@ def test_gated_shared_expert_expert_parallel():
     keep = np.setdiff1d(np.arange(8), differ)
     parts = _ep_partials(shape, w, x, 2)
     gc.assert_close(sum(parts)[keep], full["out"][keep])
+
+
+# ------------------------------------------------------------ failure path ---
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier that never completes gives up after its limit,
+    records MOE_ERR_TIMEOUT in the status word, and the GPU keeps working."""
+    torch = gc.torch()
+    lib = q.load_library()
+    ws = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    assert lib.moe_debug_wait_probe(ws.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    assert q.moe_device_status(ws) == -6                      # MOE_ERR_TIMEOUT
+    # the context is intact: a layer still runs and matches the oracle
+    test_layer_without_shared_expert()
