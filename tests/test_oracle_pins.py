@@ -33,7 +33,7 @@ def _read_golden(name):
 
 def test_format_blocks_hand_decoded():
     rows = _read_golden("format_blocks.txt")
-    assert len(rows) == 4
+    assert len(rows) == 5
     for (bb, scales, codes, expected) in rows:
         bits, block = int(bb[0]), int(bb[1])
         sc = np.array([int(s, 16) for s in scales], dtype=np.uint16)
