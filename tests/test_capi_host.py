@@ -182,3 +182,34 @@ def test_binding_fails_loudly_without_library(tmp_path):
             mod.load_library(str(tmp_path / "missing.so"))
         finally:
             mod._lib = saved
+
+
+def test_header_is_plain_c(tmp_path):
+    """The boundary header compiles as C99 (no C++ in the interface) and a C
+    caller can name every entry point with the declared types."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_capi.c"
+    src.write_text("""
+#include "moe_capi.h"
+int use(void* ws, size_t n, const uint16_t* x, uint16_t* y, float* yp, void* stream) {
+  moe_config c = {512, 2048, 768, 10, 768, 4, 32};
+  moe_layer_weights w = {0};
+  int32_t code = 0;
+  size_t need = moe_workspace_bytes(&c, 16);
+  int st = moe_layer_forward(&c, &w, x, 16, y, ws, n, stream);
+  st |= moe_layer_forward_ep(&c, &w, x, 16, 0, 2, yp, ws, n, stream);
+  st |= moe_stack_forward(&c, &w, 1, y, 16, NULL, ws, n, stream);
+  st |= moe_device_status(ws, &code);
+  moe_debug_decode_path(0);
+  (void)moe_status_str(st);
+  return st + (int)need + code;
+}
+""")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, str(src)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
