@@ -45,7 +45,8 @@ def parse():
     ap.add_argument("--tokens", type=int, default=16)
     ap.add_argument("--instances", type=int, default=48, help="distinct layer instances rotated over")
     ap.add_argument("--no-detail", action="store_true", help="skip the secondary workloads")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=2)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16,
+                    help="tokens of the headline batch the CPU oracle baseline runs (16 = the whole batch)")
     ap.add_argument("--quick", action="store_true",
                     help="headline loop only (no e2e, detail or CPU baseline): the small case used for ncu")
     return ap.parse_args()
