@@ -54,12 +54,12 @@ def parse():
 
 # ------------------------------------------------------------------ utils ---
 
-def profiled_traffic(profile: str, sources) -> float | None:
-    """DRAM bytes per launch from a committed ncu summary under profiles/, or
+def profiled_fields(profile: str, sources, profiles_dir: str | None = None, csrc_dir: str | None = None):
+    """The `key: value` lines of a committed ncu summary under profiles/, or
     None when the kernel's sources changed since that capture (the summary
     records the sha256 of the sources it was taken with)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", profile)
+    path = os.path.join(profiles_dir or os.path.join(ROOT, "profiles"), profile)
     if not os.path.exists(path):
         return None
     fields = {}
@@ -69,10 +69,30 @@ def profiled_traffic(profile: str, sources) -> float | None:
             fields[k.strip()] = v.strip().split()[0] if v.strip() else ""
     h = hashlib.sha256()
     for f in sources:
-        h.update(open(os.path.join(ROOT, "quantized_expert_ffn_moe_b200", "csrc", f), "rb").read())
-    if fields.get("source_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+        h.update(open(os.path.join(csrc_dir or os.path.join(ROOT, "quantized_expert_ffn_moe_b200", "csrc"), f),
+                      "rb").read())
+    if fields.get("source_sha256") != h.hexdigest():
+        return None
+    return fields
+
+
+def profiled_traffic(profile: str, sources) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary (None if stale)."""
+    fields = profiled_fields(profile, sources)
+    if not fields or "traffic_bytes_per_launch" not in fields:
         return None
     return float(fields["traffic_bytes_per_launch"])
+
+
+def issue_ceiling(instructions: float, launch_s: float, sms: int, sm_mhz: float = 1965.0) -> dict:
+    """Warp instructions per launch (ncu smsp__inst_executed.sum) against the
+    issue capacity of the GPU: one warp instruction per cycle per scheduler,
+    4 schedulers per SM, at the given SM clock."""
+    peak = sms * 4 * sm_mhz * 1e6
+    achieved = instructions / launch_s
+    return {"instructions_per_launch": instructions, "achieved_inst_per_s": achieved, "peak_inst_per_s": peak,
+            "peak_source": f"{sms} SMs x 4 schedulers x 1 warp instruction/cycle x {sm_mhz:.0f} MHz",
+            "frac": achieved / peak, "min_launch_us": 1e6 * instructions / peak}
 
 
 def measured_peaks():
@@ -372,8 +392,9 @@ def main():
         k_ms = phase_ms[1] / calls
         k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * GU_BYTES[4]
         kname = "ffn_tma_kernel<gate/up>"
-    traffic = profiled_traffic("fused_decode_kernel_decode4_t16.txt",
-                               ["fused.cu", "decode_common.cuh", "moe_internal.cuh"]) if fused else None
+    pf = profiled_fields("fused_decode_kernel_decode4_t16.txt",
+                         ["fused.cu", "decode_common.cuh", "moe_internal.cuh"]) if fused else None
+    traffic = float(pf["traffic_bytes_per_launch"]) if pf and "traffic_bytes_per_launch" in pf else None
     roofline = {"bound": "hbm", "kernel": kname, "achieved": k_bytes / (k_ms * 1e-3) / 1e9,
                 "peak": hbm_peak, "unit": "GB/s", "frac": None, "traffic": traffic,
                 "traffic_source": "profiles/fused_decode_kernel_decode4_t16.txt (ncu dram__bytes_read.sum + "
@@ -384,6 +405,14 @@ def main():
                              "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls,
                              "fused": 1000 * phase_ms[4] / calls}}
     roofline["frac"] = roofline["achieved"] / hbm_peak
+    try:
+        # the decode kernel's second ceiling: instruction issue (it is issue-
+        # bound, which is why the HBM fraction stays below one)
+        if pf and "instructions_per_launch" in pf:
+            sms = torch.cuda.get_device_properties(0).multi_processor_count
+            roofline["issue"] = issue_ceiling(float(pf["instructions_per_launch"]), k_ms * 1e-3, sms)
+    except Exception:
+        pass
     launches_per_step = 1 if fused else 5
 
     if args.quick:
