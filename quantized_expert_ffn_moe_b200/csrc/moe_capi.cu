@@ -202,6 +202,7 @@ int moe_layer_forward_ep(const moe_config* cfg, const moe_layer_weights* w, cons
   if (T < 0 || ep_size < 1 || ep_size > cfg->num_experts || ep_rank < 0 || ep_rank >= ep_size)
     return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
+  if (!w) return MOE_ERR_INVALID_ARG;
   moe_config c = *cfg;
   moe_layer_weights wl = *w;
   if (ep_rank != 0) {                            // the shared expert (and its gate) belong to rank 0

@@ -144,6 +144,7 @@ def test_layer_forward_ep_argument_errors(lib):
     assert _layer_ep(lib, c, _fake_weights(shared=False), 0, 2) == -1
     assert _layer_ep(lib, c, _fake_weights(shared=False), 1, 2, ws_bytes=0) == -3
     assert _layer_ep(lib, cfg(bits=3), w, 0, 2) == -2
+    assert lib.moe_layer_forward_ep(ctypes.byref(c), None, 1 << 30, 4, 0, 2, 2 << 30, 3 << 30, 1 << 30, None) == -1
 
 
 def test_wait_probe_argument_errors(lib):
