@@ -214,3 +214,25 @@ int use(void* ws, size_t n, const uint16_t* x, uint16_t* y, float* yp, void* str
     r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, str(src)],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_null_arguments_are_rejected_everywhere(lib):
+    """Every entry point turns NULL pointers into MOE_ERR_INVALID_ARG on the
+    host, without touching the device."""
+    c = cfg()
+    w = _fake_weights()
+    n = lib.moe_workspace_bytes(ctypes.byref(c), 4)
+    assert lib.moe_workspace_bytes(None, 4) == 0
+    assert lib.moe_route(None, 1 << 20, None, 1 << 30, 4, 1 << 31, 1 << 32, None, None, None, 3 << 30, n, None) == -1
+    assert lib.moe_layer_forward(ctypes.byref(c), None, 1 << 30, 4, 2 << 30, 3 << 30, n, None) == -1
+    assert lib.moe_layer_forward(ctypes.byref(c), ctypes.byref(w), 1 << 30, 4, 2 << 30, None, n, None) == -1
+    assert lib.moe_layer_forward_ep(None, ctypes.byref(w), 1 << 30, 4, 0, 2, 2 << 30, 3 << 30, n, None) == -1
+    assert lib.moe_stack_forward(ctypes.byref(c), None, 1, 1 << 30, 4, None, 3 << 30, n, None) == -1
+    assert lib.moe_stack_forward(None, None, 1, 1 << 30, 4, None, 3 << 30, n, None) == -1
+    arr = (q._Weights * 1)(_fake_weights())
+    assert lib.moe_stack_forward(ctypes.byref(c), arr, 1, None, 4, None, 3 << 30, n, None) == -1
+    assert lib.moe_device_status(None, None) == -1
+    assert lib.moe_dequant_rows(None, 1 << 20, 1 << 21, 0, 1, 256, 1 << 22, None) == -1
+    assert lib.moe_dequant_rows(ctypes.byref(c), None, 1 << 21, 0, 1, 256, 1 << 22, None) == -1
+    assert lib.moe_layer_forward_noalloc(None, ctypes.byref(w), 1 << 30, 4, 2 << 30, None) == -1
+    assert lib.moe_profile_end(None, None) == -1
