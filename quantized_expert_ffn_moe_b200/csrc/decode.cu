@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
   unsigned char* ring = smem + 256;
-  __half* xs = reinterpret_cast<__half*>(ring + kStages * Gm::STAGE_BYTES);     // [ntc][K]
+  int16_t* xs = reinterpret_cast<int16_t*>(ring + kStages * Gm::STAGE_BYTES);     // [ntc][K]
   float* tok_inv = reinterpret_cast<float*>(xs + size_t(ntc) * K);
   float* tok_w = tok_inv + kMaxNTC;
   int* tok_pos = reinterpret_cast<int*>(tok_w + kMaxNTC);
@@ -216,14 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-        int sh = 0;
-        if (vmax > 0.f) {
-          int ex;
-          frexpf(vmax, &ex);
-          sh = min(max(8 - ex, -100), 100);      // max |x * 2^sh| in [128, 256)
-        }
+        const int sh = act_shift(vmax);
         const float mul = ldexpf(1.f, sh);
-        __half* dst = xs + size_t(tl) * K;
+        int16_t* dst = xs + size_t(tl) * K;
         for (int g0 = lane * Gm::G; g0 < K; g0 += 32 * Gm::G) {
           float v[Gm::G];
           if (MODE == GATEUP) {
@@ -247,13 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
             }
           }
           uint4 parts[Gm::NPART];
-          pack_pair_order<Gm::G>(v, mul, parts);
+          pack_int_order<BITS, Gm::G>(v, mul, parts);
           const int base = staged_offset<BITS, LPR, CPL>(g0);
 #pragma unroll
           for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
         }
         if (lane == 0) {
-          tok_inv[tl] = ldexpf(1.f, -sh);
+          tok_inv[tl] = act_inv<BITS>(sh);
           tok_pos[tl] = p;
           tok_w[tl] = (MODE == DOWN && !is_shared) ? __ldcg(rv.topk_w + __ldcg(rv.pairs + p)) : 1.f;
         }
@@ -286,7 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
 
 // --------------------------------------------------------- dequant hook
 // Writes out[r][j] = q * scale for rows row0.. of a packed matrix, with the
-// same word decoders the GEMV uses (test hook, not on the timed path).
+// byte decoders the GEMV uses (q4_bytes / q2_bytes: signed bytes 16 q or
+// 64 q); test hook, not on the timed path.
 template <int BITS>
 __global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
                                     int row0, int rows, int cols, int BLOCK, float* __restrict__ out) {
@@ -298,14 +294,21 @@ __global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uin
     const int r = int(i / words_per_row), wi = int(i % words_per_row);
     const size_t row = size_t(row0 + r);
     const uint32_t v = *reinterpret_cast<const uint32_t*>(codes + row * (cols * BITS / 8) + size_t(wi) * 4);
-    __half2 q[G / 2];
-    if (BITS == 4) decode_q4x8(v, q); else decode_q2x16(v, q);
+    uint32_t f[4];
+    if (BITS == 4) {
+      q4_bytes(v, f[0], f[1]);
+    } else {
+      q2_bytes<false>(v, f);
+    }
     for (int j = 0; j < G; ++j) {
       const int col = wi * G + j;
-      const int sl = decode_slot(BITS, j);
-      const __half qh = (sl & 1) ? __high2half(q[sl >> 1]) : __low2half(q[sl >> 1]);
+      // element j: 4-bit -> byte j/2 of lo (even j) / hi (odd j);
+      //            2-bit -> byte j/4 of field j%4
+      const uint32_t word = BITS == 4 ? f[j & 1] : f[j & 3];
+      const int byte = BITS == 4 ? (j >> 1) : (j >> 2);
+      const int qb = int(int8_t(uint8_t(word >> (8 * byte))));
       const float sc = __half2float(__ushort_as_half(scales[row * (cols / BLOCK) + col / BLOCK]));
-      out[size_t(r) * cols + col] = __half2float(qh) * sc;
+      out[size_t(r) * cols + col] = ldexpf(float(qb), -CodeMul<BITS>::kLog2) * sc;
     }
   }
 }

@@ -31,9 +31,78 @@ struct Geom {
   static constexpr int STAGE_BYTES = (CODE_BYTES + SCALE_BYTES + 127) / 128 * 128;
 };
 
-// Offset (in halves) of element h of a staged activation row: the order in
-// which a lane of a row group meets the decoded half2 pairs (see decode_q4x8 /
-// decode_q2x16), laid out so that the lanes of a group read consecutive
+// Integer operands of the GEMV.  A code field shifted to the top of its byte
+// and XOR-ed with 0x80 is, read as a signed byte, the code minus its offset
+// times the field weight: for 4-bit codes c, ((c << 4) ^ 0x80) = 16 (c - 8);
+// for 2-bit codes, ((c << 6) ^ 0x80) = 64 (c - 2) and ((c << 6) ^ 0xA0) =
+// 64 (c - 1.5) (the four-level reading).  dp2a multiplies two signed 16-bit
+// activations with two of those bytes and adds them to a 32-bit sum, so a
+// block's dot product is exact in int32 and is scaled once per block in fp32.
+//
+// 4-bit word v = codes c0..c7 (c_j at bits 4j): returns the bytes
+//   lo = (16 q0, 16 q2, 16 q4, 16 q6), hi = (16 q1, 16 q3, 16 q5, 16 q7)
+__device__ __forceinline__ void q4_bytes(uint32_t v, uint32_t& lo, uint32_t& hi) {
+  lo = lop_and_xor(v << 4, 0xF0F0F0F0u, 0x80808080u);
+  hi = lop_and_xor(v, 0xF0F0F0F0u, 0x80808080u);
+}
+// 2-bit word v = codes c0..c15 (c_j at bits 2j): f[r] holds the bytes
+// 64 q of elements r, r+4, r+8, r+12.  LV4: the four-level reading
+// q = c - 1.5 instead of q = c - 2.
+template <bool LV4>
+__device__ __forceinline__ void q2_bytes(uint32_t v, uint32_t (&f)[4]) {
+  constexpr uint32_t X = LV4 ? 0xA0A0A0A0u : 0x80808080u;
+  f[3] = lop_and_xor(v, 0xC0C0C0C0u, X);
+  f[2] = lop_and_xor(v << 2, 0xC0C0C0C0u, X);
+  f[1] = lop_and_xor(v << 4, 0xC0C0C0C0u, X);
+  f[0] = lop_and_xor(v << 6, 0xC0C0C0C0u, X);
+}
+// Signed-byte weight of the code fields above: the dot products come out
+// multiplied by 2^kCodeLog2.
+template <int BITS> struct CodeMul { static constexpr int kLog2 = BITS == 4 ? 4 : 6; };
+
+// Position, inside one code word's group of G elements, of element j in the
+// operand order of the dp2a calls: 4-bit (x0 x2 x4 x6 x1 x3 x5 x7), 2-bit
+// (x0 x4 x8 x12 x1 x5 x9 x13 x2 x6 x10 x14 x3 x7 x11 x15).
+__host__ __device__ inline int dot_slot(int bits, int j) {
+  return bits == 4 ? (j & 1) * 4 + (j >> 1) : (j & 3) * 4 + (j >> 2);
+}
+// Inverse of dot_slot: the element at operand position s.
+__host__ __device__ inline int dot_elem(int bits, int s) {
+  return bits == 4 ? (s & 3) * 2 + (s >> 2) : (s & 3) * 4 + (s >> 2);
+}
+
+// Per-row power-of-two scale of the integer activations: the largest |x|
+// lands in [2^13, 2^14), so every element rounds to a value that fits int16
+// with a bit to spare.  Returns the shift sh (x_int = rint(x * 2^sh)).
+__device__ __forceinline__ int act_shift(float vmax) {
+  if (!(vmax > 0.f)) return 0;
+  int ex;
+  frexpf(vmax, &ex);
+  return min(max(14 - ex, -100), 100);
+}
+// Factor that turns a row's fp32 sum of (scale x integer dot) back into the
+// real dot product: 2^-sh for the activations, 2^-kLog2 for the code bytes.
+template <int BITS>
+__device__ __forceinline__ float act_inv(int sh) { return ldexpf(1.f, -sh - CodeMul<BITS>::kLog2); }
+
+// G consecutive activations (one code word's elements) times mul, rounded to
+// int16 and packed in dot_slot order as G/8 16-byte parts, in registers.
+template <int BITS, int G>
+__device__ __forceinline__ void pack_int_order(const float (&v)[G], float mul, uint4 (&parts)[G / 8]) {
+  uint32_t w[G / 2];
+#pragma unroll
+  for (int i = 0; i < G / 2; ++i) {
+    const int a = __float2int_rn(v[dot_elem(BITS, 2 * i)] * mul);
+    const int b = __float2int_rn(v[dot_elem(BITS, 2 * i + 1)] * mul);
+    w[i] = (uint32_t(a) & 0xFFFFu) | (uint32_t(b) << 16);
+  }
+#pragma unroll
+  for (int q = 0; q < G / 8; ++q) parts[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
+// Offset (in 16-bit units) of element h of a staged activation row: the
+// order in which a lane of a row group meets the operand pairs of its code
+// words (dot_slot), laid out so that the lanes of a group read consecutive
 // 16-byte slots.
 template <int BITS, int LPR, int CPL>
 __device__ __forceinline__ int staged_offset(int h) {
@@ -41,7 +110,7 @@ __device__ __forceinline__ int staged_offset(int h) {
   const int c = h / Gm::W16, o = h % Gm::W16;
   const int s = c / LPR, lr = c % LPR;
   const int m = o / Gm::G, j = o % Gm::G;
-  const int slot = decode_slot(BITS, j);
+  const int slot = dot_slot(BITS, j);
   const int part = slot >> 3, within = slot & 7;
   return ((((s * 4 + m) * Gm::NPART + part) * LPR + lr) << 3) + within;
 }
@@ -61,11 +130,14 @@ __host__ __device__ inline int scales_per_row(int K, int block) { return K / blo
 __host__ __device__ inline int piece_shift(int bits, int block) { return bits == 4 && block == 128 ? 2 : 0; }
 
 // Dot products of the lane group's two rows with NT staged tokens, reduced
-// over the LPR lanes of the row, then the epilogue.  Each block's products
-// accumulate in two independent fp16x2 chains (even / odd code words) and
-// are folded into fp32 with the block scale.  `nt` <= NT tokens are valid.
-template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0>
-__device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& rw, const __half* xs, int tb, int lr,
+// over the LPR lanes of the row, then the epilogue.  Per code word the lane
+// turns the codes into signed bytes (q4_bytes / q2_bytes) and runs dp2a
+// against the int16 activations (two independent int32 chains per row and
+// token); each block's exact integer sum is converted to fp32 and multiplied
+// by the block's fp16 scale.  `nt` <= NT tokens are valid; xs holds int16
+// activations staged with staged_offset.
+template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0, bool LV4 = false>
+__device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& rw, const int16_t* xs, int tb, int lr,
                                          const float* tok_inv, const float* tok_w, const int* tok_pos,
                                          int nt = NT, const int* xrow = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
@@ -96,43 +168,42 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
         sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * (Gm::SPR >> PS) * 2 + (c >> PS) * 2));
-      __half2 hacc[2][NT][2];
+      int ia[2][NT], ib[2][NT];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
 #pragma unroll
-        for (int t = 0; t < NT; ++t) hacc[rho][t][0] = hacc[rho][t][1] = __float2half2_rn(0.f);
+        for (int t = 0; t < NT; ++t) ia[rho][t] = ib[rho][t] = 0;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        __half2 q[2][4];
-        decode_q4x8(wd[0][m], q[0]);
-        decode_q4x8(wd[1][m], q[1]);
+        uint32_t lo[2], hi[2];
+        q4_bytes(wd[0][m], lo[0], hi[0]);
+        q4_bytes(wd[1][m], lo[1], hi[1]);
         const int xoff = ((s * 4 + m) * LPR + lr) * 8;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
           const uint4 xv = *reinterpret_cast<const uint4*>(xs + xr0[t] + xoff);
-          const __half2 x2[4] = {u32_as_h2(xv.x), u32_as_h2(xv.y), u32_as_h2(xv.z), u32_as_h2(xv.w)};
 #pragma unroll
-          for (int rho = 0; rho < 2; ++rho)
-#pragma unroll
-            for (int z = 0; z < 4; ++z) hacc[rho][t][m & 1] = __hfma2(q[rho][z], x2[z], hacc[rho][t][m & 1]);
+          for (int rho = 0; rho < 2; ++rho) {
+            ia[rho][t] = __dp2a_lo(int(xv.x), int(lo[rho]), ia[rho][t]);
+            ib[rho][t] = __dp2a_hi(int(xv.y), int(lo[rho]), ib[rho][t]);
+            ia[rho][t] = __dp2a_lo(int(xv.z), int(hi[rho]), ia[rho][t]);
+            ib[rho][t] = __dp2a_hi(int(xv.w), int(hi[rho]), ib[rho][t]);
+          }
         }
       }
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const float2 f = __half22float2(__hadd2(hacc[rho][t][0], hacc[rho][t][1]));
-          acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
-        }
+        for (int t = 0; t < NT; ++t) acc[rho][t] = fmaf(sc[rho], __int2float_rn(ia[rho][t] + ib[rho][t]), acc[rho][t]);
     } else {
       uint2 scp[2];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        __half2 q[2][8];
-        decode_q2x16(wd[0][m], q[0]);
-        decode_q2x16(wd[1][m], q[1]);
+        uint32_t f[2][4];
+        q2_bytes<LV4>(wd[0][m], f[0]);
+        q2_bytes<LV4>(wd[1][m], f[1]);
         const int xoff = ((s * 4 + m) * 2 * LPR + lr) * 8;
         float sc[2];
 #pragma unroll
@@ -142,21 +213,20 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const __half* xr = xs + xr0[t] + xoff;
+          const int16_t* xr = xs + xr0[t] + xoff;
           const uint4 xa = *reinterpret_cast<const uint4*>(xr);
           const uint4 xb = *reinterpret_cast<const uint4*>(xr + LPR * 8);
-          const __half2 x2[8] = {u32_as_h2(xa.x), u32_as_h2(xa.y), u32_as_h2(xa.z), u32_as_h2(xa.w),
-                                 u32_as_h2(xb.x), u32_as_h2(xb.y), u32_as_h2(xb.z), u32_as_h2(xb.w)};
 #pragma unroll
           for (int rho = 0; rho < 2; ++rho) {
-            __half2 h0 = __hmul2(q[rho][0], x2[0]), h1 = __hmul2(q[rho][1], x2[1]);
-#pragma unroll
-            for (int z = 2; z < 8; z += 2) {
-              h0 = __hfma2(q[rho][z], x2[z], h0);
-              h1 = __hfma2(q[rho][z + 1], x2[z + 1], h1);
-            }
-            const float2 f = __half22float2(__hadd2(h0, h1));
-            acc[rho][t] = fmaf(sc[rho], f.x + f.y, acc[rho][t]);
+            int ia = __dp2a_lo(int(xa.x), int(f[rho][0]), 0);
+            int ib = __dp2a_hi(int(xa.y), int(f[rho][0]), 0);
+            ia = __dp2a_lo(int(xa.z), int(f[rho][1]), ia);
+            ib = __dp2a_hi(int(xa.w), int(f[rho][1]), ib);
+            ia = __dp2a_lo(int(xb.x), int(f[rho][2]), ia);
+            ib = __dp2a_hi(int(xb.y), int(f[rho][2]), ib);
+            ia = __dp2a_lo(int(xb.z), int(f[rho][3]), ia);
+            ib = __dp2a_hi(int(xb.w), int(f[rho][3]), ib);
+            acc[rho][t] = fmaf(sc[rho], __int2float_rn(ia + ib), acc[rho][t]);
           }
         }
       }

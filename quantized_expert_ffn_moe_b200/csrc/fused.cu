@@ -6,8 +6,8 @@
 // with the shared expert; in the stack RMSNorm before and the bf16 residual
 // after each layer), reorganised so that a decode step pays one launch:
 //
-//   R  every CTA: stages the T tokens (RMSNorm factor in the stack, xhat in
-//      fp16 with a power-of-two scale) and computes the router logits of its
+//   R  every CTA: stages the T tokens (RMSNorm factor in the stack, xhat as
+//      int16 with a power-of-two scale) and computes the router logits of its
 //      slice of experts -> global; the producer thread prefetches this CTA's
 //      share of the shared expert's bytes into L2                 | grid barrier
 //   S  every CTA (the same deterministic computation): top-k, gates, stable
@@ -176,11 +176,11 @@ struct FCursor {
 
 __device__ __forceinline__ float round_bf16f(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
-// Stages one row of h (fp32, K values) as fp16 in the down decoder's order,
-// with the power-of-two scale that puts its max |h| in [128, 256); returns
-// 2^-sh through inv_out (lane 0).
+// Stages one row of h (fp32, K values) as int16 in the down pass's operand
+// order, with the power-of-two scale of act_shift; returns the row's
+// act_inv factor through inv_out (lane 0).
 template <int BITS, int LPR, int CPL>
-__device__ void stage_h_row(const float* hrow, __half* dst, float* inv_out, int lane) {
+__device__ void stage_h_row(const float* hrow, int16_t* dst, float* inv_out, int lane) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
   float vmax = 0.f;
@@ -192,12 +192,7 @@ __device__ void stage_h_row(const float* hrow, __half* dst, float* inv_out, int 
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  int sh = 0;
-  if (vmax > 0.f) {
-    int ex;
-    frexpf(vmax, &ex);
-    sh = min(max(8 - ex, -100), 100);
-  }
+  const int sh = act_shift(vmax);
   const float mul = ldexpf(1.f, sh);
   for (int g0 = lane * Gm::G; g0 < K; g0 += 32 * Gm::G) {
     float v[Gm::G];
@@ -207,19 +202,19 @@ __device__ void stage_h_row(const float* hrow, __half* dst, float* inv_out, int 
       v[4 * q] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
     }
     uint4 parts[Gm::NPART];
-    pack_pair_order<Gm::G>(v, mul, parts);
+    pack_int_order<BITS, Gm::G>(v, mul, parts);
     const int base = staged_offset<BITS, LPR, CPL>(g0);
 #pragma unroll
     for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
   }
-  if (lane == 0) *inv_out = ldexpf(1.f, -sh);
+  if (lane == 0) *inv_out = act_inv<BITS>(sh);
 }
 
 // Stages the activations of one slot chunk (gate/up: x rows, normalised and
-// rounded to bf16 in the stack; down: h rows) as fp16 in the decoder's order.
+// rounded to bf16 in the stack; down: h rows) as int16 in the operand order.
 template <int MODE, int BITS, int LPR, int CPL>
 __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCursor& cur, const uint16_t* xsrc,
-                            const float* rnorm, const float* h, __half* xs, float* tok_inv, float* tok_w,
+                            const float* rnorm, const float* h, int16_t* xs, float* tok_inv, float* tok_w,
                             int* tok_pos, int warp, int lane) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
@@ -250,14 +245,9 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-    int sh = 0;
-    if (vmax > 0.f) {
-      int ex;
-      frexpf(vmax, &ex);
-      sh = min(max(8 - ex, -100), 100);
-    }
+    const int sh = act_shift(vmax);
     const float mul = ldexpf(1.f, sh);
-    __half* dst = xs + size_t(tl) * K;
+    int16_t* dst = xs + size_t(tl) * K;
     for (int g0 = lane * Gm::G; g0 < K; g0 += 32 * Gm::G) {
       float v[Gm::G];
 #pragma unroll
@@ -271,12 +261,12 @@ __device__ void stage_chunk(const FusedParams& p, const SRoute& rt, const FCurso
         }
       }
       uint4 parts[Gm::NPART];
-      pack_pair_order<Gm::G>(v, mul, parts);
+      pack_int_order<BITS, Gm::G>(v, mul, parts);
       const int base = staged_offset<BITS, LPR, CPL>(g0);
 #pragma unroll
       for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
     }
-    if (lane == 0) tok_inv[tl] = ldexpf(1.f, -sh);
+    if (lane == 0) tok_inv[tl] = act_inv<BITS>(sh);
   }
 }
 
@@ -284,15 +274,15 @@ constexpr int kMaxRE = 8;        // router rows (experts) per CTA
 
 // Stages token t once for the whole layer: one L2 round trip for the row
 // (each lane holds whole groups of G elements), RMSNorm factor (stack),
-// xhat = bf16(x * r), and the power-of-two scale that puts max |xhat| in
-// [128, 256); stored as fp16 in the gate/up operand order.  Then, from the
+// xhat = bf16(x * r), and the power-of-two scale of act_shift; stored as
+// int16 in the gate/up operand order.  Then, from the
 // same registers, the token's router logits for the ne <= kMaxRE experts
 // whose rows (bf16) are in shared memory at rrows once `rbar` completes
 // (rbar == nullptr: they already have): sum_h Wr[e][h] * xhat[h] in fp32
-// with exact products, plus the bias.  dst == nullptr skips the fp16 row;
+// with exact products, plus the bias.  dst == nullptr skips the int16 row;
 // xb_out (if set) receives xhat as bf16 in natural order.
 template <int BITS, int LPR, int CPL>
-__device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, float* rnorm_out, float* inv_out,
+__device__ void stage_token_all(const uint16_t* row, bool stack, int16_t* dst, float* rnorm_out, float* inv_out,
                                 uint16_t* xb_out, const uint16_t* rrows, int ne, const float* rbias,
                                 float* logit_row, uint64_t* rbar, uint32_t rpar, volatile int* abort_flag,
                                 int* status, int lane) {
@@ -354,12 +344,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
   float vmax = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  int sh = 0;
-  if (vmax > 0.f) {
-    int ex;
-    frexpf(vmax, &ex);
-    sh = min(max(8 - ex, -100), 100);
-  }
+  const int sh = act_shift(vmax);
   const float mul = ldexpf(1.f, sh);
 #pragma unroll
   for (int q = 0; q < NG && dst != nullptr; ++q) {
@@ -374,7 +359,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
       }
     }
     uint4 parts[Gm::NPART];
-    pack_pair_order<G>(vf, mul, parts);
+    pack_int_order<BITS, G>(vf, mul, parts);
     const int base = staged_offset<BITS, LPR, CPL>((q * 32 + lane) * G);
 #pragma unroll
     for (int part = 0; part < Gm::NPART; ++part) *reinterpret_cast<uint4*>(dst + base + part * LPR * 8) = parts[part];
@@ -387,7 +372,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, __half* dst, fl
   }
   if (lane == 0) {
     *rnorm_out = r;
-    *inv_out = ldexpf(1.f, -sh);
+    *inv_out = act_inv<BITS>(sh);
   }
   if (ne <= 0) return;
   if (rbar != nullptr) {
@@ -497,8 +482,8 @@ template <int MODE, int BITS, int LPR, int CPL, int PS>
 __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur, long long w1, unsigned char* ring,
                              int ring_stride, uint64_t* full, uint64_t* empty, int* consumed, int grp,
                              const uint16_t* xsrc, const float* rnorm, const float* hin, float* out, int out_cols,
-                             const __half* xs_pre, const float* pre_inv, const float* pre_w, int pre_base,
-                             __half* xs_grp, const GroupTok& tk, volatile int* abort_flag, int* status,
+                             const int16_t* xs_pre, const float* pre_inv, const float* pre_w, int pre_base,
+                             int16_t* xs_grp, const GroupTok& tk, volatile int* abort_flag, int* status,
                              unsigned long long* tacc = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
@@ -555,7 +540,7 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
         const int nt = min(4, nc - tb);
-        const __half* xb = pre ? xs_pre : xs_grp + size_t(tb) * K;
+        const int16_t* xb = pre ? xs_pre : xs_grp + size_t(tb) * K;
         const int* xr = pre ? tk.xrow : nullptr;
         if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 1, xr);
         else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 2, xr);
@@ -699,7 +684,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   const int NMW = (T + 31) >> 5;                                          // token mask words per expert
   // tokens: every token (pre-staged) or router chunks in R and G; the two
   // groups' chunk buffers in G (not pre-staged) and D
-  __half* xs = reinterpret_cast<__half*>(smem + p.smem_xs_off);
+  int16_t* xs = reinterpret_cast<int16_t*>(smem + p.smem_xs_off);
 
   char* ws = p.ws;
   int* status = reinterpret_cast<int*>(ws + p.L_.status);
@@ -715,7 +700,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   float* tkb = reinterpret_cast<float*>(smem + 1024 + grp * 4 * kMaxNTC * 4);
   const GroupTok tk{tkb, tkb + kMaxNTC, reinterpret_cast<int*>(tkb + 2 * kMaxNTC),
                     reinterpret_cast<int*>(tkb + 3 * kMaxNTC)};
-  __half* xs_grp = xs + size_t(grp) * p.grp_xs;
+  int16_t* xs_grp = xs + size_t(grp) * p.grp_xs;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kFStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kNCW); }
     mbar_init(rbar, 1);
@@ -760,7 +745,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       }
     } else {
       // one warp per token: it stages the token (RMSNorm factor in the stack,
-      // fp16 xhat with its power-of-two scale) -- into the token region, where
+      // int16 xhat with its power-of-two scale) -- into the token region, where
       // it stays for gate/up, or, when the tokens do not all fit, into its own
       // row of the idle ring slots 1-2 -- and at once computes the token's
       // router logits for this CTA's experts from their rows in ring slot 0

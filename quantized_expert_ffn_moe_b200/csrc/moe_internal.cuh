@@ -222,6 +222,12 @@ __device__ __forceinline__ void report_error(int* status, int code, int aux) {
   if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, aux);
 }
 
+// (a & b) ^ c in one instruction.
+__device__ __forceinline__ uint32_t lop_and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 // (a & b) | c in one instruction.
 __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
@@ -471,6 +477,10 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
                                 uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
                                 cudaStream_t s, int hybrid = 0);
 bool prefill_supported(const moe_config& c);
+// The argument checks of moe_layer_forward short of the workspace (MOE_OK for
+// T == 0, which is a no-op).
+int check_layer_args(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
+                     const uint16_t* y);
 // Decode-path choice for single layers of 32..64 tokens: 0 = by the cost
 // model after routing, 1 = always the fused CUDA-core kernel, 2 = always the
 // grouped tensor-core kernels (measurement hook moe_debug_decode_path).

@@ -24,16 +24,26 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 }
 
 // ------------------------------------------------------------------ rmsnorm
-// xhat[t] = bf16(x[t] / sqrt(mean(x[t]^2) + 1e-6)), one CTA of 256 threads per token.
+// xhat[t] = bf16(x[t] / sqrt(mean(x[t]^2) + 1e-6)), one CTA of 256 threads per
+// token.  The sum of squares runs in the same order as the norm that
+// combine_kernel fuses into the residual add (each thread 8 consecutive
+// elements per step of 2048, then the warps in order), so a layer gets the
+// same normalised input whichever of the two computed it.
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const uint16_t* __restrict__ x,
                                                       uint16_t* __restrict__ xhat, int H) {
   pdl_wait();
   const int t = blockIdx.x;
   const uint16_t* row = x + size_t(t) * H;
   float ss = 0.f;
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    const float v = bf16_bits_to_float(row[h]);
-    ss = fmaf(v, v, ss);
+  for (int h0 = threadIdx.x * 8; h0 < H; h0 += 256 * 8) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(row + h0);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(xw[i] << 16), hi = __uint_as_float(xw[i] & 0xFFFF0000u);
+      ss = fmaf(lo, lo, ss);
+      ss = fmaf(hi, hi, ss);
+    }
   }
   __shared__ float red[8];
 #pragma unroll

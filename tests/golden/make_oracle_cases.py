@@ -31,12 +31,21 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 
 # name -> spec.  shape: MoeShape name; T: batch size; batch: x stream id;
 # tokens: which tokens of the batch are stored (None = all); zipf: router bias;
-# layers: number of stacked layers (0 = a single layer, no norm / residual).
+# layers: number of stacked layers (0 = a single layer, no norm / residual);
+# steps: stack layers evaluated one at a time (RMSNorm, MoE, residual), layer l
+# on the seeded input of x stream batch + l.
 CASES = {
     "full4_decode": dict(shape="FULL4", T=16, batch=0, tokens=None, zipf=False, layers=0),
     "full2_zipf_decode": dict(shape="FULL2", T=64, batch=0, tokens=None, zipf=True, layers=0),
     "full4_prefill": dict(shape="FULL4", T=4096, batch=1, tokens=("sample", 24, 11), zipf=False, layers=0),
     "full4_stack48_decode": dict(shape="FULL4", T=32, batch=2, tokens=(0, 1, 2, 3), zipf=False, layers=48),
+    # one stack layer (RMSNorm, MoE, residual) at sampled depths of the
+    # 48-layer stack, each on its own seeded input (x stream id batch + l)
+    "full4_stack_step_t1": dict(shape="FULL4", T=1, batch=300, tokens=None, zipf=False, steps=(0, 1, 7, 23, 47)),
+    "full4_stack_step_t32": dict(shape="FULL4", T=32, batch=400, tokens=(0, 9, 31), zipf=False,
+                                 steps=(0, 1, 23, 47)),
+    "full4_stack_step_t2048": dict(shape="FULL4", T=2048, batch=500, tokens=("sample", 6, 2048), zipf=False,
+                                   steps=(0, 1, 23, 47)),
 }
 SEED = 0
 
@@ -81,8 +90,52 @@ def _stack_job(args):
     return rows, r
 
 
+def _step_job(args):
+    name, l, rows = args
+    spec = CASES[name]
+    shape = getattr(mi, spec["shape"])
+    x = mi.hidden_states_bf16(spec["T"], shape.hidden, SEED, spec["batch"] + l)[rows]
+    r = orc.layer_forward(oracle_layer(shape, l, spec["zipf"]), x, rmsnorm=True)
+    return l, rows, r
+
+
+def compute_steps(name: str, procs: int):
+    """Stack layers one at a time: for each sampled layer l the MoE output
+    (before the residual add), the routing, and the next residual stream."""
+    spec = CASES[name]
+    shape = getattr(mi, spec["shape"])
+    toks = case_tokens(spec)
+    steps = list(spec["steps"])
+    jobs = [(name, l, toks[i::procs]) for l in steps for i in range(procs) if len(toks[i::procs])]
+    ctx = mp.get_context("spawn")
+    t0 = time.time()
+    with ctx.Pool(min(len(jobs), procs)) as pool:
+        res = pool.map(_step_job, jobs)
+    out = dict(tokens=toks, shape=np.array([shape.experts, shape.hidden, shape.inter, shape.top_k,
+                                            int(shape.shared), shape.bits, shape.block]),
+               T=np.array(spec["T"]), batch=np.array(spec["batch"]), seed=np.array(SEED),
+               zipf=np.array(int(spec["zipf"])), steps=np.array(steps))
+    L, n, H = len(steps), len(toks), shape.hidden
+    out_ = np.zeros((L, n, H), np.float64)
+    logits = np.zeros((L, n, shape.experts), np.float64)
+    idx = np.zeros((L, n, shape.top_k), np.int32)
+    pos = {int(t): i for i, t in enumerate(toks)}
+    for l, rows, r in res:
+        li = steps.index(l)
+        for j, t in enumerate(rows):
+            out_[li, pos[int(t)]] = r["out"][j]
+            logits[li, pos[int(t)]] = r["logits"][j]
+            idx[li, pos[int(t)]] = r["idx"][j]
+    out.update(out_=out_.astype(np.float32), logits=logits, idx=idx)
+    path = os.path.join(HERE, f"oracle_{name}.npz")
+    np.savez_compressed(path, **out)
+    print(f"{name}: {n} tokens x {L} layers in {time.time() - t0:.1f} s -> {path}", flush=True)
+
+
 def compute(name: str, procs: int):
     spec = CASES[name]
+    if "steps" in spec:
+        return compute_steps(name, procs)
     shape = getattr(mi, spec["shape"])
     toks = case_tokens(spec)
     chunks = [toks[i::procs] for i in range(procs) if len(toks[i::procs])]

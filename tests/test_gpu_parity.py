@@ -222,75 +222,6 @@ def test_empty_batch_and_small_workspace():
     assert q.moe_layer_forward(cfg, w, x, y, small, check=False) == -3
 
 
-# ------------------------------------------------------------------ stack ---
-
-def _gpu_stack(shape, layers_w, x_bits, trace=True):
-    torch = gc.torch()
-    cfg = gc.cfg_of(shape)
-    T = x_bits.shape[0]
-    x = gc.to_dev_bits(x_bits)
-    ws = gc.workspace(cfg, T)
-    tr = torch.empty((len(layers_w), T, shape.top_k), dtype=torch.int32, device="cuda") if trace else None
-    q.moe_stack_forward(cfg, layers_w, x, ws, topk_trace=tr)
-    torch.cuda.synchronize()
-    assert q.moe_device_status(ws) == 0
-    return mi.bf16_bits_to_f32(gc.bits_to_np(x)).astype(np.float64), (tr.cpu().numpy() if trace else None)
-
-
-STACK_BAND = 2e-3   # the residual streams of both sides differ by bf16 rounding flips after a few layers
-
-
-def test_stack_tiny_live_oracle():
-    shape = mi.TINY
-    L, T = 4, 6
-    ws = [gc.device_layer(shape, 0, l) for l in range(L)]
-    x = mi.hidden_states_bf16(T, shape.hidden, 0, 2)
-    got, trace = _gpu_stack(shape, ws, x)
-    lays = [gc.host_oracle_layer(shape, 0, l, cache_size=shape.experts + 1) for l in range(L)]
-
-    def choose(l, logits, idx):
-        over = {}
-        for t in range(T):
-            if not np.array_equal(trace[l, t], idx[t]):
-                assert orc.tie_band_ok(logits[t], trace[l, t], shape.top_k, STACK_BAND), (l, t)
-                over[t] = trace[l, t]
-        return over
-    r = orc.stack_forward(lays, x, choose_topk=choose)
-    gc.assert_close_stack(got, r["x"])
-
-
-def test_stack_full48_decode_stored_oracle():
-    """48 resident layers.  For each token the GPU's selections must equal the
-    oracle's up to the first layer l* where they differ, and that difference
-    must be a valid choice inside the tie band.  After l* the two residual
-    streams differ by a whole expert, so the comparison point is the stream
-    entering layer l*: the GPU stack is re-run on the first l* layers and
-    compared with the oracle's stream after those layers.  Tokens that never
-    diverge are compared after all 48 layers."""
-    case = gc.load_case("full4_stack48_decode")
-    shape = mi.FULL4
-    L = int(case["layers"])
-    ws = [gc.device_layer(shape, 0, l) for l in range(L)]
-    x = mi.hidden_states_bf16(int(case["T"]), shape.hidden, 0, int(case["batch"]))
-    got, trace = _gpu_stack(shape, ws, x)
-    toks = case["tokens"]
-    depth = {}
-    for i, t in enumerate(toks):
-        first = next((l for l in range(L) if not np.array_equal(trace[l, t], case["trace_idx"][l, i])), None)
-        if first is not None:
-            assert orc.tie_band_ok(case["trace_logits"][first, i], trace[first, t], shape.top_k, STACK_BAND), \
-                (t, first)
-        depth[i] = L if first is None else first
-    for d in sorted(set(depth.values())):
-        if d == 0:
-            continue
-        xd = got if d == L else _gpu_stack(shape, ws[:d], x, trace=False)[0]
-        for i, t in enumerate(toks):
-            if depth[i] == d:
-                gc.assert_close_stack(xd[t], case["trace_x"][d - 1, i].astype(np.float64))
-    assert max(depth.values()) >= 8, depth
-
-
 # --------------------------------------------------- tensor-core prefill ---
 # Shapes small enough for the live oracle that still take the tcgen05 path
 # (H and I multiples of 256): several expert groups per tile row, ragged tiles.
