@@ -156,21 +156,31 @@ int moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, in
  * themselves -- for example a plugin running inside a host application that
  * has already claimed the GPU's memory through its own pool, or code that must
  * not call cudaMalloc/cudaFree because those calls can synchronise the whole
- * device.  Inputs, outputs and results are those of moe_layer_forward; the
- * scratch is a fixed array of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) compiled into
- * libmoe.so, which every GPU that loads the library keeps until the process
- * exits.  If moe_workspace_bytes(cfg, T) exceeds that size the call returns
+ * device.  Inputs, outputs and results are those of moe_layer_forward (the
+ * same kernels on the same inputs give the same bits), and the arguments are
+ * checked in the same order with the same codes; the scratch is a fixed array
+ * of MOE_NOALLOC_SCRATCH_BYTES (4 MiB) compiled into libmoe.so, which every
+ * GPU that loads the library keeps until the process exits.  If
+ * moe_workspace_bytes(cfg, T) exceeds that size the call returns
  * MOE_ERR_WORKSPACE and launches nothing (at the 512-expert, H=2048, I=768,
- * k=10 shape this allows up to 23 tokens).  The first call on a device looks
- * up the array's device address, once per device and with that device
+ * k=10 shape this allows up to 23 tokens).  The first call on a device (and
+ * the first after its context was destroyed and re-created, e.g. by
+ * cudaDeviceReset) looks up the array's device address with that device
  * current; make that first call before any stream capture.  All calls share
- * the one array and it keeps the previous call's contents (the call clears the
- * part that must start at zero): calls that overlap on the GPU (from other
+ * the one array and it keeps the previous call's contents (the call clears
+ * the part that must start at zero): calls that overlap on the GPU (from other
  * streams or host threads) race, so the caller must serialise them.  No
  * allocating routine is called. */
 #define MOE_NOALLOC_SCRATCH_BYTES (4u << 20)
 int moe_layer_forward_noalloc(const moe_config* cfg, const moe_layer_weights* w,
                               const uint16_t* x, int32_t T, uint16_t* y, void* stream);
+
+/* The device check word of moe_layer_forward_noalloc's scratch on the current
+ * device, as moe_device_status reads it from a workspace (synchronises the
+ * device): *code_out = 0 when no kernel of the last call reported a failed
+ * check, else the moe_status code (e.g. MOE_ERR_TIMEOUT), and the return value
+ * is MOE_ERR_DEVICE_CHECK.  The pages have no counterpart. */
+int moe_noalloc_device_status(int32_t* code_out);
 
 /* Reads back the device check word kept in the workspace (synchronises the
  * device).  *code_out = 0 when no kernel reported a failed check. */

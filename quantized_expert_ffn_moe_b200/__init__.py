@@ -20,8 +20,8 @@ __all__ = [
     "MoeConfig", "LayerWeights", "MoeError", "load_library", "EXPORTS", "LIB_PATH",
     "moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
     "moe_device_status", "moe_dequant_rows", "moe_status_str", "config_of", "moe_profile_begin",
-    "moe_profile_end", "moe_layer_forward_noalloc", "NOALLOC_SCRATCH_BYTES", "moe_layer_forward_ep",
-    "ep_all_reduce",
+    "moe_profile_end", "moe_layer_forward_noalloc", "moe_noalloc_device_status", "NOALLOC_SCRATCH_BYTES",
+    "moe_layer_forward_ep", "ep_all_reduce",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
@@ -29,7 +29,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
            "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end",
            "moe_layer_forward_noalloc", "moe_last_cuda_error", "moe_debug_fused_timing",
-           "moe_debug_prefill_timing", "moe_layer_forward_ep", "moe_debug_decode_path", "moe_debug_wait_probe")
+           "moe_debug_prefill_timing", "moe_layer_forward_ep", "moe_debug_decode_path", "moe_debug_wait_probe",
+           "moe_noalloc_device_status")
 
 MOE_OK = 0
 
@@ -107,6 +108,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_dequant_rows.restype = ctypes.c_int
     lib.moe_layer_forward_noalloc.argtypes = [cfgp, ctypes.POINTER(_Weights), P, I32, P, P]
     lib.moe_layer_forward_noalloc.restype = ctypes.c_int
+    lib.moe_noalloc_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+    lib.moe_noalloc_device_status.restype = ctypes.c_int
     lib.moe_profile_begin.argtypes = [I32]
     lib.moe_profile_begin.restype = ctypes.c_int
     lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32)]
@@ -220,6 +223,17 @@ def moe_layer_forward_noalloc(cfg: MoeConfig, w: LayerWeights, x, y, *, stream=N
 
 
 NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_noalloc_device_status() -> int:
+    """The device check word of the allocation-free entry point's scratch on
+    the current device (synchronises the device); 0 when no kernel reported a
+    failed check."""
+    code = ctypes.c_int32(0)
+    st = load_library().moe_noalloc_device_status(ctypes.byref(code))
+    if st not in (MOE_OK, -5):
+        _check(st, "moe_noalloc_device_status")
+    return int(code.value)
 
 
 def moe_stack_forward(cfg: MoeConfig, layers: Sequence[LayerWeights], x_inout, workspace, *, topk_trace=None,

@@ -115,6 +115,26 @@ int run_layer(const LayerArgs& a) {
 
 }  // namespace
 
+namespace moe {
+// Everything moe_layer_forward checks before it looks at the workspace, in the
+// same order: the config, T, the weights, x and y (non-null, 16-byte aligned,
+// not overlapping).  T == 0 passes (the call is then a no-op).
+int check_layer_args(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
+                     const uint16_t* y) {
+  int st = validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if ((st = validate_weights(cfg, w)) != MOE_OK) return st;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  const size_t bytes = size_t(T) * cfg->hidden * 2;
+  const char* xb = reinterpret_cast<const char*>(x);
+  const char* yb = reinterpret_cast<const char*>(y);
+  if (xb < yb + bytes && yb < xb + bytes) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_bytes(const moe_config* cfg, int32_t max_tokens) {
@@ -150,16 +170,9 @@ int moe_route(const moe_config* cfg, const uint16_t* router_w, const float* rout
 
 int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const uint16_t* x, int32_t T,
                       uint16_t* y, void* workspace, size_t ws_bytes, void* stream) {
-  int st = validate_config(cfg);
+  int st = moe::check_layer_args(cfg, w, x, T, y);
   if (st != MOE_OK) return st;
-  if (T < 0) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  if ((st = validate_weights(cfg, w)) != MOE_OK) return st;
-  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
-  const size_t bytes = size_t(T) * cfg->hidden * 2;
-  const char* xb = reinterpret_cast<const char*>(x);
-  const char* yb = reinterpret_cast<const char*>(y);
-  if (xb < yb + bytes && yb < xb + bytes) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(cfg, T, workspace, ws_bytes)) != MOE_OK) return st;
   LayerArgs a{};
   a.cfg = *cfg; a.w = *w; a.T = T; a.x = x; a.y = y; a.residual = false; a.xhat_next = nullptr;

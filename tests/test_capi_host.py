@@ -120,6 +120,28 @@ def test_layer_forward_argument_errors(lib):
     assert lib.moe_layer_forward(None, ctypes.byref(w), 1 << 30, 4, 2 << 30, 3 << 30, 1 << 40, None) == -1
 
 
+def test_noalloc_argument_errors_match_layer_forward(lib):
+    """The allocation-free entry point checks its arguments in the same order
+    as moe_layer_forward (the size limit of its fixed scratch takes the place
+    of the workspace check), so it reports the same codes, all on the host."""
+    c = cfg()
+    w = _fake_weights()
+
+    def na(c, w, x=1 << 30, T=4, y=2 << 30):
+        return lib.moe_layer_forward_noalloc(ctypes.byref(c), ctypes.byref(w) if w is not None else None, x, T, y,
+                                             None)
+    assert na(c, w, T=0) == 0                                  # empty batch: no-op
+    assert na(c, w, T=-1) == -1
+    assert na(c, None, T=24) == -1                             # null weights beat the size limit
+    assert na(c, w, x=None, T=1000) == -1                      # null x beats the size limit
+    assert na(c, w, y=(1 << 30) + 1024) == -1                  # y overlaps x
+    assert na(cfg(bits=3), w) == -2                             # the config's own code (unsupported)
+    assert na(cfg(top_k=0), w) == -1                            # ... or invalid
+    assert na(c, _fake_weights(misalign="down_codes")) == -1
+    assert na(c, w, T=24) == -3                                 # beyond the 4 MiB scratch: MOE_ERR_WORKSPACE
+    assert lib.moe_noalloc_device_status(None) == -1
+
+
 def _layer_ep(lib, c, w, rank, size, x=1 << 30, T=4, y=2 << 30, ws=3 << 30, ws_bytes=None):
     if ws_bytes is None:
         ws_bytes = lib.moe_workspace_bytes(ctypes.byref(c), T)
@@ -205,6 +227,8 @@ int use(void* ws, size_t n, const uint16_t* x, uint16_t* y, float* yp, void* str
   st |= moe_layer_forward_ep(&c, &w, x, 16, 0, 2, yp, ws, n, stream);
   st |= moe_stack_forward(&c, &w, 1, y, 16, NULL, ws, n, stream);
   st |= moe_device_status(ws, &code);
+  st |= moe_layer_forward_noalloc(&c, &w, x, 16, y, stream);
+  st |= moe_noalloc_device_status(&code);
   moe_debug_decode_path(0);
   (void)moe_status_str(st);
   return st + (int)need + code;
