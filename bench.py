@@ -45,8 +45,6 @@ def parse():
     ap.add_argument("--tokens", type=int, default=16)
     ap.add_argument("--instances", type=int, default=48, help="distinct layer instances rotated over")
     ap.add_argument("--no-detail", action="store_true", help="skip the secondary workloads")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=16,
-                    help="tokens of the headline batch the CPU oracle baseline runs (16 = the whole batch)")
     ap.add_argument("--quick", action="store_true",
                     help="headline loop only (no e2e, detail or CPU baseline): the small case used for ncu")
     return ap.parse_args()
@@ -150,60 +148,110 @@ class Clocks:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def cpu_threads() -> int:
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return int(max(n)) if n else 1
-    except Exception:
-        return 1
-
-
 # --------------------------------------------------------------- oracle ---
+# The CPU baseline runs the float64 oracle as it stands, one process per host
+# core (spawned, one BLAS thread each), each process taking its share of the
+# batch's tokens (tokens are independent in the layer).  The packed experts a
+# process needs are generated before the clock starts; a timed step is the
+# wall time of all processes running their tokens once.
 
-def oracle_sample(tokens: int):
-    """Times the CPU oracle (as it stands) on the first `tokens` tokens of the
-    headline workload.  Input generation happens before the clock starts."""
+def _ref_env():
+    for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[v] = "1"
+
+
+_REF = {}
+
+
+def _ref_prepare(tokens):
     import moe_inputs as mi
     import oracle as orc
     shape = mi.FULL4
-    x = mi.hidden_states_bf16(16, shape.hidden, 0, 0)[:tokens]
+    x = mi.hidden_states_bf16(16, shape.hidden, 0, 0)[tokens]
     rw = mi.router_weight_bf16(shape, 0, 0)
     logits = orc.router_logits(orc.bf16_to_f64(x), rw, None)
     need = sorted(set(orc.select_topk(logits, shape.top_k).reshape(-1).tolist()))
     packed = {e: mi.expert_packed(shape, 0, 0, e) for e in need}
     sh = mi.shared_packed(shape, 0, 0)
-    lay = orc.OracleLayer(experts=shape.experts, hidden=shape.hidden, inter=shape.inter, top_k=shape.top_k,
-                          bits=shape.bits, block=shape.block, router_w_bits=rw, router_bias=None,
-                          expert=lambda e: packed[e], shared=lambda: sh, cache_size=4)
+    _REF["x"] = x
+    _REF["layer"] = orc.OracleLayer(experts=shape.experts, hidden=shape.hidden, inter=shape.inter,
+                                    top_k=shape.top_k, bits=shape.bits, block=shape.block, router_w_bits=rw,
+                                    router_bias=None, expert=lambda e: packed[e], shared=lambda: sh, cache_size=4)
+    return len(need)
+
+
+def _ref_run(_):
+    import oracle as orc
     t0 = time.perf_counter()
-    orc.layer_forward(lay, x)
-    dt = time.perf_counter() - t0
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{tokens} decode tokens of the 16-token headline batch (layer 0, seed 0), float64 numpy; "
-                      f"{dt:.1f} s wall"}
+    orc.layer_forward(_REF["layer"], _REF["x"])
+    return time.perf_counter() - t0
+
+
+def _mask(cpus) -> str:
+    m = 0
+    for c in cpus:
+        m |= 1 << c
+    return hex(m)
+
+
+class OraclePool:
+    """The oracle on the 16-token headline batch, spread over the host cores."""
+
+    def __init__(self, tokens: int = 16):
+        import multiprocessing as mp
+        try:
+            self.affinity = sorted(os.sched_getaffinity(0))
+        except AttributeError:
+            self.affinity = list(range(os.cpu_count() or 1))
+        self.procs = max(1, min(tokens, len(self.affinity)))
+        self.tokens = tokens
+        chunks = [list(range(i, tokens, self.procs)) for i in range(self.procs)]
+        _ref_env()
+        self.pool = mp.get_context("spawn").Pool(self.procs)
+        self.pool.map(_ref_prepare, chunks, chunksize=1)      # untimed: inputs and packed experts
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        self.pool.map(_ref_run, range(self.procs), chunksize=1)
+        return time.perf_counter() - t0
+
+    def describe(self, value: float, steps: int, seconds: float) -> dict:
+        return {"value": value, "unit": "tokens/s", "cores": self.procs, "kind": "oracle",
+                "nproc": os.cpu_count(), "affinity": _mask(self.affinity),
+                "sample": f"the whole {self.tokens}-token headline batch (layer 0, seed 0) per step, float64 numpy, "
+                          f"tokens split over {self.procs} spawned processes with one BLAS thread each; "
+                          f"{steps} step(s), {seconds:.1f} s wall"}
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def oracle_sample(steps: int = 1, warm: int = 1):
+    op = OraclePool()
+    try:
+        for _ in range(warm):
+            op.step()
+        tot = sum(op.step() for _ in range(steps))
+        return op.describe(steps * op.tokens / tot, steps, tot), tot
+    finally:
+        op.close()
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    steps = max(1, args.steps if args.steps < 5 else 1)
-    warm = min(max(args.warmup, 0), 3)          # untimed samples first (page cache, BLAS threads)
-    for _ in range(warm):
-        oracle_sample(1)
-    tot_tok, tot_t = 0, 0.0
-    cb = None
-    for _ in range(steps):
-        cb = oracle_sample(args.cpu_sample_tokens)
-        tot_tok += args.cpu_sample_tokens
-        tot_t += args.cpu_sample_tokens / cb["value"]
-    v = tot_tok / tot_t
-    cb["value"] = v
+    # every one of the K steps runs the oracle on the whole batch; more than
+    # 60 steps would not finish within a few minutes, so K is capped there
+    steps = max(1, min(args.steps, 60))
+    warm = min(max(args.warmup, 0), 3)
+    cb, tot = oracle_sample(steps, warm)
+    v = cb["value"]
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": warm, "ms_per_step": 1000.0 * tot_t / steps, "higher_is_better": True,
+            "steps": steps, "warmup": warm, "ms_per_step": 1000.0 * tot / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "full-shape MoE layer decode, 16 tokens, 4-bit/32 (CPU oracle on a token sample)",
+            "config": {"workload": "full-shape MoE layer decode, 16 tokens, 4-bit/32 (CPU oracle)",
                        "experts": 512, "hidden": 2048, "inter": 768, "top_k": 10, "shared": 1, "bits": 4,
                        "block": 32, "tokens": 16},
             "cpu_baseline": cb,
@@ -384,14 +432,20 @@ def main():
     phase_ms, calls = q.moe_profile_end()
     fused = phase_ms[4] > 0
     if fused:
-        # one cooperative kernel per layer: the dominant (only) kernel moves all touched bytes
-        k_ms = phase_ms[4] / calls
-        k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * EXPERT_BYTES[4] + ROUTER_BYTES
+        # one cooperative kernel per layer is the step's only launch: its mean
+        # duration is the graph-replayed step time of the timed region above
+        # (CUDA events on the launching stream; it includes the gaps between
+        # launches), and it moves all the touched bytes of those K steps
+        k_ms = ms_step
+        k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(K)])) * EXPERT_BYTES[4] + ROUTER_BYTES
         kname = "fused_decode_kernel (whole layer, one launch)"
+        timing = ("CUDA events around the K graph-replayed steps on the launching stream; one launch of this "
+                  "kernel per step")
     else:
         k_ms = phase_ms[1] / calls
         k_bytes = float(np.mean([(us[i % len(us)] + 1) for i in range(calls)])) * GU_BYTES[4]
         kname = "ffn_tma_kernel<gate/up>"
+        timing = "CUDA events around each launch of this kernel (eager loop of the same steps)"
     pf = profiled_fields("fused_decode_kernel_decode4_t16.txt",
                          ["fused.cu", "decode_common.cuh", "moe_internal.cuh"]) if fused else None
     traffic = float(pf["traffic_bytes_per_launch"]) if pf and "traffic_bytes_per_launch" in pf else None
@@ -400,17 +454,21 @@ def main():
                 "traffic_source": "profiles/fused_decode_kernel_decode4_t16.txt (ncu dram__bytes_read.sum + "
                                   "dram__bytes_write.sum, one launch of the same workload)" if traffic else None,
                 "peak_source": f"{peak_src} (copy bandwidth)",
-                "algorithmic_bytes_per_launch": k_bytes, "launch_us": 1000 * k_ms,
-                "phase_us": {"route": 1000 * phase_ms[0] / calls, "gate_up": 1000 * phase_ms[1] / calls,
-                             "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls,
-                             "fused": 1000 * phase_ms[4] / calls}}
+                "algorithmic_bytes_per_launch": k_bytes, "launch_us": 1000 * k_ms, "timing": timing,
+                "launch_us_eager": 1000 * (phase_ms[4] if fused else phase_ms[1]) / calls,
+                "phase_us_eager": {"route": 1000 * phase_ms[0] / calls, "gate_up": 1000 * phase_ms[1] / calls,
+                                   "down": 1000 * phase_ms[2] / calls, "combine": 1000 * phase_ms[3] / calls,
+                                   "fused": 1000 * phase_ms[4] / calls}}
     roofline["frac"] = roofline["achieved"] / hbm_peak
     try:
-        # the decode kernel's second ceiling: instruction issue (it is issue-
-        # bound, which is why the HBM fraction stays below one)
+        # the decode kernel's second ceiling: instruction issue at the SM
+        # clock sampled during the timed region
         if pf and "instructions_per_launch" in pf:
             sms = torch.cuda.get_device_properties(0).multi_processor_count
-            roofline["issue"] = issue_ceiling(float(pf["instructions_per_launch"]), k_ms * 1e-3, sms)
+            mhz = clocks.get("sm_mhz") or 1965.0
+            roofline["issue"] = issue_ceiling(float(pf["instructions_per_launch"]), k_ms * 1e-3, sms, mhz)
+            roofline["issue"]["clock_source"] = ("median SM clock sampled during the timed region"
+                                                 if clocks.get("sm_mhz") else "nominal maximum (no clock samples)")
     except Exception:
         pass
     launches_per_step = 1 if fused else 5
@@ -484,7 +542,7 @@ def main():
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     if world == 1:
-        line["cpu_baseline"] = oracle_sample(args.cpu_sample_tokens)
+        line["cpu_baseline"] = oracle_sample(1, 1)[0]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -565,8 +623,39 @@ def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
             graphs, full = R.timed_graph(sstep, K, 2, chunk=K)
             barrier(dist, world)
             ms = max_over_ranks(dist, world, R.replay(graphs, full))
-            out[f"stack48_t{T}"] = {"tokens": T, "steps": K, "ms_per_step": ms / K,
-                                    "tokens_per_s": T * K / (ms / 1000)}
+            r = {"tokens": T, "steps": K, "ms_per_step": ms / K, "tokens_per_s": T * K / (ms / 1000)}
+            # decode T = 1 touches 10 routed + the shared expert per layer; at
+            # T = 32 the distinct experts are counted from the routing of layer 0
+            # of each batch (near-uniform routing makes the layers alike)
+            if T == 1:
+                bytes_step = 48 * (11 * EXPERT_BYTES[4] + ROUTER_BYTES)
+                r["touched_gb_per_step"] = bytes_step / 1e9
+                r["frac_of_measured_hbm"] = bytes_step / (ms / K * 1e-3) / 1e9 / hbm_peak
+            out[f"stack48_t{T}"] = r
+        # 2048-token prefill through the 48-layer stack: every layer touches
+        # all 512 experts (2048 x 10 picks), 1.364 GB, and does 212.6 GFLOP of
+        # expert FFN (+ 4.3 GFLOP router); HBM-bound (about 142 FLOP/B)
+        xs = R.xbatches(shape, 2048, 2, base=650)
+        xw = torch.empty_like(xs[0])
+
+        def pstep(i):
+            xw.copy_(xs[i % 2])
+            q.moe_stack_forward(cfg, pool4[:48], xw, ws)
+        K = 3
+        graphs, full = R.timed_graph(pstep, K, 1, chunk=K)
+        barrier(dist, world)
+        ms = max_over_ranks(dist, world, R.replay(graphs, full))
+        del graphs
+        T = 2048
+        bytes_step = 48 * (513 * EXPERT_BYTES[4] + ROUTER_BYTES) + 2 * 2 * T * 2048 * 2
+        flops_step = 48 * (9437184.0 * (T * 10 + T) + 2.0 * T * 512 * 2048)
+        sec = ms / K * 1e-3
+        out["stack48_prefill_t2048"] = {
+            "tokens": T, "steps": K, "ms_per_step": ms / K, "tokens_per_s": T / sec,
+            "gb_per_step": bytes_step / 1e9, "achieved_gbs": bytes_step / sec / 1e9,
+            "frac_of_measured_hbm": bytes_step / sec / 1e9 / hbm_peak,
+            "tflops": flops_step / sec / 1e12, "frac_of_measured_bf16": flops_step / sec / 1e12 / tf_peak,
+            "bound": "hbm (about 142 FLOP per byte of expert weights, below the ridge)"}
     return out
 
 
