@@ -586,6 +586,13 @@ def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
     poolg = R.layers(sg, 4)
     layer_rate(cfg_g, sg, poolg, 16, 2000, "4g128", "decode4g128_t16")
     del poolg
+    # 2-bit codes read as the four half-integer levels (+-1/2, +-3/2), 16
+    # tokens, near-uniform routing (8 layer instances: 7.3 GB, far above L2)
+    sh2 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=2, block=16, half=True)
+    cfg_h = q.config_of(512, 2048, 768, 10, True, 2, 16, half_levels=True)
+    poolh = R.layers(sh2, 8)
+    layer_rate(cfg_h, sh2, poolh, 16, 2000, 2, "decode2h_t16")
+    del poolh
     layer_rate(cfg, shape, pool4, 4096, 8, 4, "prefill4_t4096")
 
     # expert-parallel share: one rank's partial of the 4096-token layer when

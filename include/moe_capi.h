@@ -19,7 +19,7 @@
  *   l_e   = sum_h x_h Wr[e,h] (+ b_e)                  fp32 accumulation
  *   S     = the k largest l_e, slots by descending logit, ties -> smaller e
  *   w_j   = softmax over the selected logits (= full softmax renormalised)
- *   FFN_e = W_down,e (silu(W_gate,e x) * (W_up,e x)),   W = (code - 2^(b-1)) * scale
+ *   FFN_e = W_down,e (silu(W_gate,e x) * (W_up,e x)),   W = q * scale (q from the code)
  *   out   = g(x) FFN_shared(x) + sum_j w_j FFN_{S_j}(x)  slot order, fp32, -> bf16
  *   g(x)  = 1, or sigmoid(sum_h x_h Wg[h]) when a shared-expert gate vector Wg is given
  *
@@ -28,6 +28,9 @@
  *   codes : one byte holds 8/bits elements of a row; element j of a row is at
  *           byte j*bits/8, bit offset (j*bits)%8 (lower element in lower bits);
  *           stored code c = q + 2^(bits-1), q in [-(2^(bits-1)-1), 2^(bits-1)-1]
+ *           (integer levels; 2-bit is then ternary), or, with half_levels,
+ *           c = q + (2^bits - 1)/2, q in {-(2^(bits-1) - 1/2), ..., 2^(bits-1) - 1/2}
+ *           (the 2^bits half-integer levels; 2-bit: +-1/2, +-3/2)
  *   scales: one IEEE fp16 per block of `block` consecutive elements of a row
  *   gate/up: one [2I, H] matrix per expert, row 2i = gate row i, row 2i+1 =
  *           up row i; down: [H, I] per expert.  Experts are stacked densely.
@@ -71,6 +74,10 @@ typedef struct moe_config {
   int32_t shared_inter;  /* 0 = no shared expert, else == inter  */
   int32_t bits;          /* 4 or 2                               */
   int32_t block;         /* 32 (4-bit) or 16 (2-bit)             */
+  int32_t half_levels;   /* 0: q = c - 2^(bits-1) (integer levels,
+                            2-bit ternary); 1: q = c - (2^bits-1)/2,
+                            the 2^bits half-integer levels (2-bit:
+                            four levels +-1/2, +-3/2)              */
 } moe_config;
 
 /* One layer's weights; every pointer is device memory owned by the caller. */
@@ -203,16 +210,21 @@ int moe_profile_begin(int32_t max_calls);
 int moe_profile_end(float* ms_out, int32_t* calls);
 
 /* Measurement hook: while device_buf is non-null, fused decode launches write
- * %globaltimer readings (ns) of each CTA's first layer to device_buf[cta][20]
- * (zero it first; the caller owns the buffer; null switches it off):
- *   [8] layer start, [14] token 0 staged (with its router logits when each
- *   warp stages one token), [15] this CTA's router logits written,
- *   [0] router logits done (CTA barrier), [1] after the first grid barrier,
- *   [9] top-k done, [10] grouping scan done, [2] work lists ready,
- *   [3] gate/up done, [4] after the second barrier, [5] down done,
- *   [6] after the third barrier, [7] combine done;
- *   [11..13] gate/up and [16..18] down, consumer group 0: ns spent waiting for
- *   stage data, ns spent staging tokens, stages taken.
+ * timestamps of each CTA's first layer to device_buf[cta][32] (zero it first;
+ * the caller owns the buffer; null switches it off).  SM clock64 cycles:
+ *   [8] layer start, [21] scratch counters cleared, [19] token 0's row loaded,
+ *   [20] token 0 staged, [14] token 0's router logits done (with its router
+ *   logits when each warp stages one token), [15] this CTA's router logits
+ *   written, [0] router logits done (CTA barrier), [1] after the first grid
+ *   barrier, [9] top-k done, [10] routing lists done, [2] work lists ready,
+ *   [3] gate/up done, [4] after the waits for other CTAs' gate/up rows,
+ *   [5] down done, [6] after the second grid barrier, [7] combine done;
+ *   consumer group 0: [24] / [25] first gate/up stage's data in / last
+ *   gate/up stage done, [26] / [27] the same for down; producer: [28] / [29]
+ *   first / last gate/up stage issued, [30] / [31] down.  %globaltimer ns
+ *   (comparable across CTAs): [22] layer start, [23] combine done.
+ *   [11..13] gate/up and [16..18] down, consumer group 0: ns spent waiting
+ *   for stage data, ns spent staging tokens, stages taken.
  * Calls made while it is set are not reentrant-safe measurements of a
  * production run; they only observe one. */
 void moe_debug_fused_timing(unsigned long long* device_buf);

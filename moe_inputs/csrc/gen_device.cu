@@ -43,7 +43,7 @@ __device__ inline float normal_at(uint64_t key, uint64_t i, float c) {
 struct PoolArgs {
   uint64_t seed;
   int layer, E, H, I, bits, block;
-  int e0, ne, shared;
+  int e0, ne, shared, half;
   float c;
   uint8_t* gu_codes;
   uint16_t* gu_scales;
@@ -89,18 +89,27 @@ __global__ void gen_pool_kernel(PoolArgs a) {
       w[j] = normal_at(key, (uint64_t)row * K + col0 + j, a.c);
       amax = fmaxf(amax, fabsf(w[j]));
     }
-    const __half s16 = __float2half_rn(__fdiv_rn(amax, float(qmax)));
+    // half-integer levels: top level qmax + 1/2, code of the level just
+    // above w / s (floor + 2^(bits-1)), clamped to the 2^bits codes
+    const float top = a.half ? float(qmax) + 0.5f : float(qmax);
+    const __half s16 = __float2half_rn(__fdiv_rn(amax, top));
     const float sf = __half2float(s16);
     uint32_t packed[16] = {0};           // up to 64 bytes of codes per block
     for (int j = 0; j < a.block; ++j) {
-      int q = 0;
+      int code = 1 << (a.bits - 1);
       if (sf != 0.f) {
-        q = int(rintf(__fdiv_rn(w[j], sf)));
-        q = q < -qmax ? -qmax : (q > qmax ? qmax : q);
+        const float ratio = __fdiv_rn(w[j], sf);
+        if (a.half) {
+          code = int(floorf(ratio)) + (1 << (a.bits - 1));
+          code = code < 0 ? 0 : (code > (1 << a.bits) - 1 ? (1 << a.bits) - 1 : code);
+        } else {
+          int q = int(rintf(ratio));
+          q = q < -qmax ? -qmax : (q > qmax ? qmax : q);
+          code = q + (1 << (a.bits - 1));
+        }
       }
-      const uint32_t code = uint32_t(q + (1 << (a.bits - 1)));
       const int bit = j * a.bits;
-      packed[bit >> 5] |= code << (bit & 31);
+      packed[bit >> 5] |= uint32_t(code) << (bit & 31);
     }
     const int code_bytes = a.block * a.bits / 8;
     const size_t row_bytes = size_t(K) * a.bits / 8;
@@ -134,14 +143,15 @@ extern "C" {
 // shared expert (shared == 1, ne == 1).  Outputs are device buffers laid out
 // as in include/moe_capi.h, starting at the first generated expert.
 // c = fp32 sigma / 75674.45 (bits 0x348de3bd for sigma 0.02).
-int moe_gen_pool(uint64_t seed, int layer, int E, int H, int I, int bits, int block, int e0, int ne, int shared,
-                 float c, uint8_t* gu_codes, uint16_t* gu_scales, uint8_t* d_codes, uint16_t* d_scales,
+int moe_gen_pool(uint64_t seed, int layer, int E, int H, int I, int bits, int block, int half, int e0, int ne,
+                 int shared, float c, uint8_t* gu_codes, uint16_t* gu_scales, uint8_t* d_codes, uint16_t* d_scales,
                  void* stream) {
   if (!((bits == 4 && (block == 32 || block == 128)) || (bits == 2 && block == 16))) return -2;
   if (ne <= 0 || (shared && ne != 1) || (!shared && (e0 < 0 || e0 + ne > E))) return -1;
   if (!gu_codes || !gu_scales || !d_codes || !d_scales) return -1;
   if (H % block || I % block) return -2;
-  PoolArgs a{(uint64_t)seed, layer, E, H, I, bits, block, e0, ne, shared, c, gu_codes, gu_scales, d_codes, d_scales};
+  PoolArgs a{(uint64_t)seed, layer, E, H, I, bits, block, e0, ne, shared, half ? 1 : 0, c, gu_codes, gu_scales,
+             d_codes, d_scales};
   gen_pool_kernel<<<148 * 16, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }

@@ -21,7 +21,7 @@ def load():
             raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m moe_inputs.build`")
         lib = ctypes.CDLL(LIB_PATH)
         u64, i32, f32, P = ctypes.c_uint64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
-        lib.moe_gen_pool.argtypes = [u64, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P, P, P, P]
+        lib.moe_gen_pool.argtypes = [u64, i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, f32, P, P, P, P, P]
         lib.moe_gen_pool.restype = ctypes.c_int
         lib.moe_gen_normal_bf16.argtypes = [u64, u64, u64, f32, P, P]
         lib.moe_gen_normal_bf16.restype = ctypes.c_int
@@ -46,7 +46,7 @@ def fill_pool(shape: gen.MoeShape, seed: int, layer: int, gu_codes, gu_scales, d
     tensors, which start at the first generated expert."""
     ne = (1 if shared else shape.experts - e0) if ne is None else ne
     st = load().moe_gen_pool(seed, layer, shape.experts, shape.hidden, shape.inter, shape.bits, shape.block,
-                             e0, ne, 1 if shared else 0, float(gen.C_SIGMA002), gu_codes.data_ptr(),
+                             1 if shape.half else 0, e0, ne, 1 if shared else 0, float(gen.C_SIGMA002), gu_codes.data_ptr(),
                              gu_scales.data_ptr(), d_codes.data_ptr(), d_scales.data_ptr(), _stream())
     if st != 0:
         raise RuntimeError(f"moe_gen_pool failed: {st}")

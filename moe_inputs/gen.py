@@ -20,7 +20,12 @@ Recipe (identical on the CUDA side, ``csrc/gen_device.cu``):
   quantiser: ``s = fp16(fp32(absmax / qmax))``, ``q = clamp(rint(w / s),
   -qmax, qmax)`` (``q = 0`` where ``s == 0``), ``qmax = 2**(bits-1) - 1``,
   stored code ``c = q + 2**(bits-1)``, lower element index in the lower bits
-  of each byte.
+  of each byte.  Half-integer levels (the format variant with 2**bits levels
+  +-1/2 ... +-(2**(bits-1) - 1/2), e.g. four for 2-bit):
+  ``s = fp16(fp32(absmax / L))`` with ``L = 2**(bits-1) - 1/2``, ``c =
+  clamp(floor(fp32(w / s)) + 2**(bits-1), 0, 2**bits - 1)`` (the level just
+  above w / s, so a value exactly on a boundary takes the upper level;
+  ``c = 2**(bits-1)`` where ``s == 0``), decoded as ``q = c - (2**bits - 1)/2``.
 
 Element indices: gate / up masters are ``[I, H]`` (index ``i*H + h``), down
 masters ``[H, I]`` (index ``r*I + i``).  The packed gate/up matrix
@@ -77,6 +82,7 @@ class MoeShape:
     shared: bool
     bits: int
     block: int
+    half: bool = False          # half-integer levels (2**bits levels, no zero)
 
     @property
     def qmax(self) -> int:
@@ -157,7 +163,7 @@ def scales_per_row(cols: int, block: int) -> int:
     return cols // block
 
 
-def quantize_blocks(w: np.ndarray, bits: int, block: int):
+def quantize_blocks(w: np.ndarray, bits: int, block: int, half: bool = False):
     """Encode fp32 masters [rows, cols] into (codes uint8 [rows, cols*bits/8],
     scales uint16 fp16-bits [rows, cols/block]).  Input preparation only."""
     w = np.asarray(w, dtype=np.float32)
@@ -166,14 +172,20 @@ def quantize_blocks(w: np.ndarray, bits: int, block: int):
     qmax = (1 << (bits - 1)) - 1
     wb = w.reshape(rows, cols // block, block)
     amax = np.max(np.abs(wb), axis=-1)
-    s16 = (amax / np.float32(qmax)).astype(np.float32).astype(np.float16)
+    top = np.float32(qmax + 0.5) if half else np.float32(qmax)
+    s16 = (amax / top).astype(np.float32).astype(np.float16)
     sf = s16.astype(np.float32)
     safe = np.where(sf == 0, np.float32(1), sf)
     with np.errstate(invalid="ignore", divide="ignore"):
-        q = np.rint(wb / safe[..., None]).astype(np.float32)
-    q = np.clip(q, -qmax, qmax)
-    q[sf == 0] = 0
-    c = (q.astype(np.int32) + (1 << (bits - 1))).astype(np.uint8).reshape(rows, cols)
+        ratio = (wb / safe[..., None]).astype(np.float32)
+    if half:
+        c = np.clip(np.floor(ratio) + (1 << (bits - 1)), 0, (1 << bits) - 1)
+        c[sf == 0] = 1 << (bits - 1)
+        c = c.astype(np.uint8).reshape(rows, cols)
+    else:
+        q = np.clip(np.rint(ratio), -qmax, qmax)
+        q[sf == 0] = 0
+        c = (q.astype(np.int32) + (1 << (bits - 1))).astype(np.uint8).reshape(rows, cols)
     if bits == 4:
         codes = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
     else:
@@ -204,8 +216,8 @@ def expert_packed(shape: MoeShape, seed: int, layer: int, expert: int):
     w13 = np.empty((2 * shape.inter, shape.hidden), dtype=np.float32)
     w13[0::2] = g
     w13[1::2] = u
-    gc, gs = quantize_blocks(w13, shape.bits, shape.block)
-    dc, ds = quantize_blocks(d, shape.bits, shape.block)
+    gc, gs = quantize_blocks(w13, shape.bits, shape.block, shape.half)
+    dc, ds = quantize_blocks(d, shape.bits, shape.block, shape.half)
     return gc, gs, dc, ds
 
 

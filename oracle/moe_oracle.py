@@ -91,15 +91,19 @@ def unpack_codes(codes: np.ndarray, bits: int, n: int) -> np.ndarray:
 
 
 def dequantize(codes: np.ndarray, scales_bits: np.ndarray, rows: int, cols: int,
-               bits: int, block: int) -> np.ndarray:
-    """Weights w[r, c] = (code - 2**(bits-1)) * scale[r, c // block] in float64
-    (exact: an integer of at most 2 bits times an fp16 value)."""
+               bits: int, block: int, half: bool = False) -> np.ndarray:
+    """Weights w[r, c] = q * scale[r, c // block] in float64, q = code -
+    2**(bits-1) (integer levels), or q = code - (2**bits - 1) / 2 for the
+    half-integer levels (2**bits levels symmetric about zero, e.g. +-1/2,
+    +-3/2 for 2 bits).  Exact: a small integer or half-integer times an fp16
+    value."""
     codes = np.asarray(codes, dtype=np.uint8).reshape(rows, cols * bits // 8)
     scales = np.asarray(scales_bits, dtype=np.uint16).view(np.float16)
     scales = scales.reshape(rows, cols // block).astype(np.float64)
+    offset = ((1 << bits) - 1) / 2.0 if half else float(1 << (bits - 1))
     w = np.empty((rows, cols), dtype=np.float64)
     for r in range(rows):
-        q = unpack_codes(codes[r], bits, cols) - (1 << (bits - 1))
+        q = unpack_codes(codes[r], bits, cols) - offset
         w[r] = q * np.repeat(scales[r], block)
     return w
 
@@ -207,6 +211,7 @@ class OracleLayer:
     shared: Callable[[], Optional[tuple]]
     cache_size: int = 48
     shared_gate_w_bits: Optional[np.ndarray] = None   # [H] bf16 bits, or None (shared weight 1)
+    half_levels: bool = False                         # codes are the half-integer levels
 
     def __post_init__(self):
         self._cache: dict = {}
@@ -216,8 +221,8 @@ class OracleLayer:
             return self._cache[key]
         gc, gs, dc, ds = packed()
         H, I = self.hidden, self.inter
-        w13 = dequantize(gc, gs, 2 * I, H, self.bits, self.block)
-        wd = dequantize(dc, ds, H, I, self.bits, self.block)
+        w13 = dequantize(gc, gs, 2 * I, H, self.bits, self.block, self.half_levels)
+        wd = dequantize(dc, ds, H, I, self.bits, self.block, self.half_levels)
         dense = (w13[0::2], w13[1::2], wd)
         if len(self._cache) >= self.cache_size:
             self._cache.pop(next(iter(self._cache)))

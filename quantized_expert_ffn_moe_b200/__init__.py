@@ -45,7 +45,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int32), ("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("shared_inter", ctypes.c_int32), ("bits", ctypes.c_int32),
-                ("block", ctypes.c_int32)]
+                ("block", ctypes.c_int32), ("half_levels", ctypes.c_int32)]
 
 
 class _Weights(ctypes.Structure):
@@ -152,8 +152,8 @@ def _check(st: int, what: str):
         raise MoeError(st, what)
 
 
-def config_of(experts, hidden, inter, top_k, shared, bits, block) -> MoeConfig:
-    return MoeConfig(experts, hidden, inter, top_k, inter if shared else 0, bits, block)
+def config_of(experts, hidden, inter, top_k, shared, bits, block, half_levels=False) -> MoeConfig:
+    return MoeConfig(experts, hidden, inter, top_k, inter if shared else 0, bits, block, 1 if half_levels else 0)
 
 
 def moe_status_str(status: int) -> str:

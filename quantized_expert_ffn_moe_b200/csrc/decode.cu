@@ -36,6 +36,7 @@ struct FfnArgs {
   size_t expert_scale_count;
   int rows;                      // rows per expert (2I gate/up, H down)
   int block;                     // elements per scale
+  uint32_t xk;                   // code_xor of the format
   int out_cols;                  // columns of the output buffer (I gate/up, H down)
   int ntc;                       // tokens staged per chunk
   const uint16_t* xin;           // GATEUP: [T][K] bf16 activations
@@ -169,8 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
         const int spr = scales_per_row(Gm::K, a.block);
         const uint32_t sbytes = uint32_t(Gm::RPS) * spr * 2;
         mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes);
-        bulk_g2s(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot]);
-        bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot]);
+        const uint64_t pol = l2_evict_first_policy();      // weight bytes are read once
+        bulk_g2s_hint(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot], pol);
+        bulk_g2s_hint(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot], pol);
         ++issued;
       }
       // never leave with copies in flight
@@ -265,7 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
     }
     if (ok) {
       const unsigned char* st = ring + slot * Gm::STAGE_BYTES;
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0};
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0,
+                      a.xk};
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += NTB) {
         const int nt = min(NTB, nc - tb);          // warp-uniform
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
 // 64 q); test hook, not on the timed path.
 template <int BITS>
 __global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
-                                    int row0, int rows, int cols, int BLOCK, float* __restrict__ out) {
+                                    int row0, int rows, int cols, int BLOCK, uint32_t xk, float* __restrict__ out) {
   constexpr int G = BITS == 4 ? 8 : 16;
   const int words_per_row = cols / G;
   const long long total = (long long)rows * words_per_row;
@@ -296,9 +299,9 @@ __global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uin
     const uint32_t v = *reinterpret_cast<const uint32_t*>(codes + row * (cols * BITS / 8) + size_t(wi) * 4);
     uint32_t f[4];
     if (BITS == 4) {
-      q4_bytes(v, f[0], f[1]);
+      q4_bytes(v, xk, f[0], f[1]);
     } else {
-      q2_bytes<false>(v, f);
+      q2_bytes(v, xk, f);
     }
     for (int j = 0; j < G; ++j) {
       const int col = wi * G + j;
@@ -399,7 +402,7 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   g.sh_codes = a.w.shared_gate_up_codes; g.sh_scales = a.w.shared_gate_up_scales;
   g.expert_code_bytes = size_t(2 * I) * H * bits / 8;
   g.expert_scale_count = size_t(2 * I) * (H / c.block);
-  g.rows = 2 * I; g.out_cols = I; g.ntc = pg.ntc; g.block = c.block;
+  g.rows = 2 * I; g.out_cols = I; g.ntc = pg.ntc; g.block = c.block; g.xk = code_xor(bits, c.half_levels);
   g.xin = a.x; g.hin = nullptr;
   g.out = reinterpret_cast<float*>(a.ws + a.L.h);
   g.status = reinterpret_cast<int*>(a.ws + a.L.status);
@@ -415,7 +418,7 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   d.sh_codes = a.w.shared_down_codes; d.sh_scales = a.w.shared_down_scales;
   d.expert_code_bytes = size_t(H) * I * bits / 8;
   d.expert_scale_count = size_t(H) * (I / c.block);
-  d.rows = H; d.out_cols = H; d.ntc = pd.ntc; d.block = c.block;
+  d.rows = H; d.out_cols = H; d.ntc = pd.ntc; d.block = c.block; d.xk = code_xor(bits, c.half_levels);
   d.xin = nullptr; d.hin = reinterpret_cast<const float*>(a.ws + a.L.h);
   d.out = reinterpret_cast<float*>(a.ws + a.L.y);
   d.status = reinterpret_cast<int*>(a.ws + a.L.status);
@@ -424,14 +427,15 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   return bits == 4 ? dispatch<DOWN, 4>(I, d, a.num_sms, a.stream) : dispatch<DOWN, 2>(I, d, a.num_sms, a.stream);
 }
 
-cudaError_t launch_dequant_rows(int bits, int block, const uint8_t* codes, const uint16_t* scales, int row0, int rows,
-                                int cols, float* out, cudaStream_t s) {
+cudaError_t launch_dequant_rows(int bits, int block, int half_levels, const uint8_t* codes, const uint16_t* scales,
+                                int row0, int rows, int cols, float* out, cudaStream_t s) {
   const int G = bits == 4 ? 8 : 16;
   const long long total = (long long)rows * (cols / G);
   const long long want = (total + 255) / 256;
   const int blocks = int(want < 4096 ? want : 4096);
-  if (bits == 4) dequant_rows_kernel<4><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, out);
-  else dequant_rows_kernel<2><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, out);
+  const uint32_t xk = code_xor(bits, half_levels);
+  if (bits == 4) dequant_rows_kernel<4><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, xk, out);
+  else dequant_rows_kernel<2><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, xk, out);
   return cudaGetLastError();
 }
 

@@ -34,27 +34,29 @@ struct Geom {
 // Integer operands of the GEMV.  A code field shifted to the top of its byte
 // and XOR-ed with 0x80 is, read as a signed byte, the code minus its offset
 // times the field weight: for 4-bit codes c, ((c << 4) ^ 0x80) = 16 (c - 8);
-// for 2-bit codes, ((c << 6) ^ 0x80) = 64 (c - 2) and ((c << 6) ^ 0xA0) =
-// 64 (c - 1.5) (the four-level reading).  dp2a multiplies two signed 16-bit
+// for 2-bit codes, ((c << 6) ^ 0x80) = 64 (c - 2).  The half-integer levels
+// only change the constant: ((c << 4) ^ 0x88) = 16 (c - 7.5) and
+// ((c << 6) ^ 0xA0) = 64 (c - 1.5).  dp2a multiplies two signed 16-bit
 // activations with two of those bytes and adds them to a 32-bit sum, so a
 // block's dot product is exact in int32 and is scaled once per block in fp32.
 //
+// The XOR constant of a format, one byte repeated.
+__host__ __device__ inline uint32_t code_xor(int bits, int half_levels) {
+  return half_levels ? (bits == 4 ? 0x88888888u : 0xA0A0A0A0u) : 0x80808080u;
+}
 // 4-bit word v = codes c0..c7 (c_j at bits 4j): returns the bytes
 //   lo = (16 q0, 16 q2, 16 q4, 16 q6), hi = (16 q1, 16 q3, 16 q5, 16 q7)
-__device__ __forceinline__ void q4_bytes(uint32_t v, uint32_t& lo, uint32_t& hi) {
-  lo = lop_and_xor(v << 4, 0xF0F0F0F0u, 0x80808080u);
-  hi = lop_and_xor(v, 0xF0F0F0F0u, 0x80808080u);
+__device__ __forceinline__ void q4_bytes(uint32_t v, uint32_t xk, uint32_t& lo, uint32_t& hi) {
+  lo = lop_and_xor(v << 4, 0xF0F0F0F0u, xk);
+  hi = lop_and_xor(v, 0xF0F0F0F0u, xk);
 }
 // 2-bit word v = codes c0..c15 (c_j at bits 2j): f[r] holds the bytes
-// 64 q of elements r, r+4, r+8, r+12.  LV4: the four-level reading
-// q = c - 1.5 instead of q = c - 2.
-template <bool LV4>
-__device__ __forceinline__ void q2_bytes(uint32_t v, uint32_t (&f)[4]) {
-  constexpr uint32_t X = LV4 ? 0xA0A0A0A0u : 0x80808080u;
-  f[3] = lop_and_xor(v, 0xC0C0C0C0u, X);
-  f[2] = lop_and_xor(v << 2, 0xC0C0C0C0u, X);
-  f[1] = lop_and_xor(v << 4, 0xC0C0C0C0u, X);
-  f[0] = lop_and_xor(v << 6, 0xC0C0C0C0u, X);
+// 64 q of elements r, r+4, r+8, r+12.
+__device__ __forceinline__ void q2_bytes(uint32_t v, uint32_t xk, uint32_t (&f)[4]) {
+  f[3] = lop_and_xor(v, 0xC0C0C0C0u, xk);
+  f[2] = lop_and_xor(v << 2, 0xC0C0C0C0u, xk);
+  f[1] = lop_and_xor(v << 4, 0xC0C0C0C0u, xk);
+  f[0] = lop_and_xor(v << 6, 0xC0C0C0C0u, xk);
 }
 // Signed-byte weight of the code fields above: the dot products come out
 // multiplied by 2^kCodeLog2.
@@ -121,6 +123,7 @@ struct Rows {
   const unsigned char* codes;     // row rl0; row rl0+1 follows at +RB
   const unsigned char* scales;    // row rl0; row rl0+1 follows at +(SPR >> PS)*2
   int r0;
+  uint32_t xk;                    // code_xor of the format
 };
 
 // Scales per row, and the piece-to-scale shift PS of a 4-bit block of 32
@@ -136,7 +139,7 @@ __host__ __device__ inline int piece_shift(int bits, int block) { return bits ==
 // token); each block's exact integer sum is converted to fp32 and multiplied
 // by the block's fp16 scale.  `nt` <= NT tokens are valid; xs holds int16
 // activations staged with staged_offset.
-template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0, bool LV4 = false>
+template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0>
 __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& rw, const int16_t* xs, int tb, int lr,
                                          const float* tok_inv, const float* tok_w, const int* tok_pos,
                                          int nt = NT, const int* xrow = nullptr) {
@@ -176,8 +179,8 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         uint32_t lo[2], hi[2];
-        q4_bytes(wd[0][m], lo[0], hi[0]);
-        q4_bytes(wd[1][m], lo[1], hi[1]);
+        q4_bytes(wd[0][m], rw.xk, lo[0], hi[0]);
+        q4_bytes(wd[1][m], rw.xk, lo[1], hi[1]);
         const int xoff = ((s * 4 + m) * LPR + lr) * 8;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -202,8 +205,8 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         uint32_t f[2][4];
-        q2_bytes<LV4>(wd[0][m], f[0]);
-        q2_bytes<LV4>(wd[1][m], f[1]);
+        q2_bytes(wd[0][m], rw.xk, f[0]);
+        q2_bytes(wd[1][m], rw.xk, f[1]);
         const int xoff = ((s * 4 + m) * 2 * LPR + lr) * 8;
         float sc[2];
 #pragma unroll

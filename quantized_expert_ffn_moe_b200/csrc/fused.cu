@@ -48,7 +48,7 @@ constexpr int kFRingOff = 3584;                   // shared-memory offset of the
 constexpr int kFMaxTokens = 64;
 constexpr int kFMaxPairs = kFMaxTokens * 16;
 constexpr int kMaxFusedLayers = 64;
-constexpr int kTimePoints = 20;
+constexpr int kTimePoints = 32;
 
 struct FusedParams {
   moe_config cfg;
@@ -57,7 +57,7 @@ struct FusedParams {
   const uint16_t* x;             // layer mode input
   uint16_t* y;                   // layer mode output, or the residual stream (stack)
   int* trace;                    // stack: [L][T][k] selections, or null
-  unsigned long long* timing;    // null, or [gridDim][20] %globaltimer stamps of layer 0
+  unsigned long long* timing;    // null, or [gridDim][32] timestamps of layer 0 (moe_debug_fused_timing)
   char* ws;
   Layout L_;
   int ntc_gu, ntc_dn;             // tokens per chunk (gate/up: T when every token is pre-staged)
@@ -285,7 +285,7 @@ template <int BITS, int LPR, int CPL>
 __device__ void stage_token_all(const uint16_t* row, bool stack, int16_t* dst, float* rnorm_out, float* inv_out,
                                 uint16_t* xb_out, const uint16_t* rrows, int ne, const float* rbias,
                                 float* logit_row, uint64_t* rbar, uint32_t rpar, volatile int* abort_flag,
-                                int* status, int lane) {
+                                int* status, int lane, unsigned long long* tstamp = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K, G = Gm::G, NG = K / (32 * G);       // groups per lane
   constexpr int NW = G / 8;                                     // 16-byte words per group
@@ -344,6 +344,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, int16_t* dst, f
   float vmax = fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  if (tstamp && lane == 0) tstamp[19] = static_cast<unsigned long long>(clock64());   // the row has arrived
   const int sh = act_shift(vmax);
   const float mul = ldexpf(1.f, sh);
 #pragma unroll
@@ -374,6 +375,7 @@ __device__ void stage_token_all(const uint16_t* row, bool stack, int16_t* dst, f
     *rnorm_out = r;
     *inv_out = act_inv<BITS>(sh);
   }
+  if (tstamp && lane == 0) tstamp[20] = static_cast<unsigned long long>(clock64());   // staged
   if (ne <= 0) return;
   if (rbar != nullptr) {
     if (*abort_flag) return;
@@ -484,7 +486,7 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
                              const uint16_t* xsrc, const float* rnorm, const float* hin, float* out, int out_cols,
                              const int16_t* xs_pre, const float* pre_inv, const float* pre_w, int pre_base,
                              int16_t* xs_grp, const GroupTok& tk, volatile int* abort_flag, int* status,
-                             unsigned long long* tacc = nullptr) {
+                             unsigned long long* tacc = nullptr, unsigned long long* tabs = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -498,6 +500,7 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
   // pre_inv / pre_w of that row
   const bool pre = xs_pre != nullptr;
   int staged_slot = -1, staged_chunk = -1;
+  bool first_data = true;
   for (; cur.valid(w1); cur.advance()) {
     const int i = (*consumed)++;
     if (i % kFGroups != grp) continue;
@@ -532,10 +535,18 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
       *abort_flag = 1;
       report_error(status, MOE_ERR_TIMEOUT, 41);
     }
-    if (timed) { tacc[0] += global_ns() - tw; tacc[2] += 1; }
+    if (timed) {
+      const unsigned long long now = global_ns();
+      tacc[0] += now - tw;
+      const unsigned long long cyc = static_cast<unsigned long long>(clock64());
+      tacc[2] += 1;
+      if (tabs && first_data) tabs[0] = cyc;            // first stage's data in
+      first_data = false;
+    }
     if (ok) {
       const unsigned char* st = ring + slot * ring_stride;
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0};
+      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0,
+                      code_xor(BITS, p.cfg.half_levels)};
       const int nc = cur.nc;
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
@@ -549,6 +560,7 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
+    if (timed && tabs) tabs[1] = static_cast<unsigned long long>(clock64());   // last stage done
   }
 }
 
@@ -602,8 +614,9 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
                              const uint8_t* sh_codes, const uint16_t* sh_scales, size_t expert_code_bytes,
                              size_t expert_scale_count, unsigned char* ring, int ring_stride, uint64_t* full,
                              uint64_t* empty, int* issued, volatile int* abort_flag, int* status, Publisher& pub,
-                             bool gate_up, int block) {
+                             bool gate_up, int block, unsigned long long* tabs = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
+  const int first_issue = *issued;
   for (; cur.valid(w1); cur.advance()) {
     const int i = *issued;
     const int slot = i % kFStages;
@@ -624,11 +637,17 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
     const int spr = scales_per_row(Gm::K, block);
     const uint32_t sbytes = uint32_t(Gm::RPS) * spr * 2;
     mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes);
-    bulk_g2s(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot]);
-    bulk_g2s(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot]);
+    const uint64_t pol = l2_evict_first_policy();
+    bulk_g2s_hint(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot], pol);
+    bulk_g2s_hint(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot], pol);
     pub.rslot[slot] = gate_up ? cur.slot : -1;
     if (gate_up) ++pub.pending;
     *issued = i + 1;
+    if (tabs) {                                  // first and last issue of the pass
+      const unsigned long long now = static_cast<unsigned long long>(clock64());
+      if (i == first_issue) tabs[0] = now;
+      tabs[1] = now;
+    }
   }
 }
 
@@ -663,8 +682,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   float* rnorm = reinterpret_cast<float*>(smem + 128);                   // [64]
   float* inv_all = reinterpret_cast<float*>(smem + 384);                 // [64]
   int* snslots = reinterpret_cast<int*>(smem + 640);
-  int* s_handover = snslots + 1;                                         // 1: tensor-core kernels take the layer
   int* scan_scratch = reinterpret_cast<int*>(smem + 768);                // [2 * kFCons]
+  int* s_handover = snslots + 1;                                         // 1: tensor-core kernels take the layer
   // [1024, 3072): per-group token metadata, 4 arrays of kMaxNTC each
   float* dinv = reinterpret_cast<float*>(smem + 3072);                   // [64] down rows staged at once
   float* dwt = dinv + kMaxNTC;                                           // [64]
@@ -717,8 +736,15 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
     if (threadIdx.x == 0 && !*abort_flag && !grid_barrier(gword, G, status)) *abort_flag = 1;
     all_sync();
   };
+  // SM clock cycles (fine-grained within the CTA); the layer start and the
+  // end of the combine also in %globaltimer ns at [22] / [23], comparable
+  // across CTAs
   auto stamp = [&](int l, int i) {
-    if (p.timing && l == 0 && threadIdx.x == 0) p.timing[blockIdx.x * kTimePoints + i] = global_ns();
+    if (p.timing && l == 0 && threadIdx.x == 0) {
+      p.timing[blockIdx.x * kTimePoints + i] = static_cast<unsigned long long>(clock64());
+      if (i == 8) p.timing[blockIdx.x * kTimePoints + 22] = global_ns();
+      if (i == 7) p.timing[blockIdx.x * kTimePoints + 23] = global_ns();
+    }
   };
 
   for (int l = 0; l < p.L; ++l) {
@@ -755,6 +781,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         const int z0 = int((long long)(E + 2) * blockIdx.x / G), z1 = int((long long)(E + 2) * (blockIdx.x + 1) / G);
         for (int u = z0 + threadIdx.x; u < z1; u += kFCons * 32) gdone[u] = 0;
       }
+      stamp(l, 21);
       // one warp per token: staging and, from the same registers, the
       // token's router logits for this CTA's experts; with fewer tokens than
       // warps, the warps keep xhat (bf16) in the idle ring slots 1-2 instead
@@ -768,7 +795,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
                                       &rnorm[t], &inv_all[t], few ? xb + size_t(t) * H : nullptr,
                                       reinterpret_cast<const uint16_t*>(ring), few ? 0 : ne,
                                       lw.router_bias ? lw.router_bias + e0 : nullptr, logits + size_t(t) * E + e0,
-                                      have_rows ? nullptr : rbar, l & 1, abort_flag, status, lane);
+                                      have_rows ? nullptr : rbar, l & 1, abort_flag, status, lane,
+                                      (p.timing && l == 0 && t == 0) ? p.timing + blockIdx.x * kTimePoints : nullptr);
         have_rows = !few;
         if (t == 0) stamp(l, 14);
         __syncwarp();
@@ -984,14 +1012,16 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
           produce_pass<BITS, LG, CG>(cg, g1, lw.gate_up_codes, lw.gate_up_scales, lw.shared_gate_up_codes,
                                       lw.shared_gate_up_scales, size_t(2 * I) * H * c.bits / 8,
                                       size_t(2 * I) * (H / c.block), ring, RING_STRIDE, full, empty, &issued,
-                                      abort_flag, status, pub, true, c.block);
+                                      abort_flag, status, pub, true, c.block,
+                                      p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 28 : nullptr);
         }
         pub.issued_all();
         if (d0 < d1) {
           cd.init(d0);
           produce_pass<BITS, LD, CD>(cd, d1, lw.down_codes, lw.down_scales, lw.shared_down_codes,
                                       lw.shared_down_scales, size_t(H) * I * c.bits / 8, size_t(H) * (I / c.block),
-                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false, c.block);
+                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false, c.block,
+                                      p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 30 : nullptr);
         }
         drain_publish(issued, empty, abort_flag, status, pub);
       }
@@ -1002,7 +1032,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         consume_pass<GATEUP, BITS, LG, CG, PS>(p, rt, cg, g1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
                                            rnorm, nullptr, hbuf, I, p.pre ? xs : nullptr, inv_all, nullptr, 0, xs_grp,
                                            tk, abort_flag, status,
-                                           p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 11 : nullptr);
+                                           p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 11 : nullptr,
+                                           p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 24 : nullptr);
       }
       all_sync();
       stamp(l, 3);
@@ -1047,7 +1078,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         consume_pass<DOWN, BITS, LD, CD, PS>(p, rt, cd, d1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
                                          rnorm, hbuf, ybuf, H, dpre ? xs : nullptr, dinv, dwt, lo, xs_grp, tk,
                                          abort_flag, status,
-                                         p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 16 : nullptr);
+                                         p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 16 : nullptr,
+                                         p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 26 : nullptr);
       }
       all_sync();
       stamp(l, 5);

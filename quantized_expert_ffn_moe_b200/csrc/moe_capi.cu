@@ -41,6 +41,7 @@ int validate_config(const moe_config* c) {
   if (c->top_k > 16 || c->top_k > c->num_experts) return MOE_ERR_UNSUPPORTED;
   if (!((c->bits == 4 && (c->block == 32 || c->block == 128)) || (c->bits == 2 && c->block == 16)))
     return MOE_ERR_UNSUPPORTED;
+  if (c->half_levels != 0 && c->half_levels != 1) return MOE_ERR_UNSUPPORTED;
   const int H = c->hidden;
   if (!(H == 256 || H == 512 || H == 1024 || H == 2048 || H == 4096)) return MOE_ERR_UNSUPPORTED;
   if (c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
@@ -300,11 +301,12 @@ int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t
   if (!cfg || !codes || !scales || !out || row0 < 0 || rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
   if (!((cfg->bits == 4 && (cfg->block == 32 || cfg->block == 128)) || (cfg->bits == 2 && cfg->block == 16)))
     return MOE_ERR_UNSUPPORTED;
+  if (cfg->half_levels != 0 && cfg->half_levels != 1) return MOE_ERR_UNSUPPORTED;
   if (cols % cfg->block != 0 || (cols * cfg->bits / 8) % 4 != 0) return MOE_ERR_UNSUPPORTED;
   if (!aligned(codes, 4) || !aligned(scales, 2) || !aligned(out, 4)) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
-  return cuda_status(launch_dequant_rows(cfg->bits, cfg->block, codes, scales, row0, rows, cols, out,
-                                         static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_dequant_rows(cfg->bits, cfg->block, cfg->half_levels, codes, scales, row0, rows, cols,
+                                         out, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_profile_begin(int32_t max_calls) {

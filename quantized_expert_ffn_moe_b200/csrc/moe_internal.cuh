@@ -211,6 +211,22 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// L2 policy for bytes read exactly once (the expert weights of a decode
+// step): evicted first, so the stream does not push the kernel's code, the
+// tokens and the routing scratch out of L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// bulk_g2s with an L2 cache policy.
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
@@ -390,6 +406,19 @@ __device__ __forceinline__ void decode_q4x8(uint32_t v, __half2 out[4]) {
   out[3] = __hfma2(u32_as_h2(hi1), mul_hi, add_hi);
 }
 
+// Half-integer levels, q = c - 7.5: every field is first placed four bits up
+// (0x6400 | (c << 4) = 1024 + 16 c), so one fused multiply-add by 1/16 and
+// -71.5 leaves q; same pair order as decode_q4x8.
+__device__ __forceinline__ void decode_q4x8_half(uint32_t v, __half2 out[4]) {
+  const uint32_t MAGIC = 0x64006400u;
+  const __half2 mul = u32_as_h2(0x2C002C00u);             // 1/16
+  const __half2 add = u32_as_h2(0xD478D478u);             // -71.5 = -(64 + 7.5)
+  out[0] = __hfma2(u32_as_h2(lop_and_or(v << 4, 0x00F000F0u, MAGIC)), mul, add);
+  out[1] = __hfma2(u32_as_h2(lop_and_or(v, 0x00F000F0u, MAGIC)), mul, add);
+  out[2] = __hfma2(u32_as_h2(lop_and_or(v >> 4, 0x00F000F0u, MAGIC)), mul, add);
+  out[3] = __hfma2(u32_as_h2(lop_and_or(v >> 8, 0x00F000F0u, MAGIC)), mul, add);
+}
+
 // 2-bit, one 32-bit word = 16 elements e0..e15 (e_j at bits 2j):
 //   out[j] = (q_j, q_{j+8}) for j = 0..7
 __device__ __forceinline__ void decode_q2x16(uint32_t v, __half2 out[8]) {
@@ -402,6 +431,23 @@ __device__ __forceinline__ void decode_q2x16(uint32_t v, __half2 out[8]) {
   for (int half = 0; half < 2; ++half) {
     const uint32_t w = half ? (v >> 8) : v;
     out[4 * half + 0] = __hsub2(u32_as_h2(lop_and_or(w, 0x00030003u, MAGIC)), sub1);
+    out[4 * half + 1] = __hfma2(u32_as_h2(lop_and_or(w, 0x000C000Cu, MAGIC)), m4, a4);
+    out[4 * half + 2] = __hfma2(u32_as_h2(lop_and_or(w, 0x00300030u, MAGIC)), m16, a16);
+    out[4 * half + 3] = __hfma2(u32_as_h2(lop_and_or(w, 0x00C000C0u, MAGIC)), m64, a64);
+  }
+}
+// Half-integer levels, q = c - 1.5 (four levels +-0.5, +-1.5): the lowest
+// field is moved up two bits first so that every offset 1024 / 2^n + 1.5 is
+// exact in fp16; same pair order as decode_q2x16.
+__device__ __forceinline__ void decode_q2x16_half(uint32_t v, __half2 out[8]) {
+  const uint32_t MAGIC = 0x64006400u;
+  const __half2 m4 = u32_as_h2(0x34003400u), a4 = u32_as_h2(0xDC06DC06u);    // 1/4,  -257.5
+  const __half2 m16 = u32_as_h2(0x2C002C00u), a16 = u32_as_h2(0xD418D418u);  // 1/16, -65.5
+  const __half2 m64 = u32_as_h2(0x24002400u), a64 = u32_as_h2(0xCC60CC60u);  // 1/64, -17.5
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const uint32_t w = half ? (v >> 8) : v;
+    out[4 * half + 0] = __hfma2(u32_as_h2(lop_and_or(w << 2, 0x000C000Cu, MAGIC)), m4, a4);
     out[4 * half + 1] = __hfma2(u32_as_h2(lop_and_or(w, 0x000C000Cu, MAGIC)), m4, a4);
     out[4 * half + 2] = __hfma2(u32_as_h2(lop_and_or(w, 0x00300030u, MAGIC)), m16, a16);
     out[4 * half + 3] = __hfma2(u32_as_h2(lop_and_or(w, 0x00C000C0u, MAGIC)), m64, a64);
@@ -489,7 +535,7 @@ int decode_path_mode();
 bool router_gemm_supported(const moe_config& c, int T);
 cudaError_t launch_router_gemm(const moe_config& c, const uint16_t* router_w, const float* bias, const uint16_t* x,
                                int T, float* logits, int* status, int num_sms, cudaStream_t s);
-cudaError_t launch_dequant_rows(int bits, int block, const uint8_t* codes, const uint16_t* scales,
+cudaError_t launch_dequant_rows(int bits, int block, int half_levels, const uint8_t* codes, const uint16_t* scales,
                                 int row0, int rows, int cols, float* out, cudaStream_t s);
 bool decode_shape_supported(int bits, int H, int I);
 

@@ -86,11 +86,22 @@ struct PrefillArgs {
   int* status;
   unsigned long long* timing;   // null, or [gridDim][16] per-role wait times (ns) of this launch
   int gated;                    // 1: no tiles unless the fused decode kernel handed the layer over
+  int half_levels;              // 1: codes are the half-integer levels q = c - (2^bits - 1)/2
 };
 
 constexpr int kPTime = 16;
 
 // ------------------------------------------------------------ primitives
+// The same with an L2 cache policy (the packed weights: read once per tile).
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar)),
+        "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
@@ -168,16 +179,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t v[32]) {
 
 // Packed word -> fp16 pairs q * s (q exact from the magic-number decode, one
 // rounding in the multiply).  Pair order as in the decode path: 4-bit
-// (q_j, q_{j+4}), 2-bit (q_j, q_{j+8}).
-__device__ __forceinline__ void dq4_f16(uint32_t v, __half2 s, uint32_t out[4]) {
+// (q_j, q_{j+4}), 2-bit (q_j, q_{j+8}).  half: the half-integer levels.
+__device__ __forceinline__ void dq4_f16(uint32_t v, __half2 s, bool half, uint32_t out[4]) {
   __half2 q[4];
-  decode_q4x8(v, q);
+  if (half) decode_q4x8_half(v, q);
+  else decode_q4x8(v, q);
 #pragma unroll
   for (int j = 0; j < 4; ++j) out[j] = h2_as_u32(__hmul2(q[j], s));
 }
-__device__ __forceinline__ void dq2_f16(uint32_t v, __half2 s, uint32_t out[8]) {
+__device__ __forceinline__ void dq2_f16(uint32_t v, __half2 s, bool half, uint32_t out[8]) {
   __half2 q[8];
-  decode_q2x16(v, q);
+  if (half) decode_q2x16_half(v, q);
+  else decode_q2x16(v, q);
 #pragma unroll
   for (int j = 0; j < 8; ++j) out[j] = h2_as_u32(__hmul2(q[j], s));
 }
@@ -328,8 +341,15 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
         }
         unsigned char* dst = sRaw + s * RAW_STRIDE;
         mbar_arrive_expect_tx(&full_raw[s], Gm::CODE_BYTES + Gm::SCALE_BYTES);
-        tma_load_2d(dst, mc, r * Gm::IB, row, &full_raw[s]);
-        tma_load_2d(dst + Gm::SCALE_OFF, ms, r * (RAWK / Gm::BLOCK), row, &full_raw[s]);
+        if (ti.n <= kPrefillTileN) {
+          // one token tile: these weight bytes are read once in the pass
+          const uint64_t pol = l2_evict_first_policy();
+          tma_load_2d_hint(dst, mc, r * Gm::IB, row, &full_raw[s], pol);
+          tma_load_2d_hint(dst + Gm::SCALE_OFF, ms, r * (RAWK / Gm::BLOCK), row, &full_raw[s], pol);
+        } else {
+          tma_load_2d(dst, mc, r * Gm::IB, row, &full_raw[s]);
+          tma_load_2d(dst + Gm::SCALE_OFF, ms, r * (RAWK / Gm::BLOCK), row, &full_raw[s]);
+        }
       }
     }
     for (int i = max(0, rc - PNR); i < rc; ++i)
@@ -400,6 +420,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     // warp w writes rows of its tensor-memory lane quarter (w % 4); the two
     // warps of a quarter take the first and second half of a packed stage
     const int r = (warp & 3) * 32 + lane;          // tile row
+    const bool hl = a.half_levels != 0;
     const int half = (warp - kWarpDq0) >> 2;       // which of the two A stages of a packed stage
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     static_assert(RAWK == 2 * PSK, "a packed stage feeds two A stages, one per dequant half");
@@ -432,7 +453,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
                 const __half2 s2 = __half2half2(hs);
                 const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) dq4_f16(wd[q], s2, o32 + (cc * 4 + q) * 4);
+                for (int q = 0; q < 4; ++q) dq4_f16(wd[q], s2, hl, o32 + (cc * 4 + q) * 4);
               }
             } else {
               // 16 bytes of codes = 64 weights in 4 words, 4 scales
@@ -449,7 +470,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
                 const uint32_t pr = svw[si >> 1];
                 const __half hs = __ushort_as_half((unsigned short)((si & 1) ? (pr >> 16) : (pr & 0xFFFFu)));
                 const __half2 s2 = __half2half2(hs);
-                dq2_f16(wd[q], s2, o32 + q * 8);
+                dq2_f16(wd[q], s2, hl, o32 + q * 8);
               }
             }
             tmem_st32(tmem_base + lane_base + kAColBase + uint32_t(as) * kAStageCols + uint32_t(hb * 32), o32);
@@ -878,6 +899,7 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   g.status = reinterpret_cast<int*>(a.ws + a.L.status);
   g.timing = g_prefill_timing;
   g.gated = a.gated;
+  g.half_levels = c.half_levels;
   const bool sh = c.shared_inter > 0;
   err = bits == 4 ? launch_gemm<0, 4>(g, a.w.gate_up_codes, a.w.gate_up_scales, a.w.shared_gate_up_codes,
                                       a.w.shared_gate_up_scales, c.num_experts, sh, xs, P, a.num_sms, a.stream)

@@ -27,7 +27,7 @@ def torch():
 
 def cfg_of(shape: mi.MoeShape) -> q.MoeConfig:
     return q.config_of(shape.experts, shape.hidden, shape.inter, shape.top_k, shape.shared, shape.bits,
-                       shape.block)
+                       shape.block, shape.half)
 
 
 def device_layer(shape: mi.MoeShape, seed: int, layer: int, zipf: bool = False,
@@ -92,7 +92,8 @@ def host_oracle_layer(shape, seed, layer, zipf=False, cache_size=16, shared_gate
         expert=lambda e: mi.expert_packed(shape, seed, layer, e),
         shared=(lambda: mi.shared_packed(shape, seed, layer)) if shape.shared else (lambda: None),
         cache_size=cache_size,
-        shared_gate_w_bits=mi.shared_gate_weight_bf16(shape, seed, layer) if shared_gate else None)
+        shared_gate_w_bits=mi.shared_gate_weight_bf16(shape, seed, layer) if shared_gate else None,
+        half_levels=shape.half)
 
 
 def check_selection(oracle_logits, oracle_idx, gpu_idx, k, band=TIE_BAND):

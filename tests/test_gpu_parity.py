@@ -20,6 +20,10 @@ SHAPE_2BIT_TINY = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared
 # 4-bit with one scale per 128 elements (the GPTQ-style group size)
 TINY_G128 = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=4, block=128)
 FULL4_G128 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=128)
+# half-integer levels (2-bit: the four levels +-1/2, +-3/2; 4-bit: sixteen)
+TINY2H = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=2, block=16, half=True)
+TINY4H = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=4, block=32, half=True)
+FULL2H = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=2, block=16, half=True)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -36,8 +40,8 @@ def _cuda():
 
 # ------------------------------------------------------------ input bytes ---
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, TINY_G128],
-                         ids=["tiny4", "tiny2", "full4", "full2", "tiny4g128"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, TINY_G128, TINY2H, TINY4H, FULL2H],
+                         ids=["tiny4", "tiny2", "full4", "full2", "tiny4g128", "tiny2h", "tiny4h", "full2h"])
 def test_device_generator_matches_host(shape):
     """The device generator writes the same bytes as the numpy generator."""
     w = gc.device_layer(shape, seed=3, layer=5)
@@ -55,8 +59,8 @@ def test_device_generator_matches_host(shape):
 
 # ----------------------------------------------------------- dequant hook ---
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, FULL4_G128],
-                         ids=["tiny4", "tiny2", "full4", "full2", "full4g128"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, FULL4_G128, TINY4H, FULL2H],
+                         ids=["tiny4", "tiny2", "full4", "full2", "full4g128", "tiny4h", "full2h"])
 def test_device_decoder_bit_exact(shape):
     torch = gc.torch()
     w = gc.device_layer(shape, seed=1, layer=0)
@@ -68,12 +72,12 @@ def test_device_decoder_bit_exact(shape):
     q.moe_dequant_rows(cfg, w.gate_up_codes[e], w.gate_up_scales[e], 0, 2 * I, H, out)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64),
-                                  orc.dequantize(gcodes, gsc, 2 * I, H, shape.bits, shape.block))
+                                  orc.dequantize(gcodes, gsc, 2 * I, H, shape.bits, shape.block, shape.half))
     out = torch.empty((H - 3, I), dtype=torch.float32, device="cuda")
     q.moe_dequant_rows(cfg, w.down_codes[e], w.down_scales[e], 3, H - 3, I, out)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64),
-                                  orc.dequantize(dcodes, dsc, H, I, shape.bits, shape.block)[3:])
+                                  orc.dequantize(dcodes, dsc, H, I, shape.bits, shape.block, shape.half)[3:])
 
 
 # ----------------------------------------------------------------- router ---
@@ -133,7 +137,8 @@ def _oracle_given(lay, x_bits, gpu_idx, differ):
     return orc.layer_forward(lay, x_bits, topk_override=over)
 
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, TINY_G128], ids=["tiny4", "tiny2", "tiny4g128"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, TINY_G128, TINY2H, TINY4H],
+                         ids=["tiny4", "tiny2", "tiny4g128", "tiny2h", "tiny4h"])
 @pytest.mark.parametrize("T", [1, 2, 7, 8, 17, 64, 100])
 def test_layer_tiny_live_oracle(shape, T):
     x = mi.hidden_states_bf16(T, shape.hidden, 0, 0)
@@ -227,9 +232,11 @@ def test_empty_batch_and_small_workspace():
 # (H and I multiples of 256): several expert groups per tile row, ragged tiles.
 MID4 = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=4, block=32)
 MID2 = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=2, block=16)
+MID2H = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=2, block=16, half=True)
+MID4H = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=4, block=32, half=True)
 
 
-@pytest.mark.parametrize("shape", [MID4, MID2], ids=["mid4", "mid2"])
+@pytest.mark.parametrize("shape", [MID4, MID2, MID2H, MID4H], ids=["mid4", "mid2", "mid2h", "mid4h"])
 @pytest.mark.parametrize("T", [65, 129, 300])
 def test_prefill_path_live_oracle(shape, T):
     x = mi.hidden_states_bf16(T, shape.hidden, 0, 21)
@@ -381,6 +388,17 @@ def test_layer_full4_g128_sampled(T):
     16 and 48 tokens, the stand-alone GEMV kernels at 100 (no tensor-core path
     for this group size)."""
     _sampled_full_case(FULL4_G128, T, 7, 0, 4, 128 + T)
+
+
+# --------------------------------------------------- half-integer levels ---
+
+@pytest.mark.parametrize("T,path", [(1, 0), (16, 0), (48, 1), (48, 2), (300, 0)],
+                         ids=["t1", "t16", "t48_cuda_cores", "t48_tensor_cores", "t300_prefill"])
+def test_layer_full2_half_levels_sampled(T, path):
+    """Full shape, 2-bit codes read as the four half-integer levels: the
+    single-launch decode kernel (1, 16 tokens; 48 tokens on each side of the
+    hand-over) and the tensor-core prefill (300 tokens)."""
+    _with_path(path, lambda: _sampled_full_case(FULL2H, T, 13, 0, min(3, T), 900 + T))
 
 
 # ----------------------------------------------------- gated shared expert ---
