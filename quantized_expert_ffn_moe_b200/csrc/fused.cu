@@ -1186,11 +1186,14 @@ unsigned long long* g_fused_timing = nullptr;
 
 // Hand-over time models, [0] 4-bit/32, [1] 2-bit/16: layer time in us as
 // f0 + f1 * (CUDA-core cost units per CTA) and t0 + t1 * (tensor-core
-// k-blocks per CTA), least-squares fits to 120 layer times measured on a B200
-// (32..64 tokens, near-uniform and Zipf-skewed routing; largest residual
-// 16 us); on those batches the comparison picked the faster path every time.
-constexpr float kHyF0[2] = {57.9f, 72.5f}, kHyF1[2] = {0.1655f, 0.1294f};
-constexpr float kHyT0[2] = {89.7f, 93.5f}, kHyT1[2] = {0.6231f, 0.5696f};
+// k-blocks per CTA), least-squares fits to layer times measured on a B200
+// with CUDA graphs (32, 40, 48, 56 and 64 tokens, near-uniform and
+// Zipf-skewed routing, 6 layer instances each, both paths: 60 batches per
+// format; largest residual 17 us).  On those batches the comparison picks the
+// faster path for 57 of 60 (4-bit) and 59 of 60 (2-bit), losing at most
+// 2.1 us when it does not.
+constexpr float kHyF0[2] = {42.80f, 49.80f}, kHyF1[2] = {0.1381f, 0.1513f};
+constexpr float kHyT0[2] = {79.03f, 77.72f}, kHyT1[2] = {0.6034f, 0.6007f};
 
 void set_fused_timing(unsigned long long* buf) { g_fused_timing = buf; }
 
@@ -1228,7 +1231,7 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
     cudaError_t err;
     const int npl = c.num_experts / 32;
     // H = 2048 and I = 768: gate/up 16 lanes x 4 pieces, down 8 lanes x 3 (4-bit)
-    //                                  32 lanes x 1 piece,   4 lanes x 3 (2-bit)
+    //                                  16 lanes x 2 pieces,  4 lanes x 3 (2-bit)
     if (c.bits == 4) {
       switch (npl) {
         case 16: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 16, 2>(p, num_sms, s)
@@ -1241,9 +1244,9 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
       }
     } else {
       switch (npl) {
-        case 16: err = launch_fused_t<2, 32, 1, 4, 3, 16>(p, num_sms, s); break;
-        case 32: err = launch_fused_t<2, 32, 1, 4, 3, 32>(p, num_sms, s); break;
-        case 8: err = launch_fused_t<2, 32, 1, 4, 3, 8>(p, num_sms, s); break;
+        case 16: err = launch_fused_t<2, 16, 2, 4, 3, 16>(p, num_sms, s); break;
+        case 32: err = launch_fused_t<2, 16, 2, 4, 3, 32>(p, num_sms, s); break;
+        case 8: err = launch_fused_t<2, 16, 2, 4, 3, 8>(p, num_sms, s); break;
         default: return cudaErrorInvalidValue;
       }
     }
