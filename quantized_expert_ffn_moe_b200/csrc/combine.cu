@@ -1,6 +1,7 @@
 // Gate-weighted combine: out[t] = g_t Y[shared, t] + sum_j Y[(t, j)] in fixed
 // slot order (the gate weight is already inside Y), fp32, rounded once to
 // bf16; g_t = 1, or sigmoid(x_t . w) when the layer has a shared-expert gate.
+// Y rows are fp32 (decode GEMV) or fp16 (tensor-core path, y_half).
 // The shared expert is added with weight 1 ("How a 125B Model Reaches 100
 // Tok/s on an RTX 4090", section "The model is large on paper, sparse in
 // practice": 10 routed experts plus one shared expert are active per token).
@@ -20,7 +21,8 @@ constexpr int kCombThreads = 256;
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const float* __restrict__ Y, const int* __restrict__ inv, int T, int k, int H, int shared,
     uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next, float* __restrict__ out_f32,
-    const int* __restrict__ gate, const uint16_t* __restrict__ xin, const uint16_t* __restrict__ sgate_w) {
+    const int* __restrict__ gate, const uint16_t* __restrict__ xin, const uint16_t* __restrict__ sgate_w,
+    int y_half) {
   pdl_wait();
   if (gate && __ldcg(gate) == 0) {                // the fused decode kernel kept (and combined) the layer
     pdl_launch_dependents();
@@ -58,23 +60,39 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
   float ss = 0.f;
   constexpr int VPT = 8;                      // elements per thread per step
   for (int h0 = threadIdx.x * VPT; h0 < H; h0 += kCombThreads * VPT) {
+    // 8 consecutive Y values of row p, in fp32
+    auto yrow = [&](int p, float (&o)[VPT]) {
+      if (y_half) {
+        const uint4 hv = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(Y) + size_t(p) * H + h0);
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __half22float2(u32_as_h2(hw[i]));
+          o[2 * i] = f.x;
+          o[2 * i + 1] = f.y;
+        }
+      } else {
+        const float4 a = *reinterpret_cast<const float4*>(Y + size_t(p) * H + h0);
+        const float4 b = *reinterpret_cast<const float4*>(Y + size_t(p) * H + h0 + 4);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+      }
+    };
     float acc[VPT];
     if (shared) {
-      const float4 a = *reinterpret_cast<const float4*>(Y + size_t(P_routed + t) * H + h0);
-      const float4 b = *reinterpret_cast<const float4*>(Y + size_t(P_routed + t) * H + h0 + 4);
-      acc[0] = gsh * a.x; acc[1] = gsh * a.y; acc[2] = gsh * a.z; acc[3] = gsh * a.w;
-      acc[4] = gsh * b.x; acc[5] = gsh * b.y; acc[6] = gsh * b.z; acc[7] = gsh * b.w;
+      float yv[VPT];
+      yrow(P_routed + t, yv);
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) acc[i] = gsh * yv[i];
     } else {
 #pragma unroll
       for (int i = 0; i < VPT; ++i) acc[i] = 0.f;
     }
     for (int j = 0; j < k; ++j) {
       if (pos[j] < 0) continue;                 // expert owned by another rank
-      const float* row = Y + size_t(pos[j]) * H + h0;
-      const float4 a = *reinterpret_cast<const float4*>(row);
-      const float4 b = *reinterpret_cast<const float4*>(row + 4);
-      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      float yv[VPT];
+      yrow(pos[j], yv);
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) acc[i] += yv[i];
     }
     if (out_f32) {
       float* fd = out_f32 + size_t(t) * H + h0;
@@ -134,7 +152,7 @@ cudaError_t launch_combine(const LayerArgs& a) {
                     reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
                     a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next,
                     a.y_f32, a.gated ? reinterpret_cast<const int*>(a.ws + a.L.status) + ST_PATH : nullptr, a.x,
-                    a.w.shared_gate_w);
+                    a.w.shared_gate_w, a.y_half);
 }
 
 }  // namespace moe

@@ -101,15 +101,17 @@ int run_layer(const LayerArgs& a) {
                                     nullptr, nullptr, a.stream, a.ep_rank, a.ep_size);
   if (e != cudaSuccess) return cuda_status(e);
   prof_mark(call, 1, a.stream);
+  LayerArgs comb = a;
   if (a.T > kDecodeMaxTokens && prefill_supported(a.cfg)) {
     e = launch_prefill_ffn(a);
     if (call >= 0) cudaEventRecord(g_prof.ev[call * 5 + 2], a.stream);
+    comb.y_half = 1;                      // the tensor-core down pass writes fp16 rows
   } else {
     e = launch_decode_ffn(a, call >= 0 ? g_prof.ev[call * 5 + 2] : nullptr);
   }
   if (e != cudaSuccess) return cuda_status(e);
   prof_mark(call, 3, a.stream);
-  e = launch_combine(a);
+  e = launch_combine(comb);
   prof_mark(call, 4, a.stream);
   return cuda_status(e);
 }
@@ -193,6 +195,7 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
     cudaError_t e = launch_fused_decode(*cfg, w, 1, x, y, false, T, nullptr, a.ws, a.L, a.num_sms, a.stream, hybrid);
     if (e == cudaSuccess && hybrid) {
       a.gated = 1;
+      a.y_half = 1;
       e = launch_prefill_ffn(a);
       if (e == cudaSuccess) e = launch_combine(a);
     }

@@ -33,7 +33,7 @@ constexpr int kGroupChunk = 64;
 
 struct Layout {
   size_t status, logits, topk_idx, topk_w, counts, offsets, pairs, inv, ulist, woff_gu, woff_dn, ntoff, xhat, h,
-      y, xs, xscale, chunk_hist, gdone, total;
+      y, xs, xscale, chunk_hist, chunk_mask, gdone, total;
   int P;
 };
 
@@ -63,6 +63,7 @@ inline Layout make_layout(const moe_config& c, int T) {
   L.xs = take(size_t(P) * c.hidden * 2);
   L.xscale = take(size_t(P) * 4);
   L.chunk_hist = take(size_t((T + kGroupChunk - 1) / kGroupChunk) * c.num_experts * 4);
+  L.chunk_mask = take(size_t((T + kGroupChunk - 1) / kGroupChunk) * 2 * c.num_experts * 4);   // 64-token chunks
   L.gdone = take(size_t(c.num_experts + 2) * 4);   // fused decode: gate/up stages finished per slot
   L.total = o;
   L.P = P;
@@ -505,6 +506,7 @@ struct LayerArgs {
   int gated = 0;                  // run the tensor-core kernels only if the fused decode kernel handed over
   int ep_rank = 0, ep_size = 1;   // expert-parallel share: experts e with e % ep_size == ep_rank
   float* y_f32 = nullptr;         // [T][H] fp32 partial output (expert-parallel share) instead of y
+  int y_half = 0;                 // the per-pair rows Y are fp16 (tensor-core path), else fp32
 };
 
 cudaError_t launch_rmsnorm(const uint16_t* x, uint16_t* xhat, int T, int H, cudaStream_t s);

@@ -82,7 +82,7 @@ struct PrefillArgs {
   const int* ntoff;       // [nslots+1] prefix of token tiles per slot
   uint16_t* hout;         // gate/up: h [P][I] fp16 bits, k permuted for the down pass
   const float* xinv;      // gate/up: [P] inverse power-of-two scale of each token row
-  float* yout;            // down: Y [P][H] fp32
+  uint16_t* yout;         // down: Y [P][H] fp16 bits (gate weight applied)
   int* status;
   unsigned long long* timing;   // null, or [gridDim][16] per-role wait times (ns) of this launch
   int gated;                    // 1: no tiles unless the fused decode kernel handed the layer over
@@ -573,7 +573,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float w = __shfl_sync(0xffffffffu, colf, c);
-            if (n0 + c < ti.nvalid) a.yout[size_t(prow + n0 + c) * a.out_cols + R] = __uint_as_float(v[c]) * w;
+            if (n0 + c < ti.nvalid)
+              a.yout[size_t(prow + n0 + c) * a.out_cols + R] = __half_as_ushort(__float2half_rn(__uint_as_float(v[c]) * w));
           }
         }
       }
@@ -909,7 +910,7 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
 
   PrefillArgs d = g;
   d.K = I; d.rows_pe = H; d.out_cols = H;
-  d.hout = nullptr; d.yout = reinterpret_cast<float*>(a.ws + a.L.y);
+  d.hout = nullptr; d.yout = reinterpret_cast<uint16_t*>(a.ws + a.L.y);
   d.timing = g_prefill_timing ? g_prefill_timing + size_t(a.num_sms) * kPTime : nullptr;
   return bits == 4 ? launch_gemm<1, 4>(d, a.w.down_codes, a.w.down_scales, a.w.shared_down_codes,
                                        a.w.shared_down_scales, c.num_experts, sh, hs, P, a.num_sms, a.stream)

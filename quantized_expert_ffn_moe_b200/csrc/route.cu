@@ -325,23 +325,71 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(
 // chunk of kGroupChunk tokens counts its pairs per expert; one CTA turns the
 // counts into per-chunk bases, offsets, the touched-expert list and the work
 // prefixes; each chunk then writes its pairs in token order.
-__global__ void __launch_bounds__(256) chunk_hist_kernel(const int* __restrict__ idx, int T, int k, int E,
-                                                         int* __restrict__ chunk_hist, int* __restrict__ status,
-                                                         int ep_rank, int ep_size) {
-  extern __shared__ int hs[];
+// Large batches: a stable counting sort over 64-token chunks, with the order
+// inside a chunk taken from per-expert token masks (bit t of chunk expert e:
+// token t of the chunk picked e).  chunk_mask_kernel builds a chunk's masks and
+// its per-expert counts; chunk_scan_kernel turns the counts into per-chunk
+// bases, offsets, the touched-expert list and the work prefixes; and
+// chunk_place_kernel puts pair (t, j) of expert e at
+//   offset(e) + base(chunk, e) + (tokens of the chunk before t that picked e),
+// every pair independently.
+__global__ void __launch_bounds__(256) chunk_mask_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                                         int* __restrict__ chunk_hist, unsigned* __restrict__ chunk_mask,
+                                                         int* __restrict__ status, int ep_rank, int ep_size) {
+  extern __shared__ unsigned msk[];                 // [2][E]
   pdl_wait();
   pdl_launch_dependents();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hs[e] = 0;
+  for (int i = threadIdx.x; i < 2 * E; i += blockDim.x) msk[i] = 0u;
   __syncthreads();
   const int t0 = blockIdx.x * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
   for (int q = t0 * k + threadIdx.x; q < t1 * k; q += blockDim.x) {
     const int e = idx[q];
     if (e < 0 || e >= E) { atomicCAS(status + ST_ERROR, 0, 2); continue; }
-    if (e % ep_size != ep_rank) continue;     // expert of another rank
-    atomicAdd(&hs[e], 1);
+    const int tl = q / k - t0;
+    atomicOr(&msk[(tl >> 5) * E + e], 1u << (tl & 31));
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[size_t(blockIdx.x) * E + e] = hs[e];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const unsigned m0 = msk[e], m1 = msk[E + e];
+    chunk_hist[size_t(blockIdx.x) * E + e] = (e % ep_size == ep_rank) ? __popc(m0) + __popc(m1) : 0;
+    chunk_mask[size_t(blockIdx.x) * 2 * E + e] = m0;
+    chunk_mask[size_t(blockIdx.x) * 2 * E + E + e] = m1;
+  }
+}
+
+// Exclusive block-wide scan of NV values per thread (all kGroupThreads
+// threads), with the totals; scr: 32 * NV ints of shared memory.
+template <int NV>
+__device__ __forceinline__ void block_scan_n(const int (&v)[NV], int (&excl)[NV], int (&tot)[NV], int* scr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    x[j] = v[j];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, x[j], o);
+      if (lane >= o) x[j] += n;
+    }
+  }
+  if (lane == 31) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) scr[j * 32 + warp] = x[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    int before = 0, all = 0;
+#pragma unroll 8
+    for (int w = 0; w < kGroupThreads / 32; ++w) {
+      const int s = scr[j * 32 + w];
+      before += w < warp ? s : 0;
+      all += s;
+    }
+    excl[j] = before + x[j] - v[j];
+    tot[j] = all;
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kGroupThreads) chunk_scan_kernel(
@@ -349,124 +397,102 @@ __global__ void __launch_bounds__(kGroupThreads) chunk_scan_kernel(
     int* __restrict__ counts_out, int* __restrict__ offsets_out, int* __restrict__ ulist_out,
     int* __restrict__ api_counts, int* __restrict__ api_offsets, PassPlan pg, PassPlan pd,
     int* __restrict__ woff_gu, int* __restrict__ woff_dn, int* __restrict__ ntoff) {
-  __shared__ int offs[1025];
-  __shared__ int scan[32];
+  __shared__ int scr[32 * 3];
+  __shared__ int cnt[1025];
   pdl_wait();
   pdl_launch_dependents();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = threadIdx.x;
   int c = 0;
   if (e < E) {
-    // per-chunk base of expert e = exclusive prefix over chunks
+    // per-chunk base of expert e = exclusive prefix over chunks; the loads of
+    // 32 chunks are in flight together
     int run = 0;
-    for (int ch0 = 0; ch0 < nchunks; ch0 += 16) {      // loads issued 16 at a time
-      int v[16];
+    for (int ch0 = 0; ch0 < nchunks; ch0 += 32) {
+      int v[32];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = ch0 + j < nchunks ? chunk_hist[size_t(ch0 + j) * E + e] : 0;
+      for (int j = 0; j < 32; ++j) v[j] = ch0 + j < nchunks ? __ldcg(chunk_hist + size_t(ch0 + j) * E + e) : 0;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 32; ++j) {
         if (ch0 + j < nchunks) chunk_hist[size_t(ch0 + j) * E + e] = run;
         run += v[j];
       }
     }
     c = run;
   }
-  // exclusive scan over experts
-  int v = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, v, o); if (lane >= o) v += n; }
-  if (lane == 31) scan[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    int s2 = scan[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, s2, o); if (lane >= o) s2 += n; }
-    scan[lane] = s2;
-  }
-  __syncthreads();
-  const int excl = v - c + (warp > 0 ? scan[warp - 1] : 0);
-  __syncthreads();
+  const int in2[2] = {c, (e < E && c > 0) ? 1 : 0};
+  int ex2[2], tot2[2];
+  block_scan_n<2>(in2, ex2, tot2, scr);
   if (e < E) {
-    counts_out[e] = c; offsets_out[e] = excl; offs[e] = excl;
+    counts_out[e] = c;
+    offsets_out[e] = ex2[0];
+    cnt[e] = c;
     if (api_counts) api_counts[e] = c;
-    if (api_offsets) api_offsets[e] = excl;
+    if (api_offsets) api_offsets[e] = ex2[0];
+    if (c > 0) ulist_out[ex2[1]] = e;
   }
-  if (e == E - 1) { offsets_out[E] = excl + c; offs[E] = excl + c; if (api_offsets) api_offsets[E] = excl + c; }
-  // touched-expert list
-  const int f = (e < E && c > 0) ? 1 : 0;
-  int fv = f;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, fv, o); if (lane >= o) fv += n; }
-  __syncthreads();
-  if (lane == 31) scan[warp] = fv;
-  __syncthreads();
-  if (warp == 0) {
-    int s2 = scan[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) { const int n = __shfl_up_sync(0xffffffffu, s2, o); if (lane >= o) s2 += n; }
-    scan[lane] = s2;
+  const int U = tot2[1];
+  if (threadIdx.x == 0) {
+    offsets_out[E] = tot2[0];
+    if (api_offsets) api_offsets[E] = tot2[0];
+    status[ST_UCOUNT] = U;
+    if (shared) ulist_out[U] = E;
   }
   __syncthreads();
-  const int fpos = fv - f + (warp > 0 ? scan[warp - 1] : 0);
-  if (f) ulist_out[fpos] = e;
-  const int U = scan[31];
-  if (threadIdx.x == 0) { status[ST_UCOUNT] = U; if (shared) ulist_out[U] = E; }
-  __syncthreads();
-  if (warp == 0) {
-    const int nslots = U + shared;
-    int run_g = 0, run_d = 0, run_t = 0;
-    for (int base = 0; base < nslots; base += 32) {
-      const int u = base + lane;
-      int n = 0;
-      if (u < U) { const int ee = ulist_out[u]; n = offs[ee + 1] - offs[ee]; }
-      else if (u < nslots) n = T;
-      int g = u < nslots ? pass_cost(pg, n) : 0, d = u < nslots ? pass_cost(pd, n) : 0;
-      int nt = u < nslots ? (n + kPrefillTileN - 1) / kPrefillTileN : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int ng = __shfl_up_sync(0xffffffffu, g, o), nd = __shfl_up_sync(0xffffffffu, d, o);
-        const int nn = __shfl_up_sync(0xffffffffu, nt, o);
-        if (lane >= o) { g += ng; d += nd; nt += nn; }
-      }
-      if (u < nslots) { woff_gu[u + 1] = run_g + g; woff_dn[u + 1] = run_d + d; ntoff[u + 1] = run_t + nt; }
-      run_g += __shfl_sync(0xffffffffu, g, 31);
-      run_d += __shfl_sync(0xffffffffu, d, 31);
-      run_t += __shfl_sync(0xffffffffu, nt, 31);
+  // work prefixes over the slots (touched experts ascending, the shared
+  // expert last): slot u of thread u, and slot 1024 (E = 1024 with every
+  // expert touched and a shared expert) on thread 0's second pass
+  const int nslots = U + shared;
+  for (int base = 0; base < nslots; base += kGroupThreads) {
+    const int u = base + threadIdx.x;
+    int n = 0;
+    if (u < U) n = cnt[ulist_out[u]];
+    else if (u < nslots) n = T;
+    const int in3[3] = {u < nslots ? pass_cost(pg, n) : 0, u < nslots ? pass_cost(pd, n) : 0,
+                        u < nslots ? (n + kPrefillTileN - 1) / kPrefillTileN : 0};
+    int ex3[3], tot3[3];
+    block_scan_n<3>(in3, ex3, tot3, scr);
+    const int g0 = base ? woff_gu[base] : 0, d0 = base ? woff_dn[base] : 0, n0 = base ? ntoff[base] : 0;
+    __syncthreads();
+    if (u < nslots) {
+      woff_gu[u + 1] = g0 + ex3[0] + in3[0];
+      woff_dn[u + 1] = d0 + ex3[1] + in3[1];
+      ntoff[u + 1] = n0 + ex3[2] + in3[2];
     }
-    if (lane == 0) { woff_gu[0] = 0; woff_dn[0] = 0; ntoff[0] = 0; }
+    __syncthreads();
   }
+  if (threadIdx.x == 0) { woff_gu[0] = 0; woff_dn[0] = 0; ntoff[0] = 0; }
 }
 
-__global__ void __launch_bounds__(32) chunk_scatter_kernel(const int* __restrict__ idx, int T, int k, int E,
-                                                           const int* __restrict__ chunk_base,
-                                                           const int* __restrict__ offsets, int* __restrict__ pairs,
-                                                           int* __restrict__ inv, int* __restrict__ api_pairs,
-                                                           int ep_rank, int ep_size) {
-  extern __shared__ int cur[];                 // [E] fill cursors, then the chunk's ids
-  int* cidx = cur + E;                         // [kGroupChunk * k]
+__global__ void __launch_bounds__(256) chunk_place_kernel(const int* __restrict__ idx, int T, int k, int E,
+                                                          const int* __restrict__ chunk_base,
+                                                          const unsigned* __restrict__ chunk_mask,
+                                                          const int* __restrict__ offsets, int* __restrict__ pairs,
+                                                          int* __restrict__ inv, int* __restrict__ api_pairs,
+                                                          int ep_rank, int ep_size) {
+  extern __shared__ unsigned pl[];             // masks [2][E], then the bases [E]
+  int* base = reinterpret_cast<int*>(pl + 2 * E);
   pdl_wait();
   pdl_launch_dependents();
-  const int lane = threadIdx.x;
-  const int t0 = blockIdx.x * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
-  // the chunk's selections in one coalesced pass, so the ordered walk below
-  // reads shared memory instead of waiting on a global load per token
-  for (int q = t0 * k + lane; q < t1 * k; q += 32) cidx[q - t0 * k] = idx[q];
-  for (int e = lane; e < E; e += 32) cur[e] = offsets[e] + chunk_base[size_t(blockIdx.x) * E + e];
-  __syncwarp();
-  for (int t = t0; t < t1; ++t) {
-    if (lane < k) {
-      const int q = t * k + lane;
-      const int e = cidx[q - t0 * k];
-      if (e >= 0 && e < E && e % ep_size == ep_rank) {
-        const int pos = cur[e]++;     // distinct experts within one token
-        pairs[pos] = q;
-        inv[q] = pos;
-        if (api_pairs) api_pairs[pos] = q;
-      } else {
-        inv[q] = -1;                  // not computed on this rank
-      }
+  const int ch = blockIdx.x;
+  for (int i = threadIdx.x; i < 2 * E; i += blockDim.x) pl[i] = __ldcg(chunk_mask + size_t(ch) * 2 * E + i);
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    base[e] = __ldcg(offsets + e) + __ldcg(chunk_base + size_t(ch) * E + e);
+  __syncthreads();
+  const int t0 = ch * kGroupChunk, t1 = min(T, t0 + kGroupChunk);
+  for (int q = t0 * k + threadIdx.x; q < t1 * k; q += blockDim.x) {
+    const int e = idx[q];
+    if (e < 0 || e >= E || e % ep_size != ep_rank) {
+      inv[q] = -1;                             // not computed on this rank
+      continue;
     }
-    __syncwarp();
+    const int tl = q / k - t0;
+    const unsigned m0 = pl[e];
+    const int r = tl < 32 ? __popc(m0 & ((1u << tl) - 1u))
+                          : __popc(m0) + __popc(pl[E + e] & ((1u << (tl - 32)) - 1u));
+    const int pos = base[e] + r;
+    pairs[pos] = q;
+    inv[q] = pos;
+    if (api_pairs) api_pairs[pos] = q;
   }
 }
 
@@ -492,8 +518,9 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
       const int nch = (T + kGroupChunk - 1) / kGroupChunk, E = c.num_experts;
       int* hist = reinterpret_cast<int*>(ws + L.chunk_hist);
       int* status = reinterpret_cast<int*>(ws + L.status);
-      err = launch_pdl(chunk_hist_kernel, dim3(nch), dim3(256), size_t(E) * 4, s, (const int*)idx, T, c.top_k, E,
-                       hist, status, ep_rank, ep_size);
+      unsigned* masks = reinterpret_cast<unsigned*>(ws + L.chunk_mask);
+      err = launch_pdl(chunk_mask_kernel, dim3(nch), dim3(256), size_t(2 * E) * 4, s, (const int*)idx, T, c.top_k,
+                       E, hist, masks, status, ep_rank, ep_size);
       if (err != cudaSuccess) return err;
       err = launch_pdl(chunk_scan_kernel, dim3(1), dim3(kGroupThreads), 0, s, nch, T, E, c.shared_inter > 0 ? 1 : 0,
                        hist, status, reinterpret_cast<int*>(ws + L.counts), reinterpret_cast<int*>(ws + L.offsets),
@@ -501,10 +528,10 @@ cudaError_t launch_topk_group(const moe_config& c, int T, char* ws, const Layout
                        reinterpret_cast<int*>(ws + L.woff_gu), reinterpret_cast<int*>(ws + L.woff_dn),
                        reinterpret_cast<int*>(ws + L.ntoff));
       if (err != cudaSuccess) return err;
-      return launch_pdl(chunk_scatter_kernel, dim3(nch), dim3(32), size_t(E + kGroupChunk * c.top_k) * 4, s,
-                        (const int*)idx, T, c.top_k, E,
-                        (const int*)hist, (const int*)(ws + L.offsets), reinterpret_cast<int*>(ws + L.pairs),
-                        reinterpret_cast<int*>(ws + L.inv), api_pairs, ep_rank, ep_size);
+      return launch_pdl(chunk_place_kernel, dim3(nch), dim3(256), size_t(3 * E) * 4, s, (const int*)idx, T,
+                        c.top_k, E, (const int*)hist, (const unsigned*)masks, (const int*)(ws + L.offsets),
+                        reinterpret_cast<int*>(ws + L.pairs), reinterpret_cast<int*>(ws + L.inv), api_pairs, ep_rank,
+                        ep_size);
     }
   }
   return launch_pdl(kern, dim3(1), dim3(kGroupThreads), smem, s, logits, fused ? 1 : 0, idx, w, T,
