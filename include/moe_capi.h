@@ -238,9 +238,9 @@ void moe_debug_fused_timing(unsigned long long* device_buf);
  *   [4] MMA waiting for a free accumulator, [5] dequantizer (first thread)
  *   waiting for packed weights, [6] dequantizer waiting for a free A stage,
  *   [7] epilogue (first thread) waiting for an accumulator, [12] cycles in the
- *   MMA issue blocks, [13] cycles in tile lookups; %globaltimer (ns): [8]
- *   start and [9] end of the MMA thread, [11] end of the epilogue; counts:
- *   [10] tiles, [14] k-blocks. */
+ *   MMA issue blocks, [13] cycles in tile lookups, [15] cycles of the whole
+ *   MMA loop; %globaltimer (ns): [8] start and [9] end of the MMA thread, [11]
+ *   end of the epilogue; counts: [10] tiles, [14] k-blocks. */
 void moe_debug_prefill_timing(unsigned long long* device_buf);
 
 /* Measurement and test hook for single-layer batches of 32..64 tokens, where

@@ -44,8 +44,15 @@ constexpr int PSK = 128;       // grouped GEMM: k per A/B stage (two swizzle ato
 constexpr int RAWK = 256;      // k per packed stage
 constexpr int PNK = 4;         // A (tensor memory) / B (shared memory) stages
 constexpr int PNR = 4;         // packed stages
-constexpr int kWarpRaw = 0, kWarpB = 1, kWarpMma = 2, kWarpDq0 = 3, kNumDq = 8, kWarpEp0 = 11, kNumEp = 4;
-constexpr int kPThreads = (kWarpEp0 + kNumEp) * 32;
+constexpr int kWarpRaw = 0, kWarpB = 1, kWarpMma = 2, kWarpDq0 = 3, kNumDq = 8, kWarpEp0 = 11;
+// Epilogue warps: two per tensor-memory lane quarter for the down GEMM, whose
+// tiles carry only I / 128 k-blocks of MMAs and whose epilogue writes a value
+// per (row, token); one per quarter for gate/up (sixteen k-blocks per tile,
+// and its register budget does not fit 19 warps).
+template <int MODE> struct PEp {
+  static constexpr int kNum = MODE == 1 ? 8 : 4;
+  static constexpr int kThreads = (kWarpEp0 + kNum) * 32;
+};
 constexpr uint32_t kTmemCols = 2 * PBN;          // router GEMM: two accumulators
 // Grouped GEMM tensor memory: two accumulators of PBN columns, then PNK
 // dequantized A stages of PSK / 2 columns (128 lanes = the tile's rows, two
@@ -131,6 +138,12 @@ __device__ __forceinline__ void tc_mma_ta(uint32_t d_tmem, uint32_t a_tmem, uint
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// True in exactly one lane of a fully active warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+  return pred != 0;
 }
 // 32 consecutive columns of this thread's tensor-memory lane (warp-wide; the
 // warp's lane quarter is fixed by its rank within the warpgroup).
@@ -235,7 +248,7 @@ __device__ __forceinline__ void tile_info(const SlotTab& st, int nslots, int mt,
 }
 
 template <int MODE, int BITS>
-__global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
+__global__ void __launch_bounds__(PEp<MODE>::kThreads, 1) prefill_gemm_kernel(
     PrefillArgs a, const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
     const __grid_constant__ CUtensorMap tm_sh_codes, const __grid_constant__ CUtensorMap tm_sh_scales,
     const __grid_constant__ CUtensorMap tm_b) {
@@ -260,7 +273,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     for (int i = 0; i < PNR; ++i) { mbar_init(&full_raw[i], 1); mbar_init(&empty_raw[i], kNumDq); }
     // full_a: the four dequant warps of the k-block's half + the token tile's bytes
     for (int i = 0; i < PNK; ++i) { mbar_init(&full_a[i], kNumDq / 2 + 1); mbar_init(&empty_ab[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], kNumEp); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], PEp<MODE>::kNum); }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -310,8 +323,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     }
   }
   __syncthreads();
-  auto get_tile = [&](int t, TileInfo* ti) {
-    const int i = (t - int(blockIdx.x)) / int(gridDim.x);
+  // tile i of this CTA (global tile t = blockIdx.x + i * gridDim.x)
+  auto get_tile = [&](int i, TileInfo* ti) {
     if (i < kTileTab) {
       const int4 v = ttab[i];
       ti->e = v.x;
@@ -320,16 +333,16 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
       ti->m = v.z & 0xFFFF;
       ti->nvalid = v.w;
     } else {
-      tile_info(stab, nslots, mt, t, ti);
+      tile_info(stab, nslots, mt, int(blockIdx.x) + i * int(gridDim.x), ti);
     }
   };
 
   if (warp == kWarpRaw && lane == 0) {
     // ------------------------------------------------ packed weight producer
     int rc = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+    for (int t = blockIdx.x, i = 0; t < ntiles && !*abort_flag; t += gridDim.x, ++i) {
       TileInfo ti;
-      get_tile(t, &ti);
+      get_tile(i, &ti);
       const bool sh = ti.e >= rv.E;
       const CUtensorMap* mc = sh ? &tm_sh_codes : &tm_codes;
       const CUtensorMap* ms = sh ? &tm_sh_scales : &tm_scales;
@@ -358,9 +371,9 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
   } else if (warp == kWarpB && lane == 0) {
     // ------------------------------------------------------ token producer
     int kc = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+    for (int t = blockIdx.x, i = 0; t < ntiles && !*abort_flag; t += gridDim.x, ++i) {
       TileInfo ti;
-      get_tile(t, &ti);
+      get_tile(i, &ti);
       const int prow = ti.p0 + ti.j * PBN;
       for (int kb = 0; kb < KB; ++kb, ++kc) {
         const int s = kc % PNK;
@@ -376,45 +389,65 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     for (int i = max(0, kc - PNK); i < kc; ++i)
       if (!mbar_wait(&full_a[i % PNK], (i / PNK) & 1, nullptr)) report_error(a.status, MOE_ERR_TIMEOUT, 13);
     if (tm) tm[1] = tw0;
-  } else if (warp == kWarpMma && lane == 0) {
+  } else if (warp == kWarpMma) {
     // ---------------------------------------------------------------- MMA
+    // The whole warp runs this loop, so its control and every MMA operand are
+    // warp-uniform; one elected lane issues each stage's MMAs and commit.  (A
+    // single-lane loop left the operands per-thread: its issue competed with
+    // the dequant warps and cost ~90 instead of ~55-70 cycles per MMA.)
     int kc = 0, tc = 0;
-    for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x, ++tc) {
+    const long long c_start = tm ? clock64() : 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
       const long long cti = tm ? clock64() : 0;
       TileInfo ti;
-      get_tile(t, &ti);
+      get_tile(tc, &ti);
       if (tm) tw4 += clock64() - cti;
       const int buf = tc & 1;
-      if (tc >= 2 && !mbar_wait_t(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag, tm ? &tw2 : nullptr)) {
-        *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 14); break;
+      if (tc >= 2) {
+        const long long cw = tm ? clock64() : 0;
+        ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty[buf], ((tc >> 1) - 1) & 1, abort_flag));
+        if (tm) tw2 += clock64() - cw;
+      }
+      if (!ok) {
+        if (lane == 0) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 14); }
+        break;
       }
       tc_fence_after();
-      const int n16 = (ti.nvalid + 15) & ~15;
-      const uint32_t idesc = idesc_f16(n16);
+      const uint32_t idesc = idesc_f16((ti.nvalid + 15) & ~15);
       const uint32_t d_tmem = tmem_base + uint32_t(buf * PBN);
-      bool ok = true;
       for (int kb = 0; kb < KB; ++kb, ++kc) {
         const int s = kc % PNK;
-        if (!mbar_wait_t(&full_a[s], (kc / PNK) & 1, abort_flag, tm ? &tw0 : nullptr)) {
-          *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 15); ok = false; break;
+        const long long cw = tm ? clock64() : 0;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full_a[s], (kc / PNK) & 1, abort_flag));
+        if (!ok) {
+          if (lane == 0) { *abort_flag = 1; report_error(a.status, MOE_ERR_TIMEOUT, 15); }
+          break;
         }
         const long long ci = tm ? clock64() : 0;
+        if (tm) tw0 += ci - cw;
         tc_fence_after();
-        const uint32_t a0 = tmem_base + kAColBase + uint32_t(s) * kAStageCols, b0 = smem_u32(sB + s * kGBStageBytes);
+        const uint32_t a0 = tmem_base + kAColBase + uint32_t(s) * kAStageCols;
+        const uint64_t bd = sw128_desc(smem_u32(sB + s * kGBStageBytes));
+        if (elect_one()) {
 #pragma unroll
-        for (int k = 0; k < PSK / 16; ++k)
-          tc_mma_ta(d_tmem, a0 + uint32_t(k * 8), sw128_desc(b0 + (k >> 2) * kBStageBytes + (k & 3) * 32), idesc,
-                    (kb | k) ? 1u : 0u);
-        tc_commit(&empty_ab[s]);
+          for (int k = 0; k < PSK / 16; ++k)
+            tc_mma_ta(d_tmem, a0 + uint32_t(k * 8), bd + uint64_t(((k >> 2) * kBStageBytes + (k & 3) * 32) >> 4),
+                      idesc, (kb | k) ? 1u : 0u);
+          tc_commit(&empty_ab[s]);
+          if (kb == KB - 1) tc_commit(&acc_full[buf]);
+        }
+        __syncwarp();
         if (tm) tw3 += clock64() - ci;
       }
       if (!ok) break;
-      tc_commit(&acc_full[buf]);
     }
-    // wait for this thread's last MMAs before the CTA tears down TMEM
-    if (kc > 0 && !mbar_wait(&empty_ab[(kc - 1) % PNK], ((kc - 1) / PNK) & 1, nullptr))
+    // wait for the last MMAs before the CTA tears down TMEM
+    if (kc > 0 && !__all_sync(0xffffffffu, mbar_wait(&empty_ab[(kc - 1) % PNK], ((kc - 1) / PNK) & 1, nullptr)) &&
+        lane == 0)
       report_error(a.status, MOE_ERR_TIMEOUT, 16);
-    if (tm) { tm[2] = tw0; tm[3] = tw1; tm[4] = tw2; tm[8] = t_start; tm[9] = global_ns(); tm[10] = tc; tm[12] = tw3; tm[13] = tw4; tm[14] = kc; }
+    if (tm && lane == 0) { tm[2] = tw0; tm[3] = tw1; tm[4] = tw2; tm[8] = t_start; tm[9] = global_ns(); tm[10] = tc; tm[12] = tw3; tm[13] = tw4; tm[14] = kc; tm[15] = clock64() - c_start; }
   } else if (warp >= kWarpDq0 && warp < kWarpDq0 + kNumDq) {
     // ----------------------------------------------------------- dequant
     // warp w writes rows of its tensor-memory lane quarter (w % 4); the two
@@ -487,10 +520,12 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
       }
     }
     if (tm && threadIdx.x == kWarpDq0 * 32) { tm[5] = tw0; tm[6] = tw1; }
-  } else if (warp >= kWarpEp0 && warp < kWarpEp0 + kNumEp) {
+  } else if (warp >= kWarpEp0 && warp < kWarpEp0 + PEp<MODE>::kNum) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                         // TMEM lane quarter of this warp
     const int r = q * 32 + lane;                    // tile row
+    constexpr int kColStep = 32 * (PEp<MODE>::kNum / 4);
+    const int c_first = ((warp - kWarpEp0) >> 2) * 32;   // the warps of a quarter take alternate 32-column chunks
     // per-column factors of a tile (gate/up: the token row's inverse scale,
     // down: the gate weight), column u*32 + lane in f[u].  They are fetched
     // one tile ahead (down: the pair ids while the current tile's columns are
@@ -521,7 +556,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
     float f_n[PBN / 32];
     int pr_n[PBN / 32];
     if (blockIdx.x < ntiles) {
-      get_tile(blockIdx.x, &ti_n);
+      get_tile(0, &ti_n);
       first_level(ti_n, f_n, pr_n);
       second_level(f_n, pr_n);
     }
@@ -540,11 +575,11 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_gemm_kernel(
       }
       const bool more = t + int(gridDim.x) < ntiles;
       if (more) {
-        get_tile(t + gridDim.x, &ti_n);
+        get_tile(tc + 1, &ti_n);
         first_level(ti_n, f_n, pr_n);
       }
       tc_fence_after();
-      for (int n0 = 0; n0 < ti.nvalid; n0 += 32) {
+      for (int n0 = c_first; n0 < ti.nvalid; n0 += kColStep) {
         uint32_t v[32];
         tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(buf * PBN + n0), v);
         const int u0 = n0 >> 5;
@@ -830,7 +865,7 @@ cudaError_t launch_gemm(const PrefillArgs& pa, const uint8_t* codes, const uint1
   auto kern = prefill_gemm_kernel<MODE, BITS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(kern, dim3(num_sms), dim3(kPThreads), smem, s, pa, mc, ms, msc, mss, mb);
+  return launch_pdl(kern, dim3(num_sms), dim3(PEp<MODE>::kThreads), smem, s, pa, mc, ms, msc, mss, mb);
 }
 
 }  // namespace
