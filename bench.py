@@ -82,6 +82,29 @@ def profiled_traffic(profile: str, sources) -> float | None:
     return float(fields["traffic_bytes_per_launch"])
 
 
+# Lane operations per weight of the integer GEMV's inner loop, counted from its
+# source: decoding a 32-bit word of codes into signed bytes (4-bit: one shift
+# and two lop3 per 8 weights; 2-bit: three shifts and four lop3 per 16), and
+# per token the dp2a dot products (two products each) plus the fold of each
+# block's integer sum (I2F + FFMA per 32 / 16 weights).
+ALU_OPS = {4: (3 / 8, 0.5 + 2 / 32), 2: (7 / 16, 0.5 + 2 / 16), "4g128": (3 / 8, 0.5 + 2 / 128)}
+WEIGHTS_PER_EXPERT = 3 * 2048 * 768
+ST_PATH = 3        # status word of the workspace: 1 when the tensor-core kernels ran the call
+
+
+def alu_ceiling(bits, distinct: float, T: int, us_step: float, sm_mhz: float | None, sms: int = 148) -> dict:
+    """The CUDA-core decode's compute ceiling: lane-ops = dequant ops x (U+1)
+    x weights per expert + per-token ops x (T k + T) x weights per expert,
+    over 148 SMs x 128 lanes at the sampled SM clock."""
+    dq, per_tok = ALU_OPS[bits]
+    lane_ops = dq * (distinct + 1) * WEIGHTS_PER_EXPERT + per_tok * (T * 10 + T) * WEIGHTS_PER_EXPERT
+    mhz = sm_mhz or 1965.0
+    min_us = 1e6 * lane_ops / (sms * 128 * mhz * 1e6)
+    return {"lane_ops_per_step": lane_ops, "min_us": min_us, "frac": min_us / us_step, "sm_mhz": mhz,
+            "ops_per_weight": {"dequant": dq, "per_token": per_tok},
+            "source": "ops counted from the integer GEMV inner loop; the path the kernel ran is the other keys'"}
+
+
 def issue_ceiling(instructions: float, launch_s: float, sms: int, sm_mhz: float = 1965.0) -> dict:
     """Warp instructions per launch (ncu smsp__inst_executed.sum) against the
     issue capacity of the GPU: one warp instruction per cycle per scheduler,
@@ -538,7 +561,7 @@ def main():
 
     # ---- secondary workloads of the same layer family
     if not args.no_detail:
-        line["detail"] = detail(R, args, pool, ws, W, hbm_peak, tf_peak, dist, world)
+        line["detail"] = detail(R, args, pool, ws, W, hbm_peak, tf_peak, dist, world, clocks.get("sm_mhz"))
 
     # ---- CPU oracle baseline (rank 0, one GPU only)
     if world == 1:
@@ -549,7 +572,7 @@ def main():
         dist.destroy_process_group()
 
 
-def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
+def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world, clock_mhz=None):
     torch, q, mi = R.torch, R.q, R.mi
     out = {}
     shape = mi.FULL4
@@ -571,10 +594,26 @@ def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world):
              "distinct_experts": float(np.mean(us)), "touched_mb": mb / 1e6,
              "achieved_gbs": mb / (ms / K * 1e-3) / 1e9}
         r["frac_of_measured_hbm"] = r["achieved_gbs"] / hbm_peak
-        if T > 64:
+        tc_share = 1.0 if T > 64 else 0.0
+        if 32 <= T <= 64:
+            # which side of the hand-over the calls took (the decode kernel
+            # records its choice in the workspace's status words)
+            picks = []
+            for i in range(8):
+                step(i)
+                torch.cuda.synchronize()
+                picks.append(int(ws[4 * ST_PATH:4 * ST_PATH + 4].view(torch.int32).item()))
+            tc_share = float(np.mean(picks))
+            r["tensor_core_share_of_calls"] = tc_share
+        if tc_share > 0:
             flops = 9437184.0 * (T * 10 + T)
             r["tflops"] = flops / (ms / K * 1e-3) / 1e12
             r["frac_of_measured_bf16"] = r["tflops"] / tf_peak
+            r["tensor_operands"] = ("fp16 x fp16 -> fp32: weights dequantized to q*s (one rounding), token rows "
+                                    "scaled by a power of two per row (exact), compared against the bf16 dense "
+                                    "peak (fp16 has the same dense rate)")
+        if T <= 64:
+            r["alu"] = alu_ceiling(bits, float(np.mean(us)), T, 1000 * ms / K, clock_mhz)
         out[name] = r
 
     for T in (1, 4):

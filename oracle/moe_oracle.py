@@ -276,7 +276,8 @@ def layer_forward(layer: OracleLayer, x_bits: np.ndarray, *, rmsnorm: bool = Fal
     return {"xhat": xhat, "logits": logits, "idx": idx, "w": w, "out": out}
 
 
-def layer_forward_ep(layer: OracleLayer, x_bits: np.ndarray, ep_rank: int, ep_size: int) -> dict:
+def layer_forward_ep(layer: OracleLayer, x_bits: np.ndarray, ep_rank: int, ep_size: int, *,
+                     topk_override: Optional[dict] = None) -> dict:
     """One rank's share of the layer when its experts are split over ep_size
     ranks by e % ep_size (expert parallelism; the pages run all experts of a
     layer on one machine, so this split is a reading of how the layer shards).
@@ -285,12 +286,16 @@ def layer_forward_ep(layer: OracleLayer, x_bits: np.ndarray, ep_rank: int, ep_si
     does; rank r then adds only the pairs (t, j) whose expert idx[t, j]
     satisfies idx % ep_size == r, weighted by w[t, j], and rank 0 alone adds
     the shared expert.  Returns float64 ``partial`` [T, H] and the routing;
-    the sum of the partials over the ranks is layer_forward's ``out``."""
+    the sum of the partials over the ranks is layer_forward's ``out``.
+    ``topk_override`` replaces selections as in layer_forward."""
     if not (1 <= ep_size <= layer.experts and 0 <= ep_rank < ep_size):
         raise ValueError("need 1 <= ep_size <= experts and 0 <= ep_rank < ep_size")
     x = bf16_to_f64(x_bits)
     logits = router_logits(x, layer.router_w_bits, layer.router_bias)
     idx = select_topk(logits, layer.top_k)
+    if topk_override:
+        for t, sel in topk_override.items():
+            idx[t] = np.asarray(sel, dtype=np.int32)
     w = gate_weights(logits, idx)
     T = x.shape[0]
     partial = np.zeros((T, layer.hidden), dtype=np.float64)

@@ -57,6 +57,24 @@ def test_partials_sum_to_the_layer(ep_size):
             assert np.abs(p - full).max() > 1e-6 * scale
 
 
+def test_partials_follow_a_substituted_selection():
+    """A replaced selection (the tie-band substitution the GPU tests use) moves
+    the token's work to the new experts' owners: the partials still sum to the
+    layer computed with the same replacement, and differ from the original."""
+    lay = _tiny_layer()
+    x = mi.hidden_states_bf16(6, mi.TINY.hidden, seed=9)
+    base = orc.layer_forward(lay, x)
+    alt = base["idx"][2].copy()
+    alt[-1] = next(e for e in range(mi.TINY.experts) if e not in alt)   # swap the last pick
+    over = {2: alt}
+    full = orc.layer_forward(lay, x, topk_override=over)
+    parts = [orc.layer_forward_ep(lay, x, r, 3, topk_override=over)["partial"] for r in range(3)]
+    scale = np.abs(full["out"]).max()
+    np.testing.assert_allclose(sum(parts), full["out"], rtol=0, atol=1e-12 * scale)
+    assert np.abs(full["out"][2] - base["out"][2]).max() > 1e-6 * scale
+    np.testing.assert_array_equal(full["out"][[0, 1, 3, 4, 5]], base["out"][[0, 1, 3, 4, 5]])
+
+
 def test_rank_reads_only_its_experts():
     for ep_size in (2, 4):
         for r in range(ep_size):
