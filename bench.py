@@ -545,7 +545,7 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp16x2 dequant-dot + fp32 accumulate (bf16 activations, 4-bit codes)", "data": "synthetic",
+            "dtype": "int8 x int16 dp2a dot products (4-bit codes as signed bytes, int16 activations with a power-of-two scale per token), one fp32 fold per 32-element block, bf16 in/out", "data": "synthetic",
             "config": {"workload": "full-shape MoE layer decode (512 experts, H 2048, I 768, top-10 + shared, "
                                    "4-bit/32 fp16 scales), 16 tokens per step",
                        "tokens": T, "experts": 512, "hidden": 2048, "inter": 768, "top_k": 10, "shared": 1,
