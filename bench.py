@@ -30,7 +30,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 EXPERT_BYTES = {4: 2654208, 2: 1769472,     # packed gate/up + down of one expert (H=2048, I=768)
-                "4g128": 2433024}            # 4-bit with one fp16 scale per 128 elements
+                "4g128": 2433024,            # 4-bit with one fp16 scale per 128 elements
+                "4f8": 2521088}              # 4-bit, one E4M3 byte per 32 elements + an fp32 scale per row
 GU_BYTES = {4: 1769472, 2: 1179648}
 ROUTER_BYTES = 512 * 2048 * 2
 METRIC = "MoE-layer decode tokens/s (512 experts, top-10 + shared, H=2048, I=768, 4-bit/32, 16 tokens)"
@@ -87,7 +88,8 @@ def profiled_traffic(profile: str, sources) -> float | None:
 # and two lop3 per 8 weights; 2-bit: three shifts and four lop3 per 16), and
 # per token the dp2a dot products (two products each) plus the fold of each
 # block's integer sum (I2F + FFMA per 32 / 16 weights).
-ALU_OPS = {4: (3 / 8, 0.5 + 2 / 32), 2: (7 / 16, 0.5 + 2 / 16), "4g128": (3 / 8, 0.5 + 2 / 128)}
+ALU_OPS = {4: (3 / 8, 0.5 + 2 / 32), 2: (7 / 16, 0.5 + 2 / 16), "4g128": (3 / 8, 0.5 + 2 / 128),
+           "4f8": (3 / 8, 0.5 + 2 / 32)}
 WEIGHTS_PER_EXPERT = 3 * 2048 * 768
 ST_PATH = 3        # status word of the workspace: 1 when the tensor-core kernels ran the call
 
@@ -632,6 +634,13 @@ def detail(R, args, pool4, ws, W, hbm_peak, tf_peak, dist, world, clock_mhz=None
     poolh = R.layers(sh2, 8)
     layer_rate(cfg_h, sh2, poolh, 16, 2000, 2, "decode2h_t16")
     del poolh
+    # 4-bit with one E4M3 scale byte per 32 elements and an fp32 scale per row
+    # (the stand-alone GEMV kernels; 8 layer instances: 10.4 GB, far above L2)
+    sf8 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=32, fp8_scales=True)
+    cfg_f8 = q.config_of(512, 2048, 768, 10, True, 4, 32, fp8_scales=True)
+    poolf8 = R.layers(sf8, 8)
+    layer_rate(cfg_f8, sf8, poolf8, 16, 2000, "4f8", "decode4f8_t16")
+    del poolf8
     layer_rate(cfg, shape, pool4, 4096, 8, 4, "prefill4_t4096")
 
     # expert-parallel share: one rank's partial of the 4096-token layer when

@@ -78,6 +78,17 @@ typedef struct moe_config {
                             2-bit ternary); 1: q = c - (2^bits-1)/2,
                             the 2^bits half-integer levels (2-bit:
                             four levels +-1/2, +-3/2)              */
+  int32_t scale_fmt;     /* 0: one fp16 scale per block; 1: one E4M3
+                            (fp8: sign, 4 exponent bits with bias 7,
+                            3 mantissa bits, no infinities, largest
+                            finite 448) byte per block, times one
+                            fp32 scale per weight row (the
+                            *_row_scales arrays); block 32 (4-bit) or
+                            16 (2-bit) only.  Layers with fp8 scales
+                            run on the stand-alone GEMV kernels at
+                            every batch size (neither the
+                            single-launch decode kernel nor the
+                            tensor-core prefill reads them).       */
 } moe_config;
 
 /* One layer's weights; every pointer is device memory owned by the caller. */
@@ -98,6 +109,14 @@ typedef struct moe_layer_weights {
                                              shared expert.  Layers with a gate
                                              run on the separate kernels, not
                                              the single-launch decode kernel.  */
+  /* scale_fmt = 1 only (NULL otherwise): the *_scales arrays above then hold
+   * one E4M3 byte per block (same shapes, one byte per element instead of
+   * two), and the weight of element j of row r is q * e4m3(scale byte) *
+   * row_scale[r].  fp32, 4-byte aligned. */
+  const float*    gate_up_row_scales;     /* [E][2I]                            */
+  const float*    down_row_scales;        /* [E][H]                             */
+  const float*    shared_gate_up_row_scales;  /* [2I]; NULL if no shared        */
+  const float*    shared_down_row_scales;     /* [H]                            */
 } moe_layer_weights;
 
 /* Bytes of device workspace needed by moe_route / moe_layer_forward /
@@ -195,9 +214,17 @@ int moe_device_status(const void* workspace, int32_t* code_out);
 
 /* Test hook: rows [row0, row0+rows) of a packed matrix with `cols` columns,
  * decoded by the same device routine the GEMV kernels use, written as fp32
- * out[rows][cols].  Not on the timed path. */
+ * out[rows][cols].  Not on the timed path.  scale_fmt 0 only; fp8 scales go
+ * through moe_dequant_rows_scaled. */
 int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t* scales,
                      int32_t row0, int32_t rows, int32_t cols, float* out, void* stream);
+
+/* The same for either scale format: with cfg->scale_fmt = 1, `scales` holds
+ * one E4M3 byte per block and row_scales (device, fp32, indexed by the row of
+ * the matrix) is required; with 0 it must be NULL. */
+int moe_dequant_rows_scaled(const moe_config* cfg, const uint8_t* codes, const void* scales,
+                            const float* row_scales, int32_t row0, int32_t rows, int32_t cols, float* out,
+                            void* stream);
 
 /* Measurement hook.  moe_profile_begin(n) makes the next n layer calls
  * record CUDA events around their four phases on the call's stream (route,

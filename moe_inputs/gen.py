@@ -83,6 +83,7 @@ class MoeShape:
     bits: int
     block: int
     half: bool = False          # half-integer levels (2**bits levels, no zero)
+    fp8_scales: bool = False    # E4M3 block scales under one fp32 scale per row
 
     @property
     def qmax(self) -> int:
@@ -193,6 +194,70 @@ def quantize_blocks(w: np.ndarray, bits: int, block: int, half: bool = False):
     return np.ascontiguousarray(codes), np.ascontiguousarray(s16.view(np.uint16))
 
 
+E4M3_MAX = 448.0
+
+
+def e4m3_encode(t: np.ndarray) -> np.ndarray:
+    """Nearest E4M3 byte (ties to even, saturating at 448) of non-negative
+    fp32 values: 4 exponent bits with bias 7, 3 mantissa bits, exponent field
+    0 for the subnormals m * 2**-9.  Input preparation only."""
+    t = np.asarray(t, dtype=np.float32)
+    out = np.zeros(t.shape, dtype=np.uint8)
+    sub = t < np.float32(2.0 ** -6)
+    m_sub = np.rint(t[sub] * np.float32(512.0)).astype(np.int32)     # exact scaling; 8 -> 2**-6, code 8
+    out[sub] = m_sub.astype(np.uint8)
+    nt = t[~sub]
+    mant, ex = np.frexp(nt)                                            # nt = mant * 2**ex, mant in [0.5, 1)
+    e = ex.astype(np.int32) - 1
+    m = np.rint((mant * np.float32(2.0) - np.float32(1.0)) * np.float32(8.0)).astype(np.int32)
+    carry = m == 8
+    e = e + carry
+    m = np.where(carry, 0, m)
+    code = ((e + 7) << 3) | m
+    out[~sub] = np.minimum(code, 0x7E).astype(np.uint8)
+    return out
+
+
+def _e4m3_f32(code: np.ndarray) -> np.ndarray:
+    """fp32 value of non-negative E4M3 codes (the encoder's own view of what it
+    chose)."""
+    code = np.asarray(code, dtype=np.int32)
+    e, m = (code >> 3) & 15, code & 7
+    val = np.where(e == 0, m * 2.0 ** -9, (8 + m) * np.exp2(e.astype(np.float64) - 10))
+    return val.astype(np.float32)
+
+
+def quantize_blocks_e4m3(w: np.ndarray, bits: int, block: int):
+    """Encode fp32 masters [rows, cols] with integer levels, one E4M3 scale
+    byte per block and one fp32 scale per row: S = rowmax|w| / (qmax * 448),
+    scale byte = e4m3(blockmax|w| / (qmax * S)), q = clamp(rint(w / (e4m3 * S))).
+    Returns (codes uint8 [rows, cols*bits/8], scale bytes uint8
+    [rows, cols/block], row scales float32 [rows]).  Input preparation only."""
+    w = np.asarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    assert cols % block == 0 and bits in (2, 4)
+    qmax = (1 << (bits - 1)) - 1
+    wb = w.reshape(rows, cols // block, block)
+    amax = np.max(np.abs(wb), axis=-1)                                  # [rows, nb]
+    rmax = np.max(amax, axis=-1)                                        # [rows]
+    S = (rmax / np.float32(qmax * E4M3_MAX)).astype(np.float32)
+    den = (S * np.float32(qmax)).astype(np.float32)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        t = np.where(den[:, None] > 0, amax / np.where(den > 0, den, np.float32(1))[:, None], 0).astype(np.float32)
+    s8 = e4m3_encode(t)
+    sf = (_e4m3_f32(s8) * S[:, None]).astype(np.float32)
+    safe = np.where(sf == 0, np.float32(1), sf)
+    ratio = (wb / safe[..., None]).astype(np.float32)
+    q = np.clip(np.rint(ratio), -qmax, qmax)
+    q[sf == 0] = 0
+    c = (q.astype(np.int32) + (1 << (bits - 1))).astype(np.uint8).reshape(rows, cols)
+    if bits == 4:
+        codes = (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+    else:
+        codes = (c[:, 0::4] | (c[:, 1::4] << 2) | (c[:, 2::4] << 4) | (c[:, 3::4] << 6)).astype(np.uint8)
+    return np.ascontiguousarray(codes), np.ascontiguousarray(s8), np.ascontiguousarray(S)
+
+
 def masters(shape: MoeShape, seed: int, layer: int, expert: int):
     """fp32 masters (gate [I,H], up [I,H], down [H,I]) of routed expert
     ``expert`` (0 <= expert < E) or of the shared expert (expert == -1)."""
@@ -211,11 +276,18 @@ def expert_packed(shape: MoeShape, seed: int, layer: int, expert: int):
     """Packed (gu_codes, gu_scales, d_codes, d_scales) of one expert.
 
     gu_codes [2I, H*bits/8] uint8, gu_scales [2I, H/block] fp16 bits,
-    d_codes [H, I*bits/8] uint8, d_scales [H, I/block] fp16 bits."""
+    d_codes [H, I*bits/8] uint8, d_scales [H, I/block] fp16 bits.  With
+    fp8 scales: gu_scales / d_scales are E4M3 bytes and two more arrays
+    follow, the fp32 row scales gu_rs [2I] and d_rs [H]."""
     g, u, d = masters(shape, seed, layer, expert)
     w13 = np.empty((2 * shape.inter, shape.hidden), dtype=np.float32)
     w13[0::2] = g
     w13[1::2] = u
+    if shape.fp8_scales:
+        assert not shape.half, "fp8 block scales come with the integer levels"
+        gc, gs, grs = quantize_blocks_e4m3(w13, shape.bits, shape.block)
+        dc, ds, drs = quantize_blocks_e4m3(d, shape.bits, shape.block)
+        return gc, gs, dc, ds, grs, drs
     gc, gs = quantize_blocks(w13, shape.bits, shape.block, shape.half)
     dc, ds = quantize_blocks(d, shape.bits, shape.block, shape.half)
     return gc, gs, dc, ds
@@ -260,6 +332,6 @@ def layer_packed_pool(shape: MoeShape, seed: int, layer: int):
     """Whole-layer packed pool on the host (small shapes only): arrays with a
     leading expert axis, plus the shared expert's arrays (or None)."""
     parts = [expert_packed(shape, seed, layer, e) for e in range(shape.experts)]
-    pool = tuple(np.stack([p[i] for p in parts]) for i in range(4))
+    pool = tuple(np.stack([p[i] for p in parts]) for i in range(len(parts[0])))
     sh = shared_packed(shape, seed, layer) if shape.shared else None
     return pool, sh

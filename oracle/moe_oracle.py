@@ -30,8 +30,13 @@ element in the lower bits of each byte; packed gate/up rows interleave (row
 2i gate i, row 2i+1 up i); in the 48-layer stack each layer is
 ``x <- bf16(x + moe(bf16(rmsnorm(x))))`` with RMSNorm weight 1, eps 1e-6.
 
+Format variants (readings of the pages' grouped symmetric quantiser): codes
+read as half-integer levels ``q = c - (2**bits - 1)/2``; one E4M3 (fp8) scale
+byte per block under one fp32 scale per weight row.
+
 Precision: everything is float64 except what the interface fixes: bf16 at the
-hidden states, the RMSNorm output and the stack's residual stream, fp16 scales.
+hidden states, the RMSNorm output and the stack's residual stream, fp16 (or
+E4M3 times fp32) scales.
 
 Pins (tests/test_oracle_*.py): hand-decoded bytes of the format
 (tests/golden/format_blocks.txt), the round-trip bound of the block encoder,
@@ -40,7 +45,10 @@ gate weights, brute-force stable grouping, the dense-SwiGLU identity of an
 E=1, k=1 layer against an independent element-by-element evaluation, a hand
 computed SwiGLU example (tests/golden/swiglu_tiny.txt), linearity in the down
 weights, permutation invariance of expert storage, the RMSNorm closed form on
-constant vectors and exact bf16 rounding cases.
+constant vectors and exact bf16 rounding cases; the stack against an
+element-by-element restatement; the half-integer levels and the E4M3 scales
+against hand-decoded bytes (tests/golden/format_blocks_half.txt,
+tests/golden/format_blocks_fp8.txt) and the format's printed values.
 """
 
 from __future__ import annotations
@@ -53,7 +61,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "bf16_to_f64", "round_bf16", "unpack_codes", "dequantize", "router_logits",
+    "bf16_to_f64", "round_bf16", "unpack_codes", "e4m3_value", "dequantize", "router_logits",
     "select_topk", "gate_weights", "group_by_expert", "silu", "swiglu_ffn",
     "rmsnorm_bf16", "OracleLayer", "layer_forward", "layer_forward_ep", "stack_forward",
     "tie_band_ok", "RMS_EPS",
@@ -90,16 +98,39 @@ def unpack_codes(codes: np.ndarray, bits: int, n: int) -> np.ndarray:
     return (byte >> ((j * bits) % 8)) & ((1 << bits) - 1)
 
 
+def e4m3_value(code) -> np.ndarray:
+    """float64 value of E4M3 bytes (the OCP 8-bit floating-point format with
+    4 exponent bits and 3 mantissa bits): sign s = bit 7, exponent field
+    e = bits 3..6 with bias 7, mantissa m = bits 0..2; e = 0 encodes the
+    subnormals (-1)**s * m/8 * 2**-6, otherwise (-1)**s * (1 + m/8) * 2**(e-7);
+    the pattern e = 15, m = 7 is NaN (there are no infinities), so the largest
+    finite value is 1.75 * 2**8 = 448."""
+    c = np.asarray(code, dtype=np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
 def dequantize(codes: np.ndarray, scales_bits: np.ndarray, rows: int, cols: int,
-               bits: int, block: int, half: bool = False) -> np.ndarray:
+               bits: int, block: int, half: bool = False, row_scale: Optional[np.ndarray] = None) -> np.ndarray:
     """Weights w[r, c] = q * scale[r, c // block] in float64, q = code -
     2**(bits-1) (integer levels), or q = code - (2**bits - 1) / 2 for the
     half-integer levels (2**bits levels symmetric about zero, e.g. +-1/2,
     +-3/2 for 2 bits).  Exact: a small integer or half-integer times an fp16
-    value."""
+    value.  With ``row_scale`` (fp32 [rows]) the block scales are E4M3 bytes
+    and scale[r, b] = e4m3(byte) * row_scale[r] (fp8 block scales under one
+    fp32 scale per row), again exact in float64."""
     codes = np.asarray(codes, dtype=np.uint8).reshape(rows, cols * bits // 8)
-    scales = np.asarray(scales_bits, dtype=np.uint16).view(np.float16)
-    scales = scales.reshape(rows, cols // block).astype(np.float64)
+    if row_scale is None:
+        scales = np.asarray(scales_bits, dtype=np.uint16).view(np.float16)
+        scales = scales.reshape(rows, cols // block).astype(np.float64)
+    else:
+        sb = np.asarray(scales_bits, dtype=np.uint8).reshape(rows, cols // block)
+        rsf = np.asarray(row_scale, dtype=np.float32).reshape(rows).astype(np.float64)
+        scales = e4m3_value(sb) * rsf[:, None]
     offset = ((1 << bits) - 1) / 2.0 if half else float(1 << (bits - 1))
     w = np.empty((rows, cols), dtype=np.float64)
     for r in range(rows):
@@ -198,7 +229,9 @@ class OracleLayer:
 
     ``expert(e)`` returns (gu_codes [2I, H*b/8], gu_scales [2I, H/bs] fp16
     bits, d_codes [H, I*b/8], d_scales [H, I/bs]); ``shared()`` the same for
-    the shared expert or None."""
+    the shared expert or None.  With fp8 block scales the scales are E4M3
+    bytes and the tuples carry two more arrays, the fp32 row scales
+    (gu_row_scale [2I], d_row_scale [H])."""
     experts: int
     hidden: int
     inter: int
@@ -219,10 +252,12 @@ class OracleLayer:
     def _dense(self, key, packed):
         if key in self._cache:
             return self._cache[key]
-        gc, gs, dc, ds = packed()
+        arrays = packed()
+        gc, gs, dc, ds = arrays[:4]
+        grs, drs = arrays[4:6] if len(arrays) == 6 else (None, None)
         H, I = self.hidden, self.inter
-        w13 = dequantize(gc, gs, 2 * I, H, self.bits, self.block, self.half_levels)
-        wd = dequantize(dc, ds, H, I, self.bits, self.block, self.half_levels)
+        w13 = dequantize(gc, gs, 2 * I, H, self.bits, self.block, self.half_levels, row_scale=grs)
+        wd = dequantize(dc, ds, H, I, self.bits, self.block, self.half_levels, row_scale=drs)
         dense = (w13[0::2], w13[1::2], wd)
         if len(self._cache) >= self.cache_size:
             self._cache.pop(next(iter(self._cache)))

@@ -19,7 +19,8 @@ from typing import Optional, Sequence
 __all__ = [
     "MoeConfig", "LayerWeights", "MoeError", "load_library", "EXPORTS", "LIB_PATH",
     "moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_forward",
-    "moe_device_status", "moe_dequant_rows", "moe_status_str", "config_of", "moe_profile_begin",
+    "moe_device_status", "moe_dequant_rows", "moe_dequant_rows_scaled", "moe_status_str", "config_of",
+    "moe_profile_begin",
     "moe_profile_end", "moe_layer_forward_noalloc", "moe_noalloc_device_status", "NOALLOC_SCRATCH_BYTES",
     "moe_layer_forward_ep", "ep_all_reduce",
 ]
@@ -30,7 +31,7 @@ EXPORTS = ("moe_workspace_bytes", "moe_route", "moe_layer_forward", "moe_stack_f
            "moe_device_status", "moe_dequant_rows", "moe_status_str", "moe_profile_begin", "moe_profile_end",
            "moe_layer_forward_noalloc", "moe_last_cuda_error", "moe_debug_fused_timing",
            "moe_debug_prefill_timing", "moe_layer_forward_ep", "moe_debug_decode_path", "moe_debug_wait_probe",
-           "moe_noalloc_device_status")
+           "moe_noalloc_device_status", "moe_dequant_rows_scaled")
 
 MOE_OK = 0
 
@@ -45,20 +46,22 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int32), ("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("shared_inter", ctypes.c_int32), ("bits", ctypes.c_int32),
-                ("block", ctypes.c_int32), ("half_levels", ctypes.c_int32)]
+                ("block", ctypes.c_int32), ("half_levels", ctypes.c_int32), ("scale_fmt", ctypes.c_int32)]
 
 
 class _Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "gate_up_codes", "gate_up_scales", "down_codes", "down_scales", "shared_gate_up_codes",
         "shared_gate_up_scales", "shared_down_codes", "shared_down_scales", "router_w", "router_bias",
-        "shared_gate_w")]
+        "shared_gate_w", "gate_up_row_scales", "down_row_scales", "shared_gate_up_row_scales",
+        "shared_down_row_scales")]
 
 
 @dataclasses.dataclass
 class LayerWeights:
     """Device tensors of one layer (layouts in include/moe_capi.h).  Scales and
-    bf16 tensors may be any 16-bit dtype; only the bytes matter."""
+    bf16 tensors may be any dtype of the right element size (fp16 scales 16-bit,
+    E4M3 scales 8-bit); only the bytes matter."""
     gate_up_codes: object
     gate_up_scales: object
     down_codes: object
@@ -70,6 +73,10 @@ class LayerWeights:
     shared_down_codes: Optional[object] = None
     shared_down_scales: Optional[object] = None
     shared_gate_w: Optional[object] = None      # [H] bf16: shared expert weighted by sigmoid(x . w)
+    gate_up_row_scales: Optional[object] = None          # fp8 block scales: fp32 [E][2I]
+    down_row_scales: Optional[object] = None             # fp32 [E][H]
+    shared_gate_up_row_scales: Optional[object] = None   # fp32 [2I]
+    shared_down_row_scales: Optional[object] = None      # fp32 [H]
 
     def to_c(self) -> _Weights:
         w = _Weights()
@@ -106,6 +113,8 @@ def load_library(path: str = LIB_PATH):
     lib.moe_device_status.restype = ctypes.c_int
     lib.moe_dequant_rows.argtypes = [cfgp, P, P, I32, I32, I32, P, P]
     lib.moe_dequant_rows.restype = ctypes.c_int
+    lib.moe_dequant_rows_scaled.argtypes = [cfgp, P, P, P, I32, I32, I32, P, P]
+    lib.moe_dequant_rows_scaled.restype = ctypes.c_int
     lib.moe_layer_forward_noalloc.argtypes = [cfgp, ctypes.POINTER(_Weights), P, I32, P, P]
     lib.moe_layer_forward_noalloc.restype = ctypes.c_int
     lib.moe_noalloc_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -152,8 +161,9 @@ def _check(st: int, what: str):
         raise MoeError(st, what)
 
 
-def config_of(experts, hidden, inter, top_k, shared, bits, block, half_levels=False) -> MoeConfig:
-    return MoeConfig(experts, hidden, inter, top_k, inter if shared else 0, bits, block, 1 if half_levels else 0)
+def config_of(experts, hidden, inter, top_k, shared, bits, block, half_levels=False, fp8_scales=False) -> MoeConfig:
+    return MoeConfig(experts, hidden, inter, top_k, inter if shared else 0, bits, block, 1 if half_levels else 0,
+                     1 if fp8_scales else 0)
 
 
 def moe_status_str(status: int) -> str:
@@ -260,6 +270,15 @@ def moe_dequant_rows(cfg: MoeConfig, codes, scales, row0: int, rows: int, cols: 
                                          _ptr(out), _stream(stream))
     if check:
         _check(st, "moe_dequant_rows")
+    return st
+
+
+def moe_dequant_rows_scaled(cfg: MoeConfig, codes, scales, row_scales, row0: int, rows: int, cols: int, out, *,
+                            stream=None, check=True) -> int:
+    st = load_library().moe_dequant_rows_scaled(ctypes.byref(cfg), _ptr(codes), _ptr(scales), _ptr(row_scales),
+                                                row0, rows, cols, _ptr(out), _stream(stream))
+    if check:
+        _check(st, "moe_dequant_rows_scaled")
     return st
 
 

@@ -10,15 +10,16 @@
 // brief": compute isn't the blocker).
 //
 // Design: every CTA takes an equal contiguous share of all (expert, row-group)
-// work units, so HBM bytes are balanced across SMs.  A warp holds the packed
-// bytes of RW x 2 rows in registers (128-bit read-only loads, each 16-byte
-// piece being one 4-bit block of 32 or four 2-bit blocks of 16), decodes them
-// to exact small integers in fp16, multiplies with the activation vector
-// staged in shared memory as fp16 (pre-scaled per token by a power of two so
-// that block partial sums cannot overflow), accumulates each block in fp16x2
-// and the blocks in fp32 with the block's fp16 scale, then reduces across the
+// work units, so HBM bytes are balanced across SMs.  A producer warp streams
+// each stage's packed rows and scales into a shared-memory ring with 1-D bulk
+// copies; the consumer warps turn each code field into a signed byte (16 q or
+// 64 q), multiply with the activations staged in shared memory as int16
+// (scaled per token by a power of two) with dp2a, sum each block exactly in
+// int32 and the blocks in fp32 with the block's scale, then reduce across the
 // lanes of the row with shuffles.  No atomics: every output element is written
-// once.
+// once.  This kernel also serves the formats the single-launch decode kernel
+// leaves out: 4-bit blocks of 128 and fp8 (E4M3) block scales with an fp32
+// scale per row.
 #include "decode_common.cuh"
 
 namespace moe {
@@ -29,9 +30,12 @@ using namespace gemv;
 
 struct FfnArgs {
   const uint8_t* codes;          // routed pool
-  const uint16_t* scales;
+  const unsigned char* scales;   // fp16 or (sf = 1) E4M3 block scales
   const uint8_t* sh_codes;       // shared expert (or null)
-  const uint16_t* sh_scales;
+  const unsigned char* sh_scales;
+  const float* row_scales;       // sf = 1: fp32 scale per row of each routed expert
+  const float* sh_row_scales;    // sf = 1: of the shared expert
+  int sf;                        // scale format: 0 fp16, 1 E4M3 + row scale
   size_t expert_code_bytes;      // per routed expert
   size_t expert_scale_count;
   int rows;                      // rows per expert (2I gate/up, H down)
@@ -104,8 +108,9 @@ struct Cursor {
   }
 };
 
-template <int MODE, int BITS, int LPR, int CPL, int PS>
+template <int MODE, int BITS, int LPR, int CPL, int PS, int SF>
 __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
+  constexpr int SSZ = SF ? 1 : 2;               // bytes per block scale
   using Gm = Geom<BITS, LPR, CPL>;
   constexpr int K = Gm::K;
   constexpr int NTB = 4;                        // tokens per register block
@@ -164,15 +169,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
         }
         const bool sh = cur.e >= rv.E;
         const uint8_t* cb = sh ? a.sh_codes : a.codes + size_t(cur.e) * a.expert_code_bytes;
-        const uint16_t* sb = sh ? a.sh_scales : a.scales + size_t(cur.e) * a.expert_scale_count;
+        const unsigned char* sb = sh ? a.sh_scales : a.scales + size_t(cur.e) * a.expert_scale_count * SSZ;
         const size_t row0 = size_t(cur.stage) * Gm::RPS;
         unsigned char* dst = ring + slot * Gm::STAGE_BYTES;
         const int spr = scales_per_row(Gm::K, a.block);
-        const uint32_t sbytes = uint32_t(Gm::RPS) * spr * 2;
+        const uint32_t sbytes = uint32_t(Gm::RPS) * spr * SSZ;
         mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes);
         const uint64_t pol = l2_evict_first_policy();      // weight bytes are read once
         bulk_g2s_hint(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot], pol);
-        bulk_g2s_hint(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot], pol);
+        bulk_g2s_hint(dst + Gm::CODE_BYTES, sb + row0 * spr * SSZ, sbytes, &full[slot], pol);
         ++issued;
       }
       // never leave with copies in flight
@@ -267,14 +272,19 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
     }
     if (ok) {
       const unsigned char* st = ring + slot * Gm::STAGE_BYTES;
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0,
-                      a.xk};
+      Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * SSZ, cur.stage * Gm::RPS + rl0,
+                a.xk};
+      if (SF) {
+        const float* rsb = cur.e >= rv.E ? a.sh_row_scales : a.row_scales + size_t(cur.e) * a.rows;
+        rows.rs0 = __ldg(rsb + rows.r0);
+        rows.rs1 = __ldg(rsb + rows.r0 + 1);
+      }
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += NTB) {
         const int nt = min(NTB, nc - tb);          // warp-uniform
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 1);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 2);
-        else rows_dot<MODE, BITS, LPR, CPL, 4, PS>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS, SF>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 1);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS, SF>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, 2);
+        else rows_dot<MODE, BITS, LPR, CPL, 4, PS, SF>(a.out, a.out_cols, rows, xs + size_t(tb) * K, tb, lr, tok_inv, tok_w, tok_pos, nt);
       }
     }
     __syncwarp();
@@ -284,11 +294,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_tma_kernel(FfnArgs a) {
 
 // --------------------------------------------------------- dequant hook
 // Writes out[r][j] = q * scale for rows row0.. of a packed matrix, with the
-// byte decoders the GEMV uses (q4_bytes / q2_bytes: signed bytes 16 q or
-// 64 q); test hook, not on the timed path.
-template <int BITS>
-__global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
-                                    int row0, int rows, int cols, int BLOCK, uint32_t xk, float* __restrict__ out) {
+// byte and scale decoders the GEMV uses (q4_bytes / q2_bytes: signed bytes
+// 16 q or 64 q; fp16 or E4M3 scales, the latter times the row's fp32 scale:
+// q * e4m3 is exact, so the product is rounded once); test hook, not on the
+// timed path.
+template <int BITS, int SF>
+__global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const unsigned char* __restrict__ scales,
+                                    const float* __restrict__ row_scales, int row0, int rows, int cols, int BLOCK,
+                                    uint32_t xk, float* __restrict__ out) {
   constexpr int G = BITS == 4 ? 8 : 16;
   const int words_per_row = cols / G;
   const long long total = (long long)rows * words_per_row;
@@ -310,8 +323,13 @@ __global__ void dequant_rows_kernel(const uint8_t* __restrict__ codes, const uin
       const uint32_t word = BITS == 4 ? f[j & 1] : f[j & 3];
       const int byte = BITS == 4 ? (j >> 1) : (j >> 2);
       const int qb = int(int8_t(uint8_t(word >> (8 * byte))));
-      const float sc = __half2float(__ushort_as_half(scales[row * (cols / BLOCK) + col / BLOCK]));
-      out[size_t(r) * cols + col] = ldexpf(float(qb), -CodeMul<BITS>::kLog2) * sc;
+      const size_t si = row * (cols / BLOCK) + col / BLOCK;
+      if (SF) {
+        out[size_t(r) * cols + col] = (ldexpf(float(qb), -CodeMul<BITS>::kLog2) * e4m3_value(scales[si])) * row_scales[row];
+      } else {
+        const float sc = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(scales)[si]));
+        out[size_t(r) * cols + col] = ldexpf(float(qb), -CodeMul<BITS>::kLog2) * sc;
+      }
     }
   }
 }
@@ -326,10 +344,10 @@ PassPlan plan_of(int rows, int K) {
   return p;
 }
 
-template <int MODE, int BITS, int LPR, int CPL, int PS>
+template <int MODE, int BITS, int LPR, int CPL, int PS, int SF>
 cudaError_t launch_one(FfnArgs fa, int num_sms, cudaStream_t s) {
   using Gm = Geom<BITS, LPR, CPL>;
-  auto kern = ffn_tma_kernel<MODE, BITS, LPR, CPL, PS>;
+  auto kern = ffn_tma_kernel<MODE, BITS, LPR, CPL, PS, SF>;
   const size_t smem = 256 + size_t(kStages) * Gm::STAGE_BYTES + size_t(fa.ntc) * Gm::K * 2 + kMaxNTC * 12;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -348,9 +366,10 @@ cudaError_t dispatch(int K, FfnArgs fa, int num_sms, cudaStream_t s) {
 #define X(c, lpr, cpl)                                                              \
   case c:                                                                           \
     if constexpr (BITS == 4) {                                                      \
-      if (fa.block == 128) return launch_one<MODE, BITS, lpr, cpl, 2>(fa, num_sms, s); \
+      if (fa.block == 128) return launch_one<MODE, BITS, lpr, cpl, 2, 0>(fa, num_sms, s); \
     }                                                                               \
-    return launch_one<MODE, BITS, lpr, cpl, 0>(fa, num_sms, s);
+    if (fa.sf) return launch_one<MODE, BITS, lpr, cpl, 0, 1>(fa, num_sms, s);       \
+    return launch_one<MODE, BITS, lpr, cpl, 0, 0>(fa, num_sms, s);
     MOE_C_CASES(X)
 #undef X
     default: return cudaErrorInvalidValue;
@@ -398,8 +417,10 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   rv.topk_w = reinterpret_cast<const float*>(a.ws + a.L.topk_w);
 
   FfnArgs g{};
-  g.codes = a.w.gate_up_codes; g.scales = a.w.gate_up_scales;
-  g.sh_codes = a.w.shared_gate_up_codes; g.sh_scales = a.w.shared_gate_up_scales;
+  g.codes = a.w.gate_up_codes; g.scales = reinterpret_cast<const unsigned char*>(a.w.gate_up_scales);
+  g.sh_codes = a.w.shared_gate_up_codes;
+  g.sh_scales = reinterpret_cast<const unsigned char*>(a.w.shared_gate_up_scales);
+  g.sf = c.scale_fmt; g.row_scales = a.w.gate_up_row_scales; g.sh_row_scales = a.w.shared_gate_up_row_scales;
   g.expert_code_bytes = size_t(2 * I) * H * bits / 8;
   g.expert_scale_count = size_t(2 * I) * (H / c.block);
   g.rows = 2 * I; g.out_cols = I; g.ntc = pg.ntc; g.block = c.block; g.xk = code_xor(bits, c.half_levels);
@@ -414,8 +435,9 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   if (between) cudaEventRecord(between, a.stream);
 
   FfnArgs d{};
-  d.codes = a.w.down_codes; d.scales = a.w.down_scales;
-  d.sh_codes = a.w.shared_down_codes; d.sh_scales = a.w.shared_down_scales;
+  d.codes = a.w.down_codes; d.scales = reinterpret_cast<const unsigned char*>(a.w.down_scales);
+  d.sh_codes = a.w.shared_down_codes; d.sh_scales = reinterpret_cast<const unsigned char*>(a.w.shared_down_scales);
+  d.sf = c.scale_fmt; d.row_scales = a.w.down_row_scales; d.sh_row_scales = a.w.shared_down_row_scales;
   d.expert_code_bytes = size_t(H) * I * bits / 8;
   d.expert_scale_count = size_t(H) * (I / c.block);
   d.rows = H; d.out_cols = H; d.ntc = pd.ntc; d.block = c.block; d.xk = code_xor(bits, c.half_levels);
@@ -427,15 +449,22 @@ cudaError_t launch_decode_ffn(const LayerArgs& a, cudaEvent_t between) {
   return bits == 4 ? dispatch<DOWN, 4>(I, d, a.num_sms, a.stream) : dispatch<DOWN, 2>(I, d, a.num_sms, a.stream);
 }
 
-cudaError_t launch_dequant_rows(int bits, int block, int half_levels, const uint8_t* codes, const uint16_t* scales,
-                                int row0, int rows, int cols, float* out, cudaStream_t s) {
+cudaError_t launch_dequant_rows(int bits, int block, int half_levels, int scale_fmt, const uint8_t* codes,
+                                const void* scales, const float* row_scales, int row0, int rows, int cols,
+                                float* out, cudaStream_t s) {
   const int G = bits == 4 ? 8 : 16;
   const long long total = (long long)rows * (cols / G);
   const long long want = (total + 255) / 256;
   const int blocks = int(want < 4096 ? want : 4096);
   const uint32_t xk = code_xor(bits, half_levels);
-  if (bits == 4) dequant_rows_kernel<4><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, xk, out);
-  else dequant_rows_kernel<2><<<blocks, 256, 0, s>>>(codes, scales, row0, rows, cols, block, xk, out);
+  const unsigned char* sc = static_cast<const unsigned char*>(scales);
+  if (bits == 4) {
+    if (scale_fmt) dequant_rows_kernel<4, 1><<<blocks, 256, 0, s>>>(codes, sc, row_scales, row0, rows, cols, block, xk, out);
+    else dequant_rows_kernel<4, 0><<<blocks, 256, 0, s>>>(codes, sc, row_scales, row0, rows, cols, block, xk, out);
+  } else {
+    if (scale_fmt) dequant_rows_kernel<2, 1><<<blocks, 256, 0, s>>>(codes, sc, row_scales, row0, rows, cols, block, xk, out);
+    else dequant_rows_kernel<2, 0><<<blocks, 256, 0, s>>>(codes, sc, row_scales, row0, rows, cols, block, xk, out);
+  }
   return cudaGetLastError();
 }
 

@@ -117,13 +117,24 @@ __device__ __forceinline__ int staged_offset(int h) {
   return ((((s * 4 + m) * Gm::NPART + part) * LPR + lr) << 3) + within;
 }
 
+// Value of an E4M3 byte (sign, 4 exponent bits with bias 7, 3 mantissa bits;
+// exponent field 0 holds the subnormals m * 2^-9), exact in fp32.  The
+// encoder never writes the two NaN codes (0x7F, 0xFF).
+__device__ __forceinline__ float e4m3_value(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  const float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : float(m) * 0.001953125f;
+  return (b & 0x80u) ? -mag : mag;
+}
+
 // Two rows of one stage (codes + scales in shared memory) and their row index
-// in the expert matrix.
+// in the expert matrix.  With fp8 block scales (SF = 1 below) a scale is one
+// E4M3 byte and the rows carry their fp32 row scales rs0, rs1.
 struct Rows {
   const unsigned char* codes;     // row rl0; row rl0+1 follows at +RB
-  const unsigned char* scales;    // row rl0; row rl0+1 follows at +(SPR >> PS)*2
+  const unsigned char* scales;    // row rl0; row rl0+1 follows at +(SPR >> PS) scales
   int r0;
   uint32_t xk;                    // code_xor of the format
+  float rs0 = 1.f, rs1 = 1.f;     // fp8 block scales only: the rows' fp32 scales
 };
 
 // Scales per row, and the piece-to-scale shift PS of a 4-bit block of 32
@@ -137,9 +148,10 @@ __host__ __device__ inline int piece_shift(int bits, int block) { return bits ==
 // turns the codes into signed bytes (q4_bytes / q2_bytes) and runs dp2a
 // against the int16 activations (two independent int32 chains per row and
 // token); each block's exact integer sum is converted to fp32 and multiplied
-// by the block's fp16 scale.  `nt` <= NT tokens are valid; xs holds int16
-// activations staged with staged_offset.
-template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0>
+// by the block's scale (fp16, or with SF = 1 an E4M3 byte, the row's fp32
+// scale then applied once per output).  `nt` <= NT tokens are valid; xs holds
+// int16 activations staged with staged_offset.
+template <int MODE, int BITS, int LPR, int CPL, int NT, int PS = 0, int SF = 0>
 __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& rw, const int16_t* xs, int tb, int lr,
                                          const float* tok_inv, const float* tok_w, const int* tok_pos,
                                          int nt = NT, const int* xrow = nullptr) {
@@ -170,7 +182,8 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
       float sc[2];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
-        sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * (Gm::SPR >> PS) * 2 + (c >> PS) * 2));
+        sc[rho] = SF ? e4m3_value(rw.scales[rho * (Gm::SPR >> PS) + (c >> PS)])
+                     : __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * (Gm::SPR >> PS) * 2 + (c >> PS) * 2));
       int ia[2][NT], ib[2][NT];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
@@ -199,9 +212,12 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[rho][t] = fmaf(sc[rho], __int2float_rn(ia[rho][t] + ib[rho][t]), acc[rho][t]);
     } else {
+      // the four scales of the piece's blocks: four fp16 (8 bytes) or four E4M3 bytes
       uint2 scp[2];
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho) scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
+      for (int rho = 0; rho < 2; ++rho)
+        scp[rho] = SF ? make_uint2(*reinterpret_cast<const uint32_t*>(rw.scales + rho * Gm::SPR + c * 4), 0u)
+                      : *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         uint32_t f[2][4];
@@ -211,8 +227,12 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
         float sc[2];
 #pragma unroll
         for (int rho = 0; rho < 2; ++rho) {
-          const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
-          sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
+          if (SF) {
+            sc[rho] = e4m3_value((scp[rho].x >> (8 * m)) & 0xFFu);
+          } else {
+            const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
+            sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
+          }
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -250,11 +270,14 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
       const float inv = tok_inv[tl];
       const int p = tok_pos[tl];
       if (MODE == GATEUP) {
-        const float g = acc[0][t] * inv, u = acc[1][t] * inv;
+        float g = acc[0][t] * inv, u = acc[1][t] * inv;
+        if (SF) { g *= rw.rs0; u *= rw.rs1; }
         out[size_t(p) * out_cols + (rw.r0 >> 1)] = g / (1.f + expf(-g)) * u;
       } else {
         const float wgt = tok_w[tl] * inv;
-        *reinterpret_cast<float2*>(out + size_t(p) * out_cols + rw.r0) = make_float2(acc[0][t] * wgt, acc[1][t] * wgt);
+        float y0 = acc[0][t] * wgt, y1 = acc[1][t] * wgt;
+        if (SF) { y0 *= rw.rs0; y1 *= rw.rs1; }
+        *reinterpret_cast<float2*>(out + size_t(p) * out_cols + rw.r0) = make_float2(y0, y1);
       }
     }
   }

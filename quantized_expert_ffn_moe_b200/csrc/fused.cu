@@ -1199,6 +1199,7 @@ void set_fused_timing(unsigned long long* buf) { g_fused_timing = buf; }
 
 bool fused_supported(const moe_config& c, int T) {
   if (T < 1 || T > kFMaxTokens || T * c.top_k > kFMaxPairs) return false;
+  if (c.scale_fmt != 0) return false;              // fp8 block scales: the stand-alone GEMV reads them
   return c.hidden == 2048 && c.inter == 768 && (c.num_experts % 32) == 0 && c.num_experts <= 1024;
 }
 

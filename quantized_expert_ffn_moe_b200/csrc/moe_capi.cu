@@ -42,6 +42,8 @@ int validate_config(const moe_config* c) {
   if (!((c->bits == 4 && (c->block == 32 || c->block == 128)) || (c->bits == 2 && c->block == 16)))
     return MOE_ERR_UNSUPPORTED;
   if (c->half_levels != 0 && c->half_levels != 1) return MOE_ERR_UNSUPPORTED;
+  if (c->scale_fmt != 0 && c->scale_fmt != 1) return MOE_ERR_UNSUPPORTED;
+  if (c->scale_fmt == 1 && c->block == 128) return MOE_ERR_UNSUPPORTED;
   const int H = c->hidden;
   if (!(H == 256 || H == 512 || H == 1024 || H == 2048 || H == 4096)) return MOE_ERR_UNSUPPORTED;
   if (c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
@@ -63,6 +65,14 @@ int validate_weights(const moe_config* c, const moe_layer_weights* w) {
   }
   if (w->router_bias && !aligned(w->router_bias, 4)) return MOE_ERR_INVALID_ARG;
   if (w->shared_gate_w && (c->shared_inter == 0 || !aligned(w->shared_gate_w, 16))) return MOE_ERR_INVALID_ARG;
+  // fp8 block scales come with one fp32 scale per row; fp16 scales with none
+  const void* rs[] = {w->gate_up_row_scales, w->down_row_scales};
+  const void* srs[] = {w->shared_gate_up_row_scales, w->shared_down_row_scales};
+  for (const void* p : rs)
+    if (c->scale_fmt == 1 ? (!p || !aligned(p, 4)) : p != nullptr) return MOE_ERR_INVALID_ARG;
+  for (const void* p : srs)
+    if (c->scale_fmt == 1 && c->shared_inter > 0 ? (!p || !aligned(p, 4)) : (c->scale_fmt == 0 && p != nullptr))
+      return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -299,17 +309,28 @@ int moe_device_status(const void* workspace, int32_t* code_out) {
   return v[0] == 0 ? MOE_OK : MOE_ERR_DEVICE_CHECK;
 }
 
-int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t* scales, int32_t row0,
-                     int32_t rows, int32_t cols, float* out, void* stream) {
+int moe_dequant_rows_scaled(const moe_config* cfg, const uint8_t* codes, const void* scales,
+                            const float* row_scales, int32_t row0, int32_t rows, int32_t cols, float* out,
+                            void* stream) {
   if (!cfg || !codes || !scales || !out || row0 < 0 || rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
   if (!((cfg->bits == 4 && (cfg->block == 32 || cfg->block == 128)) || (cfg->bits == 2 && cfg->block == 16)))
     return MOE_ERR_UNSUPPORTED;
   if (cfg->half_levels != 0 && cfg->half_levels != 1) return MOE_ERR_UNSUPPORTED;
+  if (cfg->scale_fmt != 0 && cfg->scale_fmt != 1) return MOE_ERR_UNSUPPORTED;
+  if ((cfg->scale_fmt == 1) != (row_scales != nullptr)) return MOE_ERR_INVALID_ARG;
   if (cols % cfg->block != 0 || (cols * cfg->bits / 8) % 4 != 0) return MOE_ERR_UNSUPPORTED;
-  if (!aligned(codes, 4) || !aligned(scales, 2) || !aligned(out, 4)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(codes, 4) || !aligned(scales, cfg->scale_fmt ? 1 : 2) || !aligned(out, 4) ||
+      (row_scales && !aligned(row_scales, 4)))
+    return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
-  return cuda_status(launch_dequant_rows(cfg->bits, cfg->block, cfg->half_levels, codes, scales, row0, rows, cols,
-                                         out, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_dequant_rows(cfg->bits, cfg->block, cfg->half_levels, cfg->scale_fmt, codes, scales,
+                                         row_scales, row0, rows, cols, out, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_dequant_rows(const moe_config* cfg, const uint8_t* codes, const uint16_t* scales, int32_t row0,
+                     int32_t rows, int32_t cols, float* out, void* stream) {
+  if (cfg && cfg->scale_fmt != 0) return MOE_ERR_UNSUPPORTED;
+  return moe_dequant_rows_scaled(cfg, codes, scales, nullptr, row0, rows, cols, out, stream);
 }
 
 int moe_profile_begin(int32_t max_calls) {

@@ -537,7 +537,8 @@ int decode_path_mode();
 bool router_gemm_supported(const moe_config& c, int T);
 cudaError_t launch_router_gemm(const moe_config& c, const uint16_t* router_w, const float* bias, const uint16_t* x,
                                int T, float* logits, int* status, int num_sms, cudaStream_t s);
-cudaError_t launch_dequant_rows(int bits, int block, int half_levels, const uint8_t* codes, const uint16_t* scales,
+cudaError_t launch_dequant_rows(int bits, int block, int half_levels, int scale_fmt, const uint8_t* codes,
+                                const void* scales, const float* row_scales,
                                 int row0, int rows, int cols, float* out, cudaStream_t s);
 bool decode_shape_supported(int bits, int H, int I);
 

@@ -896,6 +896,7 @@ cudaError_t launch_router_gemm(const moe_config& c, const uint16_t* router_w, co
 bool prefill_supported(const moe_config& c) {
   const int H = c.hidden, I = c.inter;
   const int bs = c.block;
+  if (c.scale_fmt != 0) return false;              // fp8 block scales: the stand-alone GEMV reads them
   // the dequantizer takes one scale per 32 (4-bit) or 16 (2-bit) elements of a
   // packed stage; 4-bit blocks of 128 run on the CUDA-core GEMV at every size
   if (bs != (c.bits == 4 ? 32 : 16)) return false;

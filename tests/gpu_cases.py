@@ -27,7 +27,7 @@ def torch():
 
 def cfg_of(shape: mi.MoeShape) -> q.MoeConfig:
     return q.config_of(shape.experts, shape.hidden, shape.inter, shape.top_k, shape.shared, shape.bits,
-                       shape.block, shape.half)
+                       shape.block, shape.half, shape.fp8_scales)
 
 
 def device_layer(shape: mi.MoeShape, seed: int, layer: int, zipf: bool = False,

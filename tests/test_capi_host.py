@@ -75,14 +75,21 @@ def test_tiny_and_2bit_configs_supported(lib):
     assert q.moe_workspace_bytes(cfg(bits=4, block=128), 64) > 0      # GPTQ-style 128-element groups
 
 
-def _fake_weights(shared=True, misalign=None):
+ROW_SCALES = ("gate_up_row_scales", "down_row_scales", "shared_gate_up_row_scales", "shared_down_row_scales")
+
+
+def _fake_weights(shared=True, misalign=None, fp8=False):
     # addresses are never dereferenced on these paths
     base = 1 << 20
     w = q._Weights()
     for i, (name, _) in enumerate(q._Weights._fields_):
         setattr(w, name, base * (i + 1))
     if not shared:
-        for n in ("shared_gate_up_codes", "shared_gate_up_scales", "shared_down_codes", "shared_down_scales"):
+        for n in ("shared_gate_up_codes", "shared_gate_up_scales", "shared_down_codes", "shared_down_scales",
+                  "shared_gate_up_row_scales", "shared_down_row_scales"):
+            setattr(w, n, None)
+    if not fp8:
+        for n in ROW_SCALES:
             setattr(w, n, None)
     w.router_bias = None
     w.shared_gate_w = None
@@ -95,6 +102,31 @@ def _layer(lib, c, w, x=1 << 30, T=4, y=2 << 30, ws=3 << 30, ws_bytes=None):
     if ws_bytes is None:
         ws_bytes = lib.moe_workspace_bytes(ctypes.byref(c), T)
     return lib.moe_layer_forward(ctypes.byref(c), ctypes.byref(w), x, T, y, ws, ws_bytes, None)
+
+
+def test_fp8_scale_arguments(lib):
+    """scale_fmt 1 needs the fp32 row scales (4-byte aligned), scale_fmt 0
+    refuses them; fp8 scales only with blocks of 32 (4-bit) / 16 (2-bit)."""
+    c8 = cfg()
+    c8.scale_fmt = 1
+    assert lib.moe_workspace_bytes(ctypes.byref(c8), 16) > 0
+    assert _layer(lib, c8, _fake_weights(fp8=True), ws_bytes=100) == -3     # arguments pass, workspace too small
+    w = _fake_weights(fp8=False)
+    assert _layer(lib, c8, w) == -1                                        # row scales missing
+    w = _fake_weights(fp8=True)
+    w.down_row_scales += 2
+    assert _layer(lib, c8, w) == -1                                        # misaligned row scales
+    w = _fake_weights(fp8=True, shared=False)
+    c8s = cfg(shared=False)
+    c8s.scale_fmt = 1
+    assert _layer(lib, c8s, w, ws_bytes=100) == -3                         # no shared expert: no shared row scales
+    assert _layer(lib, cfg(), _fake_weights(fp8=True)) == -1               # fp16 scales with row scales
+    c2 = cfg()
+    c2.scale_fmt = 2
+    assert lib.moe_workspace_bytes(ctypes.byref(c2), 16) == 0
+    cg = cfg(bits=4, block=128)
+    cg.scale_fmt = 1
+    assert lib.moe_workspace_bytes(ctypes.byref(cg), 16) == 0
 
 
 def test_layer_forward_argument_errors(lib):

@@ -24,6 +24,11 @@ FULL4_G128 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=T
 TINY2H = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=2, block=16, half=True)
 TINY4H = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=4, block=32, half=True)
 FULL2H = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=2, block=16, half=True)
+# one E4M3 scale byte per block under one fp32 scale per row
+TINY4F8 = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=4, block=32, fp8_scales=True)
+TINY2F8 = mi.MoeShape(experts=64, hidden=256, inter=128, top_k=4, shared=True, bits=2, block=16, fp8_scales=True)
+FULL4F8 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=32, fp8_scales=True)
+FULL2F8 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=2, block=16, fp8_scales=True)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -40,18 +45,26 @@ def _cuda():
 
 # ------------------------------------------------------------ input bytes ---
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, TINY_G128, TINY2H, TINY4H, FULL2H],
-                         ids=["tiny4", "tiny2", "full4", "full2", "tiny4g128", "tiny2h", "tiny4h", "full2h"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, mi.FULL4, mi.FULL2, TINY_G128, TINY2H, TINY4H, FULL2H,
+                                   TINY4F8, TINY2F8, FULL4F8, FULL2F8],
+                         ids=["tiny4", "tiny2", "full4", "full2", "tiny4g128", "tiny2h", "tiny4h", "full2h",
+                              "tiny4f8", "tiny2f8", "full4f8", "full2f8"])
 def test_device_generator_matches_host(shape):
     """The device generator writes the same bytes as the numpy generator."""
     w = gc.device_layer(shape, seed=3, layer=5)
+    f8 = shape.fp8_scales
     for e in (0, 1, shape.experts - 1):
         ref = mi.expert_packed(shape, 3, 5, e)
         got = (w.gate_up_codes[e], w.gate_up_scales[e], w.down_codes[e], w.down_scales[e])
+        if f8:
+            got += (w.gate_up_row_scales[e], w.down_row_scales[e])
+        assert len(got) == len(ref)
         for r, g in zip(ref, got):
             np.testing.assert_array_equal(g.cpu().numpy().view(r.dtype).reshape(r.shape), r)
     ref = mi.shared_packed(shape, 3, 5)
     got = (w.shared_gate_up_codes, w.shared_gate_up_scales, w.shared_down_codes, w.shared_down_scales)
+    if f8:
+        got += (w.shared_gate_up_row_scales, w.shared_down_row_scales)
     for r, g in zip(ref, got):
         np.testing.assert_array_equal(g.cpu().numpy().view(r.dtype).reshape(r.shape), r)
     np.testing.assert_array_equal(gc.bits_to_np(w.router_w), mi.router_weight_bf16(shape, 3, 5))
@@ -78,6 +91,30 @@ def test_device_decoder_bit_exact(shape):
     torch.cuda.synchronize()
     np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64),
                                   orc.dequantize(dcodes, dsc, H, I, shape.bits, shape.block, shape.half)[3:])
+
+
+@pytest.mark.parametrize("shape", [TINY4F8, TINY2F8, FULL4F8, FULL2F8], ids=["tiny4f8", "tiny2f8", "full4f8", "full2f8"])
+def test_device_decoder_bit_exact_fp8_scales(shape):
+    """E4M3 block scales times the fp32 row scale: q * e4m3 is exact, so the
+    GEMV's decoder must give the float64 weight rounded once to fp32."""
+    torch = gc.torch()
+    w = gc.device_layer(shape, seed=1, layer=0)
+    cfg = gc.cfg_of(shape)
+    e = shape.experts // 2 + 1
+    gcodes, gsc, dcodes, dsc, grs, drs = mi.expert_packed(shape, 1, 0, e)
+    H, I = shape.hidden, shape.inter
+    out = torch.empty((2 * I, H), dtype=torch.float32, device="cuda")
+    q.moe_dequant_rows_scaled(cfg, w.gate_up_codes[e], w.gate_up_scales[e], w.gate_up_row_scales[e], 0, 2 * I, H, out)
+    torch.cuda.synchronize()
+    ref = orc.dequantize(gcodes, gsc, 2 * I, H, shape.bits, shape.block, row_scale=grs)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    out = torch.empty((H - 5, I), dtype=torch.float32, device="cuda")
+    q.moe_dequant_rows_scaled(cfg, w.down_codes[e], w.down_scales[e], w.down_row_scales[e], 5, H - 5, I, out)
+    torch.cuda.synchronize()
+    ref = orc.dequantize(dcodes, dsc, H, I, shape.bits, shape.block, row_scale=drs)[5:]
+    np.testing.assert_array_equal(out.cpu().numpy(), ref.astype(np.float32))
+    # the plain hook refuses fp8 scales
+    assert q.moe_dequant_rows(cfg, w.down_codes[e], w.down_scales[e], 0, 4, I, out, check=False) == -2
 
 
 # ----------------------------------------------------------------- router ---
@@ -137,8 +174,8 @@ def _oracle_given(lay, x_bits, gpu_idx, differ):
     return orc.layer_forward(lay, x_bits, topk_override=over)
 
 
-@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, TINY_G128, TINY2H, TINY4H],
-                         ids=["tiny4", "tiny2", "tiny4g128", "tiny2h", "tiny4h"])
+@pytest.mark.parametrize("shape", [mi.TINY, SHAPE_2BIT_TINY, TINY_G128, TINY2H, TINY4H, TINY4F8, TINY2F8],
+                         ids=["tiny4", "tiny2", "tiny4g128", "tiny2h", "tiny4h", "tiny4f8", "tiny2f8"])
 @pytest.mark.parametrize("T", [1, 2, 7, 8, 17, 64, 100])
 def test_layer_tiny_live_oracle(shape, T):
     x = mi.hidden_states_bf16(T, shape.hidden, 0, 0)
@@ -409,6 +446,64 @@ def test_layer_full2_half_levels_sampled(T, path):
     single-launch decode kernel (1, 16 tokens; 48 tokens on each side of the
     hand-over) and the tensor-core prefill (300 tokens)."""
     _with_path(path, lambda: _sampled_full_case(FULL2H, T, 13, 0, min(3, T), 900 + T))
+
+
+# ------------------------------------------------------- fp8 block scales ---
+
+@pytest.mark.parametrize("shape,T", [(FULL4F8, 1), (FULL4F8, 16), (FULL4F8, 100), (FULL2F8, 16), (FULL2F8, 64)],
+                         ids=["full4_t1", "full4_t16", "full4_t100", "full2_t16", "full2_t64"])
+def test_layer_full_fp8_scales_sampled(shape, T):
+    """Full shape with E4M3 block scales and fp32 row scales: the stand-alone
+    GEMV kernels at every batch size (decode and the 100-token batch)."""
+    _sampled_full_case(shape, T, 17, 0, min(3, T), 700 + T)
+
+
+def test_fp8_scales_stack_and_expert_parallel():
+    """Two layers of fp8-scaled weights through moe_stack_forward (the
+    separate kernels with the residual and the next layer's RMSNorm), and
+    the expert-parallel partials of one of them."""
+    torch = gc.torch()
+    shape = TINY4F8
+    T = 12
+    x = mi.hidden_states_bf16(T, shape.hidden, 0, 41)
+    ws_l = [gc.device_layer(shape, 0, l) for l in range(2)]
+    cfg = gc.cfg_of(shape)
+    xd = gc.to_dev_bits(x)
+    ws = gc.workspace(cfg, T)
+    q.moe_stack_forward(cfg, ws_l, xd, ws)
+    torch.cuda.synchronize()
+    got_stack = gc.bits_to_np(xd)
+    # one layer at a time through the same entry point composes bitwise
+    xs = gc.to_dev_bits(x)
+    for l in range(2):
+        q.moe_stack_forward(cfg, ws_l[l:l + 1], xs, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(gc.bits_to_np(xs), got_stack)
+    # first step against the oracle at the layer tolerance
+    lay = gc.host_oracle_layer(shape, 0, 0, cache_size=shape.experts + 1)
+    xs = gc.to_dev_bits(x)
+    tr = torch.empty((1, T, shape.top_k), dtype=torch.int32, device="cuda")
+    q.moe_stack_forward(cfg, ws_l[:1], xs, ws, topk_trace=tr)
+    torch.cuda.synchronize()
+    idx = tr[0].cpu().numpy()
+    r = orc.layer_forward(lay, x, rmsnorm=True)
+    differ = gc.check_selection(r["logits"], r["idx"], idx, shape.top_k)
+    if differ:
+        r = orc.layer_forward(lay, x, rmsnorm=True, topk_override={t: idx[t] for t in differ})
+    xf = orc.bf16_to_f64(x)
+    eps = gc.REL_TOL * float(np.sqrt(np.mean(r["out"] ** 2)))
+    got = orc.bf16_to_f64(gc.bits_to_np(xs))
+    lo, hi = orc.round_bf16(xf + r["out"] - eps), orc.round_bf16(xf + r["out"] + eps)
+    assert np.all(got >= lo) and np.all(got <= hi)
+    # expert-parallel partials sum to the layer
+    parts = _ep_partials(shape, ws_l[0], x, 2)
+    full = orc.layer_forward(lay, x)
+    idx0 = gc.run_route(shape, ws_l[0], x)[0]
+    d0 = gc.check_selection(full["logits"], full["idx"], idx0, shape.top_k)
+    if d0:
+        full = orc.layer_forward(lay, x, topk_override={t: idx0[t] for t in d0})
+    scale = float(np.sqrt(np.mean(full["out"] ** 2)))
+    assert float(np.abs(sum(parts) - full["out"]).max()) <= gc.REL_TOL * scale
 
 
 # ----------------------------------------------------- gated shared expert ---
