@@ -84,7 +84,7 @@ typedef struct moe_config {
                             finite 448) byte per block, times one
                             fp32 scale per weight row (the
                             *_row_scales arrays); block 32 (4-bit) or
-                            16 (2-bit) only.  Layers with fp8 scales
+                            16 (2-bit), integer levels only.  Layers with fp8 scales
                             run on the stand-alone GEMV kernels at
                             every batch size (neither the
                             single-launch decode kernel nor the

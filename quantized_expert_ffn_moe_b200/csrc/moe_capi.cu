@@ -43,7 +43,7 @@ int validate_config(const moe_config* c) {
     return MOE_ERR_UNSUPPORTED;
   if (c->half_levels != 0 && c->half_levels != 1) return MOE_ERR_UNSUPPORTED;
   if (c->scale_fmt != 0 && c->scale_fmt != 1) return MOE_ERR_UNSUPPORTED;
-  if (c->scale_fmt == 1 && c->block == 128) return MOE_ERR_UNSUPPORTED;
+  if (c->scale_fmt == 1 && (c->block == 128 || c->half_levels)) return MOE_ERR_UNSUPPORTED;
   const int H = c->hidden;
   if (!(H == 256 || H == 512 || H == 1024 || H == 2048 || H == 4096)) return MOE_ERR_UNSUPPORTED;
   if (c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;

@@ -127,6 +127,10 @@ def test_fp8_scale_arguments(lib):
     cg = cfg(bits=4, block=128)
     cg.scale_fmt = 1
     assert lib.moe_workspace_bytes(ctypes.byref(cg), 16) == 0
+    ch = cfg()
+    ch.scale_fmt = 1
+    ch.half_levels = 1
+    assert lib.moe_workspace_bytes(ctypes.byref(ch), 16) == 0
 
 
 def test_layer_forward_argument_errors(lib):
