@@ -630,10 +630,13 @@ __global__ void __launch_bounds__(PEp<MODE>::kThreads, 1) prefill_gemm_kernel(
   }
 }
 
-// Token rows gathered into expert order as fp16, k permuted within each group
-// of G as the dequantized weights are, each row scaled by the power of two
-// that brings its largest magnitude into [2^13, 2^14) (exact conversion of the
-// bf16 values; xinv[p] undoes it).  One warp per pair position.
+// Token rows scattered into expert order as fp16 (routed positions, then the
+// shared expert's): one warp per token converts its row once -- exactly, after
+// the power of two that brings its largest magnitude into [2^13, 2^14), with k
+// permuted within each group of 8 (4-bit) / 16 (2-bit) to match the
+// dequantizer's pair order -- and stores it at every position of the token
+// (inv[t k + j], position -1 = another rank's expert; T k + t for the shared
+// expert), with xinv = the inverse power of two.
 template <int BITS>
 __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __restrict__ x, RouteView rv, int H,
                                                             uint16_t* __restrict__ xs, float* __restrict__ xinv,
@@ -642,16 +645,10 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
   pdl_launch_dependents();
   if (gated && __ldcg(rv.status + ST_PATH) == 0) return;     // the fused decode kernel kept the layer
   constexpr int G = BITS == 4 ? 8 : 16;
-  const int P = rv.T * rv.k + (rv.shared ? rv.T : 0);
-  // routed positions in use: all T*k, or fewer when the experts are split
-  // over ranks (this rank's pairs only)
-  const int Pr = __ldcg(rv.offsets + rv.E);
+  constexpr int kMaxChunks = 4096 / (32 * G);              // chunks of G elements per lane (H <= 4096)
   const int lane = threadIdx.x & 31;
-  for (int p = blockIdx.x * 8 + (threadIdx.x >> 5); p < P; p += gridDim.x * 8) {
-    if (p < rv.T * rv.k && p >= Pr) continue;
-    const int tok = p < rv.T * rv.k ? __ldg(rv.pairs + p) / rv.k : p - rv.T * rv.k;
+  for (int tok = blockIdx.x * 8 + (threadIdx.x >> 5); tok < rv.T; tok += gridDim.x * 8) {
     const uint16_t* src = x + size_t(tok) * H;
-    uint16_t* dst = xs + size_t(p) * H;
     float vmax = 0.f;
     for (int h0 = lane * 8; h0 < H; h0 += 256) {
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + h0));
@@ -668,9 +665,15 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
       frexpf(vmax, &ex);
       sh = min(max(14 - ex, -100), 100);
     }
-    const float mul = ldexpf(1.f, sh);
-    if (lane == 0) xinv[p] = ldexpf(1.f, -sh);
-    for (int h0 = lane * G; h0 < H; h0 += 32 * G) {
+    const float mul = ldexpf(1.f, sh), inv_mul = ldexpf(1.f, -sh);
+    // the converted row, chunk c of this lane = elements (c * 32 + lane) * G ...
+    // (H = 256 at 2-bit: 16 chunks of 16, half the lanes hold one)
+    uint4 row[kMaxChunks][G / 8];
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int h0 = (c * 32 + lane) * G;
+      if (c * 32 * G >= H) break;
+      if (h0 >= H) continue;
       float in[G];
 #pragma unroll
       for (int q = 0; q < G / 8; ++q) {
@@ -682,10 +685,23 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
           in[8 * q + 2 * z + 1] = __uint_as_float(w[z] & 0xFFFF0000u);
         }
       }
-      uint4 parts[G / 8];
-      pack_pair_order<G>(in, mul, parts);
+      pack_pair_order<G>(in, mul, row[c]);
+    }
+    // every position of the token: its k routed pairs, then the shared expert
+    const int np = rv.k + (rv.shared ? 1 : 0);
+    for (int j = 0; j < np; ++j) {
+      const int p = j < rv.k ? __ldg(rv.inv + size_t(tok) * rv.k + j) : rv.T * rv.k + tok;
+      if (p < 0) continue;                                   // another rank's expert
+      uint16_t* dst = xs + size_t(p) * H;
 #pragma unroll
-      for (int q = 0; q < G / 8; ++q) *reinterpret_cast<uint4*>(dst + h0 + 8 * q) = parts[q];
+      for (int c = 0; c < kMaxChunks; ++c) {
+        const int h0 = (c * 32 + lane) * G;
+        if (c * 32 * G >= H) break;
+        if (h0 >= H) continue;
+#pragma unroll
+        for (int q = 0; q < G / 8; ++q) *reinterpret_cast<uint4*>(dst + h0 + 8 * q) = row[c][q];
+      }
+      if (lane == 0) xinv[p] = inv_mul;
     }
   }
 }
@@ -922,11 +938,10 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   uint16_t* xs = reinterpret_cast<uint16_t*>(a.ws + a.L.xs);
   uint16_t* hs = reinterpret_cast<uint16_t*>(a.ws + a.L.h);
   float* xinv = reinterpret_cast<float*>(a.ws + a.L.xscale);
+  const int gblocks = max(1, min(a.num_sms * 8, (a.T + 7) / 8));    // one warp per token
   cudaError_t err = bits == 4
-      ? launch_pdl(gather_tokens_kernel<4>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv,
-                   a.gated)
-      : launch_pdl(gather_tokens_kernel<2>, dim3(a.num_sms * 8), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv,
-                   a.gated);
+      ? launch_pdl(gather_tokens_kernel<4>, dim3(gblocks), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv, a.gated)
+      : launch_pdl(gather_tokens_kernel<2>, dim3(gblocks), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv, a.gated);
   if (err != cudaSuccess) return err;
 
   PrefillArgs g{};
