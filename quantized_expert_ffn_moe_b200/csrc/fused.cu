@@ -727,6 +727,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
     mbar_fence_init();
   }
   __syncthreads();
+  // launched behind the kernel that clears the workspace's status words (a
+  // programmatic dependency, so this launch overlaps that one); nothing in
+  // the workspace is touched before it has completed
+  pdl_wait();
   int issued = 0, consumed = 0;
   const unsigned G = gridDim.x;
   const uint16_t* xsrc = p.stack ? p.y : p.x;
@@ -1172,12 +1176,22 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   cfg.blockDim = dim3(kFThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, q);
+  cfg.numAttrs = 2;
+  err = cudaLaunchKernelEx(&cfg, kern, q);
+  if (err == cudaErrorNotSupported || err == cudaErrorInvalidValue) {
+    // no programmatic dependency with a cooperative launch here: launch it
+    // plainly (the status words are already cleared by then)
+    (void)cudaGetLastError();
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, q);
+  }
+  return err;
 }
 
 }  // namespace

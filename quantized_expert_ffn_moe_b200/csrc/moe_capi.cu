@@ -193,8 +193,9 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
   a.L = make_layout(*cfg, T);
   a.num_sms = num_sms_current();
   a.stream = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int* status = reinterpret_cast<int*>(a.ws + a.L.status);
   if (T <= kDecodeMaxTokens && fused_supported(*cfg, T) && !w->shared_gate_w) {
+    if (launch_status_reset(status, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
     const int call = (g_prof.on && g_prof.used < g_prof.cap) ? g_prof.used++ : -1;
     prof_mark(call, 0, a.stream);
     // 32..64 tokens: the fused kernel routes and then either finishes the
@@ -217,7 +218,9 @@ int moe_layer_forward(const moe_config* cfg, const moe_layer_weights* w, const u
     if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_status(e);
     (void)cudaGetLastError();        // cannot co-schedule one CTA per SM here: separate kernels
     if (call >= 0) g_prof.used--;
+    return run_layer(a);              // the status words are already cleared
   }
+  if (cudaMemsetAsync(status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
   return run_layer(a);
 }
 
@@ -273,10 +276,16 @@ int moe_stack_forward(const moe_config* cfg, const moe_layer_weights* layers, in
   a.num_sms = num_sms_current();
   a.stream = static_cast<cudaStream_t>(stream);
   uint16_t* xhat = reinterpret_cast<uint16_t*>(a.ws + a.L.xhat);
-  if (cudaMemsetAsync(a.ws + a.L.status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int* status = reinterpret_cast<int*>(a.ws + a.L.status);
   bool gated = false;
   for (int l = 0; l < L; ++l) gated = gated || layers[l].shared_gate_w != nullptr;
-  if (T <= kDecodeMaxTokens && fused_supported(*cfg, T) && !gated) {
+  const bool fused = T <= kDecodeMaxTokens && fused_supported(*cfg, T) && !gated;
+  if (fused) {
+    if (launch_status_reset(status, a.stream) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (cudaMemsetAsync(status, 0, ST_COUNT * 4, a.stream) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
+  if (fused) {
     const cudaError_t e = launch_fused_decode(*cfg, layers, L, x_inout, x_inout, true, T, topk_trace, a.ws, a.L,
                                               a.num_sms, a.stream);
     if (e == cudaSuccess) return MOE_OK;

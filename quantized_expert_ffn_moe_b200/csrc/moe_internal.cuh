@@ -521,6 +521,7 @@ bool fused_supported(const moe_config& c, int T);
 void set_fused_timing(unsigned long long* buf);
 void set_prefill_timing(unsigned long long* buf);
 extern unsigned long long* g_prefill_timing;
+cudaError_t launch_status_reset(int* status, cudaStream_t s);
 cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* layers, int L, const uint16_t* x,
                                 uint16_t* y, bool stack, int T, int* trace, char* ws, const Layout& Lw, int num_sms,
                                 cudaStream_t s, int hybrid = 0);

@@ -584,6 +584,20 @@ cudaError_t launch_topk_group_any(const moe_config& c, int T, char* ws, const La
   }
 }
 
+// Clears the workspace's status words (error code, counts, grid-barrier words)
+// before a single-launch decode kernel; it lets that kernel launch at once
+// (programmatic dependency) and the kernel waits for its completion before it
+// touches the workspace.
+__global__ void status_reset_kernel(int* status) {
+  pdl_launch_dependents();
+  for (int i = threadIdx.x; i < ST_COUNT; i += blockDim.x) status[i] = 0;
+}
+
+cudaError_t launch_status_reset(int* status, cudaStream_t s) {
+  status_reset_kernel<<<1, 128, 0, s>>>(status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
                               const uint16_t* x, int T, char* ws, const Layout& L, int* api_counts,
                               int* api_offsets, int* api_pairs, cudaStream_t s, int ep_rank, int ep_size) {
