@@ -839,157 +839,230 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       }
       all_sync();
       stamp(l, 9);
-      {
-        // exclusive scan of the counts and the ascending touched-expert list
-        const int EPT = (E + kFCons * 32 - 1) / (kFCons * 32);     // experts per thread
-        const int eb = threadIdx.x * EPT;
-        int csum = 0, fsum = 0;
-        for (int z = 0; z < EPT; ++z) {
-          const int e = eb + z;
-          int cc = 0;
-          if (e < E)
-            for (int m = 0; m < NMW; ++m) cc += __popc(rt.tmask[m * E + e]);
-          csum += cc;
-          fsum += cc > 0 ? 1 : 0;
+      if (P <= 31) {
+        // a few pairs (one, two or three tokens): one warp ranks them by
+        // (expert, pair id) -- the stable positions -- finds each expert's run,
+        // and scans the slots' costs; later phases read offsets[e] and
+        // offsets[e + 1] of the picked experts only
+        if (warp == 0) {
+          const bool act = lane < P;
+          const int e = act ? rt.idx[lane] : 0x7FFFFFFF;
+          int rank = 0, cnt = 0;
+          bool first = act;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int ej = __shfl_sync(0xffffffffu, e, j);
+            if (j < P) {
+              rank += (ej < e || (ej == e && j < lane)) ? 1 : 0;
+              cnt += ej == e ? 1 : 0;
+              if (ej == e && j < lane) first = false;
+            }
+          }
+          const unsigned fm = __ballot_sync(0xffffffffu, first);
+          int slot = 0;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int ej = __shfl_sync(0xffffffffu, e, j);
+            slot += ((fm >> j) & 1u) && ej < e ? 1 : 0;
+          }
+          if (act) {
+            rt.pairs[rank] = lane;
+            rt.inv[lane] = rank;
+          }
+          if (first) {
+            rt.ulist[slot] = e;
+            rt.offsets[e] = rank;
+            rt.offsets[e + 1] = rank + cnt;      // the next picked expert's start, when that is e + 1
+          }
+          const int U = __popc(fm), ns = U + S;
+          if (lane == 0) {
+            rt.offsets[E] = P;
+            if (S) rt.ulist[U] = E;
+            *snslots = ns;
+          }
+          __syncwarp();
+          const PassPlan pg{p.ntc_gu, 2 * I / GU::RPS}, pd{p.ntc_dn, H / DN::RPS};
+          int gc = 0, dc = 0;
+          if (lane < ns) {
+            const int eu = rt.ulist[lane];
+            const int n = eu >= E ? T : rt.offsets[eu + 1] - rt.offsets[eu];
+            gc = pass_cost(pg, n);
+            dc = pass_cost(pd, n);
+          }
+          int gi = gc, di = dc;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int ng = __shfl_up_sync(0xffffffffu, gi, o), nd = __shfl_up_sync(0xffffffffu, di, o);
+            if (lane >= o) { gi += ng; di += nd; }
+          }
+          if (lane < ns) {
+            rt.woff_gu[lane] = gi - gc;
+            rt.woff_dn[lane] = di - dc;
+          }
+          if (lane == 31) {
+            rt.woff_gu[ns] = gi;
+            rt.woff_dn[ns] = di;
+          }
         }
-        int2 tot;
-        const int2 run = block_excl_scan2(csum, fsum, scan_scratch, &tot);
-        int crun = run.x, frun = run.y;
-        for (int z = 0; z < EPT; ++z) {
-          const int e = eb + z;
-          if (e < E) {
-            rt.offsets[e] = crun;
+        all_sync();
+        stamp(l, 10);
+        if (warp == 1 && p.trace && blockIdx.x == 0) {
+          for (int q = lane; q < P; q += 32) p.trace[size_t(l) * P + q] = rt.idx[q];
+        }
+      } else {
+        {
+          // exclusive scan of the counts and the ascending touched-expert list
+          const int EPT = (E + kFCons * 32 - 1) / (kFCons * 32);     // experts per thread
+          const int eb = threadIdx.x * EPT;
+          int csum = 0, fsum = 0;
+          for (int z = 0; z < EPT; ++z) {
+            const int e = eb + z;
             int cc = 0;
-            for (int m = 0; m < NMW; ++m) cc += __popc(rt.tmask[m * E + e]);
-            crun += cc;
-            if (cc > 0) rt.ulist[frun++] = e;
+            if (e < E)
+              for (int m = 0; m < NMW; ++m) cc += __popc(rt.tmask[m * E + e]);
+            csum += cc;
+            fsum += cc > 0 ? 1 : 0;
+          }
+          int2 tot;
+          const int2 run = block_excl_scan2(csum, fsum, scan_scratch, &tot);
+          int crun = run.x, frun = run.y;
+          for (int z = 0; z < EPT; ++z) {
+            const int e = eb + z;
+            if (e < E) {
+              rt.offsets[e] = crun;
+              int cc = 0;
+              for (int m = 0; m < NMW; ++m) cc += __popc(rt.tmask[m * E + e]);
+              crun += cc;
+              if (cc > 0) rt.ulist[frun++] = e;
+            }
+          }
+          if (threadIdx.x == 0) {
+            rt.offsets[E] = tot.x;
+            if (S) rt.ulist[tot.y] = E;
+            *snslots = tot.y + S;
           }
         }
-        if (threadIdx.x == 0) {
-          rt.offsets[E] = tot.x;
-          if (S) rt.ulist[tot.y] = E;
-          *snslots = tot.y + S;
-        }
-      }
-      all_sync();
-      stamp(l, 10);
-      // stable positions inside each expert's list (pairs in token order): a
-      // pair of token t sits after the earlier tokens in its expert's mask, so
-      // every CTA derives the same positions, which the passes of different
-      // CTAs rely on.  Meanwhile the cost-weighted work prefix of the slots
-      // for the two passes.
-      for (int q = threadIdx.x; q < P; q += kFCons * 32) {
-        const int e = rt.idx[q], t = q / k;
-        int r = 0;
-        for (int m = 0; m < NMW; ++m) {
-          const int tb = t - 32 * m;
-          if (tb <= 0) break;
-          const unsigned below = tb >= 32 ? 0xFFFFFFFFu : ((1u << tb) - 1u);
-          r += __popc(rt.tmask[m * E + e] & below);
-        }
-        const int pos = rt.offsets[e] + r;
-        rt.pairs[pos] = q;
-        rt.inv[q] = pos;
-      }
-      if (warp == 1 && p.trace && blockIdx.x == 0) {
-        for (int q = lane; q < P; q += 32) p.trace[size_t(l) * P + q] = rt.idx[q];
-      }
-      {
-        const PassPlan pg{p.ntc_gu, 2 * I / GU::RPS}, pd{p.ntc_dn, H / DN::RPS};
-        const int ns = *snslots;
-        const int SPT = (ns + kFCons * 32 - 1) / (kFCons * 32);    // slots per thread
-        const int u0 = threadIdx.x * SPT;
-        int g = 0, d = 0;
-        for (int z = 0; z < SPT; ++z) {
-          const int u = u0 + z;
-          if (u < ns) {
-            const int e = rt.ulist[u];
-            const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
-            g += pass_cost(pg, n);
-            d += pass_cost(pd, n);
+        all_sync();
+        stamp(l, 10);
+        // stable positions inside each expert's list (pairs in token order): a
+        // pair of token t sits after the earlier tokens in its expert's mask, so
+        // every CTA derives the same positions, which the passes of different
+        // CTAs rely on.  Meanwhile the cost-weighted work prefix of the slots
+        // for the two passes.
+        for (int q = threadIdx.x; q < P; q += kFCons * 32) {
+          const int e = rt.idx[q], t = q / k;
+          int r = 0;
+          for (int m = 0; m < NMW; ++m) {
+            const int tb = t - 32 * m;
+            if (tb <= 0) break;
+            const unsigned below = tb >= 32 ? 0xFFFFFFFFu : ((1u << tb) - 1u);
+            r += __popc(rt.tmask[m * E + e] & below);
           }
+          const int pos = rt.offsets[e] + r;
+          rt.pairs[pos] = q;
+          rt.inv[q] = pos;
         }
-        int2 tot;
-        const int2 run = block_excl_scan2(g, d, scan_scratch, &tot);
-        int grun = run.x, drun = run.y;
-        const int gt = tot.x, dt = tot.y;
-        for (int z = 0; z < SPT; ++z) {
-          const int u = u0 + z;
-          if (u < ns) {
-            const int e = rt.ulist[u];
-            const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
-            rt.woff_gu[u] = grun;
-            rt.woff_dn[u] = drun;
-            grun += pass_cost(pg, n);
-            drun += pass_cost(pd, n);
-          }
+        if (warp == 1 && p.trace && blockIdx.x == 0) {
+          for (int q = lane; q < P; q += 32) p.trace[size_t(l) * P + q] = rt.idx[q];
         }
-        if (threadIdx.x == 0) { rt.woff_gu[ns] = gt; rt.woff_dn[ns] = dt; }
-        if (p.hybrid) {
-          // tensor-core work of the same slots: 128-token tiles of each slot
-          // over the gate/up (2I/128 row tiles x H/128 k-blocks) and down
-          // (H/128 x I/128) matrices
-          const int kb_tile = (2 * I / 128) * (H / 128) + (H / 128) * (I / 128);
-          int tk = 0;
+        {
+          const PassPlan pg{p.ntc_gu, 2 * I / GU::RPS}, pd{p.ntc_dn, H / DN::RPS};
+          const int ns = *snslots;
+          const int SPT = (ns + kFCons * 32 - 1) / (kFCons * 32);    // slots per thread
+          const int u0 = threadIdx.x * SPT;
+          int g = 0, d = 0;
           for (int z = 0; z < SPT; ++z) {
             const int u = u0 + z;
             if (u < ns) {
               const int e = rt.ulist[u];
               const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
-              tk += (n + 127) / 128;
+              g += pass_cost(pg, n);
+              d += pass_cost(pd, n);
             }
           }
-          int2 ttot;
-          const int2 trun = block_excl_scan2(tk, 0, scan_scratch, &ttot);
-          const float per_f = float(gt + dt) / float(G), per_t = float(ttot.x) * kb_tile / float(G);
-          const bool tc = p.hybrid == 2 || p.cost_t0 + p.cost_t1 * per_t < p.cost_f0 + p.cost_f1 * per_f;
-          if (threadIdx.x == 0) *s_handover = tc ? 1 : 0;
-          if (blockIdx.x == 0) {
-            if (threadIdx.x == 0) {
-              status[ST_COST_F] = gt + dt;
-              status[ST_COST_T] = ttot.x * kb_tile;
-              status[ST_PATH] = tc ? 1 : 0;
+          int2 tot;
+          const int2 run = block_excl_scan2(g, d, scan_scratch, &tot);
+          int grun = run.x, drun = run.y;
+          const int gt = tot.x, dt = tot.y;
+          for (int z = 0; z < SPT; ++z) {
+            const int u = u0 + z;
+            if (u < ns) {
+              const int e = rt.ulist[u];
+              const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+              rt.woff_gu[u] = grun;
+              rt.woff_dn[u] = drun;
+              grun += pass_cost(pg, n);
+              drun += pass_cost(pd, n);
             }
-            if (tc) {
-              // the routing in the layout the grouped kernels read
-              int* g_counts = reinterpret_cast<int*>(ws + p.L_.counts);
-              int* g_offsets = reinterpret_cast<int*>(ws + p.L_.offsets);
-              int* g_pairs = reinterpret_cast<int*>(ws + p.L_.pairs);
-              int* g_inv = reinterpret_cast<int*>(ws + p.L_.inv);
-              int* g_ulist = reinterpret_cast<int*>(ws + p.L_.ulist);
-              int* g_ntoff = reinterpret_cast<int*>(ws + p.L_.ntoff);
-              int* g_idx = reinterpret_cast<int*>(ws + p.L_.topk_idx);
-              float* g_w = reinterpret_cast<float*>(ws + p.L_.topk_w);
-              for (int e = threadIdx.x; e <= E; e += kFCons * 32) {
-                g_offsets[e] = rt.offsets[e];
-                if (e < E) g_counts[e] = rt.offsets[e + 1] - rt.offsets[e];
+          }
+          if (threadIdx.x == 0) { rt.woff_gu[ns] = gt; rt.woff_dn[ns] = dt; }
+          if (p.hybrid) {
+            // tensor-core work of the same slots: 128-token tiles of each slot
+            // over the gate/up (2I/128 row tiles x H/128 k-blocks) and down
+            // (H/128 x I/128) matrices
+            const int kb_tile = (2 * I / 128) * (H / 128) + (H / 128) * (I / 128);
+            int tk = 0;
+            for (int z = 0; z < SPT; ++z) {
+              const int u = u0 + z;
+              if (u < ns) {
+                const int e = rt.ulist[u];
+                const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+                tk += (n + 127) / 128;
               }
-              for (int u = threadIdx.x; u < ns; u += kFCons * 32) g_ulist[u] = rt.ulist[u];
-              for (int q = threadIdx.x; q < P; q += kFCons * 32) {
-                g_pairs[q] = rt.pairs[q];
-                g_inv[q] = rt.inv[q];
-                g_idx[q] = rt.idx[q];
-                g_w[q] = rt.w[q];
-              }
-              // token-tile prefix over the slots, in this thread's SPT slots
-              int run = trun.x;
-              for (int z = 0; z < SPT; ++z) {
-                const int u = u0 + z;
-                if (u < ns) {
-                  const int e = rt.ulist[u];
-                  const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
-                  g_ntoff[u] = run;
-                  run += (n + 127) / 128;
-                }
-              }
+            }
+            int2 ttot;
+            const int2 trun = block_excl_scan2(tk, 0, scan_scratch, &ttot);
+            const float per_f = float(gt + dt) / float(G), per_t = float(ttot.x) * kb_tile / float(G);
+            const bool tc = p.hybrid == 2 || p.cost_t0 + p.cost_t1 * per_t < p.cost_f0 + p.cost_f1 * per_f;
+            if (threadIdx.x == 0) *s_handover = tc ? 1 : 0;
+            if (blockIdx.x == 0) {
               if (threadIdx.x == 0) {
-                g_ntoff[ns] = ttot.x;
-                status[ST_UCOUNT] = ns - S;
+                status[ST_COST_F] = gt + dt;
+                status[ST_COST_T] = ttot.x * kb_tile;
+                status[ST_PATH] = tc ? 1 : 0;
+              }
+              if (tc) {
+                // the routing in the layout the grouped kernels read
+                int* g_counts = reinterpret_cast<int*>(ws + p.L_.counts);
+                int* g_offsets = reinterpret_cast<int*>(ws + p.L_.offsets);
+                int* g_pairs = reinterpret_cast<int*>(ws + p.L_.pairs);
+                int* g_inv = reinterpret_cast<int*>(ws + p.L_.inv);
+                int* g_ulist = reinterpret_cast<int*>(ws + p.L_.ulist);
+                int* g_ntoff = reinterpret_cast<int*>(ws + p.L_.ntoff);
+                int* g_idx = reinterpret_cast<int*>(ws + p.L_.topk_idx);
+                float* g_w = reinterpret_cast<float*>(ws + p.L_.topk_w);
+                for (int e = threadIdx.x; e <= E; e += kFCons * 32) {
+                  g_offsets[e] = rt.offsets[e];
+                  if (e < E) g_counts[e] = rt.offsets[e + 1] - rt.offsets[e];
+                }
+                for (int u = threadIdx.x; u < ns; u += kFCons * 32) g_ulist[u] = rt.ulist[u];
+                for (int q = threadIdx.x; q < P; q += kFCons * 32) {
+                  g_pairs[q] = rt.pairs[q];
+                  g_inv[q] = rt.inv[q];
+                  g_idx[q] = rt.idx[q];
+                  g_w[q] = rt.w[q];
+                }
+                // token-tile prefix over the slots, in this thread's SPT slots
+                int run = trun.x;
+                for (int z = 0; z < SPT; ++z) {
+                  const int u = u0 + z;
+                  if (u < ns) {
+                    const int e = rt.ulist[u];
+                    const int n = e >= E ? T : rt.offsets[e + 1] - rt.offsets[e];
+                    g_ntoff[u] = run;
+                    run += (n + 127) / 128;
+                  }
+                }
+                if (threadIdx.x == 0) {
+                  g_ntoff[ns] = ttot.x;
+                  status[ST_UCOUNT] = ns - S;
+                }
               }
             }
           }
         }
       }
+
     }
     __syncthreads();                 // routing of this layer ready for all warps
     stamp(l, 2);

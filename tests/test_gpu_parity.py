@@ -224,7 +224,8 @@ def _stored_layer_case(name, T_list):
 
 
 def test_layer_full4_decode_stored_oracle():
-    _stored_layer_case("full4_decode", [1, 4, 16])
+    # 1-3 tokens: the routing lists built by one warp; 4 and 16: by the block scans
+    _stored_layer_case("full4_decode", [1, 2, 3, 4, 16])
 
 
 def test_layer_full2_zipf_decode_stored_oracle():
