@@ -18,11 +18,14 @@ namespace {
 
 constexpr int kCombThreads = 256;
 
+// YH: the Y rows are fp16 (each kernel instance holds one row format only,
+// so the fp16 one keeps its registers low enough for six CTAs per SM).
+template <bool YH>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(
     const float* __restrict__ Y, const int* __restrict__ inv, int T, int k, int H, int shared,
     uint16_t* __restrict__ out, int residual, uint16_t* __restrict__ xhat_next, float* __restrict__ out_f32,
-    const int* __restrict__ gate, const uint16_t* __restrict__ xin, const uint16_t* __restrict__ sgate_w,
-    int y_half) {
+    const int* __restrict__ gate, const uint16_t* __restrict__ xin, const uint16_t* __restrict__ sgate_w) {
+  constexpr bool y_half = YH;
   pdl_wait();
   if (gate && __ldcg(gate) == 0) {                // the fused decode kernel kept (and combined) the layer
     pdl_launch_dependents();
@@ -87,12 +90,35 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
 #pragma unroll
       for (int i = 0; i < VPT; ++i) acc[i] = 0.f;
     }
-    for (int j = 0; j < k; ++j) {
-      if (pos[j] < 0) continue;                 // expert owned by another rank
-      float yv[VPT];
-      yrow(pos[j], yv);
+    if (YH) {
+      // fp16 rows: four rows' loads in flight before their adds (slot order kept)
+      for (int j0 = 0; j0 < k; j0 += 4) {
+        uint4 hv[4];
 #pragma unroll
-      for (int i = 0; i < VPT; ++i) acc[i] += yv[i];
+        for (int j = 0; j < 4; ++j)
+          if (j0 + j < k && pos[j0 + j] >= 0)
+            hv[j] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(Y) + size_t(pos[j0 + j]) * H + h0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j0 + j < k && pos[j0 + j] >= 0) {
+            const uint32_t hw[4] = {hv[j].x, hv[j].y, hv[j].z, hv[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __half22float2(u32_as_h2(hw[i]));
+              acc[2 * i] += f.x;
+              acc[2 * i + 1] += f.y;
+            }
+          }
+        }
+      }
+    } else {
+      for (int j = 0; j < k; ++j) {
+        if (pos[j] < 0) continue;                 // expert owned by another rank
+        float yv[VPT];
+        yrow(pos[j], yv);
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) acc[i] += yv[i];
+      }
     }
     if (out_f32) {
       float* fd = out_f32 + size_t(t) * H + h0;
@@ -148,11 +174,11 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(
 
 cudaError_t launch_combine(const LayerArgs& a) {
   const moe_config& c = a.cfg;
-  return launch_pdl(combine_kernel, dim3(a.T), dim3(kCombThreads), 0, a.stream,
-                    reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
+  return launch_pdl(a.y_half ? combine_kernel<true> : combine_kernel<false>, dim3(a.T), dim3(kCombThreads), 0,
+                    a.stream, reinterpret_cast<const float*>(a.ws + a.L.y), reinterpret_cast<const int*>(a.ws + a.L.inv),
                     a.T, c.top_k, c.hidden, c.shared_inter > 0 ? 1 : 0, a.y, a.residual ? 1 : 0, a.xhat_next,
                     a.y_f32, a.gated ? reinterpret_cast<const int*>(a.ws + a.L.status) + ST_PATH : nullptr, a.x,
-                    a.w.shared_gate_w, a.y_half);
+                    a.w.shared_gate_w);
 }
 
 }  // namespace moe
