@@ -85,10 +85,11 @@ typedef struct moe_config {
                             fp32 scale per weight row (the
                             *_row_scales arrays); block 32 (4-bit) or
                             16 (2-bit), integer levels only.  Layers with fp8 scales
-                            run on the stand-alone GEMV kernels at
-                            every batch size (neither the
-                            single-launch decode kernel nor the
-                            tensor-core prefill reads them).       */
+                            run on the single-launch decode kernel
+                            (hidden 2048, inter 768) and on the
+                            stand-alone GEMV kernels at every batch
+                            size; the tensor-core prefill does not
+                            read them.                              */
 } moe_config;
 
 /* One layer's weights; every pointer is device memory owned by the caller. */
@@ -112,7 +113,8 @@ typedef struct moe_layer_weights {
   /* scale_fmt = 1 only (NULL otherwise): the *_scales arrays above then hold
    * one E4M3 byte per block (same shapes, one byte per element instead of
    * two), and the weight of element j of row r is q * e4m3(scale byte) *
-   * row_scale[r].  fp32, 4-byte aligned. */
+   * row_scale[r].  fp32, 16-byte aligned (the decode kernels copy them in
+   * bulk with the codes). */
   const float*    gate_up_row_scales;     /* [E][2I]                            */
   const float*    down_row_scales;        /* [E][H]                             */
   const float*    shared_gate_up_row_scales;  /* [2I]; NULL if no shared        */

@@ -17,9 +17,10 @@
 // (scaled per token by a power of two) with dp2a, sum each block exactly in
 // int32 and the blocks in fp32 with the block's scale, then reduce across the
 // lanes of the row with shuffles.  No atomics: every output element is written
-// once.  This kernel also serves the formats the single-launch decode kernel
-// leaves out: 4-bit blocks of 128 and fp8 (E4M3) block scales with an fp32
-// scale per row.
+// once.  This kernel also serves every shape and layer the single-launch
+// decode kernel leaves out (other hidden/intermediate sizes, the gated shared
+// expert) and, at every batch size, layers with fp8 (E4M3) block scales, which
+// the tensor-core prefill does not read.
 #include "decode_common.cuh"
 
 namespace moe {

@@ -126,6 +126,16 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
   return (b & 0x80u) ? -mag : mag;
 }
 
+// Two E4M3 bytes (v & 0xFF, then (v >> 8) & 0xFF) to fp16 in one hardware
+// conversion: every E4M3 value, subnormals included, is exact in fp16 (its
+// smallest step 2^-9 and largest value 448 lie inside fp16's range), so the
+// pair read as fp32 equals e4m3_value of each byte.
+__device__ __forceinline__ __half2 e4m3x2_to_h2(uint32_t v) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(d) : "r"(v));
+  return *reinterpret_cast<__half2*>(&d);
+}
+
 // Two rows of one stage (codes + scales in shared memory) and their row index
 // in the expert matrix.  With fp8 block scales (SF = 1 below) a scale is one
 // E4M3 byte and the rows carry their fp32 row scales rs0, rs1.
@@ -180,10 +190,16 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
     const uint32_t wd[2][4] = {{cw0.x, cw0.y, cw0.z, cw0.w}, {cw1.x, cw1.y, cw1.z, cw1.w}};
     if (BITS == 4) {
       float sc[2];
+      if (SF) {                                   // both rows' scale bytes in one conversion
+        const float2 f = __half22float2(e4m3x2_to_h2(uint32_t(rw.scales[c >> PS]) |
+                                                     (uint32_t(rw.scales[(Gm::SPR >> PS) + (c >> PS)]) << 8)));
+        sc[0] = f.x;
+        sc[1] = f.y;
+      } else {
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho)
-        sc[rho] = SF ? e4m3_value(rw.scales[rho * (Gm::SPR >> PS) + (c >> PS)])
-                     : __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * (Gm::SPR >> PS) * 2 + (c >> PS) * 2));
+        for (int rho = 0; rho < 2; ++rho)
+          sc[rho] = __half2float(*reinterpret_cast<const __half*>(rw.scales + rho * (Gm::SPR >> PS) * 2 + (c >> PS) * 2));
+      }
       int ia[2][NT], ib[2][NT];
 #pragma unroll
       for (int rho = 0; rho < 2; ++rho)
@@ -212,12 +228,19 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[rho][t] = fmaf(sc[rho], __int2float_rn(ia[rho][t] + ib[rho][t]), acc[rho][t]);
     } else {
-      // the four scales of the piece's blocks: four fp16 (8 bytes) or four E4M3 bytes
+      // the four scales of the piece's blocks as four fp16: read (8 bytes), or
+      // converted from four E4M3 bytes
       uint2 scp[2];
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho)
-        scp[rho] = SF ? make_uint2(*reinterpret_cast<const uint32_t*>(rw.scales + rho * Gm::SPR + c * 4), 0u)
-                      : *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
+      for (int rho = 0; rho < 2; ++rho) {
+        if (SF) {
+          const uint32_t b4 = *reinterpret_cast<const uint32_t*>(rw.scales + rho * Gm::SPR + c * 4);
+          const __half2 h01 = e4m3x2_to_h2(b4), h23 = e4m3x2_to_h2(b4 >> 16);
+          scp[rho] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+        } else {
+          scp[rho] = *reinterpret_cast<const uint2*>(rw.scales + rho * Gm::SPR * 2 + c * 8);
+        }
+      }
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         uint32_t f[2][4];
@@ -227,12 +250,8 @@ __device__ __forceinline__ void rows_dot(float* out, int out_cols, const Rows& r
         float sc[2];
 #pragma unroll
         for (int rho = 0; rho < 2; ++rho) {
-          if (SF) {
-            sc[rho] = e4m3_value((scp[rho].x >> (8 * m)) & 0xFFu);
-          } else {
-            const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
-            sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
-          }
+          const uint32_t pr = (m < 2) ? scp[rho].x : scp[rho].y;
+          sc[rho] = __half2float(__ushort_as_half((unsigned short)((m & 1) ? (pr >> 16) : (pr & 0xFFFFu))));
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {

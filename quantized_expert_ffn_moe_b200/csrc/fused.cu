@@ -480,7 +480,9 @@ struct GroupTok {
 // (warps grp*kNCW ...): walks the same stage sequence as the producer and
 // takes the stages whose index has the group's parity.  A group stages the
 // tokens of a (slot, chunk) itself when it meets its first stage of it.
-template <int MODE, int BITS, int LPR, int CPL, int PS>
+// SF = 1: fp8 block scales (one E4M3 byte per block), with the fp32 scales of
+// the stage's rows staged after them.
+template <int MODE, int BITS, int LPR, int CPL, int PS, int SF>
 __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur, long long w1, unsigned char* ring,
                              int ring_stride, uint64_t* full, uint64_t* empty, int* consumed, int grp,
                              const uint16_t* xsrc, const float* rnorm, const float* hin, float* out, int out_cols,
@@ -488,6 +490,7 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
                              int16_t* xs_grp, const GroupTok& tk, volatile int* abort_flag, int* status,
                              unsigned long long* tacc = nullptr, unsigned long long* tabs = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
+  constexpr int SSZ = SF ? 1 : 2;                   // bytes per block scale
   constexpr int K = Gm::K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool timed = tacc != nullptr && threadIdx.x == 0;
@@ -545,17 +548,22 @@ __device__ void consume_pass(const FusedParams& p, const SRoute& rt, FCursor cur
     }
     if (ok) {
       const unsigned char* st = ring + slot * ring_stride;
-      const Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * 2, cur.stage * Gm::RPS + rl0,
-                      code_xor(BITS, p.cfg.half_levels)};
+      Rows rows{st + rl0 * Gm::RB, st + Gm::CODE_BYTES + rl0 * (Gm::SPR >> PS) * SSZ, cur.stage * Gm::RPS + rl0,
+                code_xor(BITS, p.cfg.half_levels)};
+      if (SF) {                                   // the row scales the producer staged after the block scales
+        const float* rss = reinterpret_cast<const float*>(st + Gm::CODE_BYTES + Gm::RPS * Gm::SPR);
+        rows.rs0 = rss[rl0];
+        rows.rs1 = rss[rl0 + 1];
+      }
       const int nc = cur.nc;
 #pragma unroll 1
       for (int tb = 0; tb < nc; tb += 4) {
         const int nt = min(4, nc - tb);
         const int16_t* xb = pre ? xs_pre : xs_grp + size_t(tb) * K;
         const int* xr = pre ? tk.xrow : nullptr;
-        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 1, xr);
-        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 2, xr);
-        else rows_dot<MODE, BITS, LPR, CPL, 4, PS>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, nt, xr);
+        if (nt == 1) rows_dot<MODE, BITS, LPR, CPL, 1, PS, SF>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 1, xr);
+        else if (nt == 2) rows_dot<MODE, BITS, LPR, CPL, 2, PS, SF>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, 2, xr);
+        else rows_dot<MODE, BITS, LPR, CPL, 4, PS, SF>(out, out_cols, rows, xb, tb, lr, tk.inv, tk.w, tk.pos, nt, xr);
       }
     }
     __syncwarp();
@@ -609,10 +617,14 @@ struct Publisher {
 };
 
 // Producer side of one pass: issues this CTA's stages into the ring.
-template <int BITS, int LPR, int CPL>
-__device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, const uint16_t* scales,
-                             const uint8_t* sh_codes, const uint16_t* sh_scales, size_t expert_code_bytes,
-                             size_t expert_scale_count, unsigned char* ring, int ring_stride, uint64_t* full,
+// SF = 1: the block scales are E4M3 bytes, and the stage's fp32 row scales
+// (rs: rows_pe per routed expert; sh_rs: the shared expert) follow them in
+// the slot at CODE_BYTES + RPS * SPR.
+template <int BITS, int LPR, int CPL, int SF>
+__device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, const unsigned char* scales,
+                             const uint8_t* sh_codes, const unsigned char* sh_scales, size_t expert_code_bytes,
+                             size_t expert_scale_count, const float* rs, const float* sh_rs, int rows_pe,
+                             unsigned char* ring, int ring_stride, uint64_t* full,
                              uint64_t* empty, int* issued, volatile int* abort_flag, int* status, Publisher& pub,
                              bool gate_up, int block, unsigned long long* tabs = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
@@ -631,15 +643,21 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
     }
     const bool sh = cur.e >= cur.E;
     const uint8_t* cb = sh ? sh_codes : codes + size_t(cur.e) * expert_code_bytes;
-    const uint16_t* sb = sh ? sh_scales : scales + size_t(cur.e) * expert_scale_count;
+    constexpr int SSZ = SF ? 1 : 2;             // bytes per block scale
+    const unsigned char* sb = sh ? sh_scales : scales + size_t(cur.e) * expert_scale_count * SSZ;
     const size_t row0 = size_t(cur.stage) * Gm::RPS;
     unsigned char* dst = ring + slot * ring_stride;
     const int spr = scales_per_row(Gm::K, block);
-    const uint32_t sbytes = uint32_t(Gm::RPS) * spr * 2;
-    mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes);
+    const uint32_t sbytes = uint32_t(Gm::RPS) * spr * SSZ;
+    constexpr uint32_t RSB = SF ? Gm::RPS * 4 : 0;     // row-scale bytes of the stage
+    mbar_arrive_expect_tx(&full[slot], Gm::CODE_BYTES + sbytes + RSB);
     const uint64_t pol = l2_evict_first_policy();
     bulk_g2s_hint(dst, cb + row0 * Gm::RB, Gm::CODE_BYTES, &full[slot], pol);
-    bulk_g2s_hint(dst + Gm::CODE_BYTES, sb + row0 * spr, sbytes, &full[slot], pol);
+    bulk_g2s_hint(dst + Gm::CODE_BYTES, sb + row0 * spr * SSZ, sbytes, &full[slot], pol);
+    if (SF) {
+      const float* rb = sh ? sh_rs : rs + size_t(cur.e) * rows_pe;
+      bulk_g2s_hint(dst + Gm::CODE_BYTES + Gm::RPS * Gm::SPR, rb + row0, RSB, &full[slot], pol);
+    }
     pub.rslot[slot] = gate_up ? cur.slot : -1;
     if (gate_up) ++pub.pending;
     *issued = i + 1;
@@ -666,7 +684,7 @@ __device__ void drain_publish(int issued, uint64_t* empty, volatile int* abort_f
   pub.flush();
 }
 
-template <int BITS, int LG, int CG, int LD, int CD, int NPL, int PS>
+template <int BITS, int LG, int CG, int LD, int CD, int NPL, int PS, int SF>
 __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid_constant__ FusedParams p) {
   using GU = Geom<BITS, LG, CG>;
   using DN = Geom<BITS, LD, CD>;
@@ -1086,18 +1104,22 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
         pub.reset();
         if (g0 < g1) {
           cg.init(g0);
-          produce_pass<BITS, LG, CG>(cg, g1, lw.gate_up_codes, lw.gate_up_scales, lw.shared_gate_up_codes,
-                                      lw.shared_gate_up_scales, size_t(2 * I) * H * c.bits / 8,
-                                      size_t(2 * I) * (H / c.block), ring, RING_STRIDE, full, empty, &issued,
+          produce_pass<BITS, LG, CG, SF>(cg, g1, lw.gate_up_codes,
+                                      reinterpret_cast<const unsigned char*>(lw.gate_up_scales), lw.shared_gate_up_codes,
+                                      reinterpret_cast<const unsigned char*>(lw.shared_gate_up_scales),
+                                      size_t(2 * I) * H * c.bits / 8,
+                                      size_t(2 * I) * (H / c.block), lw.gate_up_row_scales,
+                                      lw.shared_gate_up_row_scales, 2 * I, ring, RING_STRIDE, full, empty, &issued,
                                       abort_flag, status, pub, true, c.block,
                                       p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 28 : nullptr);
         }
         pub.issued_all();
         if (d0 < d1) {
           cd.init(d0);
-          produce_pass<BITS, LD, CD>(cd, d1, lw.down_codes, lw.down_scales, lw.shared_down_codes,
-                                      lw.shared_down_scales, size_t(H) * I * c.bits / 8, size_t(H) * (I / c.block),
-                                      ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false, c.block,
+          produce_pass<BITS, LD, CD, SF>(cd, d1, lw.down_codes, reinterpret_cast<const unsigned char*>(lw.down_scales),
+                                      lw.shared_down_codes, reinterpret_cast<const unsigned char*>(lw.shared_down_scales),
+                                      size_t(H) * I * c.bits / 8, size_t(H) * (I / c.block), lw.down_row_scales,
+                                      lw.shared_down_row_scales, H, ring, RING_STRIDE, full, empty, &issued, abort_flag, status, pub, false, c.block,
                                       p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 30 : nullptr);
         }
         drain_publish(issued, empty, abort_flag, status, pub);
@@ -1106,7 +1128,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
       // ---------------------------------------------------------- phase G
       if (g0 < g1) {
         cg.init(g0);
-        consume_pass<GATEUP, BITS, LG, CG, PS>(p, rt, cg, g1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
+        consume_pass<GATEUP, BITS, LG, CG, PS, SF>(p, rt, cg, g1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
                                            rnorm, nullptr, hbuf, I, p.pre ? xs : nullptr, inv_all, nullptr, 0, xs_grp,
                                            tk, abort_flag, status,
                                            p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 11 : nullptr,
@@ -1152,7 +1174,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
           }
           all_sync();
         }
-        consume_pass<DOWN, BITS, LD, CD, PS>(p, rt, cd, d1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
+        consume_pass<DOWN, BITS, LD, CD, PS, SF>(p, rt, cd, d1, ring, RING_STRIDE, full, empty, &consumed, grp, xsrc,
                                          rnorm, hbuf, ybuf, H, dpre ? xs : nullptr, dinv, dwt, lo, xs_grp, tk,
                                          abort_flag, status,
                                          p.timing && l == 0 ? p.timing + blockIdx.x * kTimePoints + 16 : nullptr,
@@ -1202,7 +1224,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   // the ring is drained: every issued stage was waited on by the consumers
 }
 
-template <int BITS, int LG, int CG, int LD, int CD, int NPL, int PS = 0>
+template <int BITS, int LG, int CG, int LD, int CD, int NPL, int PS = 0, int SF = 0>
 cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   using GU = Geom<BITS, LG, CG>;
   using DN = Geom<BITS, LD, CD>;
@@ -1241,7 +1263,7 @@ cudaError_t launch_fused_t(const FusedParams& p, int num_sms, cudaStream_t s) {
   q.xs_halves = (long long)xs_halves;
   const size_t smem = q.smem_xs_off + xs_halves * 2;
   if (smem > size_t(kSmemMax)) return cudaErrorInvalidValue;
-  auto kern = fused_decode_kernel<BITS, LG, CG, LD, CD, NPL, PS>;
+  auto kern = fused_decode_kernel<BITS, LG, CG, LD, CD, NPL, PS, SF>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg{};
@@ -1286,7 +1308,6 @@ void set_fused_timing(unsigned long long* buf) { g_fused_timing = buf; }
 
 bool fused_supported(const moe_config& c, int T) {
   if (T < 1 || T > kFMaxTokens || T * c.top_k > kFMaxPairs) return false;
-  if (c.scale_fmt != 0) return false;              // fp8 block scales: the stand-alone GEMV reads them
   return c.hidden == 2048 && c.inter == 768 && (c.num_experts % 32) == 0 && c.num_experts <= 1024;
 }
 
@@ -1323,18 +1344,24 @@ cudaError_t launch_fused_decode(const moe_config& c, const moe_layer_weights* la
     if (c.bits == 4) {
       switch (npl) {
         case 16: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 16, 2>(p, num_sms, s)
-                                      : launch_fused_t<4, 16, 4, 8, 3, 16>(p, num_sms, s); break;
+                     : c.scale_fmt ? launch_fused_t<4, 16, 4, 8, 3, 16, 0, 1>(p, num_sms, s)
+                                   : launch_fused_t<4, 16, 4, 8, 3, 16>(p, num_sms, s); break;
         case 32: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 32, 2>(p, num_sms, s)
-                                      : launch_fused_t<4, 16, 4, 8, 3, 32>(p, num_sms, s); break;
+                     : c.scale_fmt ? launch_fused_t<4, 16, 4, 8, 3, 32, 0, 1>(p, num_sms, s)
+                                   : launch_fused_t<4, 16, 4, 8, 3, 32>(p, num_sms, s); break;
         case 8: err = c.block == 128 ? launch_fused_t<4, 16, 4, 8, 3, 8, 2>(p, num_sms, s)
-                                     : launch_fused_t<4, 16, 4, 8, 3, 8>(p, num_sms, s); break;
+                    : c.scale_fmt ? launch_fused_t<4, 16, 4, 8, 3, 8, 0, 1>(p, num_sms, s)
+                                  : launch_fused_t<4, 16, 4, 8, 3, 8>(p, num_sms, s); break;
         default: return cudaErrorInvalidValue;
       }
     } else {
       switch (npl) {
-        case 16: err = launch_fused_t<2, 16, 2, 4, 3, 16>(p, num_sms, s); break;
-        case 32: err = launch_fused_t<2, 16, 2, 4, 3, 32>(p, num_sms, s); break;
-        case 8: err = launch_fused_t<2, 16, 2, 4, 3, 8>(p, num_sms, s); break;
+        case 16: err = c.scale_fmt ? launch_fused_t<2, 16, 2, 4, 3, 16, 0, 1>(p, num_sms, s)
+                                   : launch_fused_t<2, 16, 2, 4, 3, 16>(p, num_sms, s); break;
+        case 32: err = c.scale_fmt ? launch_fused_t<2, 16, 2, 4, 3, 32, 0, 1>(p, num_sms, s)
+                                   : launch_fused_t<2, 16, 2, 4, 3, 32>(p, num_sms, s); break;
+        case 8: err = c.scale_fmt ? launch_fused_t<2, 16, 2, 4, 3, 8, 0, 1>(p, num_sms, s)
+                                  : launch_fused_t<2, 16, 2, 4, 3, 8>(p, num_sms, s); break;
         default: return cudaErrorInvalidValue;
       }
     }

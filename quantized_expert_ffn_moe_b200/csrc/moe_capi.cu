@@ -69,9 +69,9 @@ int validate_weights(const moe_config* c, const moe_layer_weights* w) {
   const void* rs[] = {w->gate_up_row_scales, w->down_row_scales};
   const void* srs[] = {w->shared_gate_up_row_scales, w->shared_down_row_scales};
   for (const void* p : rs)
-    if (c->scale_fmt == 1 ? (!p || !aligned(p, 4)) : p != nullptr) return MOE_ERR_INVALID_ARG;
+    if (c->scale_fmt == 1 ? (!p || !aligned(p, 16)) : p != nullptr) return MOE_ERR_INVALID_ARG;
   for (const void* p : srs)
-    if (c->scale_fmt == 1 && c->shared_inter > 0 ? (!p || !aligned(p, 4)) : (c->scale_fmt == 0 && p != nullptr))
+    if (c->scale_fmt == 1 && c->shared_inter > 0 ? (!p || !aligned(p, 16)) : (c->scale_fmt == 0 && p != nullptr))
       return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }

@@ -105,7 +105,7 @@ def _layer(lib, c, w, x=1 << 30, T=4, y=2 << 30, ws=3 << 30, ws_bytes=None):
 
 
 def test_fp8_scale_arguments(lib):
-    """scale_fmt 1 needs the fp32 row scales (4-byte aligned), scale_fmt 0
+    """scale_fmt 1 needs the fp32 row scales (16-byte aligned), scale_fmt 0
     refuses them; fp8 scales only with blocks of 32 (4-bit) / 16 (2-bit)."""
     c8 = cfg()
     c8.scale_fmt = 1
@@ -116,6 +116,9 @@ def test_fp8_scale_arguments(lib):
     w = _fake_weights(fp8=True)
     w.down_row_scales += 2
     assert _layer(lib, c8, w) == -1                                        # misaligned row scales
+    w = _fake_weights(fp8=True)
+    w.shared_gate_up_row_scales += 4
+    assert _layer(lib, c8, w) == -1                                        # 4-byte but not 16-byte aligned
     w = _fake_weights(fp8=True, shared=False)
     c8s = cfg(shared=False)
     c8s.scale_fmt = 1
