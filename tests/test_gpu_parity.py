@@ -451,11 +451,14 @@ def test_layer_full2_half_levels_sampled(T, path):
 
 # ------------------------------------------------------- fp8 block scales ---
 
-@pytest.mark.parametrize("shape,T", [(FULL4F8, 1), (FULL4F8, 16), (FULL4F8, 100), (FULL2F8, 16), (FULL2F8, 64)],
-                         ids=["full4_t1", "full4_t16", "full4_t100", "full2_t16", "full2_t64"])
+@pytest.mark.parametrize("shape,T", [(FULL4F8, 1), (FULL4F8, 3), (FULL4F8, 16), (FULL4F8, 48), (FULL4F8, 100),
+                                     (FULL2F8, 16), (FULL2F8, 64)],
+                         ids=["full4_t1", "full4_t3", "full4_t16", "full4_t48", "full4_t100", "full2_t16", "full2_t64"])
 def test_layer_full_fp8_scales_sampled(shape, T):
-    """Full shape with E4M3 block scales and fp32 row scales: the stand-alone
-    GEMV kernels at every batch size (decode and the 100-token batch)."""
+    """Full shape with E4M3 block scales and fp32 row scales: the
+    single-launch decode kernel up to 64 tokens (3 tokens: the one-warp
+    routing lists; 48: no tensor-core hand-over for this format) and the
+    stand-alone GEMV kernels for the 100-token batch."""
     _sampled_full_case(shape, T, 17, 0, min(3, T), 700 + T)
 
 

@@ -35,6 +35,7 @@ import quantized_expert_ffn_moe_b200 as q
 pytestmark = pytest.mark.gpu
 
 MID4 = mi.MoeShape(experts=32, hidden=512, inter=256, top_k=4, shared=True, bits=4, block=32)
+FULL4F8 = mi.MoeShape(experts=512, hidden=2048, inter=768, top_k=10, shared=True, bits=4, block=32, fp8_scales=True)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -124,6 +125,31 @@ def test_stack_layer_steps_live_oracle(shape, T):
         if differ:
             r = orc.layer_forward(lay, x, rmsnorm=True, topk_override={t: trace[0][t] for t in differ})
         assert_stack_step(orc.bf16_to_f64(x), got, r["out"])
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_stack_fp8_scales_full_live_oracle(T):
+    """fp8 block scales through the stack's single-launch decode kernel
+    (RMSNorm in its first phase, the residual in its combine): each of two
+    full-shape layers on its own seeded input against the oracle, and the
+    two-layer launch equal to two one-layer calls."""
+    shape = FULL4F8
+    ws = [gc.device_layer(shape, 0, l) for l in range(2)]
+    for l in range(2):
+        x = mi.hidden_states_bf16(T, shape.hidden, 0, 90 + l)
+        got, trace = _gpu_stack(shape, [ws[l]], x)
+        lay = gc.host_oracle_layer(shape, 0, l, cache_size=12)
+        r = orc.layer_forward(lay, x, rmsnorm=True)
+        differ = gc.check_selection(r["logits"], r["idx"], trace[0], shape.top_k)
+        if differ:
+            r = orc.layer_forward(lay, x, rmsnorm=True, topk_override={t: trace[0][t] for t in differ})
+        assert_stack_step(orc.bf16_to_f64(x), got, r["out"])
+    x = mi.hidden_states_bf16(T, shape.hidden, 0, 95)
+    whole = _stack_bits(shape, ws, x)
+    step = x
+    for w in ws:
+        step = _stack_bits(shape, [w], step)
+    np.testing.assert_array_equal(whole, step)
 
 
 # --------------------------------------------------------- composition ---
