@@ -628,6 +628,11 @@ __device__ void produce_pass(FCursor cur, long long w1, const uint8_t* codes, co
                              uint64_t* empty, int* issued, volatile int* abort_flag, int* status, Publisher& pub,
                              bool gate_up, int block, unsigned long long* tabs = nullptr) {
   using Gm = Geom<BITS, LPR, CPL>;
+  // fp8 scales: the E4M3 bytes (RPS * SPR) and the fp32 row scales (RPS * 4)
+  // share the slot's scale region, sized for RPS * SPR fp16 scales; the row
+  // scales' bulk copy needs a 16-byte aligned destination and size
+  static_assert(!SF || (Gm::SPR >= 4 && (Gm::CODE_BYTES + Gm::RPS * Gm::SPR) % 16 == 0 && (Gm::RPS * 4) % 16 == 0),
+                "fp8 row scales do not fit the stage's scale region");
   const int first_issue = *issued;
   for (; cur.valid(w1); cur.advance()) {
     const int i = *issued;

@@ -630,13 +630,29 @@ __global__ void __launch_bounds__(PEp<MODE>::kThreads, 1) prefill_gemm_kernel(
   }
 }
 
+// 1-D bulk copy from shared to global memory (both addresses 16-byte aligned,
+// bytes a multiple of 16), in this thread's bulk async-group.
+__device__ __forceinline__ void bulk_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Until this thread's bulk copies have read their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Until this thread's bulk copies have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Shared-memory stores of this thread made visible to the bulk-copy (async) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // Token rows scattered into expert order as fp16 (routed positions, then the
 // shared expert's): one warp per token converts its row once -- exactly, after
 // the power of two that brings its largest magnitude into [2^13, 2^14), with k
 // permuted within each group of 8 (4-bit) / 16 (2-bit) to match the
-// dequantizer's pair order -- and stores it at every position of the token
-// (inv[t k + j], position -1 = another rank's expert; T k + t for the shared
-// expert), with xinv = the inverse power of two.
+// dequantizer's pair order -- into its row of shared memory, and one lane
+// copies that row in bulk to every position of the token (inv[t k + j],
+// position -1 = another rank's expert; T k + t for the shared expert), with
+// xinv = the inverse power of two.  Dynamic shared memory: 8 rows of H fp16.
 template <int BITS>
 __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __restrict__ x, RouteView rv, int H,
                                                             uint16_t* __restrict__ xs, float* __restrict__ xinv,
@@ -646,7 +662,9 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
   if (gated && __ldcg(rv.status + ST_PATH) == 0) return;     // the fused decode kernel kept the layer
   constexpr int G = BITS == 4 ? 8 : 16;
   constexpr int kMaxChunks = 4096 / (32 * G);              // chunks of G elements per lane (H <= 4096)
+  extern __shared__ __align__(16) unsigned char gsm[];
   const int lane = threadIdx.x & 31;
+  uint16_t* srow = reinterpret_cast<uint16_t*>(gsm) + size_t(threadIdx.x >> 5) * H;
   for (int tok = blockIdx.x * 8 + (threadIdx.x >> 5); tok < rv.T; tok += gridDim.x * 8) {
     const uint16_t* src = x + size_t(tok) * H;
     float vmax = 0.f;
@@ -687,23 +705,34 @@ __global__ void __launch_bounds__(256) gather_tokens_kernel(const uint16_t* __re
       }
       pack_pair_order<G>(in, mul, row[c]);
     }
+    // the warp's row buffer is free again once the previous token's copies
+    // have read it
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < kMaxChunks; ++c) {
+      const int h0 = (c * 32 + lane) * G;
+      if (c * 32 * G >= H) break;
+      if (h0 >= H) continue;
+#pragma unroll
+      for (int q = 0; q < G / 8; ++q) *reinterpret_cast<uint4*>(srow + h0 + 8 * q) = row[c][q];
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
     // every position of the token: its k routed pairs, then the shared expert
-    const int np = rv.k + (rv.shared ? 1 : 0);
-    for (int j = 0; j < np; ++j) {
-      const int p = j < rv.k ? __ldg(rv.inv + size_t(tok) * rv.k + j) : rv.T * rv.k + tok;
-      if (p < 0) continue;                                   // another rank's expert
-      uint16_t* dst = xs + size_t(p) * H;
-#pragma unroll
-      for (int c = 0; c < kMaxChunks; ++c) {
-        const int h0 = (c * 32 + lane) * G;
-        if (c * 32 * G >= H) break;
-        if (h0 >= H) continue;
-#pragma unroll
-        for (int q = 0; q < G / 8; ++q) *reinterpret_cast<uint4*>(dst + h0 + 8 * q) = row[c][q];
+    if (lane == 0) {
+      const int np = rv.k + (rv.shared ? 1 : 0);
+      for (int j = 0; j < np; ++j) {
+        const int p = j < rv.k ? __ldg(rv.inv + size_t(tok) * rv.k + j) : rv.T * rv.k + tok;
+        if (p < 0) continue;                                 // another rank's expert
+        bulk_s2g(xs + size_t(p) * H, srow, uint32_t(H) * 2);
+        xinv[p] = inv_mul;
       }
-      if (lane == 0) xinv[p] = inv_mul;
+      bulk_commit();
     }
   }
+  // the rows are in global memory before the warp (and its shared memory) goes
+  if (lane == 0) bulk_wait_all();
 }
 
 // Router logits of a large batch on the tensor cores:
@@ -939,9 +968,13 @@ cudaError_t launch_prefill_ffn(const LayerArgs& a) {
   uint16_t* hs = reinterpret_cast<uint16_t*>(a.ws + a.L.h);
   float* xinv = reinterpret_cast<float*>(a.ws + a.L.xscale);
   const int gblocks = max(1, min(a.num_sms * 8, (a.T + 7) / 8));    // one warp per token
-  cudaError_t err = bits == 4
-      ? launch_pdl(gather_tokens_kernel<4>, dim3(gblocks), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv, a.gated)
-      : launch_pdl(gather_tokens_kernel<2>, dim3(gblocks), dim3(256), 0, a.stream, a.x, rv, H, xs, xinv, a.gated);
+  const size_t gsmem = size_t(8) * H * 2;                              // one fp16 row per warp
+  cudaError_t err = cudaFuncSetAttribute(bits == 4 ? gather_tokens_kernel<4> : gather_tokens_kernel<2>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(gsmem));
+  if (err != cudaSuccess) return err;
+  err = bits == 4
+      ? launch_pdl(gather_tokens_kernel<4>, dim3(gblocks), dim3(256), gsmem, a.stream, a.x, rv, H, xs, xinv, a.gated)
+      : launch_pdl(gather_tokens_kernel<2>, dim3(gblocks), dim3(256), gsmem, a.stream, a.x, rv, H, xs, xinv, a.gated);
   if (err != cudaSuccess) return err;
 
   PrefillArgs g{};
