@@ -754,6 +754,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_decode_kernel(const __grid
   // programmatic dependency, so this launch overlaps that one); nothing in
   // the workspace is touched before it has completed
   pdl_wait();
+  // the next call's status reset may be scheduled now; it waits for this
+  // grid to complete before it clears anything
+  pdl_launch_dependents();
   int issued = 0, consumed = 0;
   const unsigned G = gridDim.x;
   const uint16_t* xsrc = p.stack ? p.y : p.x;

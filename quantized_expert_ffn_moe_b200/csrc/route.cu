@@ -590,12 +590,12 @@ cudaError_t launch_topk_group_any(const moe_config& c, int T, char* ws, const La
 // touches the workspace.
 __global__ void status_reset_kernel(int* status) {
   pdl_launch_dependents();
+  pdl_wait();                    // whatever ran before on the stream has completed
   for (int i = threadIdx.x; i < ST_COUNT; i += blockDim.x) status[i] = 0;
 }
 
 cudaError_t launch_status_reset(int* status, cudaStream_t s) {
-  status_reset_kernel<<<1, 128, 0, s>>>(status);
-  return cudaGetLastError();
+  return launch_pdl(status_reset_kernel, dim3(1), dim3(128), 0, s, status);
 }
 
 cudaError_t launch_route_full(const moe_config& c, const uint16_t* router_w, const float* bias,
